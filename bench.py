@@ -1,0 +1,414 @@
+"""Benchmark of the latent-KV chunk attention hot path on B200.
+
+One step = one denoising pass of one chunk through one Wan2.1-T2V-1.3B-shaped
+latent attention layer: cache append (down-projection + ring write), window
+3D-RoPE, query absorption, and chunk attention with the fused W_uv
+up-projection -- N_q = 4680 queries x 12 heads over N_k = 32760 keys.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are replicas: every
+rank runs its own independent rollout; the timed region is bracketed by a
+barrier and CUDA synchronisation, and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from latent_kv_attention_down_b200 import synth  # noqa: E402
+
+METRIC = "MLA chunk-attention TFLOP/s and query tokens/s, Wan-1.3B layer shape, 1×B200"
+WORKLOAD = synth.WAN
+N_LAYER_SETS = 12  # distinct layer buffers cycled through: ~1 GB of inputs, far above the 126 MB L2
+
+
+def step_flops(d=WORKLOAD):
+    """Algorithmic FLOPs of one step (absorbed form)."""
+    nq, nk = d.n_queries, d.window_tokens
+    attn = 2 * nq * nk * d.n_heads * (2 * d.d_latent + d.d_rope)
+    append = 2 * nq * d.d_model * (d.d_latent + d.d_rope)
+    absorb = 2 * nq * d.n_heads * d.d_nope * d.d_latent
+    uv = 2 * nq * d.n_heads * d.d_latent * d.d_head
+    return {"attention": attn, "append": append, "q_absorb": absorb, "w_uv": uv,
+            "total": attn + append + absorb + uv}
+
+
+def dense_flops(d=WORKLOAD):
+    nq, nk = d.n_queries, d.window_tokens
+    return {"attention": 2 * nq * nk * d.n_heads * (2 * d.d_head),
+            "append": 2 * nq * d.d_model * (d.d_latent + d.d_rope) + 2 * nq * d.n_heads * d.d_latent * (d.d_nope + d.d_head)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j["hbm_gbs"], j["bf16_tflops"], j.get("bf16_tflops_sustained", j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def profiled_traffic(kernel_file, summary):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current source of the kernel (its sha256 is recorded beside it)."""
+    path = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "latent_kv_attention_down_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+
+def oracle_sample(n_queries=256, heads=None, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload: the full
+    32760-key window built from x (down-projection, per-head reconstruction,
+    3D-RoPE, softmax) for ``n_queries`` query tokens of the chunk, all heads."""
+    import oracle.vmla_oracle as O
+    d = WORKLOAD
+    w = synth.weights(d, 0, seed)
+    frame_x = {}
+    for c in range(d.window_frames // d.chunk_frames):
+        x = synth.activations(d, 0, c, base_seed=seed)[0]
+        for k in range(d.chunk_frames):
+            frame_x[c * d.chunk_frames + k] = x[k * d.tokens_per_frame:(k + 1) * d.tokens_per_frame]
+    last = d.window_frames // d.chunk_frames - 1
+    q = synth.queries(d, 0, last, base_seed=seed)[0]
+    rows = np.arange(n_queries)
+    t0 = time.perf_counter()
+    c, r, kpos, torg = O.window_latents(frame_x, d.window_frames, d.window_frames, w.w_down, d.d_latent,
+                                        d.grid_h, d.grid_w)
+    qpos = O.chunk_query_positions(last * d.chunk_frames, d.chunk_frames, torg, d.grid_h, d.grid_w)
+    O.chunk_attention(c, r, kpos, q, qpos, w.w_uk, w.w_uv, d_nope=d.d_nope, rope_pairs=d.rope_pairs,
+                      query_rows=rows, heads=heads)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(n_queries=256):
+    secs = oracle_sample(n_queries)
+    per_query = step_flops()["total"] / WORKLOAD.n_queries
+    return {"value": n_queries * per_query / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "query_tokens_per_s": n_queries / secs, "seconds": round(secs, 2),
+            "sample": f"fp64 numpy oracle, {n_queries} of the 4680 query tokens x 12 heads over the full "
+                      f"32760-key window, window built from x (down-projection, per-head K/V, 3D-RoPE, softmax); "
+                      f"TFLOP/s credited at the GPU step's FLOPs per query token"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    n = 128
+    times = []
+    for _ in range(args.warmup_ref):
+        oracle_sample(n)
+    for _ in range(args.steps_ref):
+        times.append(oracle_sample(n))
+    secs = sum(times) / len(times)
+    per_query = step_flops()["total"] / WORKLOAD.n_queries
+    value = n * per_query / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps_ref, "warmup": args.warmup_ref, "ms_per_step": secs * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "wan1.3b-layer: N_q=4680 (sampled 128), N_k=32760, n_h=12, d_c=192, d_rope=32"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} query tokens x 12 heads over the full window per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from latent_kv_attention_down_b200 import api
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    d = WORKLOAD
+    L = N_LAYER_SETS
+    cfg = api.config_from_dims(d, layers=L)
+    m = api.LatentKVAttention(cfg).allocate(device=dev, design=api.DESIGN_RECON_ONCE, dense=args.dense)
+    bf = torch.bfloat16
+    seed = 1000 * rank
+    wts = [synth.weights(d, l, seed) for l in range(L)]
+    W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv)) for w in wts]
+    chunks = d.window_frames // d.chunk_frames
+    first = (chunks - 1) * d.chunk_frames
+    # fill every layer's 21-frame window (the fill activations are shared by the layers), then give each
+    # layer set its own chunk activations, queries and output for the timed passes
+    for c in range(chunks):
+        x = torch.from_numpy(synth.activations(d, 0, c, base_seed=seed)).to(dev, bf)
+        for l in range(L):
+            m.append(l, x, W[l][0], c * d.chunk_frames, d.chunk_frames)
+            if args.dense:
+                m.dense_append(l, x, W[l][0], W[l][1], W[l][2], c * d.chunk_frames, d.chunk_frames)
+    xs, qs, outs = [], [], []
+    for l in range(L):
+        xs.append(torch.from_numpy(synth.activations(d, l, chunks - 1, pass_=1, base_seed=seed)).to(dev, bf))
+        qs.append(torch.from_numpy(synth.queries(d, l, chunks - 1, base_seed=seed)).to(dev, bf))
+        outs.append(torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev))
+    torch.cuda.synchronize()
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+
+    def step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_ABSORBED)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(fn, steps, warmup, profile=False):
+        for i in range(warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        barrier()
+        if profile:
+            m.profile(True)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s0.record()
+        for i in range(steps):
+            fn(warmup + i)
+        s1.record()
+        torch.cuda.synchronize()
+        barrier()
+        return s0.elapsed_time(s1)
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(visible.split(",")[local_rank] if visible else local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    ms = timed(step, args.steps, args.warmup, profile=True)
+    clk = clocks.stop()
+    per_kernel = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "attention")}
+    m.profile(False)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    ms_step = max_over_ranks(ms / args.steps)
+    F = step_flops()
+    value = world * F["total"] / (ms_step * 1e-3) / 1e12
+    tokens = world * d.n_queries / (ms_step * 1e-3)
+
+    # ------------------------------------------------ end to end from pinned host memory
+    xh = [xs[l].cpu().pin_memory() for l in range(2)]
+    qh = [qs[l].cpu().pin_memory() for l in range(2)]
+    oh = [torch.empty(outs[0].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    xd, qd, od = torch.empty_like(xs[0]), torch.empty_like(qs[0]), torch.empty_like(outs[0])
+
+    def e2e_step(i):
+        l = i % 2
+        m.step_host(l, xh[l], qh[l], oh[l], W[l][0], W[l][1], W[l][2], xd, qd, od, first, d.chunk_frames,
+                    api.DESIGN_ABSORBED)
+
+    e2e_steps = max(10, args.steps // 4)
+    ms_e2e = max_over_ranks(timed(e2e_step, e2e_steps, 3) / e2e_steps)
+    h2d = xh[0].numel() * 2 + qh[0].numel() * 2
+    d2h = oh[0].numel() * 4
+
+    # ------------------------------------------------ dense per-head comparison on the same box
+    dense = None
+    if args.dense:
+        def dense_step(i):
+            l = i % L
+            m.dense_append(l, xs[l], W[l][0], W[l][1], W[l][2], first, d.chunk_frames)
+            m.dense_attention(l, qs[l], outs[l], first, d.chunk_frames)
+        dsteps = max(10, args.steps // 4)
+        ms_d = timed(dense_step, dsteps, 3, profile=True)
+        da_ms, da_n = m.profile_read("dense_attention")
+        dap_ms, dap_n = m.profile_read("dense_append")
+        m.profile(False)
+        DF = dense_flops()
+        dense = {"ms_per_step": max_over_ranks(ms_d / dsteps),
+                 "attention_ms": da_ms / max(da_n, 1), "append_ms": dap_ms / max(dap_n, 1),
+                 "attention_tflops": DF["attention"] / (da_ms / max(da_n, 1) * 1e-3) / 1e12,
+                 "cache_scalars_per_token": 2 * d.n_heads * d.d_head, "window_read_bytes": d.window_tokens * 2 * d.n_heads * d.d_head * 2}
+
+    # ------------------------------------------------ design (b'): per-head K/V rebuilt once per call
+    def recon_step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_RECON_ONCE)
+    rsteps = max(10, args.steps // 4)
+    ms_r = timed(recon_step, rsteps, 3, profile=True)
+    rk = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "reconstruct_once", "dense_attention")}
+    m.profile(False)
+    DF = dense_flops()
+    ra_ms = rk["dense_attention"][0] / max(rk["dense_attention"][1], 1)
+    recon_once = {"ms_per_step": max_over_ranks(ms_r / rsteps),
+                  "tflops_effective": world * F["total"] / (max_over_ranks(ms_r / rsteps) * 1e-3) / 1e12,
+                  "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in rk.items()},
+                  "attention_tflops_issued": DF["attention"] / (ra_ms * 1e-3) / 1e12}
+
+    # ------------------------------------------------ roofline of the dominant kernel (attention)
+    hbm, tc_burst, tc_sust, src = load_peaks()
+    at_ms, at_n = per_kernel["attention"]
+    at_launch_ms = at_ms / max(at_n, 1)
+    achieved = F["attention"] / (at_launch_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": achieved / tc_burst, "peak_source": f"{src} bf16 dense (burst, cuBLAS)",
+                "frac_of_sustained": achieved / tc_sust,
+                "traffic": profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"),
+                "kernel": "attn_tc_kernel<192,false>", "launch_ms": at_launch_ms,
+                "algorithmic_flops_per_launch": F["attention"]}
+    kernels = {}
+    for k, (ms_k, n_k) in per_kernel.items():
+        kernels[k] = {"ms_per_launch": ms_k / max(n_k, 1), "launches": n_k}
+    # HBM-bound kernels: algorithmic bytes per launch
+    nq, nk = d.n_queries, d.window_tokens
+    alg_bytes = {"append": nq * d.d_model * 2 + (d.d_latent + d.d_rope) * d.d_model * 2 + nq * (d.d_latent + d.d_rope) * 2,
+                 "rope": 2 * nk * d.d_rope * 2,
+                 "q_absorb": nq * d.n_heads * d.d_head * 2 + d.n_heads * d.d_nope * d.d_latent * 2 +
+                 nq * d.n_heads * (d.d_latent + d.d_rope) * 2}
+    for k, b in alg_bytes.items():
+        kernels[k]["algorithmic_bytes"] = b
+        kernels[k]["gbs"] = b / (kernels[k]["ms_per_launch"] * 1e-3) / 1e9
+        kernels[k]["frac_of_hbm"] = kernels[k]["gbs"] / hbm
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "wan1.3b-layer chunk step: append 3 frames + rope + q-absorb + absorbed attention "
+                                   "with fused W_uv; N_q=4680, N_k=32760, n_h=12, d_c=192, d_rope=32, batch 1",
+                       "global_batch": world, "seq_len": nk, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {L} layer buffer sets cycled"},
+            "query_tokens_per_s": tokens, "roofline": roofline, "kernels": kernels,
+            "e2e": {"value": world * F["total"] / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "vmla_chunk_step_host (pinned host x, q -> device, append, attention, out -> host)"},
+            "gpu_launches": 4 * args.steps, "clocks": clk}
+    line["designs"] = {"absorbed_ms_per_step": ms_step, "recon_once": recon_once}
+    if dense:
+        line["dense"] = dense
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_queries)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    m.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-dense", dest="dense", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-queries", type=int, default=2048)
+    ap.add_argument("--steps-ref", type=int, default=None)
+    ap.add_argument("--warmup-ref", type=int, default=None)
+    args = ap.parse_args()
+    args.steps_ref = args.steps_ref if args.steps_ref is not None else min(args.steps, 5)
+    args.warmup_ref = args.warmup_ref if args.warmup_ref is not None else min(args.warmup, 1)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

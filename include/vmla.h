@@ -1,0 +1,234 @@
+/*
+ * vmla.h -- C ABI of libvmla.so: VideoMLA latent-KV chunk attention on B200 (sm_100a).
+ *
+ * The method (VideoMLA: Low-Rank Latent KV Cache for Minute-Scale
+ * Autoregressive Video Diffusion; cited below by page and section):
+ *   [paperlayer]  summary on paperlayer.ai: §3 Method, §4, App. C.1, D.1-D.5, E, F
+ *   [gist.it]     technical summary on gist.science (Italian), "Metodologia" 1-4
+ *
+ * Every token of a fixed sliding window of latent video frames is cached as a
+ * shared content latent c_KV = W_dkv x (d_latent scalars) plus one head-shared
+ * positional key k_R = W_kr x (d_rope scalars), stored before its 3D rotary
+ * embedding [gist.it pt. 1, 3; paperlayer §3, App. D.5].  A chunk of new
+ * frames attends over the whole window, itself included, with per-head queries
+ * split into a content part (d_nope) and a 3D-rotated positional part (d_rope)
+ * [paperlayer App. D.3-D.4].
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Memory.  The caller owns every device buffer (cache, workspace, weights,
+ *   activations, outputs) and passes raw device pointers.  The library owns
+ *   only its host-side handle; it never allocates device memory.  Device
+ *   pointers must be 16-byte aligned.
+ * - Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   Compute calls only enqueue work on it and return; nothing synchronises
+ *   except vmla_device_status() and vmla_profile_read().
+ * - Layout.  Row-major, contiguous, batch outermost.  dtype VMLA_BF16 means
+ *   weights, x, q and the caches are bf16 (accumulation is fp32); VMLA_FP32
+ *   means float.  Attention outputs are float32 in both cases.
+ * - Errors.  Every call validates its arguments on the host and returns a
+ *   vmla_status; nothing is enqueued when it is not VMLA_OK.  A launch
+ *   failure reported by CUDA returns VMLA_ERR_CUDA.  Device-side faults that
+ *   the kernels detect themselves (a pipeline wait that ran out of time, an
+ *   index outside its buffer) are recorded in a device status word that
+ *   vmla_device_status() reads.
+ * - Threads.  A handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef VMLA_H_
+#define VMLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VMLA_ABI_VERSION 1
+
+typedef enum vmla_status {
+  VMLA_OK = 0,
+  VMLA_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size, misaligned pointer */
+  VMLA_ERR_UNSUPPORTED_SHAPE = 2, /* shape has no kernel for this dtype (see vmla_config_check) */
+  VMLA_ERR_OUT_OF_RANGE = 3,      /* layer index, frame count or a RoPE position >= 1024 out of range */
+  VMLA_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
+  VMLA_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up on a pipeline wait (device status word) */
+  VMLA_ERR_STATE = 6,             /* frame sequence not allowed (skips or rewinds), buffers not bound */
+  VMLA_ERR_DEVICE_BOUNDS = 7      /* a kernel found an index outside its buffer (device status word) */
+} vmla_status;
+
+typedef enum vmla_dtype { VMLA_BF16 = 0, VMLA_FP32 = 1 } vmla_dtype;
+
+/* How vmla_chunk_attention evaluates the same scores and outputs. */
+typedef enum vmla_design {
+  VMLA_DESIGN_AUTO = 0,        /* ABSORBED for d_latent <= 192, RECON_ONCE from 256 on (VMLA_BF16;
+                                  VMLA_FP32 always evaluates the absorbed form) */
+  VMLA_DESIGN_ABSORBED = 1,    /* W_uk folded into the query, MQA over [c_KV | k_R], W_uv after the
+                                  softmax-weighted sum [paperlayer App. E] */
+  VMLA_DESIGN_RECONSTRUCT = 2, /* per KV tile, per-head K/V rebuilt from c_KV in shared memory, then
+                                  d_head attention [gist.it pt. 2; paperlayer §3 On-demand reconstruction] */
+  VMLA_DESIGN_RECON_ONCE = 3   /* per-head K/V of the whole window rebuilt once into the workspace, then
+                                  d_head attention */
+} vmla_design;
+
+/* When the positional key gets its 3D rotation. */
+typedef enum vmla_rope_mode {
+  VMLA_ROPE_AT_READ = 0,  /* stored unrotated, rotated at attention time with window-relative frame
+                             indices t = frame - first frame of the window [paperlayer App. D.5, App. E] */
+  VMLA_ROPE_AT_APPEND = 1 /* rotated at append with the absolute frame index (scores are identical
+                             without a sink frame, RoPE depends on offsets only) */
+} vmla_rope_mode;
+
+typedef struct vmla_config {
+  int d_model;           /* D, width of x (1536) */
+  int n_heads;           /* n_h (12) */
+  int d_nope;            /* per-head content dims of q and k (96) */
+  int d_rope;            /* positional dims, = 2*(rope_pairs[0]+rope_pairs[1]+rope_pairs[2]) (32) */
+  int d_latent;          /* d_c, width of c_KV (192) */
+  int d_value;           /* per-head value / output dims (128) */
+  int rope_pairs[3];     /* complex pairs of the t, h, w axes ((6,5,5), [paperlayer App. D.3]) */
+  int rope_base_dims[3]; /* B_a in w_{a,i} = theta^(-2i/B_a); 0 means 2*rope_pairs[a] */
+  float rope_theta;      /* 10000 */
+  int grid_h, grid_w;    /* latent frame grid; tokens per frame T_f = grid_h*grid_w (30 x 52 = 1560) */
+  int window_frames;     /* W: ring capacity in frames, current chunk included (21) */
+  int chunk_frames;      /* largest n_frames of an attention call (3) */
+  int batch;             /* independent rings (one per sample) */
+  int layers;            /* layers held by one handle's caches */
+  vmla_dtype dtype;
+  vmla_rope_mode rope_mode;
+  float softmax_rescale_log2; /* online softmax: a row's running max is raised only when a key tile's
+                                 max exceeds it by more than 2^this (8 by default); 0 raises it on
+                                 every increase.  Results are the same; only the amount of O
+                                 rescaling work differs. */
+} vmla_config;
+
+typedef struct vmla_handle vmla_handle;
+
+/* Name of a status code (static string, never NULL). */
+const char* vmla_status_string(vmla_status status);
+
+/* VMLA_ABI_VERSION of the loaded library. */
+int vmla_abi_version(void);
+
+/* Fill *cfg with one Wan2.1-T2V-1.3B attention layer [paperlayer §4, App. C.1, D.1-D.3]:
+ * D=1536, 12 heads, d_nope=96, d_rope=32 in (6,5,5) pairs, d_c=192, d_value=128,
+ * 30x52 grid, W=21 frames, chunks of 3 frames, batch 1, 1 layer, bf16, RoPE at read,
+ * softmax_rescale_log2 = 8. */
+vmla_status vmla_config_init(vmla_config* cfg);
+
+/* VMLA_OK when every field is consistent and a kernel exists for it:
+ * VMLA_FP32 accepts any positive sizes (d_latent, d_nope+d_rope, d_value <= 512);
+ * VMLA_BF16 needs d_nope + d_rope = d_value = 128, d_rope = 32 and d_latent a multiple of 64 in
+ * [64, 384].  grid_h, grid_w, window_frames must be < 1024 (RoPE range, [paperlayer App. C.1]). */
+vmla_status vmla_config_check(const vmla_config* cfg);
+
+/* Bytes of the caller-allocated caches of one handle (all layers and samples):
+ *   ckv:  [layers][batch][window_frames*T_f][d_latent]
+ *   kr:   [layers][batch][window_frames*T_f][d_rope]
+ *   dense_kv (the per-head comparison layout, 2*n_heads*d_value scalars per token):
+ *         [layers][batch][window_frames*T_f][2][n_heads][d_value]  (keys, then values)
+ * Any output pointer may be NULL. */
+vmla_status vmla_cache_bytes(const vmla_config* cfg, size_t* ckv_bytes, size_t* kr_bytes, size_t* dense_kv_bytes);
+
+/* Bytes of device workspace that vmla_bind() needs for calls with `design`
+ * (and for the dense calls, whatever design). */
+vmla_status vmla_workspace_bytes(const vmla_config* cfg, vmla_design design, size_t* bytes);
+
+/* The angular frequency of each rotary pair, t pairs first, then h, then w
+ * (w_{a,i} = theta^(-2i/B_a), i = 0..pairs_a-1 [paperlayer App. D.3]), as float. n >= pair count. */
+vmla_status vmla_rope_frequencies(const vmla_config* cfg, float* freqs, int n);
+
+/* Create / destroy a handle (host memory only; no CUDA call). */
+vmla_status vmla_create(const vmla_config* cfg, vmla_handle** out);
+vmla_status vmla_destroy(vmla_handle* h);
+
+/* Attach the caller's latent caches and workspace (sizes from vmla_cache_bytes /
+ * vmla_workspace_bytes).  Resets every layer's frame counter to 0.  The cache
+ * contents need no initialisation: no kernel reads a slot before it is written. */
+vmla_status vmla_bind(vmla_handle* h, void* ckv, void* kr, void* workspace, size_t workspace_bytes);
+
+/* Attach the caller's dense per-head cache (only for the vmla_dense_* calls). */
+vmla_status vmla_dense_bind(vmla_handle* h, void* dense_kv);
+
+/* Latent cache write [gist.it pt. 1, 3; paperlayer §3 Shared low-rank KV cache]:
+ *   [c_KV | k_R] = W_down x for n_frames frames, written into the ring slots of
+ *   frames first_frame .. first_frame+n_frames-1 (slot of frame f = f mod W: the
+ *   oldest frame is evicted, FIFO [paperlayer App. D.4]).  k_R is stored unrotated
+ *   (VMLA_ROPE_AT_READ) or rotated with the absolute frame index (VMLA_ROPE_AT_APPEND).
+ * x:      [batch][n_frames*T_f][d_model]
+ * w_down: [d_latent + d_rope][d_model]  (rows of W_dkv, then rows of W_kr)
+ * Frame rule per layer (F = frames appended so far): first_frame == F appends a new
+ * chunk; first_frame + n_frames == F rewrites the newest frames (the next denoising
+ * pass of the same chunk).  Anything else is VMLA_ERR_STATE.  1 <= n_frames <= W. */
+vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, int64_t first_frame,
+                              int n_frames, void* stream);
+
+/* Chunk attention over the window [paperlayer App. D.3-D.5, App. E]:
+ *   for query i of frame first_frame + i/T_f and head h,
+ *     out[i, h*d_value:(h+1)*d_value] = sum_j softmax_j(s_ij) W_uv,h c_j,
+ *     s_ij = ( q_nope,ih . W_uk,h c_j  +  RoPE(q_rope,ih) . RoPE(k_R,j) ) / sqrt(d_nope + d_rope)
+ *   over every key j of the window frames [max(0, F-W), F) (no mask: the chunk is
+ *   the newest frames and sees itself).
+ * q:    [batch][n_frames*T_f][n_heads][d_nope + d_rope]  (per head: content, then positional)
+ * w_uk: [n_heads][d_nope][d_latent]   w_uv: [n_heads][d_value][d_latent]
+ * out:  [batch][n_frames*T_f][n_heads*d_value], float32 for both dtypes (a bf16 rounding of the
+ *       output alone would take two thirds of a 3e-2*RMS max-error budget: max |out| is about 5 RMS)
+ * The chunk must be the newest appended frames: first_frame + n_frames == F,
+ * 1 <= n_frames <= chunk_frames; otherwise VMLA_ERR_STATE. */
+vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
+                                 void* out, int64_t first_frame, int n_frames, vmla_design design, void* stream);
+
+/* The dense per-head comparison [gist.it problem statement; paperlayer App. C.1]:
+ * the same keys and values, cached as 2*n_heads*d_value scalars per token.
+ * vmla_dense_cache_append writes k_h = [W_uk,h c | RoPE(k_R)] (rotated with the
+ * absolute frame index) and v_h = W_uv,h c into dense_kv, with c and k_R = W_down x
+ * as in vmla_cache_append (same frame rule, tracked separately from the latent
+ * cache).  vmla_dense_chunk_attention runs d_head attention per head on it, with
+ * the query's positional part rotated by the absolute frame index; out is float32 as above. */
+vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, const void* w_uk,
+                                    const void* w_uv, int64_t first_frame, int n_frames, void* stream);
+vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q, void* out, int64_t first_frame,
+                                       int n_frames, void* stream);
+
+/* One denoising pass of a chunk, end to end from HOST memory: copy x and q from
+ * (preferably pinned) host buffers into the caller's device staging buffers, append,
+ * attend, copy out back to the host buffer -- all enqueued on `stream`; the host
+ * buffers must stay valid until the stream reaches this point.  Shapes as above. */
+vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, const void* q_host,
+                                 void* out_host, const void* w_down, const void* w_uk, const void* w_uv,
+                                 void* x_dev, void* q_dev, void* out_dev, int64_t first_frame, int n_frames,
+                                 vmla_design design, void* stream);
+
+/* Host-side view of the window of `layer` after `frames_appended` frames: for each
+ * window frame, oldest first, its absolute index, ring slot (frame mod W) and
+ * window-relative index t.  `capacity` is the length of the three arrays; *n gets
+ * the number of window frames. */
+vmla_status vmla_window(const vmla_handle* h, int64_t frames_appended, int32_t* frame, int32_t* slot,
+                        int32_t* t_local, int capacity, int* n);
+
+/* Frames appended so far to a layer's latent cache (resume a rollout exactly). */
+vmla_status vmla_state_get(const vmla_handle* h, int layer, int64_t* frames_appended);
+vmla_status vmla_state_set(vmla_handle* h, int layer, int64_t frames_appended);
+
+/* Synchronise `stream`, read and clear the library's device status word:
+ * VMLA_OK, VMLA_ERR_DEVICE_TIMEOUT or VMLA_ERR_DEVICE_BOUNDS; *flags (may be NULL)
+ * gets the raw bits. */
+vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
+
+/* Per-stage CUDA-event timing of the kernels each call launches, recorded on the
+ * call's stream.  Stages: 0 append, 1 rope, 2 q-absorb, 3 attention (absorbed),
+ * 4 attention (reconstruct), 5 dense append, 6 dense attention, 7 reconstruct-once.
+ * vmla_profile_read synchronises, then returns the summed milliseconds and the
+ * launch count of one stage since profiling was enabled. */
+vmla_status vmla_profile_enable(vmla_handle* h, int enable);
+vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* launches);
+
+/* Self-test of the bounded pipeline waits: launches one CTA that waits on an
+ * mbarrier nothing arrives at, for at most `limit_ns` nanoseconds (<= 1e9), then
+ * returns.  The device status word must afterwards report VMLA_ERR_DEVICE_TIMEOUT. */
+vmla_status vmla_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VMLA_H_ */

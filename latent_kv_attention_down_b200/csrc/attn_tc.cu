@@ -1,0 +1,433 @@
+// Chunk attention on tcgen05 tensor cores (sm_100a).
+//
+// Absorbed design [paperlayer App. E]: with W_uk folded into the query
+// (q~_h = [W_uk,h^T q_nope,h | RoPE(q_rope,h)]), every head scores the SAME
+// shared key [c_KV | RoPE(k_R)] (d_latent + 32 wide) and accumulates the SAME
+// shared values c_KV (d_latent wide): multi-query attention over the latent
+// cache.  W_uv,h is applied once per output row after the softmax-weighted
+// sum (value-path absorption), fused into the epilogue as a second tcgen05
+// GEMM whose A operand is O_bar split into a bf16 pair (rounded + residual),
+// so the only roundings left on the output path are the cache's, P's and
+// q~'s.  The output is written in fp32.  The dense variant runs the same pipeline with per-head 128-wide K
+// and V tiles (the 3072-scalar comparison layout).
+//
+// One CTA owns 128 query rows of one head of one sample and streams the whole
+// window in tiles of BN = 128 keys:
+//   warp 0     TMA producer: Q once, then K/V tiles into a STAGES-deep ring
+//   warp 1     tcgen05.mma issuer (one thread) + TMEM owner
+//   warps 4-7  softmax: thread r owns query row r = TMEM lane r
+// TMEM (512 columns): S0 [0,BN), S1 [BN,2BN), O [2BN, 2BN+DV).
+//   S_j = Q K_j^T (fp32) lands in S[j&1]; the softmax threads turn it into
+//   P_j = exp2(S_j * scale*log2e - m) as bf16 pairs written back over S[j&1];
+//   O += P_j V_j reads P straight from TMEM (A operand) and V from the same
+//   shared-memory tile as K (MN-major descriptor), so V is never loaded twice.
+// While the softmax works on S_j, the tensor core already computes S_{j+1}.
+// The running max is only raised when it grows by more than 2^threshold (lazy
+// rescale, 2^8 by default); O is then rescaled in TMEM after the previous P V has finished.
+// Every mbarrier wait is bounded; a CTA that gives up records the error and
+// drains its in-flight copies and MMAs before releasing TMEM.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace vmla {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int DL_, bool DENSE_>
+struct AttnCfg {
+  static constexpr bool DENSE = DENSE_;
+  static constexpr int DL = DL_;
+  static constexpr int BN = 128;
+  static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of Q
+  static constexpr int Q_BYTES = QB * 16384 + (DENSE ? 0 : 128 * 64);
+  static constexpr int KBLK = BN * 128;  // one [BN keys x 64] SW128 block
+  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * 64;
+  static constexpr int DV = DENSE ? 128 : DL;
+  static constexpr int SMEM_CAP = 232448;
+  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - 512 - Q_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static constexpr int S_COL = 0;  // S buffer b at S_COL + b*BN
+  static constexpr int O_COL = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int SMEM = 1024 + Q_BYTES + STAGES * STAGE_BYTES + 512;
+  static_assert(STAGES >= 2, "pipeline needs two stages");
+  static_assert(O_COL + DV <= 512, "TMEM budget");
+  static_assert(SMEM <= SMEM_CAP, "shared memory budget");
+  static_assert(STAGES * STAGE_BYTES >= 2 * DV * 256 && STAGES * STAGE_BYTES >= 65536, "epilogue staging");
+  static_assert(DV % 64 == 0 && DV <= 256, "value width");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t kv_full[4];
+  uint64_t kv_empty[4];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint64_t o_final;
+  uint64_t wuv_full;
+  uint64_t ob_full;
+  uint64_t epi_done;
+  uint64_t drain;
+  uint32_t tslot;
+  int abort_flag;
+};
+
+// bf16 row of 32 floats into a 128B-swizzled K-major tile: row r, columns c0..c0+31
+// (c0 a multiple of 32) of a tile made of [128 rows x 64 cols] blocks of 16 KB.
+// With `lo` set, what is stored is the rounding residual v*scale - bf16(v*scale),
+// so that hi + lo carries the value to about 16 significant bits.
+__device__ __forceinline__ void st_swizzled_row32(uint8_t* tile, int r, int c0, const float (&v)[32], float scale,
+                                                  bool lo) {
+  uint8_t* blk = tile + (c0 >> 6) * 16384 + r * 128;
+  const int j0 = (c0 & 63) >> 3;  // first 16-byte chunk of the 64-col block
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = v[8 * q + 2 * k] * scale, b = v[8 * q + 2 * k + 1] * scale;
+      const uint32_t hi = pack_bf16x2(a, b);
+      w[k] = lo ? pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xFFFF0000u)) : hi;
+    }
+    *reinterpret_cast<uint4*>(blk + (((j0 + q) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// fp32 row of 32 floats (128 bytes) into a 128B-swizzled tile of [128 rows x 32 fp32] blocks
+// of 16 KB: the shared-memory image of one TMA box of the fp32 output.
+__device__ __forceinline__ void st_swizzled_row32_f32(uint8_t* tile, int r, int c0, const float (&v)[32],
+                                                      float scale) {
+  uint8_t* row = tile + (c0 >> 5) * 16384 + r * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(row + ((j ^ (r & 7)) << 4)) =
+        make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale, v[4 * j + 3] * scale);
+}
+
+template <class C>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t stage) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, C::BN, false, false);
+  if constexpr (C::DENSE) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ss(d_tmem, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
+             smem_desc(stage + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < C::DL / 16; ++kk)
+      mma_ss(d_tmem, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
+             smem_desc(stage + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
+    const uint32_t qr = sq + C::QB * 16384, kr = stage + C::QB * C::KBLK;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+      mma_ss(d_tmem, smem_desc(qr + kk * 32, 16, 512, LAYOUT_SW64), smem_desc(kr + kk * 32, 16, 512, LAYOUT_SW64),
+             idesc, 1);
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t stage, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, C::DV, false, true);
+  const uint32_t v = C::DENSE ? stage + 2 * C::KBLK : stage;
+#pragma unroll
+  for (int kk = 0; kk < C::BN / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc(v + kk * 2048, C::KBLK, 1024, LAYOUT_SW128), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int DL, bool DENSE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
+                   const __grid_constant__ CUtensorMap tm_wuv, const __grid_constant__ CUtensorMap tm_out,
+                   const AttnTc a) {
+  using C = AttnCfg<DL, DENSE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::Q_BYTES;
+  Bars* bars = reinterpret_cast<Bars*>(sKV + C::STAGES * C::STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int m0 = mt * 128;
+  const int n_tiles = (a.n_keys + C::BN - 1) / C::BN;
+  const Guard g{&bars->abort_flag, a.err, a.limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bars->s_full[k], 1);
+      mbar_init(&bars->p_full[k], 128);
+    }
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_final, 1);
+    mbar_init(&bars->wuv_full, 1);
+    mbar_init(&bars->ob_full, 128);
+    mbar_init(&bars->epi_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&bars->tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars->tslot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      const int qrow = b * a.n_heads + h;
+      if constexpr (C::DENSE) {
+        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+        for (int qb = 0; qb < 2; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
+      } else {
+        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+        for (int qb = 0; qb < C::QB; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
+        tma_load_3d(sQ + C::QB * 16384, &tm_qr, &bars->q_full, DL, m0, qrow);
+      }
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % C::STAGES;
+        if (!wait_phase(&bars->kv_empty[s], ((j / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+        uint8_t* st = sKV + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_BYTES);
+        if constexpr (C::DENSE) {
+          for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], h * 128 + kb * 64, j * C::BN, b);
+            tma_load_3d(st + (2 + kb) * C::KBLK, &tm_k, &bars->kv_full[s], (a.n_heads + h) * 128 + kb * 64,
+                        j * C::BN, b);
+          }
+        } else {
+          for (int kb = 0; kb < C::QB; ++kb)
+            tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], kb * 64, j * C::BN, b);
+          tma_load_3d(st + C::QB * C::KBLK, &tm_kr, &bars->kv_full[s], 0, j * C::BN, b);
+        }
+        ++issued;
+      }
+      bool wuv_issued = false;
+      if constexpr (!C::DENSE) {
+        // W_uv,h goes where the K/V ring was, once every P V has consumed it
+        if (issued == n_tiles && wait_phase(&bars->o_final, 0, g, DEV_ERR_TIMEOUT_PRODUCER)) {
+          mbar_arrive_expect_tx(&bars->wuv_full, C::DV * 256);
+          for (int kb = 0; kb < C::DV / 64; ++kb)
+            tma_load_3d(sKV + kb * 16384, &tm_wuv, &bars->wuv_full, kb * 64, 0, h);
+          wuv_issued = true;
+        }
+      }
+      if (bars->abort_flag) {
+        drain_phase(&bars->q_full, 0, g);
+        for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
+          drain_phase(&bars->kv_full[j % C::STAGES], (j / C::STAGES) & 1, g);
+        if (wuv_issued) drain_phase(&bars->wuv_full, 0, g);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t sq = smem_u32(sQ), skv = smem_u32(sKV);
+      bool ok = wait_phase(&bars->q_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
+                wait_phase(&bars->kv_full[0], 0, g, DEV_ERR_TIMEOUT_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_qk<C>(tbase + C::S_COL, sq, skv);
+        mma_commit(&bars->s_full[0]);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles) {
+          const int s1 = (j + 1) % C::STAGES;
+          if (!(ok = wait_phase(&bars->kv_full[s1], ((j + 1) / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          issue_qk<C>(tbase + C::S_COL + ((j + 1) & 1) * C::BN, sq, skv + s1 * C::STAGE_BYTES);
+          mma_commit(&bars->s_full[(j + 1) & 1]);
+        }
+        if (!(ok = wait_phase(&bars->p_full[j & 1], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+        tc_fence_after();
+        const int s = j % C::STAGES;
+        issue_pv<C>(tbase + C::O_COL, tbase + C::S_COL + (j & 1) * C::BN, skv + s * C::STAGE_BYTES, j > 0);
+        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->o_done);
+      }
+      if (ok) mma_commit(&bars->o_final);
+      if constexpr (!C::DENSE) {
+        // fused value up-projection: out_h = O_bar W_uv,h^T with O_bar (bf16, normalised) staged over Q
+        if (ok && wait_phase(&bars->ob_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
+            wait_phase(&bars->wuv_full, 0, g, DEV_ERR_TIMEOUT_MMA)) {
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+          const uint32_t ob_lo = skv + C::DV * 256;  // residual half of O_bar, after W_uv,h
+#pragma unroll
+          for (int kk = 0; kk < C::DV / 16; ++kk) {
+            const uint64_t w = smem_desc(skv + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
+            mma_ss(tbase, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), w, idesc,
+                   kk > 0);
+            mma_ss(tbase, smem_desc(ob_lo + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), w, idesc, 1);
+          }
+          mma_commit(&bars->epi_done);
+        }
+      }
+      if (bars->abort_flag) {
+        mma_commit(&bars->drain);
+        drain_phase(&bars->drain, 0, g);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / correction / epilogue
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;  // query row inside the tile == TMEM lane
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(wq * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int buf = j & 1;
+      ok = __all_sync(0xffffffffu, wait_phase(&bars->s_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sraw[C::BN];
+#pragma unroll
+      for (int c = 0; c < C::BN; c += 64)
+        tmem_ld64(lane_base + C::S_COL + buf * C::BN + c, *reinterpret_cast<uint32_t(*)[64]>(&sraw[c]));
+      const int valid = a.n_keys - j * C::BN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < C::BN; ++c) {
+        float v = __uint_as_float(sraw[c]);
+        if (c >= valid) v = -INFINITY;
+        sraw[c] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
+      }
+      const float m_tile = mx * a.scale_log2;
+      if (j == 0) {
+        m_run = m_tile;
+      } else if (__any_sync(0xffffffffu, m_tile > m_run + a.rescale_threshold)) {
+        // raise the running max of every row of this warp; rescale O once the previous P V is done
+        const float m_new = fmaxf(m_run, m_tile);
+        const float alpha = ex2_approx(m_run - m_new);
+        ok = __all_sync(0xffffffffu, wait_phase(&bars->o_done, (j - 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < C::DV; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + C::O_COL + c, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(lane_base + C::O_COL + c, o);
+        }
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float neg_m = -m_run;
+      float sum = 0.f;
+#pragma unroll
+      for (int half = 0; half < C::BN / 64; ++half) {
+        uint32_t packed[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sraw[half * 64 + 2 * k]), a.scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sraw[half * 64 + 2 * k + 1]), a.scale_log2, neg_m));
+          sum += p0 + p1;
+          packed[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(lane_base + C::S_COL + buf * C::BN + half * 32, packed);
+      }
+      l_run += sum;
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[buf]);
+    }
+    ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->o_final, 0, g, DEV_ERR_TIMEOUT_EPILOGUE));
+    if (ok) tc_fence_after();
+    const float inv_l = 1.f / l_run;
+    if constexpr (!C::DENSE) {
+      // O_bar = O / l as a bf16 pair: the rounded part over the Q region, the residual
+      // after W_uv,h in the K/V ring (A operands of the two W_uv GEMMs)
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < C::DV; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + C::O_COL + c, o);
+          st_swizzled_row32(sQ, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, false);
+          st_swizzled_row32(sKV + C::DV * 256, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, true);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->ob_full);
+      ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->epi_done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE));
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + c, o);
+          st_swizzled_row32_f32(sKV, r, c, *reinterpret_cast<float(*)[32]>(o), 1.f);
+        }
+      }
+    } else {
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + C::O_COL + c, o);
+          st_swizzled_row32_f32(sKV, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l);
+        }
+      }
+    }
+    fence_async_smem();
+    named_bar_sync(1, 128);
+    if (r == 0 && !bars->abort_flag) {
+      for (int blk = 0; blk < 4; ++blk) tma_store_3d(&tm_out, sKV + blk * 16384, h * 128 + blk * 32, m0, b);
+      bulk_commit();
+      bulk_wait_all_read();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+template <int DL, bool DENSE>
+cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk, const CUtensorMap& tkr,
+                    const CUtensorMap& tuv, const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
+  using C = AttnCfg<DL, DENSE>;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (attr != cudaSuccess) return attr;
+  if (a.n_q <= 0 || a.n_keys <= 0) return cudaSuccess;
+  attn_tc_kernel<DL, DENSE><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv, to, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_absorbed_block_n(int) { return 128; }
+
+cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
+                                    const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tuv,
+                                    const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
+  switch (d_latent) {
+    case 64: return go_attn<64, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 128: return go_attn<128, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 192: return go_attn<192, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 256: return go_attn<256, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& to,
+                                 const AttnTc& a, int batch, cudaStream_t s) {
+  return go_attn<128, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
+}
+
+}  // namespace vmla

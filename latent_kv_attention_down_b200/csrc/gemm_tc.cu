@@ -1,0 +1,449 @@
+// tcgen05 GEMM kernels of the bf16 path (sm_100a).  All three share one shape:
+// a 128-row A tile and a weight B tile staged in shared memory by TMA
+// (128-byte swizzle), one elected thread issuing tcgen05.mma into a TMEM
+// accumulator, and four epilogue warps that read their TMEM lane (= output
+// row) back with tcgen05.ld and store bf16 rows.
+//
+//  * append_tc  [gist.it pt. 1, 3; paperlayer §3]: [c_KV | k_R] = W_down x,
+//    rows scattered into the ring slot of their frame (FIFO ring of W frames,
+//    slot f mod W [paperlayer App. D.4]); k_R optionally rotated with the
+//    absolute frame index.  K = d_model, pipelined over 4 stages of 64.
+//  * qprep_tc   [paperlayer App. E, content-path absorption]: the query's
+//    content part pushed through W_uk,h (q~ = W_uk,h^T q_nope, d_latent wide)
+//    next to its rotated positional part, one head per CTA column.
+//  * recon_tc   [gist.it pt. 2; paperlayer §3 On-demand reconstruction]: the
+//    per-head dense entries k_h = [W_uk,h c | RoPE(k_R)], v_h = W_uv,h c.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace vmla {
+namespace {
+
+constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 4..7 epilogue
+
+__device__ __forceinline__ float pair_angle(const Rope& rp, int p, float t, float h, float w) {
+  const float pos = p < rp.n_t ? t : (p < rp.n_t + rp.n_h ? h : w);
+  return pos * rp.freq[p];
+}
+
+// Rotate 16 adjacent pairs held in v[0..31].
+__device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, float t, float h, float w) {
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    float s, c;
+    sincosf(pair_angle(rp, p, t, h, w), &s, &c);
+    const float u = v[2 * p], x = v[2 * p + 1];
+    v[2 * p] = u * c - x * s;
+    v[2 * p + 1] = u * s + x * c;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = s[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * q + 2 * k] = __uint_as_float(w[k] << 16);
+      v[8 * q + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ void raw_to_float(const uint32_t (&r)[32], float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared prologue: barriers, abort flag, TMEM allocation by warp 1.
+__device__ __forceinline__ uint32_t setup_cta(uint64_t* bars, int nbars, uint32_t* tslot, int* abort_flag,
+                                              uint32_t tmem_cols) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbars; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(tslot, tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tslot;
+}
+
+__device__ __forceinline__ void teardown_cta(uint32_t tbase, uint32_t tmem_cols) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, tmem_cols);
+  }
+}
+
+// ============================================================== append
+template <int N_OUT>
+struct AppendCfg {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr int NB = N_OUT <= 256 ? N_OUT : N_OUT / 2;
+  static constexpr int NSPLIT = N_OUT / NB;
+  static constexpr int B_BYTES = N_OUT * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = N_OUT <= 256 ? 256 : 512;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static_assert(N_OUT % 32 == 0 && NB % 16 == 0 && NB <= 256, "bad N");
+  static_assert(B_BYTES % 1024 == 0, "stage alignment");
+};
+
+template <int N_OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    append_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                     const AppendTc a) {
+  using C = AppendCfg<N_OUT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* done = empty + C::STAGES;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, b = blockIdx.y;
+  const int kblocks = a.d_model / 64;
+  const Guard g{abort_flag, a.err, a.limit_ns};
+  const uint32_t tbase = setup_cta(full, 2 * C::STAGES + 1, tslot, abort_flag, C::TMEM_COLS);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_w);
+      int issued = 0;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % C::STAGES;
+        if (!wait_phase(&empty[s], ((kb / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+        uint8_t* sa = smem + s * C::STAGE_BYTES;
+        uint8_t* sb = sa + C::A_BYTES;
+        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        tma_load_3d(sa, &tm_x, &full[s], kb * 64, m0, b);
+        for (int sp = 0; sp < C::NSPLIT; ++sp) tma_load_2d(sb + sp * C::NB * 128, &tm_w, &full[s], kb * 64, sp * C::NB);
+        ++issued;
+      }
+      if (*abort_flag)
+        for (int kb = issued > C::STAGES ? issued - C::STAGES : 0; kb < issued; ++kb)
+          drain_phase(&full[kb % C::STAGES], (kb / C::STAGES) & 1, g);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, C::NB, false, false);
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % C::STAGES;
+        if (!wait_phase(&full[s], (kb / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+        const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int sp = 0; sp < C::NSPLIT; ++sp)
+            mma_ss(tbase + sp * C::NB, smem_desc(sa + k * 32, 16, 1024, LAYOUT_SW128),
+                   smem_desc(sb + sp * C::NB * 128 + k * 32, 16, 1024, LAYOUT_SW128), idesc, (kb | k) != 0);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(done);
+      if (*abort_flag) drain_phase(done, 0, g);
+    }
+  } else if (warp >= 4) {
+    const int wq = warp - 4;
+    const int m = m0 + wq * 32 + lane;
+    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
+    __syncwarp();
+    tc_fence_after();
+    const bool valid = ok && m < a.rows;
+    const int T = a.ring.tokens_per_frame;
+    const int mm = valid ? m : 0;
+    const int64_t frame = a.first_frame + mm / T;
+    const int tok = mm % T;
+    __nv_bfloat16* lat;
+    __nv_bfloat16* pos;
+    if (a.contiguous) {
+      lat = a.ckv + ((int64_t)b * a.rows + mm) * N_OUT;
+      pos = lat + a.d_latent;
+    } else {
+      const int64_t row = (frame % a.ring.window_frames) * T + tok;
+      lat = a.ckv + ((int64_t)b * a.ring_rows + row) * a.d_latent;
+      pos = a.kr + ((int64_t)b * a.ring_rows + row) * 32;
+    }
+#pragma unroll 1
+    for (int c0 = 0; c0 < N_OUT; c0 += 32) {
+      uint32_t raw[32];
+      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
+      if (!valid) continue;
+      float v[32];
+      raw_to_float(raw, v);
+      if (c0 < a.d_latent) {
+        store_bf16x32(lat + c0, v);
+      } else {
+        if (a.rotate) rotate16(v, a.rope, (float)frame, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+        store_bf16x32(pos, v);
+      }
+    }
+  }
+  teardown_cta(tbase, C::TMEM_COLS);
+}
+
+// ============================================================== q-absorb
+template <int DL>
+struct QPrepCfg {
+  static constexpr int A_BYTES = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
+  static constexpr int WB = 96 * 128;            // one 64-col block of W_uk,h: 96 rows x 128 B
+  static constexpr int B_BYTES = (DL / 64) * WB;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr int SMEM = 1024 + A_BYTES + B_BYTES + 256;
+  static_assert(DL % 64 == 0 && DL <= 256, "bad d_latent");
+};
+
+template <int DL>
+__global__ void __launch_bounds__(kThreads, 1)
+    qprep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wuk,
+                    const QPrepTc a) {
+  using C = QPrepCfg<DL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::B_BYTES);
+  uint64_t* done = full + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const Guard g{abort_flag, a.err, a.limit_ns};
+  const uint32_t tbase = setup_cta(full, 2, tslot, abort_flag, C::TMEM_COLS);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(full, C::A_BYTES + C::B_BYTES);
+      tma_load_3d(sA, &tm_q, full, h * 128, m0, b);
+      tma_load_3d(sA + 16384, &tm_q, full, h * 128 + 64, m0, b);
+      for (int cb = 0; cb < DL / 64; ++cb) tma_load_3d(sB + cb * C::WB, &tm_wuk, full, cb * 64, 0, h);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
+      tc_fence_after();
+      if (ok) {
+        const uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+        for (int kk = 0; kk < 6; ++kk)  // d_nope = 96 = 6 x 16
+          mma_ss(tbase, smem_desc(a0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
+                 smem_desc(b0 + kk * 2048, C::WB, 1024, LAYOUT_SW128), idesc, kk > 0);
+      }
+      mma_commit(done);
+      if (*abort_flag) drain_phase(done, 0, g);
+    }
+    if (lane == 0 && *abort_flag) drain_phase(full, 0, g);
+  } else if (warp >= 4) {
+    const int wq = warp - 4;
+    const int i = m0 + wq * 32 + lane;
+    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
+    __syncwarp();
+    tc_fence_after();
+    const bool valid = ok && i < a.n_q;
+    const int ii = valid ? i : 0;
+    __nv_bfloat16* out = a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + ii) * (DL + 32);
+#pragma unroll 1
+    for (int c0 = 0; c0 < DL; c0 += 32) {
+      uint32_t raw[32];
+      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
+      if (!valid) continue;
+      float v[32];
+      raw_to_float(raw, v);
+      store_bf16x32(out + c0, v);
+    }
+    if (valid) {
+      float v[32];
+      load_bf16x32(a.q + (((int64_t)b * a.n_q + ii) * a.n_heads + h) * 128 + 96, v);
+      const int T = a.ring.tokens_per_frame, tok = ii % T;
+      rotate16(v, a.rope, (float)(a.t_first + ii / T), (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+      store_bf16x32(out + DL, v);
+    }
+  }
+  teardown_cta(tbase, C::TMEM_COLS);
+}
+
+// ============================================================== per-head reconstruction
+template <int DL>
+struct ReconCfg {
+  static constexpr int NKB = DL / 64;
+  static constexpr int A_BLK = 128 * 128;  // 128 latent rows x 64 cols
+  static constexpr int B_BLK = 224 * 128;  // [96 rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr int SMEM = 1024 + NKB * (A_BLK + B_BLK) + 256;
+};
+
+template <int DL>
+__global__ void __launch_bounds__(kThreads, 1)
+    recon_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wuk,
+                    const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a) {
+  using C = ReconCfg<DL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::NKB * C::A_BLK;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::NKB * C::B_BLK);
+  uint64_t* done = full + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const Guard g{abort_flag, a.err, a.limit_ns};
+  const uint32_t tbase = setup_cta(full, 2, tslot, abort_flag, C::TMEM_COLS);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(full, C::NKB * (C::A_BLK + C::B_BLK));
+      for (int kb = 0; kb < C::NKB; ++kb) {
+        tma_load_3d(sA + kb * C::A_BLK, &tm_c, full, kb * 64, m0, b);
+        tma_load_3d(sB + kb * C::B_BLK, &tm_wuk, full, kb * 64, 0, h);
+        tma_load_3d(sB + kb * C::B_BLK + 96 * 128, &tm_wuv, full, kb * 64, 0, h);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
+      tc_fence_after();
+      if (ok) {
+        const uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+        for (int kk = 0; kk < DL / 16; ++kk)
+          mma_ss(tbase, smem_desc(a0 + (kk / 4) * C::A_BLK + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
+                 smem_desc(b0 + (kk / 4) * C::B_BLK + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
+      }
+      mma_commit(done);
+      if (*abort_flag) {
+        drain_phase(done, 0, g);
+        drain_phase(full, 0, g);
+      }
+    }
+  } else if (warp >= 4) {
+    const int wq = warp - 4;
+    const int m = m0 + wq * 32 + lane;
+    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
+    __syncwarp();
+    tc_fence_after();
+    const bool valid = ok && m < a.rows;
+    const int mm = valid ? m : 0;
+    const int T = a.ring.tokens_per_frame;
+    const int64_t frame = a.first_frame + mm / T;
+    const int tok = mm % T;
+    const int64_t row = a.to_ring ? (frame % a.ring.window_frames) * T + tok : mm;
+    __nv_bfloat16* kd = a.dense + (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
+    __nv_bfloat16* vd = kd + (int64_t)a.n_heads * 128;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 224; c0 += 32) {
+      uint32_t raw[32];
+      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
+      if (!valid) continue;
+      float v[32];
+      raw_to_float(raw, v);
+      store_bf16x32(c0 < 96 ? kd + c0 : vd + (c0 - 96), v);
+    }
+    if (valid) {
+      float v[32];
+      load_bf16x32(a.kr + ((int64_t)b * a.kr_rows + mm) * a.kr_stride, v);
+      if (a.rotate) rotate16(v, a.rope, (float)frame, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+      store_bf16x32(kd + 96, v);
+    }
+  }
+  teardown_cta(tbase, C::TMEM_COLS);
+}
+
+template <class K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int N_OUT>
+cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, cudaStream_t s) {
+  using C = AppendCfg<N_OUT>;
+  static const cudaError_t attr = set_smem(append_tc_kernel<N_OUT>, C::SMEM);
+  if (attr != cudaSuccess) return attr;
+  append_tc_kernel<N_OUT><<<dim3((a.rows + 127) / 128, batch), kThreads, C::SMEM, s>>>(tx, tw, a);
+  return cudaGetLastError();
+}
+
+template <int DL>
+cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc& a, int batch, cudaStream_t s) {
+  using C = QPrepCfg<DL>;
+  static const cudaError_t attr = set_smem(qprep_tc_kernel<DL>, C::SMEM);
+  if (attr != cudaSuccess) return attr;
+  qprep_tc_kernel<DL><<<dim3((a.n_q + 127) / 128, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tw, a);
+  return cudaGetLastError();
+}
+
+template <int DL>
+cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
+                     int batch, cudaStream_t s) {
+  using C = ReconCfg<DL>;
+  static const cudaError_t attr = set_smem(recon_tc_kernel<DL>, C::SMEM);
+  if (attr != cudaSuccess) return attr;
+  recon_tc_kernel<DL><<<dim3((a.rows + 127) / 128, a.n_heads, batch), kThreads, C::SMEM, s>>>(tc, tuk, tuv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int append_tc_w_box_rows(int d_latent) {
+  const int n = d_latent + 32;
+  return n <= 256 ? n : n / 2;
+}
+
+cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch,
+                             cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  if (a.d_model % 64 != 0) return cudaErrorInvalidValue;
+  switch (a.d_latent) {
+    case 64: return go_append<96>(tx, tw, a, batch, s);
+    case 128: return go_append<160>(tx, tw, a, batch, s);
+    case 192: return go_append<224>(tx, tw, a, batch, s);
+    case 256: return go_append<288>(tx, tw, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc& a, int batch,
+                            cudaStream_t s) {
+  if (a.n_q <= 0) return cudaSuccess;
+  switch (a.d_latent) {
+    case 64: return go_qprep<64>(tq, tw, a, batch, s);
+    case 128: return go_qprep<128>(tq, tw, a, batch, s);
+    case 192: return go_qprep<192>(tq, tw, a, batch, s);
+    case 256: return go_qprep<256>(tq, tw, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
+                            int batch, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  switch (a.d_latent) {
+    case 64: return go_recon<64>(tc, tuk, tuv, a, batch, s);
+    case 128: return go_recon<128>(tc, tuk, tuv, a, batch, s);
+    case 192: return go_recon<192>(tc, tuk, tuv, a, batch, s);
+    case 256: return go_recon<256>(tc, tuk, tuv, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vmla

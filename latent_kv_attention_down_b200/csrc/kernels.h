@@ -1,0 +1,186 @@
+// Internal interface between the host library (vmla.cpp) and the CUDA kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace vmla {
+
+constexpr int kMaxPairs = 32;
+
+// Bits of the library's device status word.
+enum DeviceError : unsigned {
+  DEV_ERR_TIMEOUT_PRODUCER = 1u << 0,
+  DEV_ERR_TIMEOUT_MMA = 1u << 1,
+  DEV_ERR_TIMEOUT_SOFTMAX = 1u << 2,
+  DEV_ERR_TIMEOUT_EPILOGUE = 1u << 3,
+  DEV_ERR_TIMEOUT_SELFTEST = 1u << 4,
+  DEV_ERR_BOUNDS = 1u << 5,
+};
+constexpr unsigned DEV_ERR_BOUNDS_MASK = DEV_ERR_BOUNDS;
+
+// 3D-RoPE table: pair p < n_t turns with the frame index t, then n_h pairs
+// with the grid row h, then n_w pairs with the grid column w.
+struct Rope {
+  float freq[kMaxPairs];
+  int n_t, n_h, n_w;
+};
+
+// Ring geometry of one sample's cache: frame f lives in ring frame slot f mod W.
+struct Ring {
+  int tokens_per_frame;  // T_f
+  int grid_w;
+  int window_frames;     // W
+};
+
+// ------------------------------------------------------------------ fp32 SIMT path (any shape)
+struct SimtAppend {
+  const float* x;       // [B][rows][D]
+  const float* w_down;  // [d_c + d_r][D]
+  float* ckv;           // [B][W*T_f][d_c]   (or a contiguous [B][rows][d_c] scratch)
+  float* kr;            // [B][W*T_f][d_r]
+  int batch, rows, d_model, d_latent, d_rope;
+  int64_t first_frame;
+  int rotate;           // rotate k_R with the absolute frame index before storing
+  int contiguous;       // store row m at row m (scratch) instead of its ring slot
+  int64_t out_rows;     // rows per sample of ckv/kr
+  Ring ring;
+  Rope rope;
+};
+cudaError_t launch_append_simt(const SimtAppend& a, cudaStream_t s);
+
+struct RopeWindow {  // rotate the window's positional keys with window-relative t
+  const void* kr;    // [B][W*T_f][d_r]
+  void* kr_rot;      // [B][W*T_f][d_r]
+  int batch, n_keys, d_rope;
+  int window_start_slot;  // ring frame slot of the oldest window frame
+  Ring ring;
+  Rope rope;
+};
+cudaError_t launch_rope_window_f32(const RopeWindow& a, cudaStream_t s);
+cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s);
+
+struct SimtQPrep {  // q~ = [W_uk^T q_nope | RoPE(q_rope)]  (absorbed) or [q_nope | RoPE(q_rope)] (dense)
+  const float* q;     // [B][n_q][n_h][d_nope + d_r]
+  const float* w_uk;  // [n_h][d_nope][d_c]   (unused when absorb == 0)
+  float* qt;          // [B][n_h][n_q][width]
+  int batch, n_q, n_heads, d_nope, d_rope, d_latent, absorb;
+  int64_t t_first;    // frame index t of query row 0
+  Ring ring;
+  Rope rope;
+};
+cudaError_t launch_qprep_simt(const SimtQPrep& a, cudaStream_t s);
+
+struct SimtAttn {
+  const float* qt;    // [B][n_h][n_q][dqk]
+  const float* key;   // latent: [B][ring_rows][d_c] (+ kpos [B][ring_rows][d_r]); dense: [B][ring_rows][2][n_h][dv]
+  const float* kpos;  // rotated positional keys (latent only)
+  const float* w_uv;  // [n_h][dv][d_c] (latent only)
+  float* out;         // [B][n_q][n_h*dv]
+  int batch, n_q, n_keys, n_heads, d_latent, d_rope, d_value, dense;
+  int64_t ring_rows;
+  float scale;        // 1/sqrt(d_nope + d_rope)
+};
+cudaError_t launch_attn_simt(const SimtAttn& a, cudaStream_t s);
+
+struct SimtDenseReconstruct {  // dense per-head entries from a chunk's latents
+  const float* c;       // [B][rows][d_c]  (contiguous scratch)
+  const float* r;       // [B][rows][d_r]  (unrotated)
+  const float* w_uk;    // [n_h][d_nope][d_c]
+  const float* w_uv;    // [n_h][dv][d_c]
+  float* dense;         // [B][W*T_f][2][n_h][dv]
+  int batch, rows, n_heads, d_nope, d_rope, d_latent, d_value;
+  int64_t first_frame;
+  Ring ring;
+  Rope rope;
+};
+cudaError_t launch_dense_reconstruct_simt(const SimtDenseReconstruct& a, cudaStream_t s);
+
+// ------------------------------------------------------------------ bf16 tcgen05 path (sm_100a)
+struct AppendTc {
+  __nv_bfloat16* ckv;  // [B][ring_rows][d_c] or contiguous [B][rows][d_c + d_r] when contiguous
+  __nv_bfloat16* kr;   // [B][ring_rows][d_r]
+  int rows, d_model, d_latent;  // d_rope is 32
+  int64_t first_frame;
+  int rotate, contiguous;
+  int64_t ring_rows;
+  Ring ring;
+  Rope rope;
+  unsigned* err;
+  uint64_t limit_ns;
+};
+// x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, d_c + 32) box (64, nb) SW128
+cudaError_t launch_append_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const AppendTc& a, int batch,
+                             cudaStream_t s);
+int append_tc_w_box_rows(int d_latent);
+
+struct QPrepTc {
+  const __nv_bfloat16* q;  // [B][n_q][n_h][128]  (rope part read directly)
+  __nv_bfloat16* qt;       // [B][n_h][n_q][d_c + 32]
+  int n_q, n_heads, d_latent;
+  int64_t t_first;
+  Ring ring;
+  Rope rope;
+  unsigned* err;
+  uint64_t limit_ns;
+};
+// q map: 3D (n_h*128, n_q, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64, 96, 1) SW128
+cudaError_t launch_qprep_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_wuk, const QPrepTc& a, int batch,
+                            cudaStream_t s);
+
+struct AttnTc {
+  int n_q, n_keys, n_heads, m_tiles;
+  float scale_log2;  // log2(e) / sqrt(d_nope + d_rope)
+  float rescale_threshold;  // lazy-rescale threshold of the running max, log2 units
+  unsigned* err;
+  uint64_t limit_ns;
+};
+// Absorbed design.  qt maps: 3D (d_c+32, n_q, B*n_h): latent box (64,128,1) SW128, rope box (32,128,1) SW64;
+// ckv map: 3D (d_c, n_keys, B) box (64,BN,1) SW128; kr map: 3D (32, n_keys, B) box (32,BN,1) SW64;
+// w_uv map: 3D (d_c, 128, n_h) box (64,128,1) SW128; out map: 3D (n_h*128, n_q, B) box (64,128,1) SW128.
+cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
+                                    const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr, const CUtensorMap& tm_wuv,
+                                    const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
+int attn_absorbed_block_n(int d_latent);
+
+// Dense per-head attention, d_head = 128.  q map: 3D (128, n_q, B*n_h) box (64,128,1);
+// kv map: 3D (2*n_h*128, n_keys, B) box (64,128,1); out as above.
+cudaError_t launch_attn_dense_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_out,
+                                 const AttnTc& a, int batch, cudaStream_t s);
+
+struct DenseQTc {  // q' = [q_nope | RoPE(q_rope)] -> [B][n_h][n_q][128]
+  const __nv_bfloat16* q;
+  __nv_bfloat16* qd;
+  int batch, n_q, n_heads;
+  int64_t t_first;
+  Ring ring;
+  Rope rope;
+};
+cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s);
+
+struct ReconTc {  // per-head dense entries from latents (tcgen05)
+  const __nv_bfloat16* kr;  // positional keys [B][rows_per_sample][32] (rotated iff !rotate)
+  __nv_bfloat16* dense;     // [B][ring_rows][2][n_h][128]
+  int rows, n_heads, d_latent;
+  int64_t first_frame;      // frame of row 0 (ring placement and absolute t)
+  int rotate;               // rotate kr with the absolute frame index
+  int to_ring;              // 1: row m -> ring slot of its frame; 0: row m -> row m
+  int64_t kr_rows;          // rows per sample of kr
+  int kr_stride;            // elements between consecutive kr rows
+  int64_t ring_rows;        // rows per sample of dense
+  Ring ring;
+  Rope rope;
+  unsigned* err;
+  uint64_t limit_ns;
+};
+// c map: 3D (d_c, rows, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64,96,1);
+// w_uv map: 3D (d_c, 128, n_h) box (64,128,1)
+cudaError_t launch_recon_tc(const CUtensorMap& tm_c, const CUtensorMap& tm_wuk, const CUtensorMap& tm_wuv,
+                            const ReconTc& a, int batch, cudaStream_t s);
+
+// ------------------------------------------------------------------ device status
+unsigned* device_error_word();  // address of the library's device status word (current device)
+cudaError_t launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s);
+
+}  // namespace vmla

@@ -1,0 +1,92 @@
+// 3D-RoPE kernels of the bf16 path [paperlayer App. C.1, App. D.3, App. D.5]:
+//  * rope_window_bf16: rotate every positional key of the window with its
+//    window-relative (t, h, w) into the workspace.  HBM-bound: each thread
+//    moves one 16-byte vector (4 rotary pairs) in and out, fully coalesced.
+//  * dense_q_bf16: the dense path's query [q_nope | RoPE(q_rope)], re-laid out
+//    head-major for the attention kernel's TMA tiles.
+#include "kernels.h"
+
+namespace vmla {
+namespace {
+
+__device__ __forceinline__ float pair_angle(const Rope& rp, int p, float t, float h, float w) {
+  const float pos = p < rp.n_t ? t : (p < rp.n_t + rp.n_h ? h : w);
+  return pos * rp.freq[p];
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// rotate the 4 pairs held in one 16-byte vector; first pair index p0
+__device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, float t, float h, float w) {
+  uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float s, c;
+    sincosf(pair_angle(rp, p0 + k, t, h, w), &s, &c);
+    const float u = bf_lo(in[k]), x = bf_hi(in[k]);
+    out[k] = pack2(u * c - x * s, u * s + x * c);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// d_rope = 32: 4 threads per key, 16 bytes each
+__global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)a.batch * a.n_keys * 4;
+  if (idx >= total) return;
+  const int quad = idx & 3;
+  const int s = (idx >> 2) % a.n_keys;
+  const int b = (idx >> 2) / a.n_keys;
+  const int64_t ring_rows = (int64_t)a.ring.window_frames * a.ring.tokens_per_frame;
+  const int fslot = s / a.ring.tokens_per_frame, tok = s % a.ring.tokens_per_frame;
+  const int t = (fslot - a.window_start_slot + a.ring.window_frames) % a.ring.window_frames;
+  const int64_t off = ((int64_t)b * ring_rows + s) * 32 + quad * 8;
+  const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + off);
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + off) =
+      rotate4(v, a.rope, quad * 4, (float)t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+}
+
+// 16 threads per (sample, query, head): 12 copy the content dims, 4 rotate the positional ones
+__global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
+  if (idx >= total) return;
+  const int chunk = idx & 15;
+  const int h = (idx >> 4) % a.n_heads;
+  const int i = ((idx >> 4) / a.n_heads) % a.n_q;
+  const int b = (idx >> 4) / ((int64_t)a.n_heads * a.n_q);
+  const __nv_bfloat16* src = a.q + (((int64_t)b * a.n_q + i) * a.n_heads + h) * 128 + chunk * 8;
+  __nv_bfloat16* dst = a.qd + (((int64_t)b * a.n_heads + h) * a.n_q + i) * 128 + chunk * 8;
+  uint4 v = *reinterpret_cast<const uint4*>(src);
+  if (chunk >= 12) {
+    const int tok = i % a.ring.tokens_per_frame;
+    const float t = (float)(a.t_first + i / a.ring.tokens_per_frame);
+    v = rotate4(v, a.rope, (chunk - 12) * 4, t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+  }
+  *reinterpret_cast<uint4*>(dst) = v;
+}
+
+}  // namespace
+
+cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s) {
+  if (a.d_rope != 32) return cudaErrorInvalidValue;
+  const int64_t total = (int64_t)a.batch * a.n_keys * 4;
+  if (total == 0) return cudaSuccess;
+  rope_window_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s) {
+  const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
+  if (total == 0) return cudaSuccess;
+  dense_q_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace vmla

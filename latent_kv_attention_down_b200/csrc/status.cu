@@ -1,0 +1,40 @@
+// The library's device status word and the self-test of the bounded waits.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace vmla {
+
+__device__ unsigned g_device_error;
+
+unsigned* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<unsigned*>(p);
+}
+
+namespace {
+// One thread waits on an mbarrier that nothing arrives at; the bounded wait must
+// give up after limit_ns, record DEV_ERR_TIMEOUT_SELFTEST and return.
+__global__ void selftest_wait_kernel(unsigned* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Guard g{&abort_flag, err, limit_ns};
+    wait_phase(&bar, 0, g, DEV_ERR_TIMEOUT_SELFTEST);
+  }
+  __syncthreads();
+}
+}  // namespace
+
+cudaError_t launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace vmla

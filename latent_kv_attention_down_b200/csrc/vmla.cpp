@@ -1,0 +1,898 @@
+// Host side of libvmla.so: the C ABI declared in include/vmla.h.
+//
+// Validates every call, keeps the per-layer frame counters of the sliding
+// window (FIFO ring of window_frames frames, slot = frame mod W [paperlayer
+// App. D.4]), encodes the TMA tensor maps of each launch and enqueues the
+// kernels on the caller's stream.  It allocates no device memory.
+#include "vmla.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "kernels.h"
+
+using namespace vmla;
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any healthy pipeline wait
+constexpr int kStages = 8;
+constexpr int kMaxPos = 1024;  // RoPE range per axis [paperlayer App. C.1]
+
+size_t esize(const vmla_config& c) { return c.dtype == VMLA_BF16 ? 2 : 4; }
+int64_t tokens_per_frame(const vmla_config& c) { return (int64_t)c.grid_h * c.grid_w; }
+int64_t ring_rows(const vmla_config& c) { return (int64_t)c.window_frames * tokens_per_frame(c); }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, recon = 0;  // offsets
+  size_t base_bytes = 0;   // every design but RECON_ONCE
+  size_t recon_bytes = 0;  // extra for RECON_ONCE
+};
+
+WsLayout ws_layout(const vmla_config& c) {
+  const size_t e = esize(c);
+  const size_t B = c.batch, nq = (size_t)c.chunk_frames * tokens_per_frame(c);
+  const size_t dh = (size_t)c.d_nope + c.d_rope;
+  WsLayout w;
+  size_t off = 0;
+  w.kr_rot = off;
+  off = align256(off + B * ring_rows(c) * c.d_rope * e);
+  w.qt = off;
+  off = align256(off + B * c.n_heads * nq * (size_t)(c.d_latent + c.d_rope) * e);
+  w.dq = off;
+  off = align256(off + B * c.n_heads * nq * dh * e);
+  w.chunk = off;  // a chunk's latents: [B][rows][d_c + d_rope] (plus a d_rope copy for fp32)
+  off = align256(off + B * (size_t)c.window_frames * tokens_per_frame(c) * (size_t)(c.d_latent + 2 * c.d_rope) * e);
+  w.recon = off;
+  w.base_bytes = off;
+  w.recon_bytes = B * ring_rows(c) * 2 * (size_t)c.n_heads * c.d_value * e;
+  return w;
+}
+
+Rope make_rope(const vmla_config& c) {
+  Rope r;
+  std::memset(&r, 0, sizeof(r));
+  int p = 0;
+  for (int a = 0; a < 3; ++a) {
+    const double base = c.rope_base_dims[a] > 0 ? c.rope_base_dims[a] : 2.0 * c.rope_pairs[a];
+    for (int i = 0; i < c.rope_pairs[a]; ++i) r.freq[p++] = (float)std::pow((double)c.rope_theta, -2.0 * i / base);
+  }
+  r.n_t = c.rope_pairs[0];
+  r.n_h = c.rope_pairs[1];
+  r.n_w = c.rope_pairs[2];
+  return r;
+}
+
+Ring make_ring(const vmla_config& c) { return Ring{(int)tokens_per_frame(c), c.grid_w, c.window_frames}; }
+
+// ---------------------------------------------------------------- TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool have_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 3D map: dims (d0 innermost, d1, d2), byte strides s1, s2, box (b0, b1, 1); bf16 unless told otherwise
+bool map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+          uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw,
+          CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  if (!have_encode()) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
+          CUtensorMapSwizzle sw) {
+  if (!have_encode()) return false;
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {s1};
+  cuuint32_t box[2] = {b0, b1};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : VMLA_ERR_CUDA; }
+
+// AUTO: the absorbed design up to d_latent = 192; from 256 on the per-head K/V
+// are rebuilt once per call.  At 256 the rebuilt path is the more accurate one
+// (it rounds K and V per key, where the absorbed query carries one bf16
+// rounding for every key of a row) and the absorbed MMA work (2 d_latent +
+// d_rope per key) is over twice the per-head attention's (2 d_head).
+vmla_design resolve_design(const vmla_config& c, vmla_design d) {
+  if (d != VMLA_DESIGN_AUTO) return d;
+  if (c.dtype == VMLA_BF16 && c.d_latent >= 256) return VMLA_DESIGN_RECON_ONCE;
+  return VMLA_DESIGN_ABSORBED;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- handle
+struct vmla_handle {
+  vmla_config cfg;
+  void* ckv = nullptr;
+  void* kr = nullptr;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  void* dense = nullptr;
+  std::vector<int64_t> frames;        // latent cache, per layer
+  std::vector<int64_t> dense_frames;  // dense cache, per layer
+  unsigned* err = nullptr;            // device status word (resolved at bind)
+  bool profiling = false;
+  struct Timer {
+    std::vector<cudaEvent_t> ev;  // begin/end pairs
+    size_t used = 0;
+  } timers[kStages];
+};
+
+namespace {
+
+struct StageScope {  // CUDA events around one stage's launch(es) when profiling
+  vmla_handle* h;
+  int stage;
+  cudaStream_t s;
+  bool on = false;
+  StageScope(vmla_handle* h_, int st, cudaStream_t s_) : h(h_), stage(st), s(s_) {
+    if (!h->profiling) return;
+    auto& t = h->timers[stage];
+    if (t.used + 2 > t.ev.size()) {
+      for (int k = 0; k < 2; ++k) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return;
+        t.ev.push_back(e);
+      }
+    }
+    on = cudaEventRecord(t.ev[t.used], s) == cudaSuccess;
+  }
+  ~StageScope() {
+    if (!on) return;
+    auto& t = h->timers[stage];
+    cudaEventRecord(t.ev[t.used + 1], s);
+    t.used += 2;
+  }
+};
+
+// The device status word of the current device, resolved at the first launch.
+vmla_status ensure_err(vmla_handle* h) {
+  if (!h->err) h->err = device_error_word();
+  return h->err ? VMLA_OK : VMLA_ERR_CUDA;
+}
+
+vmla_status check_layer(const vmla_handle* h, int layer) {
+  if (!h) return VMLA_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= h->cfg.layers) return VMLA_ERR_OUT_OF_RANGE;
+  return VMLA_OK;
+}
+
+// Frame rule of an append: a new chunk right after the newest frame, or a
+// rewrite of the newest frames (a further denoising pass).
+vmla_status check_append_frames(const vmla_config& c, int64_t F, int64_t first, int n, int64_t* new_F) {
+  if (n < 1 || n > c.window_frames) return VMLA_ERR_OUT_OF_RANGE;
+  if (first < 0) return VMLA_ERR_STATE;
+  if (first == F)
+    *new_F = F + n;
+  else if (first + n == F)
+    *new_F = F;
+  else
+    return VMLA_ERR_STATE;
+  return VMLA_OK;
+}
+
+struct Window {
+  int64_t start;  // first window frame
+  int n_keys;
+  int start_slot;
+};
+
+vmla_status check_attention_frames(const vmla_config& c, int64_t F, int64_t first, int n, Window* w) {
+  if (n < 1 || n > c.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
+  if (F < 1 || first < 0 || first + n != F) return VMLA_ERR_STATE;
+  w->start = F > c.window_frames ? F - c.window_frames : 0;
+  w->n_keys = (int)((F - w->start) * tokens_per_frame(c));
+  w->start_slot = (int)(w->start % c.window_frames);
+  return VMLA_OK;
+}
+
+template <class T>
+T* at(void* base, size_t byte_off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + byte_off);
+}
+
+size_t layer_cache_offset(const vmla_config& c, int layer, int width) {
+  return (size_t)layer * c.batch * ring_rows(c) * width * esize(c);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vmla_status_string(vmla_status s) {
+  switch (s) {
+    case VMLA_OK: return "VMLA_OK";
+    case VMLA_ERR_INVALID_ARG: return "VMLA_ERR_INVALID_ARG";
+    case VMLA_ERR_UNSUPPORTED_SHAPE: return "VMLA_ERR_UNSUPPORTED_SHAPE";
+    case VMLA_ERR_OUT_OF_RANGE: return "VMLA_ERR_OUT_OF_RANGE";
+    case VMLA_ERR_CUDA: return "VMLA_ERR_CUDA";
+    case VMLA_ERR_DEVICE_TIMEOUT: return "VMLA_ERR_DEVICE_TIMEOUT";
+    case VMLA_ERR_STATE: return "VMLA_ERR_STATE";
+    case VMLA_ERR_DEVICE_BOUNDS: return "VMLA_ERR_DEVICE_BOUNDS";
+  }
+  return "VMLA_ERR_UNKNOWN";
+}
+
+int vmla_abi_version(void) { return VMLA_ABI_VERSION; }
+
+vmla_status vmla_config_init(vmla_config* c) {
+  if (!c) return VMLA_ERR_INVALID_ARG;
+  std::memset(c, 0, sizeof(*c));
+  c->d_model = 1536;
+  c->n_heads = 12;
+  c->d_nope = 96;
+  c->d_rope = 32;
+  c->d_latent = 192;
+  c->d_value = 128;
+  c->rope_pairs[0] = 6;
+  c->rope_pairs[1] = 5;
+  c->rope_pairs[2] = 5;
+  c->rope_theta = 10000.f;
+  c->grid_h = 30;
+  c->grid_w = 52;
+  c->window_frames = 21;
+  c->chunk_frames = 3;
+  c->batch = 1;
+  c->layers = 1;
+  c->dtype = VMLA_BF16;
+  c->rope_mode = VMLA_ROPE_AT_READ;
+  c->softmax_rescale_log2 = 8.f;
+  return VMLA_OK;
+}
+
+vmla_status vmla_config_check(const vmla_config* c) {
+  if (!c) return VMLA_ERR_INVALID_ARG;
+  if (c->dtype != VMLA_BF16 && c->dtype != VMLA_FP32) return VMLA_ERR_INVALID_ARG;
+  if (c->rope_mode != VMLA_ROPE_AT_READ && c->rope_mode != VMLA_ROPE_AT_APPEND) return VMLA_ERR_INVALID_ARG;
+  if (c->d_model < 1 || c->n_heads < 1 || c->d_nope < 0 || c->d_rope < 0 || c->d_latent < 1 || c->d_value < 1 ||
+      c->grid_h < 1 || c->grid_w < 1 || c->window_frames < 1 || c->chunk_frames < 1 || c->batch < 1 ||
+      c->layers < 1 || !(c->rope_theta > 0.f) || !(c->softmax_rescale_log2 >= 0.f))
+    return VMLA_ERR_INVALID_ARG;
+  int pairs = 0;
+  for (int a = 0; a < 3; ++a) {
+    if (c->rope_pairs[a] < 0 || c->rope_base_dims[a] < 0) return VMLA_ERR_INVALID_ARG;
+    pairs += c->rope_pairs[a];
+  }
+  if (2 * pairs != c->d_rope || pairs > kMaxPairs) return VMLA_ERR_INVALID_ARG;
+  if (c->chunk_frames > c->window_frames) return VMLA_ERR_INVALID_ARG;
+  if (c->d_value != c->d_nope + c->d_rope) return VMLA_ERR_UNSUPPORTED_SHAPE;  // dense layout [2][n_h][d_head]
+  if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if (c->dtype == VMLA_BF16) {
+    if (c->d_rope != 32 || c->d_nope != 96 || c->d_value != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_latent % 64 != 0 || c->d_latent < 64 || c->d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_model % 64 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  } else {
+    if (c->d_latent + c->d_rope > 1024 || c->d_value > 1024) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  }
+  return VMLA_OK;
+}
+
+vmla_status vmla_cache_bytes(const vmla_config* c, size_t* ckv, size_t* kr, size_t* dense) {
+  vmla_status st = vmla_config_check(c);
+  if (st != VMLA_OK) return st;
+  const size_t rows = (size_t)c->layers * c->batch * ring_rows(*c);
+  if (ckv) *ckv = rows * c->d_latent * esize(*c);
+  if (kr) *kr = rows * c->d_rope * esize(*c);
+  if (dense) *dense = rows * 2 * (size_t)c->n_heads * c->d_value * esize(*c);
+  return VMLA_OK;
+}
+
+vmla_status vmla_workspace_bytes(const vmla_config* c, vmla_design d, size_t* bytes) {
+  vmla_status st = vmla_config_check(c);
+  if (st != VMLA_OK) return st;
+  if (!bytes || d < VMLA_DESIGN_AUTO || d > VMLA_DESIGN_RECON_ONCE) return VMLA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(*c);
+  *bytes = w.base_bytes + (resolve_design(*c, d) == VMLA_DESIGN_RECON_ONCE ? w.recon_bytes : 0);
+  return VMLA_OK;
+}
+
+vmla_status vmla_rope_frequencies(const vmla_config* c, float* freqs, int n) {
+  vmla_status st = vmla_config_check(c);
+  if (st != VMLA_OK) return st;
+  if (!freqs || n < c->d_rope / 2) return VMLA_ERR_INVALID_ARG;
+  const Rope r = make_rope(*c);
+  for (int p = 0; p < c->d_rope / 2; ++p) freqs[p] = r.freq[p];
+  return VMLA_OK;
+}
+
+vmla_status vmla_create(const vmla_config* c, vmla_handle** out) {
+  if (!out) return VMLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  vmla_status st = vmla_config_check(c);
+  if (st != VMLA_OK) return st;
+  vmla_handle* h = new (std::nothrow) vmla_handle();
+  if (!h) return VMLA_ERR_INVALID_ARG;
+  h->cfg = *c;
+  h->frames.assign(c->layers, 0);
+  h->dense_frames.assign(c->layers, 0);
+  *out = h;
+  return VMLA_OK;
+}
+
+vmla_status vmla_destroy(vmla_handle* h) {
+  if (!h) return VMLA_ERR_INVALID_ARG;
+  for (auto& t : h->timers)
+    for (cudaEvent_t e : t.ev) cudaEventDestroy(e);
+  delete h;
+  return VMLA_OK;
+}
+
+vmla_status vmla_bind(vmla_handle* h, void* ckv, void* kr, void* ws, size_t ws_bytes) {
+  if (!h || !ckv || !kr || !ws) return VMLA_ERR_INVALID_ARG;
+  if (!aligned16(ckv) || !aligned16(kr) || !aligned16(ws)) return VMLA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(h->cfg);
+  if (ws_bytes < w.base_bytes) return VMLA_ERR_INVALID_ARG;
+  h->ckv = ckv;
+  h->kr = kr;
+  h->ws = ws;
+  h->ws_bytes = ws_bytes;
+  h->frames.assign(h->cfg.layers, 0);
+  return VMLA_OK;
+}
+
+vmla_status vmla_dense_bind(vmla_handle* h, void* dense) {
+  if (!h || !dense || !aligned16(dense)) return VMLA_ERR_INVALID_ARG;
+  h->dense = dense;
+  h->dense_frames.assign(h->cfg.layers, 0);
+  return VMLA_OK;
+}
+
+vmla_status vmla_window(const vmla_handle* h, int64_t F, int32_t* frame, int32_t* slot, int32_t* t_local,
+                        int capacity, int* n) {
+  if (!h || !n || F < 0) return VMLA_ERR_INVALID_ARG;
+  const int W = h->cfg.window_frames;
+  const int64_t start = F > W ? F - W : 0;
+  const int count = (int)(F - start);
+  *n = count;
+  if (count > capacity) return VMLA_ERR_INVALID_ARG;
+  for (int k = 0; k < count; ++k) {
+    const int64_t f = start + k;
+    if (frame) frame[k] = (int32_t)f;
+    if (slot) slot[k] = (int32_t)(f % W);
+    if (t_local) t_local[k] = (int32_t)(f - start);
+  }
+  return VMLA_OK;
+}
+
+vmla_status vmla_state_get(const vmla_handle* h, int layer, int64_t* F) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!F) return VMLA_ERR_INVALID_ARG;
+  *F = h->frames[layer];
+  return VMLA_OK;
+}
+
+vmla_status vmla_state_set(vmla_handle* h, int layer, int64_t F) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (F < 0) return VMLA_ERR_INVALID_ARG;
+  h->frames[layer] = F;
+  return VMLA_OK;
+}
+
+vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, int64_t first,
+                              int n, void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->ckv) return VMLA_ERR_STATE;
+  if (!x || !w_down || !aligned16(x) || !aligned16(w_down)) return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  int64_t new_F;
+  if ((st = check_append_frames(c, h->frames[layer], first, n, &new_F)) != VMLA_OK) return st;
+  const bool rotate = c.rope_mode == VMLA_ROPE_AT_APPEND;
+  if (rotate && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows = (int)(n * tokens_per_frame(c));
+  cudaError_t e;
+  {
+    StageScope scope(h, 0, s);
+    if (c.dtype == VMLA_FP32) {
+      SimtAppend a;
+      a.x = static_cast<const float*>(x);
+      a.w_down = static_cast<const float*>(w_down);
+      a.ckv = at<float>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
+      a.kr = at<float>(h->kr, layer_cache_offset(c, layer, c.d_rope));
+      a.batch = c.batch;
+      a.rows = rows;
+      a.d_model = c.d_model;
+      a.d_latent = c.d_latent;
+      a.d_rope = c.d_rope;
+      a.first_frame = first;
+      a.rotate = rotate;
+      a.contiguous = 0;
+      a.out_rows = ring_rows(c);
+      a.ring = make_ring(c);
+      a.rope = make_rope(c);
+      e = launch_append_simt(a, s);
+    } else {
+      CUtensorMap tx, tw;
+      const int nout = c.d_latent + 32;
+      if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_tc_w_box_rows(c.d_latent),
+                CU_TENSOR_MAP_SWIZZLE_128B))
+        return VMLA_ERR_CUDA;
+      AppendTc a;
+      a.ckv = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
+      a.kr = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
+      a.rows = rows;
+      a.d_model = c.d_model;
+      a.d_latent = c.d_latent;
+      a.first_frame = first;
+      a.rotate = rotate;
+      a.contiguous = 0;
+      a.ring_rows = ring_rows(c);
+      a.ring = make_ring(c);
+      a.rope = make_rope(c);
+      a.err = h->err;
+      a.limit_ns = kWaitLimitNs;
+      e = launch_append_tc(tx, tw, a, c.batch, s);
+    }
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  h->frames[layer] = new_F;
+  return VMLA_OK;
+}
+
+namespace {
+
+vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
+                           int64_t first, int n, const Window& win, cudaStream_t s) {
+  const vmla_config& c = h->cfg;
+  const WsLayout w = ws_layout(c);
+  const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
+  float* kr_layer = at<float>(h->kr, layer_cache_offset(c, layer, c.d_rope));
+  const float* kpos = kr_layer;
+  cudaError_t e = cudaSuccess;
+  if (at_read) {
+    StageScope scope(h, 1, s);
+    RopeWindow r{kr_layer, at<float>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
+                 make_ring(c), make_rope(c)};
+    e = launch_rope_window_f32(r, s);
+    kpos = at<float>(h->ws, w.kr_rot);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  const int nq = (int)(n * tokens_per_frame(c));
+  {
+    StageScope scope(h, 2, s);
+    SimtQPrep a{static_cast<const float*>(q), static_cast<const float*>(w_uk), at<float>(h->ws, w.qt), c.batch, nq,
+                c.n_heads, c.d_nope, c.d_rope, c.d_latent, 1, first - (at_read ? win.start : 0), make_ring(c),
+                make_rope(c)};
+    e = launch_qprep_simt(a, s);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  {
+    StageScope scope(h, 3, s);
+    SimtAttn a;
+    a.qt = at<float>(h->ws, w.qt);
+    a.key = at<float>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
+    a.kpos = kpos;
+    a.w_uv = static_cast<const float*>(w_uv);
+    a.out = static_cast<float*>(out);
+    a.batch = c.batch;
+    a.n_q = nq;
+    a.n_keys = win.n_keys;
+    a.n_heads = c.n_heads;
+    a.d_latent = c.d_latent;
+    a.d_rope = c.d_rope;
+    a.d_value = c.d_value;
+    a.dense = 0;
+    a.ring_rows = ring_rows(c);
+    a.scale = 1.f / std::sqrt((float)(c.d_nope + c.d_rope));
+    e = launch_attn_simt(a, s);
+  }
+  return cuda_status(e);
+}
+
+vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const void* kv_base, void* out, int nq,
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s);
+
+vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
+                           int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s) {
+  const vmla_config& c = h->cfg;
+  const WsLayout w = ws_layout(c);
+  const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
+  const int nq = (int)(n * tokens_per_frame(c));
+  const int64_t t_first = first - (at_read ? win.start : 0);
+  __nv_bfloat16* ckv_layer = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
+  __nv_bfloat16* kr_layer = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
+  const __nv_bfloat16* kpos = kr_layer;
+  cudaError_t e = cudaSuccess;
+  if (at_read) {
+    StageScope scope(h, 1, s);
+    RopeWindow r{kr_layer, at<__nv_bfloat16>(h->ws, w.kr_rot), c.batch, win.n_keys, 32, win.start_slot,
+                 make_ring(c), make_rope(c)};
+    e = launch_rope_window_bf16(r, s);
+    kpos = at<__nv_bfloat16>(h->ws, w.kr_rot);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  const uint64_t rr = ring_rows(c);
+
+  if (design == VMLA_DESIGN_RECON_ONCE) {
+    if (h->ws_bytes < w.base_bytes + w.recon_bytes) return VMLA_ERR_STATE;
+    __nv_bfloat16* recon = at<__nv_bfloat16>(h->ws, w.recon);
+    {
+      StageScope scope(h, 7, s);
+      CUtensorMap tc, tuk, tuv;
+      if (!map3(&tc, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64,
+                128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+        return VMLA_ERR_CUDA;
+      ReconTc a;
+      a.kr = kpos;
+      a.dense = recon;
+      a.rows = win.n_keys;
+      a.n_heads = c.n_heads;
+      a.d_latent = c.d_latent;
+      a.first_frame = 0;
+      a.rotate = 0;  // positional keys are already rotated (at read into the workspace, or at append)
+      a.to_ring = 0;
+      a.kr_rows = rr;
+      a.kr_stride = 32;
+      a.ring_rows = rr;
+      a.ring = make_ring(c);
+      a.rope = make_rope(c);
+      a.err = h->err;
+      a.limit_ns = kWaitLimitNs;
+      e = launch_recon_tc(tc, tuk, tuv, a, c.batch, s);
+    }
+    if (e != cudaSuccess) return VMLA_ERR_CUDA;
+    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s);
+  }
+  if (design == VMLA_DESIGN_RECONSTRUCT) return VMLA_ERR_UNSUPPORTED_SHAPE;
+
+  __nv_bfloat16* qt = at<__nv_bfloat16>(h->ws, w.qt);
+  const int dqk = c.d_latent + 32;
+  {
+    StageScope scope(h, 2, s);
+    CUtensorMap tq, tuk;
+    if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 2,
+              (uint64_t)nq * c.n_heads * 128 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+              CU_TENSOR_MAP_SWIZZLE_128B))
+      return VMLA_ERR_CUDA;
+    QPrepTc a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.qt = qt;
+    a.n_q = nq;
+    a.n_heads = c.n_heads;
+    a.d_latent = c.d_latent;
+    a.t_first = t_first;
+    a.ring = make_ring(c);
+    a.rope = make_rope(c);
+    a.err = h->err;
+    a.limit_ns = kWaitLimitNs;
+    e = launch_qprep_tc(tq, tuk, a, c.batch, s);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  {
+    StageScope scope(h, 3, s);
+    const int bn = attn_absorbed_block_n(c.d_latent);
+    const uint64_t bh = (uint64_t)c.batch * c.n_heads;
+    CUtensorMap tq, tqr, tk, tkr, tuv, to;
+    if (!map3(&tq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map3(&tk, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, bn,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
+              (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+      return VMLA_ERR_CUDA;
+    AttnTc a;
+    a.n_q = nq;
+    a.n_keys = win.n_keys;
+    a.n_heads = c.n_heads;
+    a.m_tiles = (nq + 127) / 128;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)(c.d_nope + c.d_rope)));
+    a.rescale_threshold = c.softmax_rescale_log2;
+    a.err = h->err;
+    a.limit_ns = kWaitLimitNs;
+    e = launch_attn_absorbed_tc(c.d_latent, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
+  }
+  return cuda_status(e);
+}
+
+// Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128].
+vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const void* kv_base, void* out, int nq,
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s) {
+  const vmla_config& c = h->cfg;
+  const WsLayout w = ws_layout(c);
+  __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
+  cudaError_t e;
+  {
+    StageScope scope(h, 2, s);
+    DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, t_first, make_ring(c),
+               make_rope(c)};
+    e = launch_dense_q_bf16(a, s);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  StageScope scope(h, stage, s);
+  const uint64_t rr = ring_rows(c);
+  const uint64_t row_bytes = 2ull * c.n_heads * 128 * 2;
+  CUtensorMap tq, tkv, to;
+  if (!map3(&tq, qd, 128, nq, (uint64_t)c.batch * c.n_heads, 256, (uint64_t)nq * 256, 64, 128,
+            CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&tkv, kv_base, 2ull * c.n_heads * 128, n_keys, c.batch, row_bytes, rr * row_bytes, 64, 128,
+            CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
+            (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+    return VMLA_ERR_CUDA;
+  AttnTc a;
+  a.n_q = nq;
+  a.n_keys = n_keys;
+  a.n_heads = c.n_heads;
+  a.m_tiles = (nq + 127) / 128;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)(c.d_nope + c.d_rope)));
+  a.rescale_threshold = c.softmax_rescale_log2;
+  a.err = h->err;
+  a.limit_ns = kWaitLimitNs;
+  return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s));
+}
+
+}  // namespace
+
+vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
+                                 void* out, int64_t first, int n, vmla_design design, void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->ckv) return VMLA_ERR_STATE;
+  if (!q || !w_uk || !w_uv || !out || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
+    return VMLA_ERR_INVALID_ARG;
+  if (design < VMLA_DESIGN_AUTO || design > VMLA_DESIGN_RECON_ONCE) return VMLA_ERR_INVALID_ARG;
+  Window win;
+  if ((st = check_attention_frames(h->cfg, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
+  if (h->cfg.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  design = resolve_design(h->cfg, design);
+  if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
+  return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s);
+}
+
+vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, const void* w_uk,
+                                    const void* w_uv, int64_t first, int n, void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->dense || !h->ws) return VMLA_ERR_STATE;
+  if (!x || !w_down || !w_uk || !w_uv || !aligned16(x) || !aligned16(w_down) || !aligned16(w_uk) || !aligned16(w_uv))
+    return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  int64_t new_F;
+  if ((st = check_append_frames(c, h->dense_frames[layer], first, n, &new_F)) != VMLA_OK) return st;
+  if (first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(c);
+  const int rows = (int)(n * tokens_per_frame(c));
+  const size_t dense_off = (size_t)layer * c.batch * ring_rows(c) * 2 * c.n_heads * c.d_value * esize(c);
+  cudaError_t e;
+  StageScope scope(h, 5, s);
+  if (c.dtype == VMLA_FP32) {
+    float* cbuf = at<float>(h->ws, w.chunk);
+    float* rbuf = cbuf + (size_t)c.batch * rows * c.d_latent;
+    SimtAppend a;
+    a.x = static_cast<const float*>(x);
+    a.w_down = static_cast<const float*>(w_down);
+    a.ckv = cbuf;
+    a.kr = rbuf;
+    a.batch = c.batch;
+    a.rows = rows;
+    a.d_model = c.d_model;
+    a.d_latent = c.d_latent;
+    a.d_rope = c.d_rope;
+    a.first_frame = first;
+    a.rotate = 0;
+    a.contiguous = 1;
+    a.out_rows = rows;
+    a.ring = make_ring(c);
+    a.rope = make_rope(c);
+    if ((e = launch_append_simt(a, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+    SimtDenseReconstruct d{cbuf, rbuf, static_cast<const float*>(w_uk), static_cast<const float*>(w_uv),
+                           at<float>(h->dense, dense_off), c.batch, rows, c.n_heads, c.d_nope, c.d_rope,
+                           c.d_latent, c.d_value, first, make_ring(c), make_rope(c)};
+    e = launch_dense_reconstruct_simt(d, s);
+  } else {
+    __nv_bfloat16* chunk = at<__nv_bfloat16>(h->ws, w.chunk);  // [B][rows][d_c + 32]
+    const int nout = c.d_latent + 32;
+    CUtensorMap tx, tw;
+    if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_tc_w_box_rows(c.d_latent),
+              CU_TENSOR_MAP_SWIZZLE_128B))
+      return VMLA_ERR_CUDA;
+    AppendTc a;
+    a.ckv = chunk;
+    a.kr = nullptr;
+    a.rows = rows;
+    a.d_model = c.d_model;
+    a.d_latent = c.d_latent;
+    a.first_frame = first;
+    a.rotate = 0;
+    a.contiguous = 1;
+    a.ring_rows = rows;
+    a.ring = make_ring(c);
+    a.rope = make_rope(c);
+    a.err = h->err;
+    a.limit_ns = kWaitLimitNs;
+    if ((e = launch_append_tc(tx, tw, a, c.batch, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+    CUtensorMap tc, tuk, tuv;
+    if (!map3(&tc, chunk, c.d_latent, rows, c.batch, (uint64_t)nout * 2, (uint64_t)rows * nout * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B))
+      return VMLA_ERR_CUDA;
+    ReconTc r;
+    r.kr = chunk + c.d_latent;  // positional key columns of the chunk rows (row stride d_c + 32)
+    r.dense = at<__nv_bfloat16>(h->dense, dense_off);
+    r.rows = rows;
+    r.n_heads = c.n_heads;
+    r.d_latent = c.d_latent;
+    r.first_frame = first;
+    r.rotate = 1;
+    r.to_ring = 1;
+    r.kr_rows = rows;
+    r.kr_stride = nout;
+    r.ring_rows = ring_rows(c);
+    r.ring = make_ring(c);
+    r.rope = make_rope(c);
+    r.err = h->err;
+    r.limit_ns = kWaitLimitNs;
+    e = launch_recon_tc(tc, tuk, tuv, r, c.batch, s);
+  }
+  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  h->dense_frames[layer] = new_F;
+  return VMLA_OK;
+}
+
+vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q, void* out, int64_t first, int n,
+                                       void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->dense || !h->ws) return VMLA_ERR_STATE;
+  if (!q || !out || !aligned16(q) || !aligned16(out)) return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  Window win;
+  if ((st = check_attention_frames(c, h->dense_frames[layer], first, n, &win)) != VMLA_OK) return st;
+  if (first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(c);
+  const int nq = (int)(n * tokens_per_frame(c));
+  const size_t dense_off = (size_t)layer * c.batch * ring_rows(c) * 2 * c.n_heads * c.d_value * esize(c);
+  if (c.dtype == VMLA_BF16)
+    return dense_attention_bf16_launch(h, q, at<char>(h->dense, dense_off), out, nq, win.n_keys, first, 6, s);
+  cudaError_t e;
+  {
+    StageScope scope(h, 2, s);
+    SimtQPrep a{static_cast<const float*>(q), nullptr, at<float>(h->ws, w.dq), c.batch, nq, c.n_heads, c.d_nope,
+                c.d_rope, c.d_latent, 0, first, make_ring(c), make_rope(c)};
+    if ((e = launch_qprep_simt(a, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+  }
+  StageScope scope(h, 6, s);
+  SimtAttn a;
+  a.qt = at<float>(h->ws, w.dq);
+  a.key = at<float>(h->dense, dense_off);
+  a.kpos = nullptr;
+  a.w_uv = nullptr;
+  a.out = static_cast<float*>(out);
+  a.batch = c.batch;
+  a.n_q = nq;
+  a.n_keys = win.n_keys;
+  a.n_heads = c.n_heads;
+  a.d_latent = c.d_latent;
+  a.d_rope = c.d_rope;
+  a.d_value = c.d_value;
+  a.dense = 1;
+  a.ring_rows = ring_rows(c);
+  a.scale = 1.f / std::sqrt((float)(c.d_nope + c.d_rope));
+  return cuda_status(launch_attn_simt(a, s));
+}
+
+vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, const void* q_host, void* out_host,
+                                 const void* w_down, const void* w_uk, const void* w_uv, void* x_dev, void* q_dev,
+                                 void* out_dev, int64_t first, int n, vmla_design design, void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!x_host || !q_host || !out_host || !x_dev || !q_dev || !out_dev) return VMLA_ERR_INVALID_ARG;
+  if (n < 1 || n > h->cfg.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
+  const vmla_config& c = h->cfg;
+  const size_t rows = (size_t)n * tokens_per_frame(c) * c.batch;
+  const size_t xb = rows * c.d_model * esize(c);
+  const size_t qb = rows * c.n_heads * (size_t)(c.d_nope + c.d_rope) * esize(c);
+  const size_t ob = rows * c.n_heads * (size_t)c.d_value * sizeof(float);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return VMLA_ERR_CUDA;
+  if ((st = vmla_cache_append(h, layer, x_dev, w_down, first, n, stream)) != VMLA_OK) return st;
+  if ((st = vmla_chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream)) != VMLA_OK)
+    return st;
+  return cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s) == cudaSuccess ? VMLA_OK : VMLA_ERR_CUDA;
+}
+
+vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
+  if (!h) return VMLA_ERR_INVALID_ARG;
+  unsigned* err = h->err ? h->err : device_error_word();
+  if (!err) return VMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VMLA_ERR_CUDA;
+  if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return VMLA_ERR_CUDA;
+  if (v && cudaMemset(err, 0, sizeof(v)) != cudaSuccess) return VMLA_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v & DEV_ERR_BOUNDS_MASK) return VMLA_ERR_DEVICE_BOUNDS;
+  if (v) return VMLA_ERR_DEVICE_TIMEOUT;
+  return VMLA_OK;
+}
+
+vmla_status vmla_profile_enable(vmla_handle* h, int enable) {
+  if (!h) return VMLA_ERR_INVALID_ARG;
+  h->profiling = enable != 0;
+  for (auto& t : h->timers) t.used = 0;
+  return VMLA_OK;
+}
+
+vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* launches) {
+  if (!h || stage < 0 || stage >= kStages || !total_ms || !launches) return VMLA_ERR_INVALID_ARG;
+  auto& t = h->timers[stage];
+  double sum = 0;
+  for (size_t k = 0; k + 1 < t.used; k += 2) {
+    if (cudaEventSynchronize(t.ev[k + 1]) != cudaSuccess) return VMLA_ERR_CUDA;
+    float ms = 0;
+    if (cudaEventElapsedTime(&ms, t.ev[k], t.ev[k + 1]) != cudaSuccess) return VMLA_ERR_CUDA;
+    sum += ms;
+  }
+  *total_ms = sum;
+  *launches = (int)(t.used / 2);
+  return VMLA_OK;
+}
+
+vmla_status vmla_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns > 1000000000ull) return VMLA_ERR_INVALID_ARG;
+  unsigned* err = device_error_word();
+  if (!err) return VMLA_ERR_CUDA;
+  return cuda_status(launch_selftest_wait(err, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+"""The C ABI on the host: the library loads and exports every declared entry
+point; configuration checks, cache accounting, RoPE frequencies, window and
+frame bookkeeping.  No CUDA compute call is made here."""
+import collections
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle.vmla_oracle as O
+from latent_kv_attention_down_b200 import api, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(vmla_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = api.lib()
+    names = declared_functions()
+    assert len(names) >= 20
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding declares a signature for each of them
+    assert set(names) <= set(api._SIGS), set(names) - set(api._SIGS)
+
+
+def test_abi_version_and_status_strings():
+    lib = api.lib()
+    assert lib.vmla_abi_version() == 1
+    for code in range(8):
+        assert lib.vmla_status_string(code).decode().startswith("VMLA_")
+    assert lib.vmla_status_string(99).decode() == "VMLA_ERR_UNKNOWN"
+
+
+def default_config():
+    c = api.Config()
+    api.check(api.lib().vmla_config_init(ctypes.byref(c)), "init")
+    return c
+
+
+def test_default_config_is_the_wan_layer(golden):
+    c = default_config()
+    g = {k: v["value"] for k, v in golden.items()}
+    assert (c.d_model, c.n_heads, c.d_latent, c.d_rope) == (g["d_model"], g["n_heads"], g["d_latent"], g["d_rope"])
+    assert c.d_nope + c.d_rope == g["d_head"] and [c.d_nope, c.d_rope] == g["nope_rope_split"]
+    assert list(c.rope_pairs) == g["rope_pairs_thw"]
+    assert c.grid_h * c.grid_w == g["tokens_per_latent_frame"]
+    assert c.window_frames == g["latent_frames_per_clip"] and c.chunk_frames == g["chunk_latent_frames"]
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == 0
+
+
+def test_cache_bytes_match_the_pages(golden):
+    """224 vs 3072 scalars per token; 3.02 B scalars / 6.0 GB for the 21-frame,
+    30-layer dense cache."""
+    g = {k: v["value"] for k, v in golden.items()}
+    c = default_config()
+    c.layers = g["layers"]
+    ckv, kr, dense = api.cache_bytes(c)
+    tokens = g["latent_frames_per_clip"] * g["tokens_per_latent_frame"] * g["layers"]
+    assert (ckv + kr) // (2 * tokens) == g["latent_scalars_per_token"]
+    assert dense // (2 * tokens) == g["dense_scalars_per_token"]
+    assert round(dense / 2 / 1e9, 2) == g["dense_cache_scalars_billion"]
+    assert round(dense / 1e9, 1) == g["dense_cache_gb_bf16"]
+    assert round(100 * (1 - (ckv + kr) / dense), 1) == g["reduction_percent"]
+    # the latent cache of one sample: 32760 tokens x 30 layers x 224 x 2 B = 0.44 GB
+    assert round((ckv + kr) / 1e9, 2) == 0.44
+
+
+def test_rope_frequencies_match_the_oracle():
+    for base in [(0, 0, 0), (44, 42, 42)]:
+        c = default_config()
+        c.rope_base_dims[:] = list(base)
+        got = np.array(api.rope_frequencies(c))
+        ref = np.concatenate(O.rope_frequencies((6, 5, 5), 10000.0, base))
+        np.testing.assert_allclose(got, ref.astype(np.float32), rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d_rope", 30, 1), ("rope_theta", 0.0, 1), ("batch", 0, 1), ("chunk_frames", 22, 1),
+    ("grid_w", 1024, 3), ("window_frames", 1024, 3), ("d_latent", 200, 2), ("d_latent", 512, 2),
+    ("d_nope", 64, 2), ("dtype", 7, 1), ("rope_mode", 3, 1),
+])
+def test_config_check_rejects(field, value, status):
+    c = default_config()
+    setattr(c, field, value)
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == status
+
+
+def test_fp32_accepts_small_shapes():
+    c = api.config_from_dims(synth.TINY)
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == 0
+
+
+def test_workspace_bytes_grow_with_reconstruct_once():
+    c = default_config()
+    a = api.workspace_bytes(c, api.DESIGN_ABSORBED)
+    b = api.workspace_bytes(c, api.DESIGN_RECON_ONCE)
+    assert b - a >= 32760 * 3072 * 2
+    assert a % 256 == 0
+
+
+def test_window_matches_a_fifo_deque():
+    """vmla_window against an independent deque model of the ring, over a
+    rollout of 20 chunks of 3 frames (eviction from chunk 7)."""
+    h = api.LatentKVAttention(default_config())
+    W = 21
+    dq = collections.deque(maxlen=W)
+    ring = {}
+    for chunk in range(20):
+        for f in range(3 * chunk, 3 * chunk + 3):
+            dq.append(f)
+        frames, slots, ts = h.window(3 * chunk + 3)
+        assert frames == list(dq)
+        assert ts == list(range(len(dq)))
+        for f, s in zip(frames, slots):
+            ring[s] = f
+        assert all(ring[s] == f for f, s in zip(frames, slots))
+        assert len(set(slots)) == len(slots)
+    h.close()
+
+
+def test_state_roundtrip_and_layer_range():
+    c = default_config()
+    c.layers = 3
+    h = api.LatentKVAttention(c)
+    assert h.state_get(2) == 0
+    h.state_set(2, 33)
+    assert h.state_get(2) == 33 and h.state_get(0) == 0
+    with pytest.raises(api.VmlaError) as e:
+        h.state_get(3)
+    assert e.value.status == 3
+    h.close()
+
+
+class _FakeDev:
+    """A 16-byte aligned fake device address (never dereferenced: every call
+    below is rejected on the host before any launch)."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return self.addr
+
+
+def test_frame_rule_rejections_before_any_launch():
+    c = default_config()
+    h = api.LatentKVAttention(c)
+    lib = api.lib()
+    ws = api.workspace_bytes(c)
+    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, ws - 256) == 1  # workspace too small
+    assert lib.vmla_bind(h._h, 0x10008, 0x20000, 0x30000, ws) == 1        # misaligned
+    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, ws) == 0
+    x = w = 0x40000
+    # skipping ahead or rewinding is refused
+    assert lib.vmla_cache_append(h._h, 0, x, w, 3, 3, None) == 6
+    assert lib.vmla_cache_append(h._h, 0, x, w, -3, 3, None) == 6
+    assert lib.vmla_cache_append(h._h, 0, x, w, 0, 0, None) == 3
+    assert lib.vmla_cache_append(h._h, 0, x, w, 0, 22, None) == 3
+    assert lib.vmla_cache_append(h._h, 1, x, w, 0, 3, None) == 3   # layer out of range
+    assert lib.vmla_cache_append(h._h, 0, 0x40008, w, 0, 3, None) == 1  # misaligned x
+    # attention needs the chunk to be the newest appended frames
+    assert lib.vmla_chunk_attention(h._h, 0, x, w, w, x, 0, 3, 0, None) == 6
+    h.state_set(0, 9)
+    assert lib.vmla_chunk_attention(h._h, 0, x, w, w, x, 3, 3, 0, None) == 6
+    assert lib.vmla_chunk_attention(h._h, 0, x, w, w, x, 6, 4, 0, None) == 3   # more than chunk_frames
+    assert lib.vmla_chunk_attention(h._h, 0, x, w, w, x, 6, 3, 9, None) == 1   # bad design
+    assert lib.vmla_cache_append(h._h, 0, x, w, 3, 3, None) == 6              # neither new nor newest
+    # the dense calls need their own cache bound first
+    assert lib.vmla_dense_cache_append(h._h, 0, x, w, w, w, 0, 3, None) == 6
+    assert h.state_get(0) == 9
+    h.close()
+
+
+def test_rope_at_append_range():
+    c = default_config()
+    c.rope_mode = api.ROPE_AT_APPEND
+    h = api.LatentKVAttention(c)
+    lib = api.lib()
+    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, api.workspace_bytes(c)) == 0
+    h.state_set(0, 1022)
+    # frames 1022..1024 would put an absolute t at 1024, outside the RoPE range
+    assert lib.vmla_cache_append(h._h, 0, 0x40000, 0x40000, 1022, 3, None) == 3
+    h.close()
