@@ -223,6 +223,37 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
 vmla_status vmla_profile_enable(vmla_handle* h, int enable);
 vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* launches);
 
+/* Allocation-free chunk attention.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- for example a
+ * plugin inside another runtime that is handed only its input and output
+ * buffers and owns no allocator, or a latency-critical loop in which a
+ * cudaMalloc (which can synchronise the device) is not allowed.  It needs no
+ * handle and no workspace.
+ *
+ * It computes exactly what vmla_chunk_attention computes with
+ * VMLA_DESIGN_ABSORBED (same kernels, same arguments and layouts; VMLA_BF16
+ * only), for the window of a layer that has `frames_appended` frames in it.
+ * `ckv` and `kr` are the caches of all layers as laid out by vmla_cache_bytes.
+ * Its scratch (the window's rotated positional keys and the absorbed queries:
+ * batch*W*T_f*32*2 bytes, rounded up to 256, plus batch*n_heads*n_frames*T_f*
+ * (d_latent + 32)*2 bytes) lives in a fixed 32 MiB array inside the library
+ * that every GPU which loads the library holds until the process exits;
+ * larger calls return VMLA_ERR_OUT_OF_RANGE and enqueue nothing.  The call
+ * makes no cudaMalloc or cudaFree and calls no allocating routine.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current) and keeps it; make that first call before any
+ *   stream capture begins.
+ * - Every call shares the one array, which keeps the last call's contents.
+ *   Nothing in it has to start at zero: each call writes every scratch byte it
+ *   reads.  Calls that overlap on the GPU (two streams, or two threads) race
+ *   on the array: order them on one stream.
+ * Returns as vmla_chunk_attention; device-side errors go to the same device
+ * status word (read with vmla_device_status). */
+vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int layer, const void* ckv, const void* kr,
+                                         int64_t frames_appended, const void* q, const void* w_uk,
+                                         const void* w_uv, void* out, int64_t first_frame, int n_frames,
+                                         void* stream);
+
 /* Self-test of the bounded pipeline waits: launches one CTA that waits on an
  * mbarrier nothing arrives at, for at most `limit_ns` nanoseconds (<= 1e9), then
  * returns.  The device status word must afterwards report VMLA_ERR_DEVICE_TIMEOUT. */

@@ -66,6 +66,8 @@ _SIGS = {
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
     "vmla_profile_read": (c_int, [c_void_p, c_int, ctypes.POINTER(c_double), ctypes.POINTER(c_int)]),
     "vmla_selftest_wait_timeout": (c_int, [c_uint64, c_void_p]),
+    "vmla_chunk_attention_noalloc": (c_int, [ctypes.POINTER(Config), c_int, c_void_p, c_void_p, c_int64, c_void_p,
+                                             c_void_p, c_void_p, c_void_p, c_int64, c_int, c_void_p]),
 }
 
 _LIB = None
