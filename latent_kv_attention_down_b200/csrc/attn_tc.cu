@@ -8,63 +8,45 @@
 // sum (value-path absorption), fused into the epilogue as a second tcgen05
 // GEMM whose A operand is O_bar split into a bf16 pair (rounded + residual),
 // so the only roundings left on the output path are the cache's, P's and
-// q~'s.  The output is written in fp32.  The dense variant runs the same pipeline with per-head 128-wide K
-// and V tiles (the 3072-scalar comparison layout).
+// q~'s.  The output is written in fp32.  The dense variant runs the same
+// pipeline with per-head 128-wide K and V tiles (the 3072-scalar layout).
 //
 // One CTA owns 128 query rows of one head of one sample and streams the whole
-// window in tiles of BN = 128 keys:
-//   warp 0     TMA producer: Q once, then K/V tiles into a STAGES-deep ring
-//   warp 1     tcgen05.mma issuer (one thread) + TMEM owner
-//   warps 4-7  softmax: thread r owns query row r = TMEM lane r
+// window in tiles of BN keys:
+//   warp 0      TMA producer: the query tile once, then K/V tiles into a ring
+//   warp 1      tcgen05.mma issuer (one thread) + TMEM owner
+//   warps 4-11  two softmax warpgroups; thread r of either group owns query
+//               row r = TMEM lane r, each group half of every tile's keys
 // TMEM (512 columns): S0 [0,BN), S1 [BN,2BN), O [2BN, 2BN+DV).
 //   S_j = Q K_j^T (fp32) lands in S[j&1]; the softmax threads turn it into
 //   P_j = exp2(S_j * scale*log2e - m) as bf16 pairs written back over S[j&1];
 //   O += P_j V_j reads P straight from TMEM (A operand) and V from the same
 //   shared-memory tile as K (MN-major descriptor), so V is never loaded twice.
-// While the softmax works on S_j, the tensor core already computes S_{j+1}.
+//   While the softmax works on S_j, the tensor core computes S_{j+1}; S_{j+2}
+//   reuses S[j&1] once P V_j has read P_j (in-order tensor pipe).  Letting QK
+//   run further ahead would need a third resident K/V tile, and the 227 KB of
+//   shared memory then leave no room to prefetch the next one.
 // The running max is only raised when it grows by more than 2^threshold (lazy
-// rescale, 2^8 by default); O is then rescaled in TMEM after the previous P V has finished.
-// Every mbarrier wait is bounded; a CTA that gives up records the error and
-// drains its in-flight copies and MMAs before releasing TMEM.
+// rescale, 2^8 by default); O is then rescaled in TMEM after the previous P V
+// has finished.  Every mbarrier wait is bounded; a CTA that gives up records
+// the error and drains its in-flight copies and MMAs before releasing TMEM.
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace vmla {
 namespace {
 
-constexpr int kThreads = 256;
-
-template <int DL_, bool DENSE_>
-struct AttnCfg {
-  static constexpr bool DENSE = DENSE_;
-  static constexpr int DL = DL_;
-  static constexpr int BN = 128;
-  static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of Q
-  static constexpr int Q_BYTES = QB * 16384 + (DENSE ? 0 : 128 * 64);
-  static constexpr int KBLK = BN * 128;  // one [BN keys x 64] SW128 block
-  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * 64;
-  static constexpr int DV = DENSE ? 128 : DL;
-  static constexpr int SMEM_CAP = 232448;
-  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - 512 - Q_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  static constexpr int S_COL = 0;  // S buffer b at S_COL + b*BN
-  static constexpr int O_COL = 2 * BN;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int SMEM = 1024 + Q_BYTES + STAGES * STAGE_BYTES + 512;
-  static_assert(STAGES >= 2, "pipeline needs two stages");
-  static_assert(O_COL + DV <= 512, "TMEM budget");
-  static_assert(SMEM <= SMEM_CAP, "shared memory budget");
-  static_assert(STAGES * STAGE_BYTES >= 2 * DV * 256 && STAGES * STAGE_BYTES >= 65536, "epilogue staging");
-  static_assert(DV % 64 == 0 && DV <= 256, "value width");
-};
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA + TMEM, warps 4-11 two softmax warpgroups
+constexpr int kMaxStages = 6;
+constexpr int kSoftmaxWarps = 8;
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[4];
-  uint64_t kv_empty[4];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
+  uint64_t s_full[2];  // S_j computed (MMA commit)
+  uint64_t p_full[2];  // P_j stored over S_j by every softmax warp
+  uint64_t p_done[2];  // P V_j has completed (MMA commit), by tile parity
   uint64_t o_final;
   uint64_t wuv_full;
   uint64_t ob_full;
@@ -72,6 +54,37 @@ struct Bars {
   uint64_t drain;
   uint32_t tslot;
   int abort_flag;
+  float red[2][2][128];  // per-tile half-row maxima of the two softmax groups (tile parity, group, row)
+};
+
+template <int DL_, bool DENSE_>
+struct AttnCfg {
+  static constexpr bool DENSE = DENSE_;
+  static constexpr int DL = DL_;
+  static constexpr int DQK = DENSE ? 128 : DL + 32;  // contraction width of S = Q K^T
+  static constexpr int DV = DENSE ? 128 : DL;
+  static constexpr int BN = 128;
+  static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of a query or key row
+  static constexpr int Q_BYTES = QB * 16384 + (DENSE ? 0 : 128 * 64);
+  static constexpr int KBLK = BN * 128;           // one [BN keys x 64] SW128 block
+  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * 64;
+  static constexpr int SMEM_CAP = 232448;
+  static constexpr int BARS = (sizeof(Bars) + 127) / 128 * 128;
+  static constexpr int STAGES_FIT = (SMEM_CAP - BARS - Q_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
+  static constexpr int S_COL = 0;  // S buffer b (and P_j over it) at S_COL + b*BN
+  static constexpr int O_COL = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int SMEM = Q_BYTES + STAGES * STAGE_BYTES + BARS;
+  // epilogue images: O_bar rounded over the query tile, W_uv,h then O_bar residual in the drained ring
+  static constexpr int EPI_WUV = 0;
+  static constexpr int EPI_OB_LO = DV * 256;
+  static_assert(STAGES >= 2, "the K/V ring needs two stages");
+  static_assert(O_COL + DV <= 512, "TMEM budget");
+  static_assert(SMEM <= SMEM_CAP, "shared memory budget");
+  static_assert(STAGES * STAGE_BYTES >= (DENSE ? 0 : EPI_OB_LO + DV * 256) && STAGES * STAGE_BYTES >= 65536,
+                "epilogue staging");
+  static_assert(DV % 64 == 0 && DV <= 256 && BN % 32 == 0, "tile shapes");
 };
 
 // bf16 row of 32 floats into a 128B-swizzled K-major tile: row r, columns c0..c0+31
@@ -106,35 +119,70 @@ __device__ __forceinline__ void st_swizzled_row32_f32(uint8_t* tile, int r, int 
         make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale, v[4 * j + 3] * scale);
 }
 
+// S = Q K^T for one tile.  Query tile and key tile in shared memory: QB [rows x 64] SW128
+// blocks of latent (or per-head key) columns, then (absorbed) one [rows x 32] SW64 block of
+// rotated positional columns.  Descriptors are built once and advanced by compile-time offsets.
 template <class C>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t stage) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, C::BN, false, false);
-  if constexpr (C::DENSE) {
+  constexpr int KL = C::QB * 4;  // k-steps over the SW128 blocks
+  const uint64_t kd = smem_desc(stage, 16, 1024, LAYOUT_SW128);
+  const uint64_t qd = smem_desc(sq, 16, 1024, LAYOUT_SW128);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_ss(d_tmem, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
-             smem_desc(stage + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
-  } else {
+  for (int kk = 0; kk < KL; ++kk) {
+    const uint64_t a = desc_add(qd, (kk >> 2) * 16384 + (kk & 3) * 32);
+    const uint64_t b = desc_add(kd, (kk >> 2) * C::KBLK + (kk & 3) * 32);
+    if (kk == 0)
+      mma_ss_c<false>(d_tmem, a, b, idesc);
+    else
+      mma_ss_c<true>(d_tmem, a, b, idesc);
+  }
+  if constexpr (!C::DENSE) {
+    const uint64_t krd = smem_desc(stage + C::QB * C::KBLK, 16, 512, LAYOUT_SW64);
+    const uint64_t qrd = smem_desc(sq + C::QB * 16384, 16, 512, LAYOUT_SW64);
 #pragma unroll
-    for (int kk = 0; kk < C::DL / 16; ++kk)
-      mma_ss(d_tmem, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
-             smem_desc(stage + (kk >> 2) * C::KBLK + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
-    const uint32_t qr = sq + C::QB * 16384, kr = stage + C::QB * C::KBLK;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk)
-      mma_ss(d_tmem, smem_desc(qr + kk * 32, 16, 512, LAYOUT_SW64), smem_desc(kr + kk * 32, 16, 512, LAYOUT_SW64),
-             idesc, 1);
+    for (int kk = 0; kk < 2; ++kk) mma_ss_c<true>(d_tmem, desc_add(qrd, kk * 32), desc_add(krd, kk * 32), idesc);
   }
 }
 
 template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t stage, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, C::DV, false, true);
-  const uint32_t v = C::DENSE ? stage + 2 * C::KBLK : stage;
+  const uint64_t vd = smem_desc(C::DENSE ? stage + 2 * C::KBLK : stage, C::KBLK, 1024, LAYOUT_SW128);
+  if (accumulate)
+    mma_ts_c<true>(o_tmem, p_tmem, vd, idesc);
+  else
+    mma_ts_c<false>(o_tmem, p_tmem, vd, idesc);
 #pragma unroll
-  for (int kk = 0; kk < C::BN / 16; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc(v + kk * 2048, C::KBLK, 1024, LAYOUT_SW128), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 1; kk < C::BN / 16; ++kk) mma_ts_c<true>(o_tmem, p_tmem + kk * 8, desc_add(vd, kk * 2048), idesc);
+}
+
+template <int HS>
+__device__ __forceinline__ void ld_half_tile(uint32_t taddr, uint32_t (&r)[HS]) {
+  if constexpr (HS == 64) {
+    tmem_ld64(taddr, r);
+  } else if constexpr (HS == 48) {
+    tmem_ld48(taddr, r);
+  } else {
+    tmem_ld32(taddr, r);
+  }
+}
+
+template <int NP>
+__device__ __forceinline__ void st_packed(uint32_t taddr, const uint32_t (&r)[NP]) {
+  if constexpr (NP == 32) {
+    tmem_st32(taddr, r);
+  } else if constexpr (NP == 24) {
+    tmem_st24(taddr, r);
+  } else {
+    tmem_st16(taddr, r);
+  }
+}
+
+// One warp's share of an arrival: every lane has fenced its own tcgen05 traffic.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 template <int DL, bool DENSE>
@@ -144,10 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_wuv, const __grid_constant__ CUtensorMap tm_out,
                    const AttnTc a) {
   using C = AttnCfg<DL, DENSE>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::Q_BYTES;
+  // The dynamic shared memory window starts 1024-byte aligned (the swizzled TMA tiles need it);
+  // the whole 227 KB budget may be in use, so there is no slack to realign: check instead.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(a.err, DEV_ERR_BOUNDS);
+    return;
+  }
+  uint8_t* sQ = smem_raw;
+  uint8_t* sKV = smem_raw + C::Q_BYTES;
   Bars* bars = reinterpret_cast<Bars*>(sKV + C::STAGES * C::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -163,12 +216,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars->s_full[k], 1);
-      mbar_init(&bars->p_full[k], 128);
+      mbar_init(&bars->p_full[k], kSoftmaxWarps);
+      mbar_init(&bars->p_done[k], 1);
     }
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_final, 1);
     mbar_init(&bars->wuv_full, 1);
-    mbar_init(&bars->ob_full, 128);
+    mbar_init(&bars->ob_full, kSoftmaxWarps);
     mbar_init(&bars->epi_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -183,17 +236,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
       const int qrow = b * a.n_heads + h;
-      if constexpr (C::DENSE) {
-        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-        for (int qb = 0; qb < 2; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
-      } else {
-        mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-        for (int qb = 0; qb < C::QB; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
-        tma_load_3d(sQ + C::QB * 16384, &tm_qr, &bars->q_full, DL, m0, qrow);
-      }
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+      for (int qb = 0; qb < C::QB; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
+      if constexpr (!C::DENSE) tma_load_3d(sQ + C::QB * 16384, &tm_qr, &bars->q_full, DL, m0, qrow);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % C::STAGES;
@@ -219,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (issued == n_tiles && wait_phase(&bars->o_final, 0, g, DEV_ERR_TIMEOUT_PRODUCER)) {
           mbar_arrive_expect_tx(&bars->wuv_full, C::DV * 256);
           for (int kb = 0; kb < C::DV / 64; ++kb)
-            tma_load_3d(sKV + kb * 16384, &tm_wuv, &bars->wuv_full, kb * 64, 0, h);
+            tma_load_3d(sKV + C::EPI_WUV + kb * 16384, &tm_wuv, &bars->wuv_full, kb * 64, 0, h);
           wuv_issued = true;
         }
       }
@@ -232,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // order: QK_0, then per tile j: QK_{j+1}, P V_j
     if (lane == 0) {
       const uint32_t sq = smem_u32(sQ), skv = smem_u32(sKV);
       bool ok = wait_phase(&bars->q_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
@@ -242,34 +291,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars->s_full[0]);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
+        const int buf = j & 1;
         if (j + 1 < n_tiles) {
           const int s1 = (j + 1) % C::STAGES;
           if (!(ok = wait_phase(&bars->kv_full[s1], ((j + 1) / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
           tc_fence_after();
-          issue_qk<C>(tbase + C::S_COL + ((j + 1) & 1) * C::BN, sq, skv + s1 * C::STAGE_BYTES);
-          mma_commit(&bars->s_full[(j + 1) & 1]);
+          issue_qk<C>(tbase + C::S_COL + (buf ^ 1) * C::BN, sq, skv + s1 * C::STAGE_BYTES);
+          mma_commit(&bars->s_full[buf ^ 1]);
         }
-        if (!(ok = wait_phase(&bars->p_full[j & 1], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+        if (!(ok = wait_phase(&bars->p_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
         tc_fence_after();
         const int s = j % C::STAGES;
-        issue_pv<C>(tbase + C::O_COL, tbase + C::S_COL + (j & 1) * C::BN, skv + s * C::STAGE_BYTES, j > 0);
+        issue_pv<C>(tbase + C::O_COL, tbase + C::S_COL + buf * C::BN, skv + s * C::STAGE_BYTES, j > 0);
         mma_commit(&bars->kv_empty[s]);
-        mma_commit(&bars->o_done);
+        mma_commit(&bars->p_done[buf]);
       }
       if (ok) mma_commit(&bars->o_final);
       if constexpr (!C::DENSE) {
-        // fused value up-projection: out_h = O_bar W_uv,h^T with O_bar (bf16, normalised) staged over Q
+        // fused value up-projection: out_h = O_bar W_uv,h^T, O_bar as a bf16 pair (rounded + residual)
         if (ok && wait_phase(&bars->ob_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
             wait_phase(&bars->wuv_full, 0, g, DEV_ERR_TIMEOUT_MMA)) {
           tc_fence_after();
           constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
-          const uint32_t ob_lo = skv + C::DV * 256;  // residual half of O_bar, after W_uv,h
+          const uint64_t hd = smem_desc(sq, 16, 1024, LAYOUT_SW128);
+          const uint64_t ld = smem_desc(skv + C::EPI_OB_LO, 16, 1024, LAYOUT_SW128);
+          const uint64_t wd = smem_desc(skv + C::EPI_WUV, 16, 1024, LAYOUT_SW128);
 #pragma unroll
           for (int kk = 0; kk < C::DV / 16; ++kk) {
-            const uint64_t w = smem_desc(skv + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
-            mma_ss(tbase, smem_desc(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), w, idesc,
-                   kk > 0);
-            mma_ss(tbase, smem_desc(ob_lo + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, LAYOUT_SW128), w, idesc, 1);
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            if (kk == 0)
+              mma_ss_c<false>(tbase, desc_add(hd, off), desc_add(wd, off), idesc);
+            else
+              mma_ss_c<true>(tbase, desc_add(hd, off), desc_add(wd, off), idesc);
+            mma_ss_c<true>(tbase, desc_add(ld, off), desc_add(wd, off), idesc);
           }
           mma_commit(&bars->epi_done);
         }
@@ -281,91 +335,125 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / correction / epilogue
-    const int wq = warp - 4;
+    // Two warpgroups share the 128 rows: group wg takes score columns [wg*BN/2, (wg+1)*BN/2)
+    // of every tile and O columns [wg*DV/2, (wg+1)*DV/2); warp w of either group reads TMEM
+    // lanes 32*(w%4).. (the same rows).  The row max of a tile is the larger of the two
+    // halves' maxima, swapped through shared memory once per tile.  Every thread of both
+    // groups passes the same named barriers in the same order, whatever happens: a thread
+    // that gave up skips the work, never the barrier.
+    const int wg = (warp - 4) >> 2;
+    const int wq = (warp - 4) & 3;
     const int r = wq * 32 + lane;  // query row inside the tile == TMEM lane
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(wq * 32) << 16);
+    constexpr int HS = C::BN / 2;  // score columns per group
+    constexpr int HO = C::DV / 2;  // O columns per group
+    const int sc0 = wg * HS;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int buf = j & 1;
-      ok = __all_sync(0xffffffffu, wait_phase(&bars->s_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sraw[C::BN];
-#pragma unroll
-      for (int c = 0; c < C::BN; c += 64)
-        tmem_ld64(lane_base + C::S_COL + buf * C::BN + c, *reinterpret_cast<uint32_t(*)[64]>(&sraw[c]));
-      const int valid = a.n_keys - j * C::BN;
+      ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->s_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+      uint32_t sraw[HS];
       float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < C::BN; ++c) {
-        float v = __uint_as_float(sraw[c]);
-        if (c >= valid) v = -INFINITY;
-        sraw[c] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
-      }
-      const float m_tile = mx * a.scale_log2;
-      if (j == 0) {
-        m_run = m_tile;
-      } else if (__any_sync(0xffffffffu, m_tile > m_run + a.rescale_threshold)) {
-        // raise the running max of every row of this warp; rescale O once the previous P V is done
-        const float m_new = fmaxf(m_run, m_tile);
-        const float alpha = ex2_approx(m_run - m_new);
-        ok = __all_sync(0xffffffffu, wait_phase(&bars->o_done, (j - 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
-        if (!ok) break;
+      if (ok) {
         tc_fence_after();
+        ld_half_tile<HS>(lane_base + C::S_COL + buf * C::BN + sc0, sraw);
+        const int valid = a.n_keys - j * C::BN - sc0;
+        if (valid < HS) {  // only the last tile is ragged (warp-uniform branch)
+#pragma unroll
+          for (int c = 0; c < HS; ++c)
+            if (c >= valid) sraw[c] = __float_as_uint(-INFINITY);
+        }
+        // half-row max: independent chains of 3-input max over 16 scores each
+        float mxc[HS / 16];
+#pragma unroll
+        for (int k = 0; k < HS / 16; ++k) {
+          const uint32_t* v = &sraw[16 * k];
+          float m = max3f(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+          for (int i = 3; i < 15; i += 2) m = max3f(m, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+          mxc[k] = fmaxf(m, __uint_as_float(v[15]));
+        }
+        mx = mxc[0];
+#pragma unroll
+        for (int k = 1; k < HS / 16; ++k) mx = fmaxf(mx, mxc[k]);
+      }
+      bars->red[buf][wg][r] = mx;
+      named_bar_sync(2, 256);
+      const float m_tile = fmaxf(mx, bars->red[buf][wg ^ 1][r]) * a.scale_log2;
+      if (ok) {
+        if (j == 0) {
+          m_run = m_tile;
+        } else if (__any_sync(0xffffffffu, m_tile > m_run + a.rescale_threshold)) {
+          // raise the running max of every row of this warp; rescale this group's half of O
+          // once the previous P V is done (both groups take the same decision for a row)
+          const float m_new = fmaxf(m_run, m_tile);
+          const float alpha = ex2_approx(m_run - m_new);
+          ok = __all_sync(0xffffffffu,
+                          wait_phase(&bars->p_done[(j - 1) & 1], ((j - 1) >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+          if (ok) {
+            tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < C::DV; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + C::O_COL + c, o);
+            for (int c = wg * HO; c < (wg + 1) * HO; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(lane_base + C::O_COL + c, o);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(lane_base + C::O_COL + c, o);
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(lane_base + C::O_COL + c, o);
+            }
+            l_run *= alpha;
+            m_run = m_new;
+          }
         }
-        l_run *= alpha;
-        m_run = m_new;
       }
-      const float neg_m = -m_run;
-      float sum = 0.f;
+      if (ok) {
+        // p = 2^(s*scale - m): scale-and-subtract two scores per instruction, exp2 on the MUFU,
+        // row sum in four independent packed accumulators, bf16 pairs back into TMEM over S
+        const float2 nm2 = make_float2(-m_run, -m_run);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t packed[HS / 2];
 #pragma unroll
-      for (int half = 0; half < C::BN / 64; ++half) {
-        uint32_t packed[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sraw[half * 64 + 2 * k]), a.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sraw[half * 64 + 2 * k + 1]), a.scale_log2, neg_m));
-          sum += p0 + p1;
-          packed[k] = pack_bf16x2(p0, p1);
+        for (int k = 0; k < HS / 2; ++k) {
+          const float2 x = make_float2(__uint_as_float(sraw[2 * k]), __uint_as_float(sraw[2 * k + 1]));
+          const float2 y = __ffma2_rn(x, sc2, nm2);
+          const float2 pr = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+          acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
+          packed[k] = pack_bf16x2(pr.x, pr.y);
         }
-        tmem_st32(lane_base + C::S_COL + buf * C::BN + half * 32, packed);
+        st_packed<HS / 2>(lane_base + C::S_COL + buf * C::BN + wg * (HS / 2), packed);
+        const float2 acc4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l_run += acc4.x + acc4.y;
+        tc_fence_before();
       }
-      l_run += sum;
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[buf]);
+      warp_arrive(&bars->p_full[buf]);
     }
     ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->o_final, 0, g, DEV_ERR_TIMEOUT_EPILOGUE));
     if (ok) tc_fence_after();
-    const float inv_l = 1.f / l_run;
+    // row sum = both halves' partial sums (the other parity's exchange slot is free by now)
+    bars->red[n_tiles & 1][wg][r] = l_run;
+    named_bar_sync(2, 256);
+    const float inv_l = 1.f / (l_run + bars->red[n_tiles & 1][wg ^ 1][r]);
     if constexpr (!C::DENSE) {
-      // O_bar = O / l as a bf16 pair: the rounded part over the Q region, the residual
-      // after W_uv,h in the K/V ring (A operands of the two W_uv GEMMs)
+      // O_bar = O / l as a bf16 pair (A operands of the two W_uv GEMMs): rounded part over the
+      // query tile, residual after W_uv,h in the drained K/V ring
       if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < C::DV; c += 32) {
+        for (int c = wg * HO; c < (wg + 1) * HO; c += 32) {
           uint32_t o[32];
           tmem_ld32(lane_base + C::O_COL + c, o);
           st_swizzled_row32(sQ, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, false);
-          st_swizzled_row32(sKV + C::DV * 256, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, true);
+          st_swizzled_row32(sKV + C::EPI_OB_LO, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, true);
         }
       }
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->ob_full);
+      warp_arrive(&bars->ob_full);
       ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->epi_done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE));
       if (ok) {
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
           uint32_t o[32];
           tmem_ld32(lane_base + c, o);
           st_swizzled_row32_f32(sKV, r, c, *reinterpret_cast<float(*)[32]>(o), 1.f);
@@ -374,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
           uint32_t o[32];
           tmem_ld32(lane_base + C::O_COL + c, o);
           st_swizzled_row32_f32(sKV, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l);
@@ -382,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     fence_async_smem();
-    named_bar_sync(1, 128);
-    if (r == 0 && !bars->abort_flag) {
+    named_bar_sync(1, 256);
+    if (wg == 0 && r == 0 && !bars->abort_flag) {
       for (int blk = 0; blk < 4; ++blk) tma_store_3d(&tm_out, sKV + blk * 16384, h * 128 + blk * 32, m0, b);
       bulk_commit();
       bulk_wait_all_read();
@@ -411,7 +499,17 @@ cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtenso
 
 }  // namespace
 
-int attn_absorbed_block_n(int) { return 128; }
+int attn_absorbed_block_n(int d_latent) {
+  switch (d_latent) {
+    case 64: return AttnCfg<64, false>::BN;
+    case 128: return AttnCfg<128, false>::BN;
+    case 192: return AttnCfg<192, false>::BN;
+    case 256: return AttnCfg<256, false>::BN;
+  }
+  return 128;
+}
+
+int attn_dense_block_n() { return AttnCfg<128, true>::BN; }
 
 cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
                                     const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tuv,

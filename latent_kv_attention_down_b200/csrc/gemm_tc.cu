@@ -143,19 +143,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, C::NB, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::NB, false, false);
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % C::STAGES;
         if (!wait_phase(&full[s], (kb / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-        const uint32_t sb = sa + C::A_BYTES;
+        const uint64_t ad = smem_desc(sa, 16, 1024, LAYOUT_SW128);
+        const uint64_t bd = smem_desc(sa + C::A_BYTES, 16, 1024, LAYOUT_SW128);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-          for (int sp = 0; sp < C::NSPLIT; ++sp)
-            mma_ss(tbase + sp * C::NB, smem_desc(sa + k * 32, 16, 1024, LAYOUT_SW128),
-                   smem_desc(sb + sp * C::NB * 128 + k * 32, 16, 1024, LAYOUT_SW128), idesc, (kb | k) != 0);
+          for (int sp = 0; sp < C::NSPLIT; ++sp) {
+            const uint64_t a = desc_add(ad, k * 32), b = desc_add(bd, sp * C::NB * 128 + k * 32);
+            if (k == 0 && kb == 0)
+              mma_ss_c<false>(tbase + sp * C::NB, a, b, idesc);
+            else
+              mma_ss_c<true>(tbase + sp * C::NB, a, b, idesc);
+          }
         mma_commit(&empty[s]);
       }
       mma_commit(done);
@@ -241,12 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
       tc_fence_after();
       if (ok) {
-        const uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        constexpr uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
+        const uint64_t ad = smem_desc(smem_u32(sA), 16, 1024, LAYOUT_SW128);
+        const uint64_t bd = smem_desc(smem_u32(sB), C::WB, 1024, LAYOUT_SW128);
 #pragma unroll
-        for (int kk = 0; kk < 6; ++kk)  // d_nope = 96 = 6 x 16
-          mma_ss(tbase, smem_desc(a0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
-                 smem_desc(b0 + kk * 2048, C::WB, 1024, LAYOUT_SW128), idesc, kk > 0);
+        for (int kk = 0; kk < 6; ++kk) {  // d_nope = 96 = 6 x 16
+          const uint64_t a = desc_add(ad, (kk / 4) * 16384 + (kk % 4) * 32), b = desc_add(bd, kk * 2048);
+          if (kk == 0)
+            mma_ss_c<false>(tbase, a, b, idesc);
+          else
+            mma_ss_c<true>(tbase, a, b, idesc);
+        }
       }
       mma_commit(done);
       if (*abort_flag) drain_phase(done, 0, g);
@@ -323,12 +333,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
       tc_fence_after();
       if (ok) {
-        const uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        constexpr uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
+        const uint64_t ad = smem_desc(smem_u32(sA), 16, 1024, LAYOUT_SW128);
+        const uint64_t bd = smem_desc(smem_u32(sB), 16, 1024, LAYOUT_SW128);
 #pragma unroll
-        for (int kk = 0; kk < DL / 16; ++kk)
-          mma_ss(tbase, smem_desc(a0 + (kk / 4) * C::A_BLK + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
-                 smem_desc(b0 + (kk / 4) * C::B_BLK + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
+        for (int kk = 0; kk < DL / 16; ++kk) {
+          const uint64_t a = desc_add(ad, (kk / 4) * C::A_BLK + (kk % 4) * 32);
+          const uint64_t b = desc_add(bd, (kk / 4) * C::B_BLK + (kk % 4) * 32);
+          if (kk == 0)
+            mma_ss_c<false>(tbase, a, b, idesc);
+          else
+            mma_ss_c<true>(tbase, a, b, idesc);
+        }
       }
       mma_commit(done);
       if (*abort_flag) {

@@ -142,7 +142,8 @@ struct AttnTc {
 cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
                                     const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr, const CUtensorMap& tm_wuv,
                                     const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
-int attn_absorbed_block_n(int d_latent);
+int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the key maps)
+int attn_dense_block_n();
 
 // Dense per-head attention, d_head = 128.  q map: 3D (128, n_q, B*n_h) box (64,128,1);
 // kv map: 3D (2*n_h*128, n_keys, B) box (64,128,1); out as above.

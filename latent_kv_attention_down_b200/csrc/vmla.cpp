@@ -651,8 +651,8 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
   CUtensorMap tq, tkv, to;
   if (!map3(&tq, qd, 128, nq, (uint64_t)c.batch * c.n_heads, 256, (uint64_t)nq * 256, 64, 128,
             CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map3(&tkv, kv_base, 2ull * c.n_heads * 128, n_keys, c.batch, row_bytes, rr * row_bytes, 64, 128,
-            CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&tkv, kv_base, 2ull * c.n_heads * 128, n_keys, c.batch, row_bytes, rr * row_bytes, 64,
+            attn_dense_block_n(), CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
             (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
     return VMLA_ERR_CUDA;
