@@ -366,6 +366,9 @@ def run_ours(args, rank, world, local_rank):
                     "api": "vmla_chunk_step_host (pinned host x, q -> device, append, attention, out -> host)"},
             "gpu_launches": 4 * args.steps, "clocks": clk}
     line["designs"] = {"absorbed_ms_per_step": ms_step, "recon_once": recon_once}
+    if args.legs:
+        line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
+                        "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed)}
     if dense:
         line["dense"] = dense
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -373,6 +376,136 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         print(json.dumps(line), flush=True)
     m.close()
+
+
+def _pool_fill(m, d, pool, xp, W, layer, chunks):
+    for c in range(chunks):
+        m.append(layer, pool.activations(layer, c, 0, pool=xp), W[0], c * d.chunk_frames, d.chunk_frames)
+
+
+def batch8_leg(m_timed, dev, hbm, tc, seed):
+    """The same layer at batch 8: 8 independent rings, 37440 queries per call;
+    two layer sets (x, q: 460 MB) alternate so inputs stay above L2."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    d = WORKLOAD.replace(batch=8)
+    L = 2
+    m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+    pool = synth.FramePool(d, base_seed=seed)
+    bf = torch.bfloat16
+    xp = torch.from_numpy(pool.x).to(dev, bf)
+    qp = torch.from_numpy(pool.q).to(dev, bf)
+    W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv))
+         for w in (synth.weights(d, l, seed) for l in range(L))]
+    chunks = d.window_frames // d.chunk_frames
+    first = (chunks - 1) * d.chunk_frames
+    for l in range(L):
+        _pool_fill(m, d, pool, xp, W[l], l, chunks)
+    xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
+    qs = [pool.queries(l, chunks - 1, 1, pool=qp) for l in range(L)]
+    out = torch.empty((d.batch, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
+    del xp, qp
+
+    def step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, api.DESIGN_ABSORBED)
+
+    steps = 20
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    m.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(3 + i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    k = {n: m.profile_read(n) for n in ("append", "rope", "q_absorb", "attention")}
+    m.profile(False)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    F = step_flops(WORKLOAD)
+    B = d.batch
+    nq, nk = d.n_queries, d.window_tokens
+    alg = {"append": B * nq * d.d_model * 2 + (d.d_latent + d.d_rope) * d.d_model * 2 + B * nq * (d.d_latent + d.d_rope) * 2,
+           "rope": B * 2 * nk * d.d_rope * 2,
+           "q_absorb": B * nq * d.n_heads * d.d_head * 2 + d.n_heads * d.d_nope * d.d_latent * 2 +
+           B * nq * d.n_heads * (d.d_latent + d.d_rope) * 2}
+    res = {"workload": "wan1.3b-layer chunk step at batch 8 (8 rings, N_q=37440 per call, N_k=32760 per sample)",
+           "ms_per_step": ms, "tflops": B * F["total"] / (ms * 1e-3) / 1e12,
+           "query_tokens_per_s": B * nq / (ms * 1e-3), "kernels": {}}
+    for n, (t, c) in k.items():
+        per = t / max(c, 1)
+        e = {"ms_per_launch": per}
+        if n in alg:
+            e["algorithmic_bytes"] = alg[n]
+            e["gbs"] = alg[n] / (per * 1e-3) / 1e9
+            e["frac_of_hbm"] = e["gbs"] / hbm
+        else:
+            e["tflops"] = B * F["attention"] / (per * 1e-3) / 1e12
+            e["frac_of_bf16_peak"] = e["tflops"] / tc
+        res["kernels"][n] = e
+    m.close()
+    return res
+
+
+def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256)):
+    """Latent width sweep on the Wan layer: attention time of every built design
+    and of the dense per-head cache for the same seeded x and q."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    res = {}
+    steps = 10
+    bf = torch.bfloat16
+    for dc in widths:
+        d = WORKLOAD.replace(d_latent=dc)
+        L = 2
+        m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev, design=api.DESIGN_RECON_ONCE,
+                                                                              dense=True)
+        pool = synth.FramePool(d, base_seed=seed)
+        xp = torch.from_numpy(pool.x).to(dev, bf)
+        qp = torch.from_numpy(pool.q).to(dev, bf)
+        W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv))
+             for w in (synth.weights(d, l, seed) for l in range(L))]
+        chunks = d.window_frames // d.chunk_frames
+        first = (chunks - 1) * d.chunk_frames
+        for l in range(L):
+            for c in range(chunks):
+                x = pool.activations(l, c, 0, pool=xp)
+                m.append(l, x, W[l][0], c * d.chunk_frames, d.chunk_frames)
+                m.dense_append(l, x, W[l][0], W[l][1], W[l][2], c * d.chunk_frames, d.chunk_frames)
+        qs = [pool.queries(l, chunks - 1, 0, pool=qp) for l in range(L)]
+        out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
+        F = step_flops(d)
+        entry = {"absorbed_flops": F["attention"], "dense_flops": dense_flops(d)["attention"]}
+        for name, design in (("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE), ("dense", None)):
+            def call(i):
+                l = i % L
+                if design is None:
+                    m.dense_attention(l, qs[l], out, first, d.chunk_frames)
+                else:
+                    m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, design)
+            for i in range(3):
+                call(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(steps):
+                call(i)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            entry[name] = {"ms_per_call": ms, "tflops_effective": F["attention"] / (ms * 1e-3) / 1e12}
+        st, flags = m.device_status()
+        assert st == 0, f"device status {st} flags {flags:#x}"
+        res[str(dc)] = entry
+        m.close()
+        del xp, qp, W, qs, out, m
+        torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -383,6 +516,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", dest="dense", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-legs", dest="legs", action="store_false",
+                    help="skip the batch-8 and latent-width legs")
     ap.add_argument("--cpu-queries", type=int, default=2048)
     ap.add_argument("--steps-ref", type=int, default=None)
     ap.add_argument("--warmup-ref", type=int, default=None)

@@ -15,27 +15,17 @@
 //    per-head dense entries k_h = [W_uk,h c | RoPE(k_R)], v_h = W_uv,h c.
 #include "kernels.h"
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace vmla {
 namespace {
 
 constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 4..7 epilogue
 
-__device__ __forceinline__ float pair_angle(const Rope& rp, int p, float t, float h, float w) {
-  const float pos = p < rp.n_t ? t : (p < rp.n_t + rp.n_h ? h : w);
-  return pos * rp.freq[p];
-}
-
-// Rotate 16 adjacent pairs held in v[0..31].
-__device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, float t, float h, float w) {
+// Rotate 16 adjacent pairs held in v[0..31] at grid position (t, h, w).
+__device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, int t, int h, int w) {
 #pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    float s, c;
-    sincosf(pair_angle(rp, p, t, h, w), &s, &c);
-    const float u = v[2 * p], x = v[2 * p + 1];
-    v[2 * p] = u * c - x * s;
-    v[2 * p + 1] = u * s + x * c;
-  }
+  for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], rope_cs(rp, p, t, h, w));
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
@@ -197,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c0 < a.d_latent) {
         store_bf16x32(lat + c0, v);
       } else {
-        if (a.rotate) rotate16(v, a.rope, (float)frame, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+        if (a.rotate) rotate16(v, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
         store_bf16x32(pos, v);
       }
     }
@@ -284,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float v[32];
       load_bf16x32(a.q + (((int64_t)b * a.n_q + ii) * a.n_heads + h) * 128 + 96, v);
       const int T = a.ring.tokens_per_frame, tok = ii % T;
-      rotate16(v, a.rope, (float)(a.t_first + ii / T), (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+      rotate16(v, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
       store_bf16x32(out + DL, v);
     }
   }
@@ -378,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (valid) {
       float v[32];
       load_bf16x32(a.kr + ((int64_t)b * a.kr_rows + mm) * a.kr_stride, v);
-      if (a.rotate) rotate16(v, a.rope, (float)frame, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+      if (a.rotate) rotate16(v, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
       store_bf16x32(kd + 96, v);
     }
   }

@@ -20,8 +20,8 @@ enum DeviceError : unsigned {
 };
 constexpr unsigned DEV_ERR_BOUNDS_MASK = DEV_ERR_BOUNDS;
 
-// 3D-RoPE table: pair p < n_t turns with the frame index t, then n_h pairs
-// with the grid row h, then n_w pairs with the grid column w.
+// 3D-RoPE: pair p < n_t turns with the frame index t, then n_h pairs with the
+// grid row h, then n_w pairs with the grid column w, by position * freq[p].
 struct Rope {
   float freq[kMaxPairs];
   int n_t, n_h, n_w;

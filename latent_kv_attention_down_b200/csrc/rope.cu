@@ -5,14 +5,10 @@
 //  * dense_q_bf16: the dense path's query [q_nope | RoPE(q_rope)], re-laid out
 //    head-major for the attention kernel's TMA tiles.
 #include "kernels.h"
+#include "rope.cuh"
 
 namespace vmla {
 namespace {
-
-__device__ __forceinline__ float pair_angle(const Rope& rp, int p, float t, float h, float w) {
-  const float pos = p < rp.n_t ? t : (p < rp.n_t + rp.n_h ? h : w);
-  return pos * rp.freq[p];
-}
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -23,14 +19,13 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 // rotate the 4 pairs held in one 16-byte vector; first pair index p0
-__device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, float t, float h, float w) {
+__device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, int t, int h, int w) {
   uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float s, c;
-    sincosf(pair_angle(rp, p0 + k, t, h, w), &s, &c);
-    const float u = bf_lo(in[k]), x = bf_hi(in[k]);
-    out[k] = pack2(u * c - x * s, u * s + x * c);
+    float u = bf_lo(in[k]), x = bf_hi(in[k]);
+    rope_apply(u, x, rope_cs(rp, p0 + k, t, h, w));
+    out[k] = pack2(u, x);
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
@@ -49,7 +44,7 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   const int64_t off = ((int64_t)b * ring_rows + s) * 32 + quad * 8;
   const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + off);
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + off) =
-      rotate4(v, a.rope, quad * 4, (float)t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+      rotate4(v, a.rope, quad * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
 }
 
 // 16 threads per (sample, query, head): 12 copy the content dims, 4 rotate the positional ones
@@ -66,8 +61,8 @@ __global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
   uint4 v = *reinterpret_cast<const uint4*>(src);
   if (chunk >= 12) {
     const int tok = i % a.ring.tokens_per_frame;
-    const float t = (float)(a.t_first + i / a.ring.tokens_per_frame);
-    v = rotate4(v, a.rope, (chunk - 12) * 4, t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w));
+    const int t = (int)(a.t_first + i / a.ring.tokens_per_frame);
+    v = rotate4(v, a.rope, (chunk - 12) * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
   }
   *reinterpret_cast<uint4*>(dst) = v;
 }

@@ -2,14 +2,10 @@
 // VMLA_FP32 handles.  They are plain CUDA (one thread per output element or a
 // block per query row) and make no attempt at speed.
 #include "kernels.h"
+#include "rope.cuh"
 
 namespace vmla {
 namespace {
-
-__device__ __forceinline__ float rope_angle(const Rope& rp, int p, float t, float h, float w) {
-  const float pos = p < rp.n_t ? t : (p < rp.n_t + rp.n_h ? h : w);
-  return pos * rp.freq[p];
-}
 
 // Row m of a call (frames first_frame ..) -> ring row of its sample.
 __device__ __forceinline__ int64_t ring_row(const Ring& g, int64_t first_frame, int m) {
@@ -45,12 +41,8 @@ __global__ void append_simt_kernel(const SimtAppend a) {
     }
     if (a.rotate) {
       const int tok = m % a.ring.tokens_per_frame;
-      const float t = (float)(a.first_frame + m / a.ring.tokens_per_frame);
-      float s, c;
-      sincosf(rope_angle(a.rope, p, t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w)), &s, &c);
-      const float u2 = u * c - v * s, v2 = u * s + v * c;
-      u = u2;
-      v = v2;
+      const int t = (int)(a.first_frame + m / a.ring.tokens_per_frame);
+      rope_apply(u, v, rope_cs(a.rope, p, t, tok / a.ring.grid_w, tok % a.ring.grid_w));
     }
     float* kr = a.kr + ((int64_t)b * a.out_rows + row) * a.d_rope + 2 * p;
     kr[0] = u;
@@ -72,11 +64,10 @@ __global__ void rope_window_f32_kernel(const RopeWindow a) {
   const int t = (fslot - a.window_start_slot + a.ring.window_frames) % a.ring.window_frames;
   const float* src = static_cast<const float*>(a.kr) + ((int64_t)b * ring_rows + s) * a.d_rope + 2 * p;
   float* dst = static_cast<float*>(a.kr_rot) + ((int64_t)b * ring_rows + s) * a.d_rope + 2 * p;
-  float sn, cs;
-  sincosf(rope_angle(a.rope, p, (float)t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w)), &sn, &cs);
-  const float u = src[0], v = src[1];
-  dst[0] = u * cs - v * sn;
-  dst[1] = u * sn + v * cs;
+  float u = src[0], v = src[1];
+  rope_apply(u, v, rope_cs(a.rope, p, t, tok / a.ring.grid_w, tok % a.ring.grid_w));
+  dst[0] = u;
+  dst[1] = v;
 }
 
 // ---- query preparation
@@ -107,12 +98,11 @@ __global__ void qprep_simt_kernel(const SimtQPrep a) {
   } else {
     const int p = j - lead;
     const int tok = i % a.ring.tokens_per_frame;
-    const float t = (float)(a.t_first + i / a.ring.tokens_per_frame);
-    float s, c;
-    sincosf(rope_angle(a.rope, p, t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w)), &s, &c);
-    const float u = q[a.d_nope + 2 * p], v = q[a.d_nope + 2 * p + 1];
-    out[lead + 2 * p] = u * c - v * s;
-    out[lead + 2 * p + 1] = u * s + v * c;
+    const int t = (int)(a.t_first + i / a.ring.tokens_per_frame);
+    float u = q[a.d_nope + 2 * p], v = q[a.d_nope + 2 * p + 1];
+    rope_apply(u, v, rope_cs(a.rope, p, t, tok / a.ring.grid_w, tok % a.ring.grid_w));
+    out[lead + 2 * p] = u;
+    out[lead + 2 * p + 1] = v;
   }
 }
 
@@ -229,11 +219,11 @@ __global__ void dense_reconstruct_simt_kernel(const SimtDenseReconstruct a) {
     const int p = j - a.d_nope;
     const float* r = a.r + ((int64_t)b * a.rows + m) * a.d_rope + 2 * p;
     const int tok = m % a.ring.tokens_per_frame;
-    const float t = (float)(a.first_frame + m / a.ring.tokens_per_frame);
-    float s, cs;
-    sincosf(rope_angle(a.rope, p, t, (float)(tok / a.ring.grid_w), (float)(tok % a.ring.grid_w)), &s, &cs);
-    kdst[a.d_nope + 2 * p] = r[0] * cs - r[1] * s;
-    kdst[a.d_nope + 2 * p + 1] = r[0] * s + r[1] * cs;
+    const int t = (int)(a.first_frame + m / a.ring.tokens_per_frame);
+    float u = r[0], v = r[1];
+    rope_apply(u, v, rope_cs(a.rope, p, t, tok / a.ring.grid_w, tok % a.ring.grid_w));
+    kdst[a.d_nope + 2 * p] = u;
+    kdst[a.d_nope + 2 * p + 1] = v;
   } else {
     const int e = j - a.d_nope - n_pairs;
     const float* w = a.w_uv + ((int64_t)h * a.d_value + e) * a.d_latent;

@@ -147,3 +147,56 @@ def queries(dims: Dims, layer: int, chunk: int, pass_: int = 0, n_frames: int | 
     nf = dims.chunk_frames if n_frames is None else n_frames
     return gaussian(dims, (dims.batch, nf * dims.tokens_per_frame, dims.n_heads, dims.d_head), std,
                     layer, chunk, pass_, _T_Q, base_seed)
+
+
+# ---------------------------------------------------------------- long rollouts
+_T_XPOOL, _T_QPOOL, _T_PICK = 6, 7, 8
+
+
+class FramePool:
+    """Inputs for rollouts of thousands of calls (30 layers x 20 chunks x 4
+    passes at the Wan-1.3B layer shape) without drawing 7 M fresh normals per
+    call: a pool of ``n_pool`` seeded Gaussian frames of activations and of
+    queries is drawn once; frame k of a call is pool entry e, its token rows
+    cyclically shifted by s and its sign flipped by g, with (e, s, g) drawn from
+    the call's own seeded stream.  The values stay N(0, 1) (bf16 where the
+    workload is bf16), every call still sees different content at every token,
+    and the pick is exact on either a NumPy array or a torch tensor, so the
+    oracle and the CUDA path get the same bits."""
+
+    def __init__(self, dims: Dims, n_pool: int = 8, base_seed: int = 0):
+        self.dims = dims
+        self.base_seed = base_seed
+        T = dims.tokens_per_frame
+        self.x = gaussian(dims, (n_pool, T, dims.d_model), 1.0, 0, 0, 0, _T_XPOOL, base_seed)
+        self.q = gaussian(dims, (n_pool, T, dims.n_heads, dims.d_head), 1.0, 0, 0, 0, _T_QPOOL, base_seed)
+
+    def picks(self, layer: int, chunk: int, pass_: int, tensor: int):
+        """[(entry, shift, sign)] for every (sample, frame) of the call, sample-major."""
+        d = self.dims
+        g = rng(d, layer, chunk, pass_, _T_PICK * 16 + tensor, self.base_seed)
+        n = d.batch * d.chunk_frames
+        e = g.integers(0, self.x.shape[0], n)
+        s = g.integers(0, d.tokens_per_frame, n)
+        sg = np.where(g.integers(0, 2, n) == 1, -1.0, 1.0)
+        return list(zip(e.tolist(), s.tolist(), sg.tolist()))
+
+    @staticmethod
+    def _take(pool, picks, batch):
+        if isinstance(pool, np.ndarray):
+            frames = [np.roll(pool[e], s, axis=0) * np.float32(g) for e, s, g in picks]
+            out = np.concatenate(frames, axis=0)
+        else:
+            import torch
+            frames = [torch.roll(pool[e], s, dims=0) * g for e, s, g in picks]
+            out = torch.cat(frames, dim=0)
+        return out.reshape((batch, -1) + tuple(out.shape[1:]))
+
+    def activations(self, layer: int, chunk: int, pass_: int = 0, pool=None):
+        """x of one chunk [batch, chunk_frames * T, d_model]; ``pool`` may be a
+        device copy of ``self.x`` (same values) to build it on the device."""
+        return self._take(self.x if pool is None else pool, self.picks(layer, chunk, pass_, _T_X), self.dims.batch)
+
+    def queries(self, layer: int, chunk: int, pass_: int = 0, pool=None):
+        """q of one chunk [batch, chunk_frames * T, n_heads, d_head]."""
+        return self._take(self.q if pool is None else pool, self.picks(layer, chunk, pass_, _T_Q), self.dims.batch)

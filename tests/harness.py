@@ -95,14 +95,26 @@ class Rollout:
 
     def oracle(self, layer, chunk, q, b=0, rows=None, heads=None):
         """The fp64 definition for sample b (window rebuilt from x, window-relative positions)."""
-        d = self.dims
-        first = chunk * d.chunk_frames
-        F = first + d.chunk_frames
-        w = self.w[layer]
-        c, r, kpos, t0 = O.window_latents(self.frame_x[layer][b], F, d.window_frames, w.w_down, d.d_latent,
-                                          d.grid_h, d.grid_w, rope_at="read")
-        qpos = O.chunk_query_positions(first, d.chunk_frames, t0, d.grid_h, d.grid_w)
-        ref = O.chunk_attention(c, r, kpos, q[b], qpos, w.w_uk, w.w_uv, d_nope=d.d_nope, rope_pairs=d.rope_pairs,
-                                rope_theta=d.rope_theta, rope_base_dims=d.rope_base_dims, query_rows=rows,
-                                heads=heads)
-        return ref.reshape(ref.shape[0], -1)
+        return oracle_chunk(self.dims, self.w[layer], self.frame_x[layer][b], chunk, q[b], rows, heads)
+
+
+def oracle_chunk(d, w, frame_x, chunk, q, rows=None, heads=None):
+    """fp64 output of one chunk call for one sample: ``frame_x`` maps every
+    appended frame index to its x [T, d_model] (the last pass written), ``q``
+    is that sample's [n_queries, n_heads, d_head]; [rows, n_heads * d_head]."""
+    first = chunk * d.chunk_frames
+    F = first + d.chunk_frames
+    c, r, kpos, t0 = O.window_latents(frame_x, F, d.window_frames, w.w_down, d.d_latent,
+                                      d.grid_h, d.grid_w, rope_at="read")
+    qpos = O.chunk_query_positions(first, d.chunk_frames, t0, d.grid_h, d.grid_w)
+    ref = O.chunk_attention(c, r, kpos, q, qpos, w.w_uk, w.w_uv, d_nope=d.d_nope, rope_pairs=d.rope_pairs,
+                            rope_theta=d.rope_theta, rope_base_dims=d.rope_base_dims, query_rows=rows,
+                            heads=heads)
+    return ref.reshape(ref.shape[0], -1)
+
+
+def sampled_rows(n_queries, count=256, seed=0):
+    """``count`` seeded query rows, the last row of the call always among them."""
+    rows = np.sort(np.random.default_rng(seed).choice(n_queries, min(count, n_queries), replace=False))
+    rows[-1] = n_queries - 1
+    return rows
