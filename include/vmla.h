@@ -223,6 +223,17 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
 vmla_status vmla_profile_enable(vmla_handle* h, int enable);
 vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* launches);
 
+/* Work split of the bf16 append kernel (the down-projection GEMM [c_KV | k_R] =
+ * W_down x of the paperlayer paper, Sec. 3): a persistent kernel over work items
+ * (sample, 128-row tile of x, column part of [c_KV | k_R]).  `n_split` column
+ * parts: 0 chooses per call (two when the row tiles alone would leave SMs idle,
+ * and always when d_latent > 224), 1 or 2 forces it.  `max_ctas` caps the grid
+ * (0: one CTA per SM); a small cap makes each CTA run many items.  Every split
+ * gives the same bits.  n_split = 1 with d_latent > 224 makes later appends
+ * return VMLA_ERR_UNSUPPORTED_SHAPE.  Host only; VMLA_ERR_INVALID_ARG for
+ * n_split outside 0..2 or a negative cap. */
+vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas);
+
 /* Allocation-free chunk attention.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for example a
  * plugin inside another runtime that is handed only its input and output

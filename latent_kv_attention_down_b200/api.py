@@ -64,6 +64,7 @@ _SIGS = {
     "vmla_state_set": (c_int, [c_void_p, c_int, c_int64]),
     "vmla_device_status": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
+    "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int]),
     "vmla_profile_read": (c_int, [c_void_p, c_int, ctypes.POINTER(c_double), ctypes.POINTER(c_int)]),
     "vmla_selftest_wait_timeout": (c_int, [c_uint64, c_void_p]),
     "vmla_chunk_attention_noalloc": (c_int, [ctypes.POINTER(Config), c_int, c_void_p, c_void_p, c_int64, c_void_p,
@@ -234,6 +235,10 @@ class LatentKVAttention:
         flags = c_uint32()
         st = lib().vmla_device_status(self._h, _stream(stream), ctypes.byref(flags))
         return st, flags.value
+
+    def set_append_tiling(self, n_split: int = 0, max_ctas: int = 0):
+        """Column parts (0: chosen per call) and grid cap (0: one CTA per SM) of the append kernel."""
+        check(lib().vmla_set_append_tiling(self._h, n_split, max_ctas), "vmla_set_append_tiling")
 
     def profile(self, enable: bool = True):
         check(lib().vmla_profile_enable(self._h, int(enable)), "vmla_profile_enable")

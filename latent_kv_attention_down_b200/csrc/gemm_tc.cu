@@ -80,119 +80,202 @@ __device__ __forceinline__ void teardown_cta(uint32_t tbase, uint32_t tmem_cols)
 }
 
 // ============================================================== append
-template <int N_OUT>
+// Persistent: each CTA takes work items (sample, 128-row tile, column part) in
+// a grid-stride loop.  The column parts split [c_KV | k_R] into NP pieces of
+// N_PART columns (NP = 2 gives small calls -- one chunk of one sample, 37 row
+// tiles -- work for twice as many SMs, at the price of reading x twice from
+// L2).  Two TMEM accumulators alternate, so the epilogue of one item overlaps
+// the loads and MMAs of the next; the epilogue parks the bf16 tile in shared
+// memory and writes it out row-contiguous (ring rows of one frame are
+// consecutive).
+template <int N_PART>
 struct AppendCfg {
-  static constexpr int STAGES = 4;
   static constexpr int A_BYTES = 128 * 128;  // 128 rows x 64 bf16
-  static constexpr int NB = N_OUT <= 256 ? N_OUT : N_OUT / 2;
-  static constexpr int NSPLIT = N_OUT / NB;
-  static constexpr int B_BYTES = N_OUT * 128;
+  static constexpr int B_BYTES = N_PART * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t TMEM_COLS = N_OUT <= 256 ? 256 : 512;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
-  static_assert(N_OUT % 32 == 0 && NB % 16 == 0 && NB <= 256, "bad N");
-  static_assert(B_BYTES % 1024 == 0, "stage alignment");
+  static constexpr int OUT_STRIDE = N_PART * 2 + 16;  // bytes per parked row: an odd number of 16-byte chunks
+  static constexpr int OUT_BYTES = 64 * OUT_STRIDE;   // half a tile is parked at a time
+  static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = FIT > 8 ? 8 : FIT;
+  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators, at columns 0 and 256
+  static constexpr int SMEM_USED = 1024 + STAGES * STAGE_BYTES + OUT_BYTES + 2 * 128 * 8 + 256;
+  // more than half of an SM's shared memory: one CTA per SM, so the 512 TMEM columns are always free
+  static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
+  static_assert(N_PART % 16 == 0 && N_PART <= 256, "bad N");
+  static_assert(B_BYTES % 1024 == 0 && OUT_BYTES % 16 == 0, "alignment");
+  static_assert(STAGES >= 3 && SMEM <= 227 * 1024, "does not fit");
 };
 
-template <int N_OUT>
+template <int N_PART>
 __global__ void __launch_bounds__(kThreads, 1)
     append_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const AppendTc a) {
-  using C = AppendCfg<N_OUT>;
+                     const AppendTc a, int n_parts, int items) {
+  using C = AppendCfg<N_PART>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* sout = smem + C::STAGES * C::STAGE_BYTES;
+  int64_t* row_lat = reinterpret_cast<int64_t*>(sout + C::OUT_BYTES);  // element offsets of each row's
+  int64_t* row_pos = row_lat + 128;                                    // latent / positional destination
+  uint64_t* full = reinterpret_cast<uint64_t*>(row_pos + 128);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* done = empty + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, b = blockIdx.y;
   const int kblocks = a.d_model / 64;
+  const int m_tiles = (a.rows + 127) / 128;
   const Guard g{abort_flag, a.err, a.limit_ns};
-  const uint32_t tbase = setup_cta(full, 2 * C::STAGES + 1, tslot, abort_flag, C::TMEM_COLS);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 4);  // one arrival per epilogue warp
+    mbar_init(&acc_empty[1], 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
 
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_w);
-      int issued = 0;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % C::STAGES;
-        if (!wait_phase(&empty[s], ((kb / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
-        uint8_t* sa = smem + s * C::STAGE_BYTES;
-        uint8_t* sb = sa + C::A_BYTES;
-        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-        tma_load_3d(sa, &tm_x, &full[s], kb * 64, m0, b);
-        for (int sp = 0; sp < C::NSPLIT; ++sp) tma_load_2d(sb + sp * C::NB * 128, &tm_w, &full[s], kb * 64, sp * C::NB);
-        ++issued;
+      int it = 0;  // global stage counter
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+        const int part = item % n_parts, mt = (item / n_parts) % m_tiles, b = item / (n_parts * m_tiles);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          tma_load_3d(sa, &tm_x, &full[s], kb * 64, mt * 128, b);
+          tma_load_2d(sa + C::A_BYTES, &tm_w, &full[s], kb * 64, part * N_PART);
+        }
       }
-      if (*abort_flag)
-        for (int kb = issued > C::STAGES ? issued - C::STAGES : 0; kb < issued; ++kb)
-          drain_phase(&full[kb % C::STAGES], (kb / C::STAGES) & 1, g);
+      if (*abort_flag)  // let the copies in flight land before the CTA goes away
+        for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+          drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
     }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, C::NB, false, false);
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % C::STAGES;
-        if (!wait_phase(&full[s], (kb / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+      constexpr uint32_t idesc = idesc_bf16_f32(128, N_PART, false, false);
+      int it = 0, j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        const int acc = j & 1;
+        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-        const uint64_t ad = smem_desc(sa, 16, 1024, LAYOUT_SW128);
-        const uint64_t bd = smem_desc(sa + C::A_BYTES, 16, 1024, LAYOUT_SW128);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int sp = 0; sp < C::NSPLIT; ++sp) {
-            const uint64_t a = desc_add(ad, k * 32), b = desc_add(bd, sp * C::NB * 128 + k * 32);
-            if (k == 0 && kb == 0)
-              mma_ss_c<false>(tbase + sp * C::NB, a, b, idesc);
-            else
-              mma_ss_c<true>(tbase + sp * C::NB, a, b, idesc);
+        const uint32_t d = tbase + acc * 256;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!wait_phase(&full[s], (it / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
           }
-        mma_commit(&empty[s]);
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint64_t ad = smem_desc(sa, 16, 1024, LAYOUT_SW128);
+          const uint64_t bd = smem_desc(sa + C::A_BYTES, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (k == 0 && kb == 0)
+              mma_ss_c<false>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+            else
+              mma_ss_c<true>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
       }
       mma_commit(done);
       if (*abort_flag) drain_phase(done, 0, g);
     }
-  } else if (warp >= 4) {
-    const int wq = warp - 4;
-    const int m = m0 + wq * 32 + lane;
-    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
     __syncwarp();
-    tc_fence_after();
-    const bool valid = ok && m < a.rows;
+  } else if (warp >= 4) {
+    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
-    const int mm = valid ? m : 0;
-    const int64_t frame = a.first_frame + mm / T;
-    const int tok = mm % T;
-    __nv_bfloat16* lat;
-    __nv_bfloat16* pos;
-    if (a.contiguous) {
-      lat = a.ckv + ((int64_t)b * a.rows + mm) * N_OUT;
-      pos = lat + a.d_latent;
-    } else {
-      const int64_t row = (frame % a.ring.window_frames) * T + tok;
-      lat = a.ckv + ((int64_t)b * a.ring_rows + row) * a.d_latent;
-      pos = a.kr + ((int64_t)b * a.ring_rows + row) * 32;
-    }
-#pragma unroll 1
-    for (int c0 = 0; c0 < N_OUT; c0 += 32) {
-      uint32_t raw[32];
-      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
-      if (!valid) continue;
-      float v[32];
-      raw_to_float(raw, v);
-      if (c0 < a.d_latent) {
-        store_bf16x32(lat + c0, v);
+    constexpr int CH = N_PART / 8;  // 16-byte chunks per row
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const int part = item % n_parts, mt = (item / n_parts) % m_tiles, b = item / (n_parts * m_tiles);
+      const int acc = j & 1;
+      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      __syncwarp();
+      tc_fence_after();
+      const int m = mt * 128 + r;
+      const int mm = m < a.rows ? m : 0;
+      const int64_t frame = a.first_frame + mm / T;
+      const int tok = mm % T;
+      if (a.contiguous) {
+        row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + 32);
+        row_pos[r] = row_lat[r] + a.d_latent;
       } else {
-        if (a.rotate) rotate16(v, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
-        store_bf16x32(pos, v);
+        const int64_t rr = (int64_t)b * a.ring_rows + (frame % a.ring.window_frames) * T + tok;
+        row_lat[r] = rr * a.d_latent;
+        row_pos[r] = rr * 32;
+      }
+      named_bar_sync(1, 128);  // row table complete
+      const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        if ((wq >> 1) == half) {  // warps of this half hold TMEM lanes 64*half .. 64*half + 63
+          uint8_t* orow = sout + (r - 64 * half) * C::OUT_STRIDE;
+#pragma unroll 1
+          for (int c0 = 0; c0 < N_PART; c0 += 16) {
+            uint32_t raw[16];
+            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(raw[q]);
+            const int col = part * N_PART + c0;  // 16 columns never straddle d_latent (a multiple of 64)
+            if (a.rotate && col >= a.d_latent) {
+              const int p0 = (col - a.d_latent) >> 1;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                rope_apply(v[2 * q], v[2 * q + 1],
+                           rope_cs(a.rope, p0 + q, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w));
+            }
+            uint4* o = reinterpret_cast<uint4*>(orow + c0 * 2);
+            o[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                              pack_bf16x2(v[6], v[7]));
+            o[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                              pack_bf16x2(v[14], v[15]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read; all four free it for item j + 2
+        }
+        named_bar_sync(1, 128);  // this half is parked
+        const int rows_h = min(64, valid_rows - 64 * half);
+#pragma unroll 4
+        for (int id = tid; id < rows_h * CH; id += 128) {
+          const int row = id / CH, ch = id - row * CH;
+          const int col = part * N_PART + ch * 8;
+          const bool lat = col < a.d_latent;
+          __nv_bfloat16* dst = (lat || a.contiguous ? a.ckv : a.kr) +
+                               (lat ? row_lat[64 * half + row] + col : row_pos[64 * half + row] + (col - a.d_latent));
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + row * C::OUT_STRIDE + ch * 16);
+        }
+        named_bar_sync(1, 128);  // the parked half is written out before it is reused
       }
     }
   }
-  teardown_cta(tbase, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
 }
 
 // ============================================================== q-absorb
@@ -380,13 +463,32 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int N_OUT>
-cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, cudaStream_t s) {
-  using C = AppendCfg<N_OUT>;
-  static const cudaError_t attr = set_smem(append_tc_kernel<N_OUT>, C::SMEM);
+template <int N_PART>
+cudaError_t run_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, int n_parts,
+                       int ctas, cudaStream_t s) {
+  using C = AppendCfg<N_PART>;
+  static const cudaError_t attr = set_smem(append_tc_kernel<N_PART>, C::SMEM);
   if (attr != cudaSuccess) return attr;
-  append_tc_kernel<N_OUT><<<dim3((a.rows + 127) / 128, batch), kThreads, C::SMEM, s>>>(tx, tw, a);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((a.rows + 127) / 128) * n_parts * batch;
+  const int grid = std::min(items, ctas > 0 ? ctas : sms);
+  append_tc_kernel<N_PART><<<grid, kThreads, C::SMEM, s>>>(tx, tw, a, n_parts, items);
   return cudaGetLastError();
+}
+
+template <int N_OUT>
+cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, cudaStream_t s,
+                      const AppendPlan& p) {
+  if constexpr (N_OUT <= 256) {
+    if (p.parts == 1) return run_append<N_OUT>(tx, tw, a, batch, 1, p.ctas, s);
+  }
+  if (p.parts == 2) return run_append<N_OUT / 2>(tx, tw, a, batch, 2, p.ctas, s);
+  return cudaErrorInvalidValue;
 }
 
 template <int DL>
@@ -410,20 +512,25 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
 
 }  // namespace
 
-int append_tc_w_box_rows(int d_latent) {
-  const int n = d_latent + 32;
-  return n <= 256 ? n : n / 2;
+
+AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ctas) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    cudaGetLastError();
+  AppendPlan p{n_split, ctas};
+  if (p.parts == 0) p.parts = (d_latent + 32 > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
+  return p;
 }
 
 cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch,
-                             cudaStream_t s) {
+                             cudaStream_t s, const AppendPlan& p) {
   if (a.rows <= 0) return cudaSuccess;
   if (a.d_model % 64 != 0) return cudaErrorInvalidValue;
   switch (a.d_latent) {
-    case 64: return go_append<96>(tx, tw, a, batch, s);
-    case 128: return go_append<160>(tx, tw, a, batch, s);
-    case 192: return go_append<224>(tx, tw, a, batch, s);
-    case 256: return go_append<288>(tx, tw, a, batch, s);
+    case 64: return go_append<96>(tx, tw, a, batch, s, p);
+    case 128: return go_append<160>(tx, tw, a, batch, s, p);
+    case 192: return go_append<224>(tx, tw, a, batch, s, p);
+    case 256: return go_append<288>(tx, tw, a, batch, s, p);
   }
   return cudaErrorInvalidValue;
 }

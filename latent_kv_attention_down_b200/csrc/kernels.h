@@ -110,10 +110,17 @@ struct AppendTc {
   unsigned* err;
   uint64_t limit_ns;
 };
-// x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, d_c + 32) box (64, nb) SW128
+// Work split of the persistent append kernel for a call: `parts` column parts
+// of [c_KV | k_R] (1 or 2) and a grid cap `ctas` (0: one CTA per SM).  n_split 0
+// chooses two parts when the 128-row tiles alone would leave SMs idle (and
+// always past 256 columns).
+struct AppendPlan {
+  int parts, ctas;
+};
+AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ctas);
+// x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, d_c + 32) box (64, (d_c + 32) / parts) SW128.
 cudaError_t launch_append_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const AppendTc& a, int batch,
-                             cudaStream_t s);
-int append_tc_w_box_rows(int d_latent);
+                             cudaStream_t s, const AppendPlan& plan);
 
 struct QPrepTc {
   const __nv_bfloat16* q;  // [B][n_q][n_h][128]  (rope part read directly)

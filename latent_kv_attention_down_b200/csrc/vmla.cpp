@@ -70,6 +70,11 @@ Rope make_rope(const vmla_config& c) {
   return r;
 }
 
+// A forced append column split the shape can take: one MMA covers at most 256 columns.
+bool append_tiling_fits(const vmla_config& c, int n_split) {
+  return n_split != 1 || c.d_latent + 32 <= 256;
+}
+
 Ring make_ring(const vmla_config& c) { return Ring{(int)tokens_per_frame(c), c.grid_w, c.window_frames}; }
 
 // ---------------------------------------------------------------- TMA tensor maps
@@ -143,6 +148,8 @@ struct vmla_handle {
   std::vector<int64_t> frames;        // latent cache, per layer
   std::vector<int64_t> dense_frames;  // dense cache, per layer
   unsigned* err = nullptr;            // device status word (resolved at bind)
+  int append_split = 0;               // append work split (0: chosen per call), see vmla_set_append_tiling
+  int append_ctas = 0;
   bool profiling = false;
   struct Timer {
     std::vector<cudaEvent_t> ev;  // begin/end pairs
@@ -413,6 +420,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
   if ((st = check_append_frames(c, h->frames[layer], first, n, &new_F)) != VMLA_OK) return st;
   const bool rotate = c.rope_mode == VMLA_ROPE_AT_APPEND;
   if (rotate && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if (c.dtype == VMLA_BF16 && !append_tiling_fits(c, h->append_split)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   if ((st = ensure_err(h)) != VMLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = (int)(n * tokens_per_frame(c));
@@ -440,9 +448,12 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
     } else {
       CUtensorMap tx, tw;
       const int nout = c.d_latent + 32;
+      const AppendPlan plan =
+          append_tc_plan(c.d_latent, rows, c.batch, h->append_split, h->append_ctas);
+      const int parts = plan.parts;
       if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_tc_w_box_rows(c.d_latent),
+          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
                 CU_TENSOR_MAP_SWIZZLE_128B))
         return VMLA_ERR_CUDA;
       AppendTc a;
@@ -459,7 +470,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
       a.rope = make_rope(c);
       a.err = h->err;
       a.limit_ns = kWaitLimitNs;
-      e = launch_append_tc(tx, tw, a, c.batch, s);
+      e = launch_append_tc(tx, tw, a, c.batch, s, plan);
     }
   }
   if (e != cudaSuccess) return VMLA_ERR_CUDA;
@@ -699,6 +710,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
   int64_t new_F;
   if ((st = check_append_frames(c, h->dense_frames[layer], first, n, &new_F)) != VMLA_OK) return st;
   if (first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if (c.dtype == VMLA_BF16 && !append_tiling_fits(c, h->append_split)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   if ((st = ensure_err(h)) != VMLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(c);
@@ -733,10 +745,13 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
   } else {
     __nv_bfloat16* chunk = at<__nv_bfloat16>(h->ws, w.chunk);  // [B][rows][d_c + 32]
     const int nout = c.d_latent + 32;
+    const AppendPlan plan =
+          append_tc_plan(c.d_latent, rows, c.batch, h->append_split, h->append_ctas);
+      const int parts = plan.parts;
     CUtensorMap tx, tw;
     if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_tc_w_box_rows(c.d_latent),
+        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
               CU_TENSOR_MAP_SWIZZLE_128B))
       return VMLA_ERR_CUDA;
     AppendTc a;
@@ -753,7 +768,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     a.rope = make_rope(c);
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    if ((e = launch_append_tc(tx, tw, a, c.batch, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+    if ((e = launch_append_tc(tx, tw, a, c.batch, s, plan)) != cudaSuccess) return VMLA_ERR_CUDA;
     CUtensorMap tc, tuk, tuv;
     if (!map3(&tc, chunk, c.d_latent, rows, c.batch, (uint64_t)nout * 2, (uint64_t)rows * nout * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -863,6 +878,13 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
   if (flags) *flags = v;
   if (v & DEV_ERR_BOUNDS_MASK) return VMLA_ERR_DEVICE_BOUNDS;
   if (v) return VMLA_ERR_DEVICE_TIMEOUT;
+  return VMLA_OK;
+}
+
+vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas) {
+  if (!h || n_split < 0 || n_split > 2 || max_ctas < 0) return VMLA_ERR_INVALID_ARG;
+  h->append_split = n_split;
+  h->append_ctas = max_ctas;
   return VMLA_OK;
 }
 

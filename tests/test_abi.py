@@ -196,3 +196,22 @@ def test_rope_at_append_range():
     # frames 1022..1024 would put an absolute t at 1024, outside the RoPE range
     assert lib.vmla_cache_append(h._h, 0, 0x40000, 0x40000, 1022, 3, None) == 3
     h.close()
+
+
+def test_append_tiling_arguments():
+    c = default_config()
+    h = api.LatentKVAttention(c)
+    lib = api.lib()
+    for t in ((3, 0), (-1, 0), (1, -1)):
+        assert lib.vmla_set_append_tiling(h._h, *t) == 1, t
+    for t in ((0, 0), (1, 0), (2, 0), (1, 3), (2, 148), (0, 7)):
+        assert lib.vmla_set_append_tiling(h._h, *t) == 0, t
+    # one MMA covers at most 256 columns: d_latent 256 (+32) needs two column parts
+    c256 = default_config()
+    c256.d_latent = 256
+    h2 = api.LatentKVAttention(c256)
+    assert lib.vmla_bind(h2._h, 0x10000, 0x20000, 0x30000, api.workspace_bytes(c256)) == 0
+    assert lib.vmla_set_append_tiling(h2._h, 1, 0) == 0
+    assert lib.vmla_cache_append(h2._h, 0, 0x40000, 0x40000, 0, 3, None) == 2
+    for x in (h, h2):
+        x.close()

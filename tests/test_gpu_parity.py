@@ -186,6 +186,58 @@ def test_small_append_writes_only_its_slots():
     assert np.all(raw_ckv == 0x7F) and np.all(raw_kr == 0x7F)
 
 
+TILINGS = [(0, 0), (1, 0), (2, 0), (1, 1), (2, 3)]
+
+
+@pytest.mark.parametrize("tiling", TILINGS, ids=lambda t: "np%d_ctas%d" % t)
+@pytest.mark.parametrize("rope_mode", [api.ROPE_AT_READ, api.ROPE_AT_APPEND])
+def test_append_tilings(tiling, rope_mode):
+    """Every work split of the persistent append kernel (one or two column
+    parts; a grid of one CTA per SM, or capped so each CTA runs many items
+    through both TMEM accumulators) writes bf16(W_down x) -- k_R rotated with the absolute frame
+    when RoPE is applied at append -- into exactly its ring rows, for two
+    samples and a ragged last tile (600 rows per sample)."""
+    import torch
+    import oracle.vmla_oracle as O
+    d = SMALL.replace(name="small_b2", batch=2)
+    ro = Rollout(d, rope_mode=rope_mode)
+    ro.m.set_append_tiling(*tiling)
+    ro.m.ckv.fill_(0x7F)
+    ro.m.kr.fill_(0x7F)
+    for c in range(3):  # frames 0..8; the ring holds 21
+        ro.append_chunk(0, c)
+    torch.cuda.synchronize()
+    assert ro.m.device_status()[0] == 0
+    T, R = d.tokens_per_frame, d.window_frames * d.tokens_per_frame
+    n = 9 * T
+    ckv = ro.m.ckv.view(torch.bfloat16).view(d.batch, R, d.d_latent).float().cpu().numpy()
+    kr = ro.m.kr.view(torch.bfloat16).view(d.batch, R, d.d_rope).float().cpu().numpy()
+    freqs = O.rope_frequencies(d.rope_pairs, d.rope_theta, d.rope_base_dims)
+    pos = O.key_positions(range(9), 0, d.grid_h, d.grid_w)
+    for b in range(d.batch):
+        x = np.concatenate([ro.frame_x[0][b][f] for f in range(9)])
+        c, r = O.down_project(x, ro.w[0].w_down, d.d_latent)
+        if rope_mode == api.ROPE_AT_APPEND:
+            r = O.rope_rotate(r, O.rope_angles(pos[:, 0], pos[:, 1], pos[:, 2], freqs))
+        for got, ref, what in ((ckv[b, :n], c, "c_KV"), (kr[b, :n], r, "k_R")):
+            err = np.abs(got - ref)
+            bound = 2.0 ** -8 * np.abs(ref) + 1e-5 * np.abs(ref).max()
+            assert np.all(err <= bound), f"{what} sample {b}: worst excess {np.max(err - bound):.3e}"
+    raw_ckv = ro.m.ckv.view(d.batch, R, -1)[:, n:].cpu().numpy()
+    raw_kr = ro.m.kr.view(d.batch, R, -1)[:, n:].cpu().numpy()
+    assert np.all(raw_ckv == 0x7F) and np.all(raw_kr == 0x7F)
+
+
+@pytest.mark.parametrize("tiling", [(1, 0), (2, 0), (2, 1)], ids=lambda t: "np%d_ctas%d" % t)
+def test_small_bf16_attention_after_tiled_appends(tiling):
+    """The full path with a forced append tiling, against the oracle."""
+    ro = Rollout(SMALL)
+    ro.m.set_append_tiling(*tiling)
+    _fill(ro, 8)
+    out, q = ro.attend(0, 7)
+    assert_bf16_close(out[0], ro.oracle(0, 7, q), f"tiling {tiling}")
+
+
 def test_small_output_rows_and_guards():
     """Attention writes exactly its output tensor: guard rows around it stay
     bit-identical."""
