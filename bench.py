@@ -125,6 +125,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks_of(v: float, dist=None, device="cpu") -> float:
+    """The largest of every rank's v (every rank gets it); v itself without a process group."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, ms_per_step_max: float, world: int) -> float:
+    """Whole-job rate of independent replicas: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
+
+
 # ----------------------------------------------------------------------------- CPU oracle baseline
 
 def oracle_sample(n_queries=256, heads=None, seed=0):
@@ -240,11 +257,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(v, dist, dev)
 
     def timed(fn, steps, warmup, profile=False):
         for i in range(warmup):
@@ -275,8 +288,8 @@ def run_ours(args, rank, world, local_rank):
     assert st == 0, f"device status {st} flags {flags:#x}"
     ms_step = max_over_ranks(ms / args.steps)
     F = step_flops()
-    value = world * F["total"] / (ms_step * 1e-3) / 1e12
-    tokens = world * d.n_queries / (ms_step * 1e-3)
+    value = replica_throughput(F["total"], ms_step, world) / 1e12
+    tokens = replica_throughput(d.n_queries, ms_step, world)
 
     # ------------------------------------------------ end to end from pinned host memory
     xh = [xs[l].cpu().pin_memory() for l in range(2)]

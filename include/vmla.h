@@ -107,6 +107,11 @@ typedef struct vmla_handle vmla_handle;
 /* Name of a status code (static string, never NULL). */
 const char* vmla_status_string(vmla_status status);
 
+/* Text of the CUDA error (name: description), or of the tensor-map encoding
+ * failure, behind the last VMLA_ERR_CUDA this thread received; "" before any.
+ * The pointer stays valid until the thread's next failing call. */
+const char* vmla_last_error_detail(void);
+
 /* VMLA_ABI_VERSION of the loaded library. */
 int vmla_abi_version(void);
 
@@ -264,6 +269,13 @@ vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int layer, cons
                                          int64_t frames_appended, const void* q, const void* w_uk,
                                          const void* w_uv, void* out, int64_t first_frame, int n_frames,
                                          void* stream);
+
+/* Self-test of the polynomial exp2 that the attention kernels evaluate on the
+ * FMA pipe for part of each softmax tile (the rest goes to the MUFU unit):
+ * y[i] = 2^x[i] for n (even) fp32 values in device memory, both arrays 8-byte
+ * aligned.  Relative error <= 7.5e-5 for x >= -125; below that the result is at
+ * most 2^-124.  VMLA_ERR_INVALID_ARG for odd n or misaligned arrays. */
+vmla_status vmla_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /* Self-test of the bounded pipeline waits: launches one CTA that waits on an
  * mbarrier nothing arrives at, for at most `limit_ns` nanoseconds (<= 1e9), then

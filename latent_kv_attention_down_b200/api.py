@@ -34,11 +34,15 @@ class Config(ctypes.Structure):
 class VmlaError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {lib().vmla_status_string(status).decode()}")
+        msg = f"{what}: {lib().vmla_status_string(status).decode()}"
+        if status == 4:  # VMLA_ERR_CUDA: say which CUDA error
+            msg += f" ({lib().vmla_last_error_detail().decode()})"
+        super().__init__(msg)
 
 
 _SIGS = {
     "vmla_status_string": (ctypes.c_char_p, [c_int]),
+    "vmla_last_error_detail": (ctypes.c_char_p, []),
     "vmla_abi_version": (c_int, []),
     "vmla_config_init": (c_int, [ctypes.POINTER(Config)]),
     "vmla_config_check": (c_int, [ctypes.POINTER(Config)]),
@@ -65,6 +69,7 @@ _SIGS = {
     "vmla_device_status": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
     "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int]),
+    "vmla_selftest_exp2": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
     "vmla_profile_read": (c_int, [c_void_p, c_int, ctypes.POINTER(c_double), ctypes.POINTER(c_int)]),
     "vmla_selftest_wait_timeout": (c_int, [c_uint64, c_void_p]),
     "vmla_chunk_attention_noalloc": (c_int, [ctypes.POINTER(Config), c_int, c_void_p, c_void_p, c_int64, c_void_p,
@@ -248,6 +253,11 @@ class LatentKVAttention:
         ms, n = c_double(), c_int()
         check(lib().vmla_profile_read(self._h, st, ctypes.byref(ms), ctypes.byref(n)), "vmla_profile_read")
         return ms.value, n.value
+
+
+def selftest_exp2(x, y, stream=None):
+    """y = the kernels' polynomial 2^x (fp32 device tensors, even length)."""
+    check(lib().vmla_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)), "vmla_selftest_exp2")
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None):

@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < HS / 2; ++k) {
           const float2 x = make_float2(__uint_as_float(sraw[2 * k]), __uint_as_float(sraw[2 * k + 1]));
           const float2 y = __ffma2_rn(x, sc2, nm2);
-          const float2 pr = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+          const float2 pr = exp2_mixed(y, k);
           acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
           packed[k] = pack_bf16x2(pr.x, pr.y);
         }
@@ -511,6 +511,11 @@ int attn_absorbed_block_n(int d_latent) {
 
 int attn_dense_block_n() { return AttnCfg<128, true>::BN; }
 
+cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& to,
+                                 const AttnTc& a, int batch, cudaStream_t s) {
+  return go_attn<128, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
+}
+
 cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
                                     const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tuv,
                                     const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
@@ -523,9 +528,5 @@ cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tq, const C
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& to,
-                                 const AttnTc& a, int batch, cudaStream_t s) {
-  return go_attn<128, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
-}
 
 }  // namespace vmla

@@ -153,7 +153,7 @@ int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the 
 int attn_dense_block_n();
 
 // Dense per-head attention, d_head = 128.  q map: 3D (128, n_q, B*n_h) box (64,128,1);
-// kv map: 3D (2*n_h*128, n_keys, B) box (64,128,1); out as above.
+// kv map: 3D (2*n_h*128, n_keys, B) box (64,128,1); out: 3D fp32 (n_h*128, n_q, B) box (32,128,1) SW128.
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_out,
                                  const AttnTc& a, int batch, cudaStream_t s);
 
@@ -190,5 +190,7 @@ cudaError_t launch_recon_tc(const CUtensorMap& tm_c, const CUtensorMap& tm_wuk, 
 // ------------------------------------------------------------------ device status
 unsigned* device_error_word();  // address of the library's device status word (current device)
 cudaError_t launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s);
+// y[i] = the attention kernels' polynomial 2^x[i] (exp2_poly2), n even, 8-byte aligned arrays.
+cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t s);
 
 }  // namespace vmla

@@ -368,4 +368,41 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^y for two values on the FMA pipe, leaving the MUFU unit (16 exp2 per clock
+// per SM, the softmax bottleneck) to the other elements.  Range reduction
+// y = n + f with n = round(y), taken from the low bits of y + 1.5*2^23, and f in
+// [-1/2, 1/2]; 2^f by the degree-3 polynomial of least maximum relative error on
+// that interval (Remez exchange, see exp2_fit.py: relative error <= 7.5e-5, far
+// below the bf16 rounding of P); 2^n is added to the exponent field as an
+// integer.  y is clamped below at -125, where the result is already negligible
+// for a softmax whose largest term is 1.
+// Of every 8 score pairs, the softmax loops send this many to exp2_poly2.  On
+// B200 a packed FFMA2/FADD2 takes two issue cycles, so the polynomial costs
+// about as much pipe time as the MUFU exp2 it replaces; at the Wan-1.3B layer
+// shape no share measured faster than 0 (all MUFU), which is the default.
+#ifndef VMLA_EXP2_POLY_PAIRS
+#define VMLA_EXP2_POLY_PAIRS 0
+#endif
+constexpr int kExp2PolyPairs = VMLA_EXP2_POLY_PAIRS;
+constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ float2 exp2_poly2(float2 y) {
+  y.x = fmaxf(y.x, -125.f);
+  y.y = fmaxf(y.y, -125.f);
+  const float2 t = __fadd2_rn(y, make_float2(12582912.f, 12582912.f));   // 1.5 * 2^23 + round(y)
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));  // round(y)
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), y);            // y - round(y), exact
+  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  // the low 9 bits of t hold n (two's complement); shifted by 23 they land on the exponent
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// 2^y of score pair k of a softmax loop: the polynomial for kExp2PolyPairs of every 8 pairs.
+__device__ __forceinline__ float2 exp2_mixed(float2 y, int k) {
+  return (k & 7) < kExp2PolyPairs ? exp2_poly2(y) : make_float2(ex2_approx(y.x), ex2_approx(y.y));
+}
+
 }  // namespace vmla

@@ -32,6 +32,21 @@ __global__ void selftest_wait_kernel(unsigned* err, uint64_t limit_ns) {
 }
 }  // namespace
 
+namespace {
+__global__ void selftest_exp2_kernel(const float2* x, float2* y, int64_t pairs) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < pairs) y[i] = exp2_poly2(x[i]);
+}
+}  // namespace
+
+cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t s) {
+  const int64_t pairs = n / 2;
+  if (pairs == 0) return cudaSuccess;
+  selftest_exp2_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float2*>(x),
+                                                                        reinterpret_cast<float2*>(y), pairs);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s) {
   selftest_wait_kernel<<<1, 32, 0, s>>>(err, limit_ns);
   return cudaGetLastError();

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -122,7 +123,18 @@ bool map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : VMLA_ERR_CUDA; }
+// Detail of the last VMLA_ERR_CUDA returned on this thread (vmla_last_error_detail).
+thread_local char g_detail[160] = "";
+
+vmla_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_detail, sizeof(g_detail), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return VMLA_ERR_CUDA;
+}
+vmla_status map_fail() {
+  std::snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled refused a tensor map (or the driver entry point is missing)");
+  return VMLA_ERR_CUDA;
+}
+vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : cuda_fail(e); }
 
 // AUTO: the absorbed design up to d_latent = 192; from 256 on the per-head K/V
 // are rebuilt once per call.  At 256 the rebuilt path is the more accurate one
@@ -455,7 +467,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
                 CU_TENSOR_MAP_SWIZZLE_128B))
-        return VMLA_ERR_CUDA;
+        return map_fail();
       AppendTc a;
       a.ckv = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
       a.kr = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
@@ -473,7 +485,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
       e = launch_append_tc(tx, tw, a, c.batch, s, plan);
     }
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   h->frames[layer] = new_F;
   return VMLA_OK;
 }
@@ -495,7 +507,7 @@ vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void*
     e = launch_rope_window_f32(r, s);
     kpos = at<float>(h->ws, w.kr_rot);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   const int nq = (int)(n * tokens_per_frame(c));
   {
     StageScope scope(h, 2, s);
@@ -504,7 +516,7 @@ vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void*
                 make_rope(c)};
     e = launch_qprep_simt(a, s);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   {
     StageScope scope(h, 3, s);
     SimtAttn a;
@@ -549,7 +561,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     e = launch_rope_window_bf16(r, s);
     kpos = at<__nv_bfloat16>(h->ws, w.kr_rot);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   const uint64_t rr = ring_rows(c);
 
   if (design == VMLA_DESIGN_RECON_ONCE) {
@@ -564,7 +576,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B))
-        return VMLA_ERR_CUDA;
+        return map_fail();
       ReconTc a;
       a.kr = kpos;
       a.dense = recon;
@@ -583,7 +595,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       a.limit_ns = kWaitLimitNs;
       e = launch_recon_tc(tc, tuk, tuv, a, c.batch, s);
     }
-    if (e != cudaSuccess) return VMLA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e);
     return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s);
   }
   if (design == VMLA_DESIGN_RECONSTRUCT) return VMLA_ERR_UNSUPPORTED_SHAPE;
@@ -597,7 +609,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
               (uint64_t)nq * c.n_heads * 128 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
               CU_TENSOR_MAP_SWIZZLE_128B))
-      return VMLA_ERR_CUDA;
+      return map_fail();
     QPrepTc a;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.qt = qt;
@@ -611,7 +623,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.limit_ns = kWaitLimitNs;
     e = launch_qprep_tc(tq, tuk, a, c.batch, s);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   {
     StageScope scope(h, 3, s);
     const int bn = attn_absorbed_block_n(c.d_latent);
@@ -627,7 +639,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
         !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
               (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
-      return VMLA_ERR_CUDA;
+      return map_fail();
     AttnTc a;
     a.n_q = nq;
     a.n_keys = win.n_keys;
@@ -655,7 +667,7 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
                make_rope(c)};
     e = launch_dense_q_bf16(a, s);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   StageScope scope(h, stage, s);
   const uint64_t rr = ring_rows(c);
   const uint64_t row_bytes = 2ull * c.n_heads * 128 * 2;
@@ -666,7 +678,7 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
             attn_dense_block_n(), CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
             (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
-    return VMLA_ERR_CUDA;
+    return map_fail();
   AttnTc a;
   a.n_q = nq;
   a.n_keys = n_keys;
@@ -737,7 +749,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     a.out_rows = rows;
     a.ring = make_ring(c);
     a.rope = make_rope(c);
-    if ((e = launch_append_simt(a, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+    if ((e = launch_append_simt(a, s)) != cudaSuccess) return cuda_fail(e);
     SimtDenseReconstruct d{cbuf, rbuf, static_cast<const float*>(w_uk), static_cast<const float*>(w_uv),
                            at<float>(h->dense, dense_off), c.batch, rows, c.n_heads, c.d_nope, c.d_rope,
                            c.d_latent, c.d_value, first, make_ring(c), make_rope(c)};
@@ -753,7 +765,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
               CU_TENSOR_MAP_SWIZZLE_128B))
-      return VMLA_ERR_CUDA;
+      return map_fail();
     AppendTc a;
     a.ckv = chunk;
     a.kr = nullptr;
@@ -768,7 +780,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     a.rope = make_rope(c);
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    if ((e = launch_append_tc(tx, tw, a, c.batch, s, plan)) != cudaSuccess) return VMLA_ERR_CUDA;
+    if ((e = launch_append_tc(tx, tw, a, c.batch, s, plan)) != cudaSuccess) return cuda_fail(e);
     CUtensorMap tc, tuk, tuv;
     if (!map3(&tc, chunk, c.d_latent, rows, c.batch, (uint64_t)nout * 2, (uint64_t)rows * nout * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -776,7 +788,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B))
-      return VMLA_ERR_CUDA;
+      return map_fail();
     ReconTc r;
     r.kr = chunk + c.d_latent;  // positional key columns of the chunk rows (row stride d_c + 32)
     r.dense = at<__nv_bfloat16>(h->dense, dense_off);
@@ -795,7 +807,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     r.limit_ns = kWaitLimitNs;
     e = launch_recon_tc(tc, tuk, tuv, r, c.batch, s);
   }
-  if (e != cudaSuccess) return VMLA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   h->dense_frames[layer] = new_F;
   return VMLA_OK;
 }
@@ -822,7 +834,7 @@ vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q,
     StageScope scope(h, 2, s);
     SimtQPrep a{static_cast<const float*>(q), nullptr, at<float>(h->ws, w.dq), c.batch, nq, c.n_heads, c.d_nope,
                 c.d_rope, c.d_latent, 0, first, make_ring(c), make_rope(c)};
-    if ((e = launch_qprep_simt(a, s)) != cudaSuccess) return VMLA_ERR_CUDA;
+    if ((e = launch_qprep_simt(a, s)) != cudaSuccess) return cuda_fail(e);
   }
   StageScope scope(h, 6, s);
   SimtAttn a;
@@ -857,13 +869,14 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   const size_t qb = rows * c.n_heads * (size_t)(c.d_nope + c.d_rope) * esize(c);
   const size_t ob = rows * c.n_heads * (size_t)c.d_value * sizeof(float);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return VMLA_ERR_CUDA;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e);
   if ((st = vmla_cache_append(h, layer, x_dev, w_down, first, n, stream)) != VMLA_OK) return st;
   if ((st = vmla_chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream)) != VMLA_OK)
     return st;
-  return cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s) == cudaSuccess ? VMLA_OK : VMLA_ERR_CUDA;
+  return cuda_status(cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s));
 }
 
 vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
@@ -872,9 +885,10 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
   if (!err) return VMLA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned v = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return VMLA_ERR_CUDA;
-  if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return VMLA_ERR_CUDA;
-  if (v && cudaMemset(err, 0, sizeof(v)) != cudaSuccess) return VMLA_ERR_CUDA;
+  cudaError_t e;
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
+  if (v && (e = cudaMemset(err, 0, sizeof(v))) != cudaSuccess) return cuda_fail(e);
   if (flags) *flags = v;
   if (v & DEV_ERR_BOUNDS_MASK) return VMLA_ERR_DEVICE_BOUNDS;
   if (v) return VMLA_ERR_DEVICE_TIMEOUT;
@@ -887,6 +901,8 @@ vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas) {
   h->append_ctas = max_ctas;
   return VMLA_OK;
 }
+
+const char* vmla_last_error_detail(void) { return g_detail; }
 
 vmla_status vmla_profile_enable(vmla_handle* h, int enable) {
   if (!h) return VMLA_ERR_INVALID_ARG;
@@ -908,6 +924,12 @@ vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* 
   *total_ms = sum;
   *launches = (int)(t.used / 2);
   return VMLA_OK;
+}
+
+vmla_status vmla_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0 || (n & 1) || (reinterpret_cast<uintptr_t>(x) & 7) || (reinterpret_cast<uintptr_t>(y) & 7))
+    return VMLA_ERR_INVALID_ARG;
+  return cuda_status(launch_selftest_exp2(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 
 vmla_status vmla_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

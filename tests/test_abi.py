@@ -215,3 +215,10 @@ def test_append_tiling_arguments():
     assert lib.vmla_cache_append(h2._h, 0, 0x40000, 0x40000, 0, 3, None) == 2
     for x in (h, h2):
         x.close()
+
+
+def test_selftest_exp2_arguments():
+    lib = api.lib()
+    assert lib.vmla_selftest_exp2(0x10000, 0x20000, 3, None) == 1   # odd count
+    assert lib.vmla_selftest_exp2(0x10004, 0x20000, 4, None) == 1   # misaligned
+    assert lib.vmla_selftest_exp2(0, 0x20000, 4, None) == 1         # null

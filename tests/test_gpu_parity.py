@@ -289,6 +289,26 @@ def test_wan_layer_sampled_rows():
     assert_bf16_close(out[0][rows], ref, "wan layer")
 
 
+# ------------------------------------------------------------------ numerics of the kernels' helpers
+
+def test_polynomial_exp2_error_bound():
+    """The FMA-pipe 2^x of the softmax loops against fp64 exp2: relative error
+    within the fitted minimax bound (7.5e-5) for x >= -125, tiny below."""
+    import torch
+    x = np.concatenate([np.linspace(-125.0, 10.0, 1 << 20), np.linspace(-0.5, 0.5, 4096),
+                        np.arange(-125, 11, dtype=np.float64) + 0.5, [-126.0, -200.0, -1e30, -np.inf]])
+    x = x[: len(x) // 2 * 2].astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    api.selftest_exp2(xd, yd)
+    y = yd.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    ok = x >= -125
+    rel = np.abs(y[ok] - ref[ok]) / ref[ok]
+    assert rel.max() <= 7.6e-5, rel.max()
+    assert np.all(np.isfinite(y)) and np.all(y[~ok] >= 0) and np.all(y[~ok] <= 2.0 ** -124)
+
+
 # ------------------------------------------------------------------ failure detection
 
 def test_bounded_wait_times_out_and_reports():
