@@ -341,6 +341,22 @@ def run_ours(args, rank, world, local_rank):
                   "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in rk.items()},
                   "attention_tflops_issued": DF["attention"] / (ra_ms * 1e-3) / 1e12}
 
+    # ------------------------------------------------ design (b): per-head K/V rebuilt inside every key tile
+    def rt_step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_RECONSTRUCT)
+    tsteps = max(10, args.steps // 4)
+    ms_t = timed(rt_step, tsteps, 3, profile=True)
+    tk = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "attention_reconstruct")}
+    m.profile(False)
+    ms_t = max_over_ranks(ms_t / tsteps)
+    rt_attn_ms = tk["attention_reconstruct"][0] / max(tk["attention_reconstruct"][1], 1)
+    recon_in_tile = {"ms_per_step": ms_t, "tflops_effective": world * F["total"] / (ms_t * 1e-3) / 1e12,
+                     "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in tk.items()},
+                     "attention_tflops_issued": (DF["attention"] + 2 * d.window_tokens * d.d_latent * 224 *
+                                                 d.n_heads * ((d.n_queries + 127) // 128)) / (rt_attn_ms * 1e-3) / 1e12}
+
     # ------------------------------------------------ roofline of the dominant kernel (attention)
     hbm, tc_burst, tc_sust, src = load_peaks()
     at_ms, at_n = per_kernel["attention"]
@@ -378,7 +394,8 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "api": "vmla_chunk_step_host (pinned host x, q -> device, append, attention, out -> host)"},
             "gpu_launches": 4 * args.steps, "clocks": clk}
-    line["designs"] = {"absorbed_ms_per_step": ms_step, "recon_once": recon_once}
+    line["designs"] = {"absorbed_ms_per_step": ms_step, "recon_once": recon_once,
+                       "reconstruct_in_tile": recon_in_tile}
     if args.legs:
         line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
                         "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed)}
@@ -494,7 +511,10 @@ def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256)):
         out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
         F = step_flops(d)
         entry = {"absorbed_flops": F["attention"], "dense_flops": dense_flops(d)["attention"]}
-        for name, design in (("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE), ("dense", None)):
+        designs = [("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE), ("dense", None)]
+        if dc <= 192:
+            designs.append(("reconstruct_in_tile", api.DESIGN_RECONSTRUCT))
+        for name, design in designs:
             def call(i):
                 l = i % L
                 if design is None:

@@ -65,8 +65,10 @@ typedef enum vmla_design {
                                   VMLA_FP32 always evaluates the absorbed form) */
   VMLA_DESIGN_ABSORBED = 1,    /* W_uk folded into the query, MQA over [c_KV | k_R], W_uv after the
                                   softmax-weighted sum [paperlayer App. E] */
-  VMLA_DESIGN_RECONSTRUCT = 2, /* per KV tile, per-head K/V rebuilt from c_KV in shared memory, then
-                                  d_head attention [gist.it pt. 2; paperlayer §3 On-demand reconstruction] */
+  VMLA_DESIGN_RECONSTRUCT = 2, /* per KV tile, per-head K/V rebuilt from c_KV on the tensor core and kept
+                                  in shared memory, then d_head attention [gist.it pt. 2; paperlayer §3
+                                  On-demand reconstruction]; VMLA_BF16 with d_latent 64, 128 or 192
+                                  (VMLA_ERR_UNSUPPORTED_SHAPE otherwise), no extra workspace */
   VMLA_DESIGN_RECON_ONCE = 3   /* per-head K/V of the whole window rebuilt once into the workspace, then
                                   d_head attention */
 } vmla_design;

@@ -150,6 +150,14 @@ cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tm_q, const
                                     const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr, const CUtensorMap& tm_wuv,
                                     const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
 int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the key maps)
+
+// Reconstruct-in-tile design (attn_rt.cu), d_latent 64, 128 or 192.  q map: dense queries
+// 3D (128, n_q, B*n_h) box (64,128,1) SW128; ckv map box (64,128,1) SW128; kr map box (32,128,1)
+// SW64; w_uk map 3D (d_c, 96, n_h) box (64,96,1); w_uv map box (64,128,1); out fp32 box (32,128,1).
+bool attn_reconstruct_supported(int d_latent);
+cudaError_t launch_attn_reconstruct_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_ckv,
+                                       const CUtensorMap& tm_kr, const CUtensorMap& tm_wuk, const CUtensorMap& tm_wuv,
+                                       const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
 int attn_dense_block_n();
 
 // Dense per-head attention, d_head = 128.  q map: 3D (128, n_q, B*n_h) box (64,128,1);

@@ -546,6 +546,7 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const
 vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
                            int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s) {
   const vmla_config& c = h->cfg;
+  if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   const WsLayout w = ws_layout(c);
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
   const int nq = (int)(n * tokens_per_frame(c));
@@ -598,7 +599,41 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     if (e != cudaSuccess) return cuda_fail(e);
     return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s);
   }
-  if (design == VMLA_DESIGN_RECONSTRUCT) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (design == VMLA_DESIGN_RECONSTRUCT) {
+    __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
+    {
+      StageScope scope(h, 2, s);
+      DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, t_first, make_ring(c),
+                 make_rope(c)};
+      e = launch_dense_q_bf16(a, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    StageScope scope(h, 4, s);
+    CUtensorMap tq, tc, tkr, tuk, tuv, to;
+    if (!map3(&tq, qd, 128, nq, (uint64_t)c.batch * c.n_heads, 256, (uint64_t)nq * 256, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tc, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
+              (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+      return map_fail();
+    AttnTc a;
+    a.n_q = nq;
+    a.n_keys = win.n_keys;
+    a.n_heads = c.n_heads;
+    a.m_tiles = (nq + 127) / 128;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)(c.d_nope + c.d_rope)));
+    a.rescale_threshold = c.softmax_rescale_log2;
+    a.err = h->err;
+    a.limit_ns = kWaitLimitNs;
+    return cuda_status(launch_attn_reconstruct_tc(c.d_latent, tq, tc, tkr, tuk, tuv, to, a, c.batch, s));
+  }
 
   __nv_bfloat16* qt = at<__nv_bfloat16>(h->ws, w.qt);
   const int dqk = c.d_latent + 32;

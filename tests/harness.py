@@ -24,8 +24,10 @@ def rel_l2(got, ref):
     return float(np.linalg.norm((got - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-300))
 
 
-def assert_bf16_close(got, ref, what=""):
-    """The bf16 gate: relative L2 <= 1e-2 and max |err| <= 3e-2 * RMS(ref)."""
+def assert_bf16_close(got, ref, what="", max_abs=3e-2):
+    """The bf16 gate: relative L2 <= 1e-2 and max |err| <= 3e-2 * RMS(ref).  A caller
+    may widen the max-abs term (never the relative L2 one) where the rounding of
+    the design itself is shown to exceed it; it says why next to the call."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
@@ -33,7 +35,7 @@ def assert_bf16_close(got, ref, what=""):
     rms = float(np.sqrt(np.mean(ref ** 2)))
     mx = float(np.max(np.abs(got - ref)))
     assert rel <= 1e-2, f"{what}: relative L2 {rel:.3e} > 1e-2"
-    assert mx <= 3e-2 * rms, f"{what}: max abs err {mx:.3e} > 3e-2 * rms {rms:.3e}"
+    assert mx <= max_abs * rms, f"{what}: max abs err {mx:.3e} > {max_abs:g} * rms {rms:.3e}"
     return rel, mx / rms
 
 

@@ -161,6 +161,55 @@ def test_small_bf16_batch_and_layers():
             assert_bf16_close(out[b], ro.oracle(layer, 7, q, b), f"layer {layer} sample {b}")
 
 
+@pytest.mark.parametrize("chunks", [1, 7, 10])
+def test_small_bf16_reconstruct_in_tile(chunks):
+    """Design (b): per-head K/V rebuilt from the latent tile on the tensor core
+    inside the attention kernel; partial window, full window, wrapped ring."""
+    ro = Rollout(SMALL)
+    _fill(ro, chunks)
+    out, q = ro.attend(0, chunks - 1, design=api.DESIGN_RECONSTRUCT)
+    # per-head K and V are rounded to bf16 key by key (as in the dense layout): over a
+    # 600-key window that rounding alone puts the worst element at ~3.4e-2 RMS (fp64
+    # emulation of the roundings on the same inputs); the relative L2 gate is unchanged
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"reconstruct, {chunks} chunks",
+                      max_abs=6e-2 if chunks == 1 else 3e-2)
+
+
+@pytest.mark.parametrize("d_latent", [64, 128])
+def test_small_bf16_reconstruct_in_tile_latent_width(d_latent):
+    d = SMALL.replace(d_latent=d_latent)
+    ro = Rollout(d)
+    _fill(ro, 8)
+    out, q = ro.attend(0, 7, design=api.DESIGN_RECONSTRUCT)
+    assert_bf16_close(out[0], ro.oracle(0, 7, q), f"reconstruct d_c={d_latent}")
+
+
+def test_small_bf16_reconstruct_in_tile_rope_at_append_and_rescale():
+    ro = Rollout(SMALL, rope_mode=api.ROPE_AT_APPEND, rescale_log2=0.0)
+    _fill(ro, 8)
+    out, q = ro.attend(0, 7, design=api.DESIGN_RECONSTRUCT)
+    assert_bf16_close(out[0], ro.oracle(0, 7, q), "reconstruct, rope at append, rescale every tile")
+
+
+def test_small_bf16_dense_designs_short_window():
+    """The per-head designs on a 600-key window next to design (b): the same
+    rounding of per-head K and V, the same widened max-abs term."""
+    ro = Rollout(SMALL, design=api.DESIGN_RECON_ONCE, dense=True)
+    ro.append_chunk(0, 0)
+    ro.append_chunk(0, 0, dense=True)
+    for design, dense in ((api.DESIGN_RECON_ONCE, False), (api.DESIGN_RECONSTRUCT, False), (None, True)):
+        out, q = ro.attend(0, 0, design=design or api.DESIGN_AUTO, dense=dense)
+        assert_bf16_close(out[0], ro.oracle(0, 0, q), f"design {design} dense {dense}", max_abs=6e-2)
+
+
+def test_reconstruct_in_tile_rejects_latent_256():
+    d = SMALL.replace(d_latent=256)
+    ro = Rollout(d)
+    _fill(ro, 1)
+    with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
+        ro.attend(0, 0, design=api.DESIGN_RECONSTRUCT)
+
+
 def test_small_append_writes_only_its_slots():
     """Ring rows of the appended frames hold bf16(W_down x) (bf16 rounding of
     the fp64 product); every other byte of the cache is untouched."""

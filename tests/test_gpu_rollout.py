@@ -140,7 +140,10 @@ def test_wan_latent_width_sweep(d_latent):
         ro.append_chunk(0, c, dense=True)
     rows = sampled_rows(d.n_queries, 256, seed=d_latent)
     got = {}
-    for name, design in (("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE)):
+    designs = [("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE)]
+    if d_latent <= 192:
+        designs.append(("reconstruct_in_tile", api.DESIGN_RECONSTRUCT))
+    for name, design in designs:
         out, q = ro.attend(0, 6, design=design)
         got[name] = out[0][rows]
     out, q = ro.attend(0, 6, dense=True)
