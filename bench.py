@@ -482,7 +482,7 @@ def batch8_leg(m_timed, dev, hbm, tc, seed):
     return res
 
 
-def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256)):
+def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384)):
     """Latent width sweep on the Wan layer: attention time of every built design
     and of the dense per-head cache for the same seeded x and q."""
     import torch
@@ -511,7 +511,9 @@ def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256)):
         out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
         F = step_flops(d)
         entry = {"absorbed_flops": F["attention"], "dense_flops": dense_flops(d)["attention"]}
-        designs = [("absorbed", api.DESIGN_ABSORBED), ("recon_once", api.DESIGN_RECON_ONCE), ("dense", None)]
+        designs = [("recon_once", api.DESIGN_RECON_ONCE), ("dense", None)]
+        if dc <= 256:
+            designs.append(("absorbed", api.DESIGN_ABSORBED))
         if dc <= 192:
             designs.append(("reconstruct_in_tile", api.DESIGN_RECONSTRUCT))
         for name, design in designs:

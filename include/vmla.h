@@ -125,8 +125,9 @@ vmla_status vmla_config_init(vmla_config* cfg);
 
 /* VMLA_OK when every field is consistent and a kernel exists for it:
  * VMLA_FP32 accepts any positive sizes (d_latent, d_nope+d_rope, d_value <= 512);
- * VMLA_BF16 needs d_nope + d_rope = d_value = 128, d_rope = 32 and d_latent a multiple of 64 in
- * [64, 384].  grid_h, grid_w, window_frames must be < 1024 (RoPE range, [paperlayer App. C.1]). */
+ * VMLA_BF16 needs d_nope + d_rope = d_value = 128, d_rope = 32 and d_latent one of 64, 128,
+ * 192, 256, 384 (VMLA_DESIGN_ABSORBED up to 256, VMLA_DESIGN_RECONSTRUCT up to 192).
+ * grid_h, grid_w, window_frames must be < 1024 (RoPE range, [paperlayer App. C.1]). */
 vmla_status vmla_config_check(const vmla_config* cfg);
 
 /* Bytes of the caller-allocated caches of one handle (all layers and samples):

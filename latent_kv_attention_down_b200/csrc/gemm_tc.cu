@@ -36,6 +36,15 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
+// 32 floats as bf16 into 64 bytes of shared memory (16-byte aligned)
+__device__ __forceinline__ void store_bf16x32_smem(uint8_t* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -365,97 +374,183 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================== per-head reconstruction
+// Persistent over (sample, 128-row tile, head) items, head fastest so that the
+// CTAs working at one time share the latent tile in L2.  Per item the
+// reduction over d_latent runs through a ring of [128 rows x 64] latent blocks
+// and [224 x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
+// two TMEM accumulators alternate so the epilogue of one item overlaps the
+// next; the epilogue parks 64 rows at a time as [k_h (128) | v_h (128)] bf16
+// and writes each row's two 256-byte runs out contiguously.
 template <int DL>
 struct ReconCfg {
   static constexpr int NKB = DL / 64;
   static constexpr int A_BLK = 128 * 128;  // 128 latent rows x 64 cols
   static constexpr int B_BLK = 224 * 128;  // [96 rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr int SMEM = 1024 + NKB * (A_BLK + B_BLK) + 256;
+  static constexpr int STAGE = A_BLK + B_BLK;
+  static constexpr int OUT_STRIDE = 256 * 2 + 16;  // parked row [k_h | v_h]: an odd number of 16-byte chunks
+  static constexpr int OUT_BYTES = 64 * OUT_STRIDE;
+  static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
+  static constexpr int STAGES = FIT > 6 ? 6 : FIT;
+  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of 224 columns, at 0 and 256
+  static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 128 * 8 + 256;
+  static_assert(DL % 64 == 0 && STAGES >= 3 && SMEM <= 227 * 1024 && SMEM > 116 * 1024, "does not fit");
 };
 
 template <int DL>
 __global__ void __launch_bounds__(kThreads, 1)
     recon_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wuk,
-                    const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a) {
+                    const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a, int items) {
   using C = ReconCfg<DL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + C::NKB * C::A_BLK;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::NKB * C::B_BLK);
-  uint64_t* done = full + 1;
+  uint8_t* sout = smem + C::STAGES * C::STAGE;
+  int64_t* row_k = reinterpret_cast<int64_t*>(sout + C::OUT_BYTES);  // element offset of each row's k_h
+  uint64_t* full = reinterpret_cast<uint64_t*>(row_k + 128);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const int m_tiles = (a.rows + 127) / 128;
   const Guard g{abort_flag, a.err, a.limit_ns};
-  const uint32_t tbase = setup_cta(full, 2, tslot, abort_flag, C::TMEM_COLS);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 4);  // one arrival per epilogue warp
+    mbar_init(&acc_empty[1], 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(full, C::NKB * (C::A_BLK + C::B_BLK));
-      for (int kb = 0; kb < C::NKB; ++kb) {
-        tma_load_3d(sA + kb * C::A_BLK, &tm_c, full, kb * 64, m0, b);
-        tma_load_3d(sB + kb * C::B_BLK, &tm_wuk, full, kb * 64, 0, h);
-        tma_load_3d(sB + kb * C::B_BLK + 96 * 128, &tm_wuv, full, kb * 64, 0, h);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
-      tc_fence_after();
-      if (ok) {
-        constexpr uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
-        const uint64_t ad = smem_desc(smem_u32(sA), 16, 1024, LAYOUT_SW128);
-        const uint64_t bd = smem_desc(smem_u32(sB), 16, 1024, LAYOUT_SW128);
-#pragma unroll
-        for (int kk = 0; kk < DL / 16; ++kk) {
-          const uint64_t a = desc_add(ad, (kk / 4) * C::A_BLK + (kk % 4) * 32);
-          const uint64_t b = desc_add(bd, (kk / 4) * C::B_BLK + (kk % 4) * 32);
-          if (kk == 0)
-            mma_ss_c<false>(tbase, a, b, idesc);
-          else
-            mma_ss_c<true>(tbase, a, b, idesc);
+      prefetch_tmap(&tm_c);
+      prefetch_tmap(&tm_wuk);
+      prefetch_tmap(&tm_wuv);
+      int it = 0;
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+        const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+        for (int kb = 0; kb < C::NKB; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          uint8_t* st = smem + s * C::STAGE;
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          tma_load_3d(st, &tm_c, &full[s], kb * 64, mt * 128, b);
+          tma_load_3d(st + C::A_BLK, &tm_wuk, &full[s], kb * 64, 0, h);
+          tma_load_3d(st + C::A_BLK + 96 * 128, &tm_wuv, &full[s], kb * 64, 0, h);
         }
       }
+      if (*abort_flag)
+        for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+          drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
+      int it = 0, j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        const int acc = j & 1;
+        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < C::NKB; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!(ok = wait_phase(&full[s], (it / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::STAGE);
+          const uint64_t ad = smem_desc(st, 16, 1024, LAYOUT_SW128);
+          const uint64_t bd = smem_desc(st + C::A_BLK, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (k == 0 && kb == 0)
+              mma_ss_c<false>(tbase + acc * 256, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+            else
+              mma_ss_c<true>(tbase + acc * 256, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+      }
       mma_commit(done);
-      if (*abort_flag) {
-        drain_phase(done, 0, g);
-        drain_phase(full, 0, g);
+      if (*abort_flag) drain_phase(done, 0, g);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int T = a.ring.tokens_per_frame;
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+      const int acc = j & 1;
+      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      __syncwarp();
+      tc_fence_after();
+      const int m = mt * 128 + r;
+      const bool valid = ok && m < a.rows;
+      const int mm = m < a.rows ? m : 0;
+      const int64_t frame = a.first_frame + mm / T;
+      const int tok = mm % T;
+      const int64_t row = a.to_ring ? (frame % a.ring.window_frames) * T + tok : mm;
+      row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
+      float kr[32];
+      if (valid) {
+        load_bf16x32(a.kr + ((int64_t)b * a.kr_rows + mm) * a.kr_stride, kr);
+        if (a.rotate) rotate16(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) kr[i] = 0.f;
+      }
+      named_bar_sync(1, 128);  // row table complete
+      const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        if ((wq >> 1) == half) {  // warps of this half hold TMEM lanes 64*half .. 64*half + 63
+          uint8_t* orow = sout + (r - 64 * half) * C::OUT_STRIDE;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 224; c0 += 32) {
+            uint32_t raw[32];
+            tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            float v[32];
+            raw_to_float(raw, v);
+            // TMEM columns 0..95 are k_h's content part, 96..223 are v_h (parked from column 128)
+            store_bf16x32_smem(orow + (c0 < 96 ? c0 : c0 + 32) * 2, v);
+          }
+          store_bf16x32_smem(orow + 96 * 2, kr);  // positional part of k_h
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
+        }
+        named_bar_sync(1, 128);  // this half is parked
+        const int rows_h = min(64, valid_rows - 64 * half);
+#pragma unroll 4
+        for (int id = tid; id < rows_h * 32; id += 128) {
+          const int rr = id >> 5, ch = id & 31;
+          __nv_bfloat16* dst =
+              a.dense + row_k[64 * half + rr] + (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
+        }
+        named_bar_sync(1, 128);  // the parked half is written out before it is reused
       }
     }
-  } else if (warp >= 4) {
-    const int wq = warp - 4;
-    const int m = m0 + wq * 32 + lane;
-    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
-    __syncwarp();
-    tc_fence_after();
-    const bool valid = ok && m < a.rows;
-    const int mm = valid ? m : 0;
-    const int T = a.ring.tokens_per_frame;
-    const int64_t frame = a.first_frame + mm / T;
-    const int tok = mm % T;
-    const int64_t row = a.to_ring ? (frame % a.ring.window_frames) * T + tok : mm;
-    __nv_bfloat16* kd = a.dense + (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
-    __nv_bfloat16* vd = kd + (int64_t)a.n_heads * 128;
-#pragma unroll 1
-    for (int c0 = 0; c0 < 224; c0 += 32) {
-      uint32_t raw[32];
-      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
-      if (!valid) continue;
-      float v[32];
-      raw_to_float(raw, v);
-      store_bf16x32(c0 < 96 ? kd + c0 : vd + (c0 - 96), v);
-    }
-    if (valid) {
-      float v[32];
-      load_bf16x32(a.kr + ((int64_t)b * a.kr_rows + mm) * a.kr_stride, v);
-      if (a.rotate) rotate16(v, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
-      store_bf16x32(kd + 96, v);
-    }
   }
-  teardown_cta(tbase, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
 }
 
 template <class K>
@@ -506,7 +601,14 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
   using C = ReconCfg<DL>;
   static const cudaError_t attr = set_smem(recon_tc_kernel<DL>, C::SMEM);
   if (attr != cudaSuccess) return attr;
-  recon_tc_kernel<DL><<<dim3((a.rows + 127) / 128, a.n_heads, batch), kThreads, C::SMEM, s>>>(tc, tuk, tuv, a);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((a.rows + 127) / 128) * a.n_heads * batch;
+  recon_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tuk, tuv, a, items);
   return cudaGetLastError();
 }
 
@@ -531,6 +633,7 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
     case 128: return go_append<160>(tx, tw, a, batch, s, p);
     case 192: return go_append<224>(tx, tw, a, batch, s, p);
     case 256: return go_append<288>(tx, tw, a, batch, s, p);
+    case 384: return go_append<416>(tx, tw, a, batch, s, p);
   }
   return cudaErrorInvalidValue;
 }
@@ -555,6 +658,7 @@ cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const
     case 128: return go_recon<128>(tc, tuk, tuv, a, batch, s);
     case 192: return go_recon<192>(tc, tuk, tuv, a, batch, s);
     case 256: return go_recon<256>(tc, tuk, tuv, a, batch, s);
+    case 384: return go_recon<384>(tc, tuk, tuv, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -84,6 +84,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   if (!aligned16(ckv) || !aligned16(kr) || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
   const int64_t F = frames_appended;
+  if (c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;  // absorbed kernels: up to 256 latent dims
   if (n_frames < 1 || n_frames > c.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
   if (F < 1 || first_frame < 0 || first_frame + n_frames != F) return VMLA_ERR_STATE;
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;

@@ -310,7 +310,8 @@ vmla_status vmla_config_check(const vmla_config* c) {
   if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c->dtype == VMLA_BF16) {
     if (c->d_rope != 32 || c->d_nope != 96 || c->d_value != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
-    if (c->d_latent % 64 != 0 || c->d_latent < 64 || c->d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (!(c->d_latent == 64 || c->d_latent == 128 || c->d_latent == 192 || c->d_latent == 256 || c->d_latent == 384))
+      return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (c->d_model % 64 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
   } else {
     if (c->d_latent + c->d_rope > 1024 || c->d_value > 1024) return VMLA_ERR_UNSUPPORTED_SHAPE;
@@ -742,6 +743,9 @@ vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const
   if ((st = ensure_err(h)) != VMLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   design = resolve_design(h->cfg, design);
+  // the absorbed kernels keep d_latent + 32 query and key columns resident: up to 256 latent dims
+  if (h->cfg.dtype == VMLA_BF16 && design == VMLA_DESIGN_ABSORBED && h->cfg.d_latent > 256)
+    return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
   return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s);
 }

@@ -222,3 +222,10 @@ def test_selftest_exp2_arguments():
     assert lib.vmla_selftest_exp2(0x10000, 0x20000, 3, None) == 1   # odd count
     assert lib.vmla_selftest_exp2(0x10004, 0x20000, 4, None) == 1   # misaligned
     assert lib.vmla_selftest_exp2(0, 0x20000, 4, None) == 1         # null
+
+
+@pytest.mark.parametrize("d_latent,status", [(64, 0), (128, 0), (192, 0), (256, 0), (384, 0), (320, 2), (448, 2), (32, 2)])
+def test_latent_widths_with_kernels(d_latent, status):
+    c = default_config()
+    c.d_latent = d_latent
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == status

@@ -123,7 +123,7 @@ def test_small_bf16_reconstruct_once():
     assert_bf16_close(out[0], ro.oracle(0, 7, q), "reconstruct once")
 
 
-@pytest.mark.parametrize("d_latent", [64, 128, 256])
+@pytest.mark.parametrize("d_latent", [64, 128, 256, 384])
 def test_small_bf16_latent_width(d_latent):
     """The design AUTO picks (absorbed up to 192, reconstruct-once above) at the gate."""
     ro = Rollout(SMALL.replace(name=f"small_dc{d_latent}", d_latent=d_latent))
@@ -200,6 +200,14 @@ def test_small_bf16_dense_designs_short_window():
     for design, dense in ((api.DESIGN_RECON_ONCE, False), (api.DESIGN_RECONSTRUCT, False), (None, True)):
         out, q = ro.attend(0, 0, design=design or api.DESIGN_AUTO, dense=dense)
         assert_bf16_close(out[0], ro.oracle(0, 0, q), f"design {design} dense {dense}", max_abs=6e-2)
+
+
+def test_absorbed_rejects_latent_384():
+    d = SMALL.replace(d_latent=384)
+    ro = Rollout(d)
+    _fill(ro, 1)
+    with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
+        ro.attend(0, 0, design=api.DESIGN_ABSORBED)
 
 
 def test_reconstruct_in_tile_rejects_latent_256():
