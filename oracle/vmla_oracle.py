@@ -74,10 +74,35 @@ def window_frame_range(frames_appended: int, window_frames: int) -> tuple[int, i
     return max(0, frames_appended - window_frames), frames_appended
 
 
-def ring_slot(frame: int, window_frames: int) -> int:
-    """Ring slot of a frame in a cache of ``window_frames`` frames: the slot
-    that the frame evicted when it arrived (the oldest one)."""
-    return frame % window_frames
+def window_frames_list(frames_appended: int, window_frames: int, sink_frames: int = 0) -> list[int]:
+    """Frames in the active context after ``frames_appended`` frames, in cache
+    order: the ``sink_frames`` first frames of the rollout stay for good, the
+    other ``window_frames - sink_frames`` slots hold the newest frames, the
+    oldest evicted first [paperlayer App. D.4: one sink latent frame and the
+    six most recent latent frames, FIFO eviction outside the sink]."""
+    F, S, W = frames_appended, sink_frames, window_frames
+    sink = list(range(min(S, F)))
+    local_start = max(S, F - (W - S))
+    return sink + list(range(local_start, F))
+
+
+def window_frame_t(frames_appended: int, window_frames: int, sink_frames: int = 0) -> dict:
+    """Window-relative temporal coordinate of every frame of the active context
+    [paperlayer App. D.5: cached positional keys get local temporal coordinates
+    in the sink-plus-window context]: the sink frames keep 0..S-1, the local
+    frames follow them in order, S, S+1, ... -- so t never exceeds
+    window_frames - 1 however long the rollout."""
+    frames = window_frames_list(frames_appended, window_frames, sink_frames)
+    return {f: t for t, f in enumerate(frames)}
+
+
+def ring_slot(frame: int, window_frames: int, sink_frames: int = 0) -> int:
+    """Ring slot of a frame in a cache of ``window_frames`` frames: a sink frame
+    keeps its own slot, any other frame takes the slot of the local frame it
+    evicts (the oldest one)."""
+    if frame < sink_frames:
+        return frame
+    return sink_frames + (frame - sink_frames) % (window_frames - sink_frames)
 
 
 def token_grid_position(token: np.ndarray | int, grid_w: int):
@@ -258,19 +283,28 @@ def dense_cache_entries(c, r, key_pos, w_uk, w_uv, *, rope_pairs, rope_theta=100
 
 
 def window_latents(frame_x: dict, frames_appended: int, window_frames: int, w_down, d_latent,
-                   grid_h: int, grid_w: int, rope_at: str = "read"):
-    """Latents of the window after ``frames_appended`` frames, oldest frame first.
+                   grid_h: int, grid_w: int, rope_at: str = "read", sink_frames: int = 0):
+    """Latents of the active context after ``frames_appended`` frames: the sink
+    frames, then the local frames oldest first.
 
     frame_x maps a frame index to the x rows [tokens_per_frame, d_model] it
-    was last appended with.  rope_at="read" numbers the window's frames from
-    0 (window-relative, [paperlayer App. D.5]); "append" keeps the absolute
-    frame index.  Returns (c, r, key_pos, t_origin)."""
-    start, end = window_frame_range(frames_appended, window_frames)
-    frames = list(range(start, end))
+    was last appended with.  rope_at="read" gives every frame its
+    window-relative t ([paperlayer App. D.5], ``window_frame_t``); "append"
+    keeps the absolute frame index.  Returns (c, r, key_pos, t_origin), where
+    a local frame f has t = f - t_origin (the chunk's queries use it)."""
+    frames = window_frames_list(frames_appended, window_frames, sink_frames)
     x = np.concatenate([np.asarray(frame_x[f], dtype=np.float64) for f in frames], axis=0)
     c, r = down_project(x, w_down, d_latent)
-    t_origin = start if rope_at == "read" else 0
-    return c, r, key_positions(frames, t_origin, grid_h, grid_w), t_origin
+    if rope_at == "read":
+        t_of = window_frame_t(frames_appended, window_frames, sink_frames)
+        t_origin = frames[-1] - t_of[frames[-1]]
+    else:
+        t_of = {f: f for f in frames}
+        t_origin = 0
+    tok = np.arange(grid_h * grid_w)
+    hh, ww = token_grid_position(tok, grid_w)
+    pos = np.concatenate([np.stack([np.full_like(tok, t_of[f]), hh, ww], axis=1) for f in frames], axis=0)
+    return c, r, pos.astype(np.int64), t_origin
 
 
 def chunk_query_positions(first_frame: int, n_frames: int, t_origin: int, grid_h: int, grid_w: int):

@@ -381,3 +381,63 @@ def test_planted_mistake_is_caught(name, golden):
 
 def test_unmutated_passes_all(golden):
     _all_checks(_mutant(), golden)
+
+
+# ---------------------------------------------------------------- sink frame + local window
+def _simulate_sink_ring(n_frames, W, S):
+    """An explicit slot array: sink frames take their own slot; a later frame takes
+    the first never-used local slot, else the slot of the oldest local frame."""
+    slots = [None] * W
+    states = []
+    for f in range(n_frames):
+        if f < S:
+            s = f
+        else:
+            free = [k for k in range(S, W) if slots[k] is None]
+            s = free[0] if free else min(range(S, W), key=lambda k: slots[k])
+        slots[s] = f
+        states.append(list(slots))
+    return states
+
+
+@pytest.mark.parametrize("W,S", [(7, 1), (4, 1), (5, 2), (21, 0)])
+def test_sink_window_matches_an_explicit_slot_array(W, S):
+    states = _simulate_sink_ring(60, W, S)
+    for F in range(1, 61):
+        slots = states[F - 1]
+        frames = O.window_frames_list(F, W, S)
+        assert sorted(frames) == sorted(f for f in slots if f is not None)
+        for k, f in enumerate(slots):
+            if f is not None:
+                assert O.ring_slot(f, W, S) == k
+        # sink first, locals oldest first, window-relative t = position in that order
+        t = O.window_frame_t(F, W, S)
+        sink = [f for f in frames if f < S]
+        local = [f for f in frames if f >= S]
+        assert frames == sink + sorted(local)
+        assert [t[f] for f in frames] == list(range(len(frames)))
+        if S == 0:
+            assert frames == list(range(*O.window_frame_range(F, W)))
+
+
+def test_sink_window_keeps_rope_positions_bounded():
+    """One sink frame and a six-frame local window [paperlayer App. D.4, D.5]: after
+    1000 frames the temporal coordinates are still 0..6 and the sink is frame 0."""
+    frames = O.window_frames_list(1000, 7, 1)
+    t = O.window_frame_t(1000, 7, 1)
+    assert frames == [0] + list(range(994, 1000))
+    assert sorted(t.values()) == list(range(7)) and t[0] == 0 and t[999] == 6
+
+
+def test_sink_window_latents_positions():
+    rng = np.random.default_rng(3)
+    T, D, dc = 6, 8, 4
+    frame_x = {f: rng.standard_normal((T, D)) for f in range(12)}
+    w = rng.standard_normal((dc + 2, D))
+    c, r, pos, t0 = O.window_latents(frame_x, 12, 4, w, dc, 2, 3, sink_frames=1)
+    assert c.shape == (4 * T, dc)
+    np.testing.assert_allclose(c[:T], frame_x[0] @ w[:dc].T)     # the sink's rows come first
+    np.testing.assert_allclose(c[T:2 * T], frame_x[9] @ w[:dc].T)
+    assert list(pos[::T, 0]) == [0, 1, 2, 3] and t0 == 8         # frames 9, 10, 11 at t = 1, 2, 3
+    q = O.chunk_query_positions(11, 1, t0, 2, 3)
+    assert q[0, 0] == 3
