@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define VMLA_ABI_VERSION 1
+#define VMLA_ABI_VERSION 2
 
 typedef enum vmla_status {
   VMLA_OK = 0,
@@ -92,7 +92,7 @@ typedef struct vmla_config {
   int rope_base_dims[3]; /* B_a in w_{a,i} = theta^(-2i/B_a); 0 means 2*rope_pairs[a] */
   float rope_theta;      /* 10000 */
   int grid_h, grid_w;    /* latent frame grid; tokens per frame T_f = grid_h*grid_w (30 x 52 = 1560) */
-  int window_frames;     /* W: ring capacity in frames, current chunk included (21) */
+  int window_frames;     /* W: ring capacity in frames, sink and current chunk included (21; 7 with a sink) */
   int chunk_frames;      /* largest n_frames of an attention call (3) */
   int batch;             /* independent rings (one per sample) */
   int layers;            /* layers held by one handle's caches */
@@ -102,6 +102,12 @@ typedef struct vmla_config {
                                  max exceeds it by more than 2^this (8 by default); 0 raises it on
                                  every increase.  Results are the same; only the amount of O
                                  rescaling work differs. */
+  int sink_frames;       /* S: the first S frames of a rollout stay in the ring for good (slots 0..S-1);
+                            later frames rotate FIFO through the other W-S slots.  Keys take
+                            window-relative t: the sink 0..S-1, the local frames S.. in order
+                            [paperlayer App. D.4: one sink latent frame + six recent ones; App. D.5
+                            re-indexing].  0 (default): plain FIFO window.  Needs rope_mode
+                            VMLA_ROPE_AT_READ and chunk_frames <= W-S; no dense cache. */
 } vmla_config;
 
 typedef struct vmla_handle vmla_handle;

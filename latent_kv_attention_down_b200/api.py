@@ -23,12 +23,15 @@ STAGES = {"append": 0, "rope": 1, "q_absorb": 2, "attention": 3, "attention_reco
           "dense_append": 5, "dense_attention": 6, "reconstruct_once": 7}
 
 
+ABI_VERSION = 2  # VMLA_ABI_VERSION of include/vmla.h that this binding's structures follow
+
+
 class Config(ctypes.Structure):
     _fields_ = [("d_model", c_int), ("n_heads", c_int), ("d_nope", c_int), ("d_rope", c_int),
                 ("d_latent", c_int), ("d_value", c_int), ("rope_pairs", c_int * 3), ("rope_base_dims", c_int * 3),
                 ("rope_theta", c_float), ("grid_h", c_int), ("grid_w", c_int), ("window_frames", c_int),
                 ("chunk_frames", c_int), ("batch", c_int), ("layers", c_int), ("dtype", c_int),
-                ("rope_mode", c_int), ("softmax_rescale_log2", c_float)]
+                ("rope_mode", c_int), ("softmax_rescale_log2", c_float), ("sink_frames", c_int)]
 
 
 class VmlaError(RuntimeError):
@@ -90,6 +93,9 @@ def lib() -> ctypes.CDLL:
             fn = getattr(handle, name)
             fn.restype = res
             fn.argtypes = args
+        if handle.vmla_abi_version() != ABI_VERSION:
+            raise RuntimeError(f"{LIB_PATH} has ABI version {handle.vmla_abi_version()}, this binding needs "
+                               f"{ABI_VERSION}: rebuild it")
         _LIB = handle
     return _LIB
 
@@ -113,6 +119,7 @@ def config_from_dims(dims, layers: int = 1, rope_mode: int = ROPE_AT_READ) -> Co
     c.dtype = BF16 if dims.dtype == "bf16" else FP32
     c.rope_mode = rope_mode
     c.softmax_rescale_log2 = 8.0
+    c.sink_frames = dims.sink_frames
     return c
 
 

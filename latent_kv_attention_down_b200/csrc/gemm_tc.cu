@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + 32);
         row_pos[r] = row_lat[r] + a.d_latent;
       } else {
-        const int64_t rr = (int64_t)b * a.ring_rows + (frame % a.ring.window_frames) * T + tok;
+        const int64_t rr = (int64_t)b * a.ring_rows + ring_frame_slot(a.ring, frame) * T + tok;
         row_lat[r] = rr * a.d_latent;
         row_pos[r] = rr * 32;
       }
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mm = m < a.rows ? m : 0;
       const int64_t frame = a.first_frame + mm / T;
       const int tok = mm % T;
-      const int64_t row = a.to_ring ? (frame % a.ring.window_frames) * T + tok : mm;
+      const int64_t row = a.to_ring ? ring_frame_slot(a.ring, frame) * T + tok : mm;
       row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
       float kr[32];
       if (valid) {

@@ -31,8 +31,22 @@ struct Rope {
 struct Ring {
   int tokens_per_frame;  // T_f
   int grid_w;
-  int window_frames;     // W
+  int window_frames;     // W, sink included
+  int sink_frames;       // S: frames 0..S-1 keep slots 0..S-1; later frames rotate through S..W-1
 };
+
+// Ring slot of frame f: a sink frame keeps its own slot, any other frame takes the slot
+// of the local frame it evicts (the oldest) [paperlayer App. D.4].
+__host__ __device__ inline int64_t ring_frame_slot(const Ring& g, int64_t f) {
+  return f < g.sink_frames ? f : g.sink_frames + (f - g.sink_frames) % (g.window_frames - g.sink_frames);
+}
+// Window-relative t of the keys in ring slot `slot` [paperlayer App. D.5]: sink slots keep
+// t = slot; local slots count from the oldest local frame, whose slot is S + local_start_slot.
+__host__ __device__ inline int ring_slot_t(const Ring& g, int slot, int local_start_slot) {
+  if (slot < g.sink_frames) return slot;
+  const int L = g.window_frames - g.sink_frames;
+  return g.sink_frames + (slot - g.sink_frames - local_start_slot + L) % L;
+}
 
 // ------------------------------------------------------------------ fp32 SIMT path (any shape)
 struct SimtAppend {
@@ -54,7 +68,7 @@ struct RopeWindow {  // rotate the window's positional keys with window-relative
   const void* kr;    // [B][W*T_f][d_r]
   void* kr_rot;      // [B][W*T_f][d_r]
   int batch, n_keys, d_rope;
-  int window_start_slot;  // ring frame slot of the oldest window frame
+  int window_start_slot;  // (ring slot of the oldest local frame) - sink_frames
   Ring ring;
   Rope rope;
 };

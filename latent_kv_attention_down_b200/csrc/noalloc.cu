@@ -92,8 +92,12 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
 
   const int64_t T = (int64_t)c.grid_h * c.grid_w;
   const int64_t rr = (int64_t)c.window_frames * T;
-  const int64_t start = F > c.window_frames ? F - c.window_frames : 0;
-  const int n_keys = (int)((F - start) * T);
+  // active context [paperlayer App. D.4, D.5]: sink frames, then the newest W - S frames
+  const int64_t S = c.sink_frames, L = c.window_frames - c.sink_frames;
+  const bool full = F > c.window_frames;
+  const int64_t t_origin = full ? F - L - S : 0;
+  const int start_slot = full ? (int)((F - L - S) % L) : 0;
+  const int n_keys = (int)((full ? c.window_frames : F) * T);
   const int nq = (int)(n_frames * T);
   const int dqk = c.d_latent + 32;
   const size_t kr_rot_bytes = at_read ? align256((size_t)c.batch * rr * 32 * 2) : 0;
@@ -115,7 +119,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   rope.n_t = c.rope_pairs[0];
   rope.n_h = c.rope_pairs[1];
   rope.n_w = c.rope_pairs[2];
-  const Ring ring{(int)T, c.grid_w, c.window_frames};
+  const Ring ring{(int)T, c.grid_w, c.window_frames, c.sink_frames};
 
   const size_t layer_rows = (size_t)layer * c.batch * rr;
   const __nv_bfloat16* ckv_layer = static_cast<const __nv_bfloat16*>(ckv) + layer_rows * c.d_latent;
@@ -125,7 +129,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
 
   const __nv_bfloat16* kpos = kr_layer;
   if (at_read) {
-    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, 32, (int)(start % c.window_frames), ring, rope};
+    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, 32, start_slot, ring, rope};
     if (launch_rope_window_bf16(r, s) != cudaSuccess) return VMLA_ERR_CUDA;
     kpos = kr_rot;
   }
@@ -143,7 +147,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   qa.n_q = nq;
   qa.n_heads = c.n_heads;
   qa.d_latent = c.d_latent;
-  qa.t_first = first_frame - (at_read ? start : 0);
+  qa.t_first = first_frame - (at_read ? t_origin : 0);
   qa.ring = ring;
   qa.rope = rope;
   qa.err = err;

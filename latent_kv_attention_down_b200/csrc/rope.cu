@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   const int b = (idx >> 2) / a.n_keys;
   const int64_t ring_rows = (int64_t)a.ring.window_frames * a.ring.tokens_per_frame;
   const int fslot = s / a.ring.tokens_per_frame, tok = s % a.ring.tokens_per_frame;
-  const int t = (fslot - a.window_start_slot + a.ring.window_frames) % a.ring.window_frames;
+  const int t = ring_slot_t(a.ring, fslot, a.window_start_slot);
   const int64_t off = ((int64_t)b * ring_rows + s) * 32 + quad * 8;
   const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + off);
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + off) =

@@ -10,7 +10,7 @@ namespace {
 // Row m of a call (frames first_frame ..) -> ring row of its sample.
 __device__ __forceinline__ int64_t ring_row(const Ring& g, int64_t first_frame, int m) {
   const int64_t f = first_frame + m / g.tokens_per_frame;
-  return (f % g.window_frames) * g.tokens_per_frame + (m % g.tokens_per_frame);
+  return ring_frame_slot(g, f) * g.tokens_per_frame + (m % g.tokens_per_frame);
 }
 
 // ---- append: [c | k_R] = W_down x
@@ -61,7 +61,7 @@ __global__ void rope_window_f32_kernel(const RopeWindow a) {
   const int b = idx / ((int64_t)n_pairs * a.n_keys);
   const int64_t ring_rows = (int64_t)a.ring.window_frames * a.ring.tokens_per_frame;
   const int fslot = s / a.ring.tokens_per_frame, tok = s % a.ring.tokens_per_frame;
-  const int t = (fslot - a.window_start_slot + a.ring.window_frames) % a.ring.window_frames;
+  const int t = ring_slot_t(a.ring, fslot, a.window_start_slot);
   const float* src = static_cast<const float*>(a.kr) + ((int64_t)b * ring_rows + s) * a.d_rope + 2 * p;
   float* dst = static_cast<float*>(a.kr_rot) + ((int64_t)b * ring_rows + s) * a.d_rope + 2 * p;
   float u = src[0], v = src[1];

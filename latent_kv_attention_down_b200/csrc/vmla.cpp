@@ -1,9 +1,10 @@
 // Host side of libvmla.so: the C ABI declared in include/vmla.h.
 //
 // Validates every call, keeps the per-layer frame counters of the sliding
-// window (FIFO ring of window_frames frames, slot = frame mod W [paperlayer
-// App. D.4]), encodes the TMA tensor maps of each launch and enqueues the
-// kernels on the caller's stream.  It allocates no device memory.
+// window (a ring of window_frames frames: the first sink_frames frames keep
+// their slots, later ones rotate FIFO through the rest [paperlayer App. D.4]),
+// encodes the TMA tensor maps of each launch and enqueues the kernels on the
+// caller's stream.  It allocates no device memory.
 #include "vmla.h"
 
 #include <cuda.h>
@@ -76,7 +77,9 @@ bool append_tiling_fits(const vmla_config& c, int n_split) {
   return n_split != 1 || c.d_latent + 32 <= 256;
 }
 
-Ring make_ring(const vmla_config& c) { return Ring{(int)tokens_per_frame(c), c.grid_w, c.window_frames}; }
+Ring make_ring(const vmla_config& c) {
+  return Ring{(int)tokens_per_frame(c), c.grid_w, c.window_frames, c.sink_frames};
+}
 
 // ---------------------------------------------------------------- TMA tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -211,7 +214,8 @@ vmla_status check_layer(const vmla_handle* h, int layer) {
 // Frame rule of an append: a new chunk right after the newest frame, or a
 // rewrite of the newest frames (a further denoising pass).
 vmla_status check_append_frames(const vmla_config& c, int64_t F, int64_t first, int n, int64_t* new_F) {
-  if (n < 1 || n > c.window_frames) return VMLA_ERR_OUT_OF_RANGE;
+  // one append never wraps onto its own frames: at most the ring's local part
+  if (n < 1 || n > c.window_frames - c.sink_frames) return VMLA_ERR_OUT_OF_RANGE;
   if (first < 0) return VMLA_ERR_STATE;
   if (first == F)
     *new_F = F + n;
@@ -222,18 +226,36 @@ vmla_status check_append_frames(const vmla_config& c, int64_t F, int64_t first, 
   return VMLA_OK;
 }
 
+// The active context after F frames [paperlayer App. D.4, D.5]: ring slots [0, n_keys / T_f);
+// a local frame f has window-relative t = f - t_origin, a sink frame t = f.
 struct Window {
-  int64_t start;  // first window frame
+  int64_t t_origin;
+  int64_t local_start;  // oldest local frame
   int n_keys;
-  int start_slot;
+  int start_slot;       // ring slot of the oldest local frame, minus sink_frames
 };
+
+Window window_of(const vmla_config& c, int64_t F) {
+  const int64_t S = c.sink_frames, L = c.window_frames - c.sink_frames;
+  Window w;
+  if (F <= c.window_frames) {
+    w.local_start = std::min<int64_t>(S, F);
+    w.t_origin = 0;
+    w.n_keys = (int)(F * tokens_per_frame(c));
+    w.start_slot = 0;
+  } else {
+    w.local_start = F - L;
+    w.t_origin = w.local_start - S;
+    w.n_keys = (int)((int64_t)c.window_frames * tokens_per_frame(c));
+    w.start_slot = (int)((w.local_start - S) % L);
+  }
+  return w;
+}
 
 vmla_status check_attention_frames(const vmla_config& c, int64_t F, int64_t first, int n, Window* w) {
   if (n < 1 || n > c.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
   if (F < 1 || first < 0 || first + n != F) return VMLA_ERR_STATE;
-  w->start = F > c.window_frames ? F - c.window_frames : 0;
-  w->n_keys = (int)((F - w->start) * tokens_per_frame(c));
-  w->start_slot = (int)(w->start % c.window_frames);
+  *w = window_of(c, F);
   return VMLA_OK;
 }
 
@@ -288,6 +310,7 @@ vmla_status vmla_config_init(vmla_config* c) {
   c->dtype = VMLA_BF16;
   c->rope_mode = VMLA_ROPE_AT_READ;
   c->softmax_rescale_log2 = 8.f;
+  c->sink_frames = 0;
   return VMLA_OK;
 }
 
@@ -306,6 +329,9 @@ vmla_status vmla_config_check(const vmla_config* c) {
   }
   if (2 * pairs != c->d_rope || pairs > kMaxPairs) return VMLA_ERR_INVALID_ARG;
   if (c->chunk_frames > c->window_frames) return VMLA_ERR_INVALID_ARG;
+  // a sink needs room for a whole chunk beside it, and window-relative positions
+  if (c->sink_frames < 0 || c->sink_frames + c->chunk_frames > c->window_frames) return VMLA_ERR_INVALID_ARG;
+  if (c->sink_frames > 0 && c->rope_mode != VMLA_ROPE_AT_READ) return VMLA_ERR_INVALID_ARG;
   if (c->d_value != c->d_nope + c->d_rope) return VMLA_ERR_UNSUPPORTED_SHAPE;  // dense layout [2][n_h][d_head]
   if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c->dtype == VMLA_BF16) {
@@ -384,6 +410,8 @@ vmla_status vmla_bind(vmla_handle* h, void* ckv, void* kr, void* ws, size_t ws_b
 
 vmla_status vmla_dense_bind(vmla_handle* h, void* dense) {
   if (!h || !dense || !aligned16(dense)) return VMLA_ERR_INVALID_ARG;
+  // the dense layout stores keys rotated at absolute positions: no window-relative re-indexing
+  if (h->cfg.sink_frames > 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
   h->dense = dense;
   h->dense_frames.assign(h->cfg.layers, 0);
   return VMLA_OK;
@@ -392,16 +420,18 @@ vmla_status vmla_dense_bind(vmla_handle* h, void* dense) {
 vmla_status vmla_window(const vmla_handle* h, int64_t F, int32_t* frame, int32_t* slot, int32_t* t_local,
                         int capacity, int* n) {
   if (!h || !n || F < 0) return VMLA_ERR_INVALID_ARG;
-  const int W = h->cfg.window_frames;
-  const int64_t start = F > W ? F - W : 0;
-  const int count = (int)(F - start);
+  const vmla_config& c = h->cfg;
+  const Ring g = make_ring(c);
+  const Window w = window_of(c, F);
+  const int sink = (int)std::min<int64_t>(c.sink_frames, F);
+  const int count = sink + (int)(F - w.local_start);
   *n = count;
   if (count > capacity) return VMLA_ERR_INVALID_ARG;
-  for (int k = 0; k < count; ++k) {
-    const int64_t f = start + k;
+  for (int k = 0; k < count; ++k) {  // sink frames, then local frames oldest first
+    const int64_t f = k < sink ? k : w.local_start + (k - sink);
     if (frame) frame[k] = (int32_t)f;
-    if (slot) slot[k] = (int32_t)(f % W);
-    if (t_local) t_local[k] = (int32_t)(f - start);
+    if (slot) slot[k] = (int32_t)ring_frame_slot(g, f);
+    if (t_local) t_local[k] = (int32_t)(k < sink ? f : f - w.t_origin);
   }
   return VMLA_OK;
 }
@@ -513,7 +543,7 @@ vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void*
   {
     StageScope scope(h, 2, s);
     SimtQPrep a{static_cast<const float*>(q), static_cast<const float*>(w_uk), at<float>(h->ws, w.qt), c.batch, nq,
-                c.n_heads, c.d_nope, c.d_rope, c.d_latent, 1, first - (at_read ? win.start : 0), make_ring(c),
+                c.n_heads, c.d_nope, c.d_rope, c.d_latent, 1, first - (at_read ? win.t_origin : 0), make_ring(c),
                 make_rope(c)};
     e = launch_qprep_simt(a, s);
   }
@@ -551,7 +581,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   const WsLayout w = ws_layout(c);
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
   const int nq = (int)(n * tokens_per_frame(c));
-  const int64_t t_first = first - (at_read ? win.start : 0);
+  const int64_t t_first = first - (at_read ? win.t_origin : 0);
   __nv_bfloat16* ckv_layer = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
   __nv_bfloat16* kr_layer = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
   const __nv_bfloat16* kpos = kr_layer;

@@ -46,6 +46,7 @@ class Dims:
     dtype: str = "bf16"  # storage type of every tensor: "bf16" or "fp32"
     rope_theta: float = 10000.0
     rope_base_dims: tuple = (0, 0, 0)  # 0 = twice the pair count of the axis
+    sink_frames: int = 0  # leading frames pinned in the ring (window_frames counts them)
 
     @property
     def d_head(self) -> int:
@@ -85,7 +86,12 @@ WAN = Dims("wan", d_model=1536, n_heads=12, d_nope=96, d_rope=32, d_latent=192,
 # second, large enough for several query and key tiles with ragged tails.
 WAN_SMALL = WAN.replace(name="wan_small", grid_h=10, grid_w=20)
 
-WORKLOADS = {d.name: d for d in (TINY, WAN, WAN_SMALL)}
+# Long-horizon inference as the pages run it: one sink latent frame and the six most recent latent
+# frames (the current chunk among them), 7 x 1560 = 10920 keys.
+WAN_SINK = WAN.replace(name="wan_sink", window_frames=7, sink_frames=1)
+WAN_SMALL_SINK = WAN_SMALL.replace(name="wan_small_sink", window_frames=7, sink_frames=1)
+
+WORKLOADS = {d.name: d for d in (TINY, WAN, WAN_SMALL, WAN_SINK, WAN_SMALL_SINK)}
 
 
 def _workload_id(name: str) -> int:

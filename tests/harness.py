@@ -107,7 +107,7 @@ def oracle_chunk(d, w, frame_x, chunk, q, rows=None, heads=None):
     first = chunk * d.chunk_frames
     F = first + d.chunk_frames
     c, r, kpos, t0 = O.window_latents(frame_x, F, d.window_frames, w.w_down, d.d_latent,
-                                      d.grid_h, d.grid_w, rope_at="read")
+                                      d.grid_h, d.grid_w, rope_at="read", sink_frames=d.sink_frames)
     qpos = O.chunk_query_positions(first, d.chunk_frames, t0, d.grid_h, d.grid_w)
     ref = O.chunk_attention(c, r, kpos, q, qpos, w.w_uk, w.w_uv, d_nope=d.d_nope, rope_pairs=d.rope_pairs,
                             rope_theta=d.rope_theta, rope_base_dims=d.rope_base_dims, query_rows=rows,

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = api.lib()
-    assert lib.vmla_abi_version() == 1
+    assert lib.vmla_abi_version() == api.ABI_VERSION == 2
     for code in range(8):
         assert lib.vmla_status_string(code).decode().startswith("VMLA_")
     assert lib.vmla_status_string(99).decode() == "VMLA_ERR_UNKNOWN"
@@ -229,3 +229,40 @@ def test_latent_widths_with_kernels(d_latent, status):
     c = default_config()
     c.d_latent = d_latent
     assert api.lib().vmla_config_check(ctypes.byref(c)) == status
+
+
+def test_sink_window_matches_the_oracle_rule():
+    """vmla_window with one sink frame and a six-frame local part (7-frame ring):
+    frames, ring slots and window-relative t as the oracle's sink rule gives them."""
+    import oracle.vmla_oracle as O
+    c = default_config()
+    c.window_frames, c.sink_frames = 7, 1
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == 0
+    h = api.LatentKVAttention(c)
+    for F in range(1, 40):
+        frames, slots, ts = h.window(F)
+        want = O.window_frames_list(F, 7, 1)
+        t = O.window_frame_t(F, 7, 1)
+        assert list(frames) == want
+        assert list(slots) == [O.ring_slot(f, 7, 1) for f in want]
+        assert list(ts) == [t[f] for f in want]
+    h.close()
+
+
+def test_sink_config_rules():
+    lib = api.lib()
+    c = default_config()
+    c.window_frames, c.sink_frames = 7, 1
+    c.rope_mode = api.ROPE_AT_APPEND          # the sink context needs window-relative positions
+    assert lib.vmla_config_check(ctypes.byref(c)) == 1
+    c.rope_mode = api.ROPE_AT_READ
+    c.sink_frames = 5                         # no room for a 3-frame chunk beside the sink
+    assert lib.vmla_config_check(ctypes.byref(c)) == 1
+    c.sink_frames = -1
+    assert lib.vmla_config_check(ctypes.byref(c)) == 1
+    c.sink_frames = 1
+    h = api.LatentKVAttention(c)
+    assert lib.vmla_dense_bind(h._h, 0x10000) == 2  # dense keys are rotated at absolute positions
+    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, api.workspace_bytes(c)) == 0
+    assert lib.vmla_cache_append(h._h, 0, 0x40000, 0x40000, 0, 7, None) == 3  # more than the local part
+    h.close()

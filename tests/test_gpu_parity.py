@@ -346,6 +346,53 @@ def test_wan_layer_sampled_rows():
     assert_bf16_close(out[0][rows], ref, "wan layer")
 
 
+# ------------------------------------------------------------------ sink frame + local window
+
+def test_tiny_fp32_sink_window():
+    """One pinned sink frame and a 3-frame local part, 1-frame chunks: partial
+    windows, then every later chunk evicts the oldest local frame only."""
+    d = TINY.replace(window_frames=4, sink_frames=1)
+    ro = Rollout(d)
+    for chunk in range(10):
+        ro.append_chunk(0, chunk)
+        out, q = ro.attend(0, chunk)
+        assert_fp32_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk}")
+
+
+@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE, api.DESIGN_RECONSTRUCT])
+def test_small_bf16_sink_window_rolling(design):
+    """The long-horizon context of the pages (one sink frame + six recent frames,
+    window-relative RoPE) over 9 chunks of 3 frames: the sink stays, the local
+    frames rotate, positions stay within 0..6; every chunk checked in full."""
+    d = synth.WAN_SMALL_SINK
+    ro = Rollout(d, design=api.DESIGN_RECON_ONCE)
+    for chunk in range(9):
+        ro.append_chunk(0, chunk)
+        out, q = ro.attend(0, chunk, design=design)
+        # per-head bf16 K/V on the 600-key first window: see test_small_bf16_dense_designs_short_window
+        loose = design != api.DESIGN_ABSORBED and chunk == 0
+        assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk}", max_abs=6e-2 if loose else 3e-2)
+
+
+def test_small_bf16_sink_window_passes_and_noalloc():
+    import torch
+    d = synth.WAN_SMALL_SINK
+    ro = Rollout(d)
+    for chunk in range(5):
+        for p in range(2):
+            ro.append_chunk(0, chunk, pass_=p)
+            out, q = ro.attend(0, chunk, pass_=p)
+            assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk} pass {p}")
+    qd = to_dev(q, d)
+    out2 = torch.empty_like(torch.from_numpy(out)).cuda()
+    api.check(api.lib().vmla_chunk_attention_noalloc(ro.cfg, 0, ro.m.ckv.data_ptr(), ro.m.kr.data_ptr(), 15,
+                                                     qd.data_ptr(), ro.wd[0][1].data_ptr(), ro.wd[0][2].data_ptr(),
+                                                     out2.data_ptr(), 12, 3, torch.cuda.current_stream().cuda_stream),
+              "noalloc")
+    assert ro.m.device_status()[0] == 0
+    assert torch.equal(out2.cpu(), torch.from_numpy(out)), "allocation-free path differs on the sink window"
+
+
 # ------------------------------------------------------------------ numerics of the kernels' helpers
 
 def test_polynomial_exp2_error_bound():

@@ -77,7 +77,7 @@ class PoolRollout:
         q = self.pool.queries(layer, chunk, pass_)
         for b in samples:
             frame_x = {}
-            for c in range(max(0, chunk - d.window_frames // d.chunk_frames), chunk + 1):
+            for c in sorted({0} | set(range(max(0, chunk - d.window_frames // d.chunk_frames), chunk + 1))):
                 x = self.pool.activations(layer, c, pass_ if c == chunk else self.last_pass[(layer, c)])
                 for k in range(d.chunk_frames):
                     frame_x[c * d.chunk_frames + k] = x[b, k * T:(k + 1) * T]
@@ -160,3 +160,13 @@ def test_wan_latent_width_sweep(d_latent):
             assert rel <= 1e-2 and mx <= 5e-2, f"absorbed d_c={d_latent}: rel {rel:.3e} max {mx:.3e}"
         else:
             assert_bf16_close(o, ref, f"{name} d_c={d_latent}")
+
+
+def test_wan_sink_window_sampled_rows():
+    """The Wan layer in the pages' long-horizon context (one sink frame + six
+    recent frames: 10920 keys) after 12 chunks, 256 seeded rows of every head."""
+    d = synth.WAN_SINK
+    ro = PoolRollout(d, 1)
+    for chunk in range(12):
+        ro.step(0, chunk, 0)
+    ro.check(0, 11, 0, what="sink window")
