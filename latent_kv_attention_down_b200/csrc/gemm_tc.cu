@@ -1,16 +1,18 @@
-// tcgen05 GEMM kernels of the bf16 path (sm_100a).  All three share one shape:
-// a 128-row A tile and a weight B tile staged in shared memory by TMA
-// (128-byte swizzle), one elected thread issuing tcgen05.mma into a TMEM
-// accumulator, and four epilogue warps that read their TMEM lane (= output
-// row) back with tcgen05.ld and store bf16 rows.
+// tcgen05 GEMM kernels of the bf16 path (sm_100a).  All three are persistent
+// (one CTA per SM taking work items in a grid-stride loop) and share one
+// shape: A and B tiles staged in shared memory by TMA (128-byte swizzle) in a
+// ring, one elected thread issuing tcgen05.mma into one of two TMEM
+// accumulators, and four epilogue warps that read their TMEM lane (= output
+// row) back with tcgen05.ld, park 64 rows at a time in shared memory and write
+// them out contiguously, while the next item's loads and MMAs proceed.
 //
 //  * append_tc  [gist.it pt. 1, 3; paperlayer §3]: [c_KV | k_R] = W_down x,
-//    rows scattered into the ring slot of their frame (FIFO ring of W frames,
-//    slot f mod W [paperlayer App. D.4]); k_R optionally rotated with the
-//    absolute frame index.  K = d_model, pipelined over 4 stages of 64.
+//    rows placed in the ring slot of their frame (sink frames pinned, the
+//    rest FIFO [paperlayer App. D.4]); k_R optionally rotated with the
+//    absolute frame index.  K = d_model.
 //  * qprep_tc   [paperlayer App. E, content-path absorption]: the query's
 //    content part pushed through W_uk,h (q~ = W_uk,h^T q_nope, d_latent wide)
-//    next to its rotated positional part, one head per CTA column.
+//    next to its rotated positional part.
 //  * recon_tc   [gist.it pt. 2; paperlayer §3 On-demand reconstruction]: the
 //    per-head dense entries k_h = [W_uk,h c | RoPE(k_R)], v_h = W_uv,h c.
 #include "kernels.h"
@@ -20,20 +22,12 @@
 namespace vmla {
 namespace {
 
-constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 4..7 epilogue
+constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 4..7 epilogue; every kernel is persistent
 
 // Rotate 16 adjacent pairs held in v[0..31] at grid position (t, h, w).
 __device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, int t, int h, int w) {
 #pragma unroll
   for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], rope_cs(rp, p, t, h, w));
-}
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
 // 32 floats as bf16 into 64 bytes of shared memory (16-byte aligned)
@@ -62,30 +56,6 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v
 __device__ __forceinline__ void raw_to_float(const uint32_t (&r)[32], float (&v)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Shared prologue: barriers, abort flag, TMEM allocation by warp 1.
-__device__ __forceinline__ uint32_t setup_cta(uint64_t* bars, int nbars, uint32_t* tslot, int* abort_flag,
-                                              uint32_t tmem_cols) {
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nbars; ++i) mbar_init(&bars[i], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if ((threadIdx.x >> 5) == 1) tmem_alloc(tslot, tmem_cols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  return *tslot;
-}
-
-__device__ __forceinline__ void teardown_cta(uint32_t tbase, uint32_t tmem_cols) {
-  tc_fence_before();
-  __syncthreads();
-  if ((threadIdx.x >> 5) == 1) {
-    tc_fence_after();
-    tmem_dealloc(tbase, tmem_cols);
-  }
 }
 
 // ============================================================== append
@@ -288,89 +258,171 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================== q-absorb
+// Persistent over (sample, 128-query tile, head) items, head fastest.  Per item one
+// stage holds the head's 128-column slice of q (two [128 x 64] blocks) and W_uk,h
+// ([96 x 64] blocks, read as the MN-major B operand); a single MMA chain of 6
+// k-steps gives W_uk,h^T q_nope in TMEM (two accumulators alternate); the epilogue
+// parks the item's rows of [q~_nope (d_c) | RoPE(q_rope) (32)] unpadded (all 128 when
+// they fit, else 64 at a time) and one bulk copy writes each park out (an item's
+// output rows are consecutive in memory); the copy runs while the next item's
+// positional part is rotated and its accumulator awaited.
 template <int DL>
 struct QPrepCfg {
   static constexpr int A_BYTES = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
   static constexpr int WB = 96 * 128;            // one 64-col block of W_uk,h: 96 rows x 128 B
   static constexpr int B_BYTES = (DL / 64) * WB;
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr int SMEM = 1024 + A_BYTES + B_BYTES + 256;
-  static_assert(DL % 64 == 0 && DL <= 256, "bad d_latent");
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int ROW = DL + 32;                 // output row, elements
+  static constexpr int OUT_STRIDE = ROW * 2;          // parked rows are the output's bytes, unpadded
+  static constexpr int PARK_ROWS = 2 * STAGE + 128 * OUT_STRIDE <= 212 * 1024 ? 128 : 64;
+  static constexpr int OUT_BYTES = PARK_ROWS * OUT_STRIDE;
+  static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
+  static constexpr int STAGES = FIT > 4 ? 4 : FIT;
+  static constexpr uint32_t TMEM_COLS = 512;          // two accumulators, at 0 and 256
+  static constexpr int SMEM_USED = 1024 + STAGES * STAGE + OUT_BYTES + 256;
+  static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;  // one CTA per SM
+  static_assert(DL % 64 == 0 && DL <= 256 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
 };
 
 template <int DL>
 __global__ void __launch_bounds__(kThreads, 1)
     qprep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wuk,
-                    const QPrepTc a) {
+                    const QPrepTc a, int items) {
   using C = QPrepCfg<DL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::B_BYTES);
-  uint64_t* done = full + 1;
+  uint8_t* sout = smem + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sout + C::OUT_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const int m_tiles = (a.n_q + 127) / 128;
   const Guard g{abort_flag, a.err, a.limit_ns};
-  const uint32_t tbase = setup_cta(full, 2, tslot, abort_flag, C::TMEM_COLS);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 4);
+    mbar_init(&acc_empty[1], 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(full, C::A_BYTES + C::B_BYTES);
-      tma_load_3d(sA, &tm_q, full, h * 128, m0, b);
-      tma_load_3d(sA + 16384, &tm_q, full, h * 128 + 64, m0, b);
-      for (int cb = 0; cb < DL / 64; ++cb) tma_load_3d(sB + cb * C::WB, &tm_wuk, full, cb * 64, 0, h);
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_wuk);
+      int it = 0;
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x, ++it) {
+        const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+        const int s = it % C::STAGES;
+        if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&full[s], C::STAGE);
+        tma_load_3d(st, &tm_q, &full[s], h * 128, mt * 128, b);
+        tma_load_3d(st + 16384, &tm_q, &full[s], h * 128 + 64, mt * 128, b);
+        for (int cb = 0; cb < DL / 64; ++cb) tma_load_3d(st + C::A_BYTES + cb * C::WB, &tm_wuk, &full[s], cb * 64, 0, h);
+      }
+      if (*abort_flag)
+        for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+          drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
     }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const bool ok = wait_phase(full, 0, g, DEV_ERR_TIMEOUT_MMA);
-      tc_fence_after();
-      if (ok) {
-        constexpr uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
-        const uint64_t ad = smem_desc(smem_u32(sA), 16, 1024, LAYOUT_SW128);
-        const uint64_t bd = smem_desc(smem_u32(sB), C::WB, 1024, LAYOUT_SW128);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
+      int j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        const int acc = j & 1, s = j % C::STAGES;
+        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        if (!wait_phase(&full[s], (j / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::STAGE);
+        const uint64_t ad = smem_desc(st, 16, 1024, LAYOUT_SW128);
+        const uint64_t bd = smem_desc(st + C::A_BYTES, C::WB, 1024, LAYOUT_SW128);
 #pragma unroll
         for (int kk = 0; kk < 6; ++kk) {  // d_nope = 96 = 6 x 16
-          const uint64_t a = desc_add(ad, (kk / 4) * 16384 + (kk % 4) * 32), b = desc_add(bd, kk * 2048);
+          const uint64_t ak = desc_add(ad, (kk / 4) * 16384 + (kk % 4) * 32), bk = desc_add(bd, kk * 2048);
           if (kk == 0)
-            mma_ss_c<false>(tbase, a, b, idesc);
+            mma_ss_c<false>(tbase + acc * 256, ak, bk, idesc);
           else
-            mma_ss_c<true>(tbase, a, b, idesc);
+            mma_ss_c<true>(tbase + acc * 256, ak, bk, idesc);
         }
+        mma_commit(&empty[s]);
+        mma_commit(&acc_full[acc]);
       }
       mma_commit(done);
       if (*abort_flag) drain_phase(done, 0, g);
     }
-    if (lane == 0 && *abort_flag) drain_phase(full, 0, g);
-  } else if (warp >= 4) {
-    const int wq = warp - 4;
-    const int i = m0 + wq * 32 + lane;
-    const bool ok = wait_phase(done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE);
     __syncwarp();
-    tc_fence_after();
-    const bool valid = ok && i < a.n_q;
-    const int ii = valid ? i : 0;
-    __nv_bfloat16* out = a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + ii) * (DL + 32);
+  } else if (warp >= 4) {
+    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int T = a.ring.tokens_per_frame;
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+      const int acc = j & 1;
+      // the positional part does not wait for the tensor core
+      const int i = mt * 128 + r;
+      const int ii = i < a.n_q ? i : 0;
+      float qr[32];
+      {
+        load_bf16x32(a.q + (((int64_t)b * a.n_q + ii) * a.n_heads + h) * 128 + 96, qr);
+        const int tok = ii % T;
+        rotate16(qr, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
+      }
+      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      __syncwarp();
+      tc_fence_after();
+      const int valid_rows = ok ? min(128, a.n_q - mt * 128) : 0;
+      __nv_bfloat16* out_tile = a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + mt * 128) * C::ROW;
 #pragma unroll 1
-    for (int c0 = 0; c0 < DL; c0 += 32) {
-      uint32_t raw[32];
-      tmem_ld32(tmem_addr(tbase, wq * 32, c0), raw);
-      if (!valid) continue;
-      float v[32];
-      raw_to_float(raw, v);
-      store_bf16x32(out + c0, v);
+      for (int part = 0; part < 128 / C::PARK_ROWS; ++part) {
+        if (tid == 0) bulk_wait_all_read();  // the previous park has been read by its copy
+        named_bar_sync(1, 128);
+        if ((r / C::PARK_ROWS) == part) {  // warps whose TMEM lanes are this park's rows
+          uint8_t* orow = sout + (r - C::PARK_ROWS * part) * C::OUT_STRIDE;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DL; c0 += 32) {
+            uint32_t raw[32];
+            tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            float v[32];
+            raw_to_float(raw, v);
+            store_bf16x32_smem(orow + c0 * 2, v);
+          }
+          store_bf16x32_smem(orow + DL * 2, qr);
+          fence_async_smem();  // the bulk copy (async proxy) reads what these threads wrote
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        named_bar_sync(1, 128);  // this park is complete
+        const int rows_p = min(C::PARK_ROWS, valid_rows - C::PARK_ROWS * part);
+        if (tid == 0 && rows_p > 0) {
+          bulk_store(out_tile + (int64_t)C::PARK_ROWS * part * C::ROW, sout, (uint32_t)(rows_p * C::OUT_STRIDE));
+          bulk_commit();
+        }
+      }
     }
-    if (valid) {
-      float v[32];
-      load_bf16x32(a.q + (((int64_t)b * a.n_q + ii) * a.n_heads + h) * 128 + 96, v);
-      const int T = a.ring.tokens_per_frame, tok = ii % T;
-      rotate16(v, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
-      store_bf16x32(out + DL, v);
-    }
+    if (tid == 0) bulk_wait_all_read();  // shared memory stays until the last copy has read it
   }
-  teardown_cta(tbase, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
 }
 
 // ============================================================== per-head reconstruction
@@ -591,7 +643,14 @@ cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc
   using C = QPrepCfg<DL>;
   static const cudaError_t attr = set_smem(qprep_tc_kernel<DL>, C::SMEM);
   if (attr != cudaSuccess) return attr;
-  qprep_tc_kernel<DL><<<dim3((a.n_q + 127) / 128, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tw, a);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
+  qprep_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tq, tw, a, items);
   return cudaGetLastError();
 }
 

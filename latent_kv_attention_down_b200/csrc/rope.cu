@@ -30,21 +30,35 @@ __device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, int t,
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// d_rope = 32: 4 threads per key, 16 bytes each
+// d_rope = 32: 4 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its
+// slot in every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.
 __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)a.batch * a.n_keys * 4;
-  if (idx >= total) return;
+  if (idx >= (int64_t)a.n_keys * 4) return;
   const int quad = idx & 3;
-  const int s = (idx >> 2) % a.n_keys;
-  const int b = (idx >> 2) / a.n_keys;
+  const int s = (int)(idx >> 2);
   const int64_t ring_rows = (int64_t)a.ring.window_frames * a.ring.tokens_per_frame;
   const int fslot = s / a.ring.tokens_per_frame, tok = s % a.ring.tokens_per_frame;
   const int t = ring_slot_t(a.ring, fslot, a.window_start_slot);
-  const int64_t off = ((int64_t)b * ring_rows + s) * 32 + quad * 8;
-  const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + off);
-  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + off) =
-      rotate4(v, a.rope, quad * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
+  const int hh = tok / a.ring.grid_w, ww = tok % a.ring.grid_w;
+  float2 cs[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) cs[k] = rope_cs(a.rope, quad * 4 + k, t, hh, ww);
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * 32 + quad * 8);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * 32 + quad * 8);
+  const int64_t stride = ring_rows * 32 / 8;  // one sample's ring, in 16-byte units
+#pragma unroll 4
+  for (int b = 0; b < a.batch; ++b) {
+    const uint4 v = __ldg(src + b * stride);
+    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float u = bf_lo(in[k]), x = bf_hi(in[k]);
+      rope_apply(u, x, cs[k]);
+      out[k] = pack2(u, x);
+    }
+    dst[b * stride] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
 }
 
 // 16 threads per (sample, query, head): 12 copy the content dims, 4 rotate the positional ones
@@ -71,8 +85,8 @@ __global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
 
 cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s) {
   if (a.d_rope != 32) return cudaErrorInvalidValue;
-  const int64_t total = (int64_t)a.batch * a.n_keys * 4;
-  if (total == 0) return cudaSuccess;
+  const int64_t total = (int64_t)a.n_keys * 4;
+  if (total == 0 || a.batch == 0) return cudaSuccess;
   rope_window_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
