@@ -398,7 +398,9 @@ def run_ours(args, rank, world, local_rank):
                        "reconstruct_in_tile": recon_in_tile}
     if args.legs:
         line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
-                        "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed)}
+                        "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed),
+                        "sink_window": sink_leg(dev=dev, tc=tc_burst, seed=seed),
+                        "folded_output_mixer": folded_leg(dev=dev, tc=tc_burst, seed=seed)}
     if dense:
         line["dense"] = dense
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -480,6 +482,115 @@ def batch8_leg(m_timed, dev, hbm, tc, seed):
         res["kernels"][n] = e
     m.close()
     return res
+
+
+def sink_leg(dev, tc, seed, steps=50):
+    """The pages' long-horizon context: one sink frame + six recent frames (10920 keys),
+    window-relative RoPE, after 12 chunks; one chunk step (append + attention) timed."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    d = synth.WAN_SINK
+    L = 8
+    m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+    pool = synth.FramePool(d, base_seed=seed)
+    bf = torch.bfloat16
+    xp = torch.from_numpy(pool.x).to(dev, bf)
+    qp = torch.from_numpy(pool.q).to(dev, bf)
+    W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv))
+         for w in (synth.weights(d, l, seed) for l in range(L))]
+    chunks = 12
+    for l in range(L):
+        for c in range(chunks):
+            m.append(l, pool.activations(l, c, 0, pool=xp), W[l][0], c * d.chunk_frames, d.chunk_frames)
+    first = (chunks - 1) * d.chunk_frames
+    xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
+    qs = [pool.queries(l, chunks - 1, 1, pool=qp) for l in range(L)]
+    out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
+
+    def step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, api.DESIGN_ABSORBED)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    m.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    at_ms, at_n = m.profile_read("attention")
+    m.profile(False)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    nk = d.window_tokens
+    attn_flops = 2 * d.n_queries * nk * d.n_heads * (2 * d.d_latent + d.d_rope)
+    att = at_ms / max(at_n, 1)
+    m.close()
+    return {"workload": "wan1.3b-layer, 1 sink frame + 6 recent frames (N_k=10920), window-relative RoPE, "
+                        "chunk 12", "ms_per_step": ms, "query_tokens_per_s": d.n_queries / (ms * 1e-3),
+            "attention_ms": att, "attention_tflops": attn_flops / (att * 1e-3) / 1e12,
+            "frac_of_bf16_peak": attn_flops / (att * 1e-3) / 1e12 / tc}
+
+
+def folded_leg(dev, tc, seed, steps=50):
+    """W_uv folded into the output mixer: the chunk step with out = sum_h (W_O,h W_uv,h) o~_h
+    (absorbed attention + one K = 12 x 192 GEMM to d_model = 1536 columns)."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    d = WORKLOAD
+    L = 4
+    m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+    pool = synth.FramePool(d, base_seed=seed)
+    bf = torch.bfloat16
+    xp = torch.from_numpy(pool.x).to(dev, bf)
+    qp = torch.from_numpy(pool.q).to(dev, bf)
+    ws = [synth.weights(d, l, seed) for l in range(L)]
+    W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv, w.w_o)) for w in ws]
+    folds = []
+    for l in range(L):
+        f = torch.empty(d.d_model, d.n_heads * d.d_latent, dtype=bf, device=dev)
+        m.fold_output_weights(W[l][3], W[l][2], f)
+        folds.append(f)
+    chunks = d.window_frames // d.chunk_frames
+    for l in range(L):
+        for c in range(chunks):
+            m.append(l, pool.activations(l, c, 0, pool=xp), W[l][0], c * d.chunk_frames, d.chunk_frames)
+    first = (chunks - 1) * d.chunk_frames
+    xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
+    qs = [pool.queries(l, chunks - 1, 1, pool=qp) for l in range(L)]
+    out = torch.empty((1, d.n_queries, d.d_model), dtype=torch.float32, device=dev)
+
+    def step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention_folded(l, qs[l], W[l][1], folds[l], out, first, d.chunk_frames)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    m.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    k = {n: m.profile_read(n) for n in ("attention", "folded_mixer")}
+    m.profile(False)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    gemm_ms = k["folded_mixer"][0] / max(k["folded_mixer"][1], 1)
+    gemm_flops = 2 * 2 * d.n_queries * d.d_model * d.n_heads * d.d_latent  # rounded part + residual
+    m.close()
+    return {"workload": "wan1.3b-layer chunk step with W_O W_uv folded (K=2304, d_out=1536)", "ms_per_step": ms,
+            "attention_ms": k["attention"][0] / max(k["attention"][1], 1), "mixer_gemm_ms": gemm_ms,
+            "mixer_gemm_tflops": gemm_flops / (gemm_ms * 1e-3) / 1e12}
 
 
 def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384)):

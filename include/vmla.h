@@ -231,7 +231,8 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
 
 /* Per-stage CUDA-event timing of the kernels each call launches, recorded on the
  * call's stream.  Stages: 0 append, 1 rope, 2 q-absorb, 3 attention (absorbed),
- * 4 attention (reconstruct), 5 dense append, 6 dense attention, 7 reconstruct-once.
+ * 4 attention (reconstruct), 5 dense append, 6 dense attention, 7 reconstruct-once,
+ * 8 folded output mixer.
  * vmla_profile_read synchronises, then returns the summed milliseconds and the
  * launch count of one stage since profiling was enabled. */
 vmla_status vmla_profile_enable(vmla_handle* h, int enable);
@@ -247,6 +248,23 @@ vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* 
  * return VMLA_ERR_UNSUPPORTED_SHAPE.  Host only; VMLA_ERR_INVALID_ARG for
  * n_split outside 0..2 or a negative cap. */
 vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas);
+
+/* The value path absorbed all the way into the layer's output mixer [paperlayer App. E]:
+ * with B_h = W_O,h W_uv,h (W_O,h the d_value columns of W_O that read head h),
+ *   out = sum_h B_h o~_h,   o~_h = softmax-weighted latents of head h (d_latent wide),
+ * one GEMM with K = n_heads * d_latent in place of the per-head W_uv,h and W_O.
+ * vmla_fold_output_weights writes w_fold [d_out][n_heads*d_latent] (bf16) from
+ * w_o [d_out][n_heads*d_value] and w_uv [n_heads][d_value][d_latent] (bf16, fp32 sums;
+ * a one-time weight preparation).  vmla_chunk_attention_folded is vmla_chunk_attention
+ * with VMLA_DESIGN_ABSORBED followed by that GEMM: o~ is handed over as a bf16 pair
+ * (rounded part + residual, in the workspace), out is [batch][n_frames*T_f][d_out] fp32.
+ * VMLA_BF16 with d_latent <= 256 and d_out a multiple of 128, else
+ * VMLA_ERR_UNSUPPORTED_SHAPE; frame rules and errors as vmla_chunk_attention. */
+vmla_status vmla_fold_output_weights(const vmla_config* cfg, const void* w_o, const void* w_uv, void* w_fold,
+                                     int d_out, void* stream);
+vmla_status vmla_chunk_attention_folded(vmla_handle* h, int layer, const void* q, const void* w_uk,
+                                        const void* w_fold, int d_out, void* out, int64_t first_frame,
+                                        int n_frames, void* stream);
 
 /* Allocation-free chunk attention.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for example a

@@ -20,7 +20,7 @@ BF16, FP32 = 0, 1
 DESIGN_AUTO, DESIGN_ABSORBED, DESIGN_RECONSTRUCT, DESIGN_RECON_ONCE = 0, 1, 2, 3
 ROPE_AT_READ, ROPE_AT_APPEND = 0, 1
 STAGES = {"append": 0, "rope": 1, "q_absorb": 2, "attention": 3, "attention_reconstruct": 4,
-          "dense_append": 5, "dense_attention": 6, "reconstruct_once": 7}
+          "dense_append": 5, "dense_attention": 6, "reconstruct_once": 7, "folded_mixer": 8}
 
 
 ABI_VERSION = 2  # VMLA_ABI_VERSION of include/vmla.h that this binding's structures follow
@@ -72,6 +72,9 @@ _SIGS = {
     "vmla_device_status": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
     "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int]),
+    "vmla_fold_output_weights": (c_int, [ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
+    "vmla_chunk_attention_folded": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int64,
+                                            c_int, c_void_p]),
     "vmla_selftest_exp2": (c_int, [c_void_p, c_void_p, ctypes.c_int64, c_void_p]),
     "vmla_profile_read": (c_int, [c_void_p, c_int, ctypes.POINTER(c_double), ctypes.POINTER(c_int)]),
     "vmla_selftest_wait_timeout": (c_int, [c_uint64, c_void_p]),
@@ -247,6 +250,17 @@ class LatentKVAttention:
         flags = c_uint32()
         st = lib().vmla_device_status(self._h, _stream(stream), ctypes.byref(flags))
         return st, flags.value
+
+    def fold_output_weights(self, w_o, w_uv, w_fold, stream=None):
+        """w_fold [d_out][n_h * d_c] = W_O,h W_uv,h side by side."""
+        check(lib().vmla_fold_output_weights(ctypes.byref(self.cfg), _ptr(w_o), _ptr(w_uv), _ptr(w_fold),
+                                             w_fold.shape[0], _stream(stream)), "vmla_fold_output_weights")
+
+    def attention_folded(self, layer, q, w_uk, w_fold, out, first_frame, n_frames, stream=None):
+        """Absorbed chunk attention with W_uv folded into the output mixer: out [B][rows][d_out] fp32."""
+        check(lib().vmla_chunk_attention_folded(self._h, layer, _ptr(q), _ptr(w_uk), _ptr(w_fold), w_fold.shape[0],
+                                                _ptr(out), first_frame, n_frames, _stream(stream)),
+              "vmla_chunk_attention_folded")
 
     def set_append_tiling(self, n_split: int = 0, max_ctas: int = 0):
         """Column parts (0: chosen per call) and grid cap (0: one CTA per SM) of the append kernel."""

@@ -76,14 +76,13 @@ struct AttnCfg {
   static constexpr int O_COL = 2 * BN;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int SMEM = Q_BYTES + STAGES * STAGE_BYTES + BARS;
-  // epilogue images: O_bar rounded over the query tile, W_uv,h then O_bar residual in the drained ring
-  static constexpr int EPI_WUV = 0;
-  static constexpr int EPI_OB_LO = DV * 256;
+  // epilogue images: O_bar rounded over the query tile; W_uv,h in the ring stage that tile n_tiles
+  // would have used (free two tiles before the end, so its load hides behind the last tiles), the
+  // O_bar residual in the stage after it
   static_assert(STAGES >= 2, "the K/V ring needs two stages");
   static_assert(O_COL + DV <= 512, "TMEM budget");
   static_assert(SMEM <= SMEM_CAP, "shared memory budget");
-  static_assert(STAGES * STAGE_BYTES >= (DENSE ? 0 : EPI_OB_LO + DV * 256) && STAGES * STAGE_BYTES >= 65536,
-                "epilogue staging");
+  static_assert((DENSE || STAGE_BYTES >= DV * 256) && STAGES * STAGE_BYTES >= 65536, "epilogue staging");
   static_assert(DV % 64 == 0 && DV <= 256 && BN % 32 == 0, "tile shapes");
 };
 
@@ -185,7 +184,9 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-template <int DL, bool DENSE>
+// FOLD (absorbed only): the epilogue stores O_bar itself, as its bf16 pair, for an output
+// mixer that folds W_uv,h in (tm_wuv then maps O_bar's rounded part, tm_out its residual).
+template <int DL, bool DENSE, bool FOLD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
@@ -206,6 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int m0 = mt * 128;
   const int n_tiles = (a.n_keys + C::BN - 1) / C::BN;
+  const int epi_wuv = (n_tiles % C::STAGES) * C::STAGE_BYTES;           // W_uv,h
+  const int epi_lo = ((n_tiles + 1) % C::STAGES) * C::STAGE_BYTES;      // O_bar residual
   const Guard g{&bars->abort_flag, a.err, a.limit_ns};
 
   if (threadIdx.x == 0) {
@@ -262,12 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++issued;
       }
       bool wuv_issued = false;
-      if constexpr (!C::DENSE) {
-        // W_uv,h goes where the K/V ring was, once every P V has consumed it
-        if (issued == n_tiles && wait_phase(&bars->o_final, 0, g, DEV_ERR_TIMEOUT_PRODUCER)) {
+      if constexpr (!C::DENSE && !FOLD) {
+        // W_uv,h goes into the stage a further tile would take, as soon as P V has freed it
+        const int sw = n_tiles % C::STAGES;
+        if (issued == n_tiles &&
+            wait_phase(&bars->kv_empty[sw], ((n_tiles / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) {
           mbar_arrive_expect_tx(&bars->wuv_full, C::DV * 256);
           for (int kb = 0; kb < C::DV / 64; ++kb)
-            tma_load_3d(sKV + C::EPI_WUV + kb * 16384, &tm_wuv, &bars->wuv_full, kb * 64, 0, h);
+            tma_load_3d(sKV + epi_wuv + kb * 16384, &tm_wuv, &bars->wuv_full, kb * 64, 0, h);
           wuv_issued = true;
         }
       }
@@ -307,15 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars->p_done[buf]);
       }
       if (ok) mma_commit(&bars->o_final);
-      if constexpr (!C::DENSE) {
+      if constexpr (!C::DENSE && !FOLD) {
         // fused value up-projection: out_h = O_bar W_uv,h^T, O_bar as a bf16 pair (rounded + residual)
         if (ok && wait_phase(&bars->ob_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
             wait_phase(&bars->wuv_full, 0, g, DEV_ERR_TIMEOUT_MMA)) {
           tc_fence_after();
           constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
           const uint64_t hd = smem_desc(sq, 16, 1024, LAYOUT_SW128);
-          const uint64_t ld = smem_desc(skv + C::EPI_OB_LO, 16, 1024, LAYOUT_SW128);
-          const uint64_t wd = smem_desc(skv + C::EPI_WUV, 16, 1024, LAYOUT_SW128);
+          const uint64_t ld = smem_desc(skv + epi_lo, 16, 1024, LAYOUT_SW128);
+          const uint64_t wd = smem_desc(skv + epi_wuv, 16, 1024, LAYOUT_SW128);
 #pragma unroll
           for (int kk = 0; kk < C::DV / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -436,18 +441,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv_l = 1.f / (l_run + bars->red[n_tiles & 1][wg ^ 1][r]);
     if constexpr (!C::DENSE) {
       // O_bar = O / l as a bf16 pair (A operands of the two W_uv GEMMs): rounded part over the
-      // query tile, residual after W_uv,h in the drained K/V ring
+      // query tile, residual in the ring stage after W_uv,h's
       if (ok) {
 #pragma unroll 1
         for (int c = wg * HO; c < (wg + 1) * HO; c += 32) {
           uint32_t o[32];
           tmem_ld32(lane_base + C::O_COL + c, o);
           st_swizzled_row32(sQ, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, false);
-          st_swizzled_row32(sKV + C::EPI_OB_LO, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, true);
+          st_swizzled_row32(sKV + epi_lo, r, c, *reinterpret_cast<float(*)[32]>(o), inv_l, true);
         }
       }
       fence_async_smem();
       tc_fence_before();
+      if constexpr (FOLD) {
+        named_bar_sync(1, 256);
+        if (wg == 0 && r == 0 && ok && !bars->abort_flag) {
+          for (int blk = 0; blk < C::DV / 64; ++blk) {
+            tma_store_3d(&tm_wuv, sQ + blk * 16384, h * DL + blk * 64, m0, b);
+            tma_store_3d(&tm_out, sKV + epi_lo + blk * 16384, h * DL + blk * 64, m0, b);
+          }
+          bulk_commit();
+          bulk_wait_all_read();
+        }
+      } else {
       warp_arrive(&bars->ob_full);
       ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->epi_done, 0, g, DEV_ERR_TIMEOUT_EPILOGUE));
       if (ok) {
@@ -459,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_swizzled_row32_f32(sKV, r, c, *reinterpret_cast<float(*)[32]>(o), 1.f);
         }
       }
+      }
     } else {
       if (ok) {
 #pragma unroll 1
@@ -469,12 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    fence_async_smem();
-    named_bar_sync(1, 256);
-    if (wg == 0 && r == 0 && !bars->abort_flag) {
-      for (int blk = 0; blk < 4; ++blk) tma_store_3d(&tm_out, sKV + blk * 16384, h * 128 + blk * 32, m0, b);
-      bulk_commit();
-      bulk_wait_all_read();
+    if constexpr (!FOLD) {
+      fence_async_smem();
+      named_bar_sync(1, 256);
+      if (wg == 0 && r == 0 && !bars->abort_flag) {
+        for (int blk = 0; blk < 4; ++blk) tma_store_3d(&tm_out, sKV + blk * 16384, h * 128 + blk * 32, m0, b);
+        bulk_commit();
+        bulk_wait_all_read();
+      }
     }
   }
   tc_fence_before();
@@ -485,15 +504,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DL, bool DENSE>
+template <int DL, bool DENSE, bool FOLD = false>
 cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk, const CUtensorMap& tkr,
                     const CUtensorMap& tuv, const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
   using C = AttnCfg<DL, DENSE>;
   static const cudaError_t attr =
-      cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (attr != cudaSuccess) return attr;
   if (a.n_q <= 0 || a.n_keys <= 0) return cudaSuccess;
-  attn_tc_kernel<DL, DENSE><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv, to, a);
+  attn_tc_kernel<DL, DENSE, FOLD><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv,
+                                                                                               to, a);
   return cudaGetLastError();
 }
 
@@ -510,6 +530,18 @@ int attn_absorbed_block_n(int d_latent) {
 }
 
 int attn_dense_block_n() { return AttnCfg<128, true>::BN; }
+
+cudaError_t launch_attn_absorbed_obar_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
+                                         const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tob_hi,
+                                         const CUtensorMap& tob_lo, const AttnTc& a, int batch, cudaStream_t s) {
+  switch (d_latent) {
+    case 64: return go_attn<64, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 128: return go_attn<128, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 192: return go_attn<192, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 256: return go_attn<256, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& to,
                                  const AttnTc& a, int batch, cudaStream_t s) {

@@ -605,6 +605,172 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================== folded output mixer
+// out = O_bar W_fold^T, W_fold = [B_1 | ... | B_n_h], B_h = W_O,h W_uv,h [paperlayer App. E, value
+// path absorbed into the output mixer]: one GEMM with K = n_h * d_c over the softmax-weighted
+// latents of all heads.  O_bar arrives as a bf16 pair (rounded part + residual): two MMAs per
+// k-step into one fp32 accumulator.  Persistent over (128-row tile, 128-column part) items,
+// column part fastest so the CTAs working together share the O_bar rows in L2; K streamed in
+// 64-column blocks through a 3-stage ring; two accumulators alternate; the epilogue parks the
+// fp32 tile as four [128 x 32] SW128 boxes and stores them with TMA.
+struct FoldCfg {
+  static constexpr int BLK = 128 * 128;        // [128 rows x 64 bf16]
+  static constexpr int STAGE = 3 * BLK;        // O_bar rounded, O_bar residual, W_fold rows
+  static constexpr int STAGES = 3;
+  static constexpr int OUT_BYTES = 4 * 16384;  // 128 rows x 128 fp32
+  static constexpr uint32_t TMEM_COLS = 256;   // two accumulators of 128 columns
+  static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 256;
+  static_assert(SMEM <= 227 * 1024, "does not fit");
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fold_gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
+                        const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_out,
+                        const FoldTc a, int items) {
+  using C = FoldCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sout = smem + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sout + C::OUT_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_parts = a.n_out / 128, kblocks = a.k / 64;
+  const Guard g{abort_flag, a.err, a.limit_ns};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 4);
+    mbar_init(&acc_empty[1], 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_hi);
+      prefetch_tmap(&tm_lo);
+      prefetch_tmap(&tm_w);
+      int it = 0;
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+        const int np = item % n_parts, mt = item / n_parts;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          uint8_t* st = smem + s * C::STAGE;
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          tma_load_3d(st, &tm_hi, &full[s], kb * 64, mt * 128, 0);
+          tma_load_3d(st + C::BLK, &tm_lo, &full[s], kb * 64, mt * 128, 0);
+          tma_load_3d(st + 2 * C::BLK, &tm_w, &full[s], kb * 64, np * 128, 0);
+        }
+      }
+      if (*abort_flag)
+        for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+          drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      int it = 0, j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        const int acc = j & 1;
+        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!(ok = wait_phase(&full[s], (it / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::STAGE);
+          const uint64_t hd = smem_desc(st, 16, 1024, LAYOUT_SW128);
+          const uint64_t ld = smem_desc(st + C::BLK, 16, 1024, LAYOUT_SW128);
+          const uint64_t wd = smem_desc(st + 2 * C::BLK, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (k == 0 && kb == 0)
+              mma_ss_c<false>(tbase + acc * 128, desc_add(hd, k * 32), desc_add(wd, k * 32), idesc);
+            else
+              mma_ss_c<true>(tbase + acc * 128, desc_add(hd, k * 32), desc_add(wd, k * 32), idesc);
+            mma_ss_c<true>(tbase + acc * 128, desc_add(ld, k * 32), desc_add(wd, k * 32), idesc);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+      }
+      mma_commit(done);
+      if (*abort_flag) drain_phase(done, 0, g);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const int np = item % n_parts, mt = item / n_parts;
+      const int acc = j & 1;
+      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      __syncwarp();
+      tc_fence_after();
+      if (tid == 0) bulk_wait_all_read();  // the previous tile's stores have read the parked image
+      named_bar_sync(1, 128);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_addr(tbase, wq * 32, acc * 128 + c0), v);
+        uint8_t* row = sout + (c0 >> 5) * 16384 + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(row + ((q ^ (r & 7)) << 4)) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      named_bar_sync(1, 128);
+      if (tid == 0 && ok && !*abort_flag) {
+        for (int blk = 0; blk < 4; ++blk) tma_store_3d(&tm_out, sout + blk * 16384, np * 128 + blk * 32, mt * 128, 0);
+        bulk_commit();
+      }
+    }
+    if (tid == 0) bulk_wait_all_read();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// B_h = W_O,h W_uv,h side by side (one-time weight preparation; fp32 sums, bf16 out):
+// w_fold[o][h*d_c + c] = sum_e w_o[o][h*d_v + e] * w_uv[h][e][c]
+__global__ void fold_weights_kernel(const __nv_bfloat16* w_o, const __nv_bfloat16* w_uv, __nv_bfloat16* w_fold,
+                                    int d_out, int n_heads, int d_v, int d_c) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)d_out * n_heads * d_c;
+  if (idx >= total) return;
+  const int c = idx % d_c, h = (idx / d_c) % n_heads;
+  const int64_t o = idx / ((int64_t)d_c * n_heads);
+  const __nv_bfloat16* wo = w_o + o * n_heads * d_v + (int64_t)h * d_v;
+  const __nv_bfloat16* wu = w_uv + (int64_t)h * d_v * d_c + c;
+  float acc = 0.f;
+  for (int e = 0; e < d_v; ++e) acc = fmaf(__bfloat162float(wo[e]), __bfloat162float(wu[(int64_t)e * d_c]), acc);
+  w_fold[idx] = __float2bfloat16_rn(acc);
+}
+
 template <class K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -673,6 +839,31 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
 
 }  // namespace
 
+
+cudaError_t launch_fold_gemm_tc(const CUtensorMap& thi, const CUtensorMap& tlo, const CUtensorMap& tw,
+                                const CUtensorMap& to, const FoldTc& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  if (a.k % 64 != 0 || a.n_out % 128 != 0) return cudaErrorInvalidValue;
+  static const cudaError_t attr = set_smem(fold_gemm_tc_kernel, FoldCfg::SMEM);
+  if (attr != cudaSuccess) return attr;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((a.rows + 127) / 128) * (a.n_out / 128);
+  fold_gemm_tc_kernel<<<std::min(items, sms), kThreads, FoldCfg::SMEM, s>>>(thi, tlo, tw, to, a, items);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_weights(const __nv_bfloat16* w_o, const __nv_bfloat16* w_uv, __nv_bfloat16* w_fold, int d_out,
+                                int n_heads, int d_v, int d_c, cudaStream_t s) {
+  const int64_t total = (int64_t)d_out * n_heads * d_c;
+  if (total == 0) return cudaSuccess;
+  fold_weights_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(w_o, w_uv, w_fold, d_out, n_heads, d_v, d_c);
+  return cudaGetLastError();
+}
 
 AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ctas) {
   int dev = 0, sms = 148;

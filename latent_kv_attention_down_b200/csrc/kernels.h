@@ -165,6 +165,28 @@ cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tm_q, const
                                     const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
 int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the key maps)
 
+// Absorbed attention that stores O_bar = softmax-weighted latents / l (per head, d_c wide) as a
+// bf16 pair instead of applying W_uv,h: maps 3D (n_h*d_c, n_q, B) bf16 box (64,128,1) SW128 for
+// the rounded part (tob_hi) and the residual (tob_lo).
+cudaError_t launch_attn_absorbed_obar_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
+                                         const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr,
+                                         const CUtensorMap& tob_hi, const CUtensorMap& tob_lo, const AttnTc& a,
+                                         int batch, cudaStream_t s);
+
+// Folded output mixer: out [rows][n_out] fp32 = (O_bar hi + lo) [rows][k] x w_fold[n_out][k]^T.
+// Maps 3D with a unit last extent: hi/lo (k, rows, 1) bf16 box (64,128,1) SW128; w_fold (k, n_out, 1)
+// box (64,128,1) SW128; out (n_out, rows, 1) fp32 box (32,128,1) SW128.  k % 64 == 0, n_out % 128 == 0.
+struct FoldTc {
+  int rows, k, n_out;
+  unsigned* err;
+  uint64_t limit_ns;
+};
+cudaError_t launch_fold_gemm_tc(const CUtensorMap& tm_hi, const CUtensorMap& tm_lo, const CUtensorMap& tm_w,
+                                const CUtensorMap& tm_out, const FoldTc& a, cudaStream_t s);
+// w_fold [d_out][n_h*d_c] = W_O,h W_uv,h side by side (w_o [d_out][n_h*d_v], w_uv [n_h][d_v][d_c]).
+cudaError_t launch_fold_weights(const __nv_bfloat16* w_o, const __nv_bfloat16* w_uv, __nv_bfloat16* w_fold, int d_out,
+                                int n_heads, int d_v, int d_c, cudaStream_t s);
+
 // Reconstruct-in-tile design (attn_rt.cu), d_latent 64, 128 or 192.  q map: dense queries
 // 3D (128, n_q, B*n_h) box (64,128,1) SW128; ckv map box (64,128,1) SW128; kr map box (32,128,1)
 // SW64; w_uk map 3D (d_c, 96, n_h) box (64,96,1); w_uv map box (64,128,1); out fp32 box (32,128,1).

@@ -24,7 +24,7 @@ using namespace vmla;
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any healthy pipeline wait
-constexpr int kStages = 8;
+constexpr int kStages = 9;
 constexpr int kMaxPos = 1024;  // RoPE range per axis [paperlayer App. C.1]
 
 size_t esize(const vmla_config& c) { return c.dtype == VMLA_BF16 ? 2 : 4; }
@@ -33,7 +33,7 @@ int64_t ring_rows(const vmla_config& c) { return (int64_t)c.window_frames * toke
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, recon = 0;  // offsets
+  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, obar = 0, recon = 0;  // offsets
   size_t base_bytes = 0;   // every design but RECON_ONCE
   size_t recon_bytes = 0;  // extra for RECON_ONCE
 };
@@ -52,6 +52,8 @@ WsLayout ws_layout(const vmla_config& c) {
   off = align256(off + B * c.n_heads * nq * dh * e);
   w.chunk = off;  // a chunk's latents: [B][rows][d_c + d_rope] (plus a d_rope copy for fp32)
   off = align256(off + B * (size_t)c.window_frames * tokens_per_frame(c) * (size_t)(c.d_latent + 2 * c.d_rope) * e);
+  w.obar = off;  // the folded output mixer's input: O_bar as a bf16 pair [2][B][rows][n_h * d_c]
+  off = align256(off + (c.dtype == VMLA_BF16 ? 2 * B * nq * c.n_heads * (size_t)c.d_latent * 2 : 0));
   w.recon = off;
   w.base_bytes = off;
   w.recon_bytes = B * ring_rows(c) * 2 * (size_t)c.n_heads * c.d_value * e;
@@ -574,8 +576,15 @@ vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void*
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const void* kv_base, void* out, int nq,
                                         int n_keys, int64_t t_first, int stage, cudaStream_t s);
 
+// The folded output mixer: out = O_bar W_fold^T instead of the per-head W_uv,h.
+struct FoldArgs {
+  const void* w_fold;  // [d_out][n_h * d_c]
+  int d_out;
+};
+
 vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
-                           int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s) {
+                           int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s,
+                           const FoldArgs* fold = nullptr) {
   const vmla_config& c = h->cfg;
   if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   const WsLayout w = ws_layout(c);
@@ -699,12 +708,14 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
         !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !map3(&tk, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, bn,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
-              CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
-              (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+        !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B))
+      return map_fail();
+    if (!fold &&
+        (!map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+               CU_TENSOR_MAP_SWIZZLE_128B) ||
+         !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
+               (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_DATA_TYPE_FLOAT32)))
       return map_fail();
     AttnTc a;
     a.n_q = nq;
@@ -715,9 +726,34 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.rescale_threshold = c.softmax_rescale_log2;
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    e = launch_attn_absorbed_tc(c.d_latent, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
+    if (!fold) {
+      e = launch_attn_absorbed_tc(c.d_latent, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
+    } else {
+      const uint64_t kf = (uint64_t)c.n_heads * c.d_latent;
+      __nv_bfloat16* ob_hi = at<__nv_bfloat16>(h->ws, w.obar);
+      __nv_bfloat16* ob_lo = ob_hi + (size_t)c.batch * nq * kf;
+      CUtensorMap thi, tlo;
+      if (!map3(&thi, ob_hi, kf, nq, c.batch, kf * 2, (uint64_t)nq * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map3(&tlo, ob_lo, kf, nq, c.batch, kf * 2, (uint64_t)nq * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return map_fail();
+      e = launch_attn_absorbed_obar_tc(c.d_latent, tq, tqr, tk, tkr, thi, tlo, a, c.batch, s);
+    }
   }
-  return cuda_status(e);
+  if (e != cudaSuccess || !fold) return cuda_status(e);
+  StageScope scope(h, 8, s);
+  const uint64_t kf = (uint64_t)c.n_heads * c.d_latent, rows = (uint64_t)c.batch * nq;
+  __nv_bfloat16* ob_hi = at<__nv_bfloat16>(h->ws, w.obar);
+  __nv_bfloat16* ob_lo = ob_hi + rows * kf;
+  CUtensorMap thi, tlo, tw, to;
+  if (!map3(&thi, ob_hi, kf, rows, 1, kf * 2, rows * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&tlo, ob_lo, kf, rows, 1, kf * 2, rows * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&tw, fold->w_fold, kf, fold->d_out, 1, kf * 2, (uint64_t)fold->d_out * kf * 2, 64, 128,
+            CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3(&to, out, fold->d_out, rows, 1, (uint64_t)fold->d_out * 4, rows * fold->d_out * 4, 32, 128,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+    return map_fail();
+  FoldTc fa{(int)rows, (int)kf, fold->d_out, h->err, kWaitLimitNs};
+  return cuda_status(launch_fold_gemm_tc(thi, tlo, tw, to, fa, s));
 }
 
 // Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128].
@@ -778,6 +814,38 @@ vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const
     return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
   return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s);
+}
+
+vmla_status vmla_fold_output_weights(const vmla_config* cfg, const void* w_o, const void* w_uv, void* w_fold,
+                                     int d_out, void* stream) {
+  if (!cfg || !w_o || !w_uv || !w_fold) return VMLA_ERR_INVALID_ARG;
+  vmla_status st = vmla_config_check(cfg);
+  if (st != VMLA_OK) return st;
+  if (cfg->dtype != VMLA_BF16) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (d_out < 1) return VMLA_ERR_INVALID_ARG;
+  return cuda_status(launch_fold_weights(static_cast<const __nv_bfloat16*>(w_o),
+                                         static_cast<const __nv_bfloat16*>(w_uv), static_cast<__nv_bfloat16*>(w_fold),
+                                         d_out, cfg->n_heads, cfg->d_value, cfg->d_latent,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+vmla_status vmla_chunk_attention_folded(vmla_handle* h, int layer, const void* q, const void* w_uk,
+                                        const void* w_fold, int d_out, void* out, int64_t first, int n,
+                                        void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->ckv) return VMLA_ERR_STATE;
+  if (!q || !w_uk || !w_fold || !out || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_fold) || !aligned16(out))
+    return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  if (c.dtype != VMLA_BF16 || c.d_latent > 256 || d_out < 128 || d_out % 128 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  Window win;
+  if ((st = check_attention_frames(c, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
+  if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  const FoldArgs fold{w_fold, d_out};
+  return attention_bf16(h, layer, q, w_uk, nullptr, out, first, n, win, VMLA_DESIGN_ABSORBED,
+                        static_cast<cudaStream_t>(stream), &fold);
 }
 
 vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, const void* w_uk,

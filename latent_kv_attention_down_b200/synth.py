@@ -25,6 +25,7 @@ import numpy as np
 
 # tensor ids inside a seed sequence
 _T_X, _T_Q, _T_WDOWN, _T_WUK, _T_WUV = 1, 2, 3, 4, 5
+_T_WO, _T_CQ, _T_WUQ, _T_WQR = 9, 10, 11, 12
 
 
 @dataclasses.dataclass(frozen=True)
@@ -128,6 +129,7 @@ class LayerWeights:
     w_down: np.ndarray  # [d_latent + d_rope, d_model]: rows 0..d_latent-1 are W_dkv, the rest W_kr
     w_uk: np.ndarray    # [n_heads, d_nope, d_latent]
     w_uv: np.ndarray    # [n_heads, d_head, d_latent]
+    w_o: np.ndarray = None  # [d_model, n_heads * d_head], the output mixer
 
 
 def weights(dims: Dims, layer: int = 0, base_seed: int = 0) -> LayerWeights:
@@ -135,7 +137,9 @@ def weights(dims: Dims, layer: int = 0, base_seed: int = 0) -> LayerWeights:
     w_down = gaussian(d, (d.d_latent + d.d_rope, d.d_model), d.d_model ** -0.5, layer, 0, 0, _T_WDOWN, base_seed)
     w_uk = gaussian(d, (d.n_heads, d.d_nope, d.d_latent), d.d_latent ** -0.5, layer, 0, 0, _T_WUK, base_seed)
     w_uv = gaussian(d, (d.n_heads, d.d_head, d.d_latent), d.d_latent ** -0.5, layer, 0, 0, _T_WUV, base_seed)
-    return LayerWeights(w_down, w_uk, w_uv)
+    w_o = gaussian(d, (d.d_model, d.n_heads * d.d_head), (d.n_heads * d.d_head) ** -0.5, layer, 0, 0, _T_WO,
+                   base_seed)
+    return LayerWeights(w_down, w_uk, w_uv, w_o)
 
 
 def activations(dims: Dims, layer: int, chunk: int, pass_: int = 0, n_frames: int | None = None,

@@ -267,6 +267,43 @@ def chunk_attention_absorbed(c, r, key_pos, q, query_pos, w_uk, w_uv, *, d_nope,
     return out
 
 
+def output_projection(o_heads: np.ndarray, w_o: np.ndarray) -> np.ndarray:
+    """The layer's output mixer after attention: out = W_O [o_1 | ... | o_n_h] with
+    o_heads [N, n_h, d_v] and W_O [d_out, n_h * d_v]."""
+    o = np.asarray(o_heads, dtype=np.float64)
+    return o.reshape(o.shape[0], -1) @ np.asarray(w_o, dtype=np.float64).T
+
+
+def fold_output_weights(w_o: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """B_h = W_O,h W_uv,h for every head, side by side: [d_out, n_h * d_c]
+    [paperlayer App. E: the value path's W_uv,h is absorbed after accumulation,
+    here all the way into the output mixer]."""
+    n_h, d_v, d_c = w_uv.shape
+    w_o = np.asarray(w_o, dtype=np.float64)
+    return np.concatenate([w_o[:, h * d_v:(h + 1) * d_v] @ np.asarray(w_uv[h], np.float64) for h in range(n_h)],
+                          axis=1)
+
+
+def chunk_attention_folded(c, r, key_pos, q, query_pos, w_uk, w_fold, *, d_nope, rope_pairs,
+                           rope_theta=10000.0, rope_base_dims=None) -> np.ndarray:
+    """The absorbed form end to end: out = sum_h B_h o~_h with o~_h = sum_j p_hj c_j
+    the softmax-weighted latents of head h and w_fold = [B_1 | ... | B_n_h].  Used
+    only to check it against output_projection(chunk_attention(...), W_O)."""
+    freqs = rope_frequencies(rope_pairs, rope_theta, rope_base_dims)
+    key_pos = np.asarray(key_pos)
+    k_rope = rope_rotate(r, rope_angles(key_pos[:, 0], key_pos[:, 1], key_pos[:, 2], freqs))
+    qr = rotate_queries(q, np.asarray(query_pos), d_nope, freqs)
+    c64 = np.asarray(c, dtype=np.float64)
+    key = np.concatenate([c64, k_rope], axis=1)
+    scale = 1.0 / math.sqrt(qr.shape[2])
+    n_h, d_c = w_uk.shape[0], c64.shape[1]
+    o_lat = np.zeros((q.shape[0], n_h * d_c))
+    for h in range(n_h):
+        q_tilde = np.concatenate([qr[:, h, :d_nope] @ np.asarray(w_uk[h], np.float64), qr[:, h, d_nope:]], axis=1)
+        o_lat[:, h * d_c:(h + 1) * d_c] = softmax_attention(q_tilde, key, c64, scale)
+    return o_lat @ np.asarray(w_fold, dtype=np.float64).T
+
+
 def dense_cache_entries(c, r, key_pos, w_uk, w_uv, *, rope_pairs, rope_theta=10000.0,
                         rope_base_dims=None):
     """The per-head dense layout of the same keys and values (2 n_h d_h scalars

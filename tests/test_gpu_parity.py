@@ -346,6 +346,31 @@ def test_wan_layer_sampled_rows():
     assert_bf16_close(out[0][rows], ref, "wan layer")
 
 
+# ------------------------------------------------------------------ W_uv folded into the output mixer
+
+def test_small_bf16_folded_output_mixer():
+    """out = sum_h (W_O,h W_uv,h) o~_h through the library (weight fold, absorbed
+    attention handing o~ over as a bf16 pair, one K = 12 x 192 GEMM) against W_O
+    applied to the oracle's per-head outputs."""
+    import torch
+    import oracle.vmla_oracle as O
+    d = SMALL
+    ro = Rollout(d)
+    _fill(ro, 7)
+    w = ro.w[0]
+    w_fold = torch.empty(d.d_model, d.n_heads * d.d_latent, dtype=torch.bfloat16, device="cuda")
+    ro.m.fold_output_weights(to_dev(w.w_o, d), ro.wd[0][2], w_fold)
+    ref_fold = O.fold_output_weights(w.w_o, w.w_uv)
+    got_fold = w_fold.float().cpu().numpy()
+    assert np.all(np.abs(got_fold - ref_fold) <= 2.0 ** -8 * np.abs(ref_fold) + 1e-6 * np.abs(ref_fold).max())
+    q = synth.queries(d, 0, 6)
+    out = torch.full((1, d.n_queries, d.d_model), float("nan"), dtype=torch.float32, device="cuda")
+    ro.m.attention_folded(0, to_dev(q, d), ro.wd[0][1], w_fold, out, 18, 3)
+    assert ro.m.device_status()[0] == 0
+    heads = ro.oracle(0, 6, q).reshape(d.n_queries, d.n_heads, d.d_head)
+    assert_bf16_close(out[0].cpu().numpy(), O.output_projection(heads, w.w_o), "folded output mixer")
+
+
 # ------------------------------------------------------------------ sink frame + local window
 
 def test_tiny_fp32_sink_window():

@@ -170,3 +170,29 @@ def test_wan_sink_window_sampled_rows():
     for chunk in range(12):
         ro.step(0, chunk, 0)
     ro.check(0, 11, 0, what="sink window")
+
+
+def test_wan_folded_output_mixer_sampled_rows():
+    """The folded output mixer at the Wan layer shape (K = 12 x 192, d_out = 1536)."""
+    import torch
+    import oracle.vmla_oracle as O
+    d = WAN
+    ro = PoolRollout(d, 1)
+    for chunk in range(7):
+        ro.step(0, chunk, 0)
+    w = ro.w[0]
+    w_fold = torch.empty(d.d_model, d.n_heads * d.d_latent, dtype=torch.bfloat16, device="cuda")
+    ro.m.fold_output_weights(to_dev(w.w_o, d), ro.wd[0][2], w_fold)
+    out = torch.empty(1, d.n_queries, d.d_model, dtype=torch.float32, device="cuda")
+    ro.m.attention_folded(0, ro.pool.queries(0, 6, 0, pool=ro.qp), ro.wd[0][1], w_fold, out, 18, 3)
+    assert ro.m.device_status()[0] == 0
+    rows = sampled_rows(d.n_queries, 256, seed=5)
+    frame_x = {}
+    T = d.tokens_per_frame
+    for c in range(7):
+        x = ro.pool.activations(0, c, 0)
+        for k in range(d.chunk_frames):
+            frame_x[c * d.chunk_frames + k] = x[0, k * T:(k + 1) * T]
+    heads = oracle_chunk(d, w, frame_x, 6, ro.pool.queries(0, 6, 0)[0], rows=rows)
+    ref = O.output_projection(heads.reshape(len(rows), d.n_heads, d.d_head), w.w_o)
+    assert_bf16_close(out[0].cpu().numpy()[rows], ref, "folded output mixer, Wan layer")

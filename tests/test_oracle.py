@@ -441,3 +441,28 @@ def test_sink_window_latents_positions():
     assert list(pos[::T, 0]) == [0, 1, 2, 3] and t0 == 8         # frames 9, 10, 11 at t = 1, 2, 3
     q = O.chunk_query_positions(11, 1, t0, 2, 3)
     assert q[0, 0] == 3
+
+
+# ---------------------------------------------------------------- output mixer folded into the value path
+def test_folded_output_equals_projected_heads():
+    """sum_h (W_O,h W_uv,h) o~_h (absorbed all the way into the output mixer) equals
+    W_O applied to the concatenated per-head outputs of the non-absorbed definition."""
+    rng = np.random.default_rng(11)
+    n_h, d_nope, d_rope, d_c, N_k, N_q, d_out = 3, 6, 4, 5, 17, 7, 9
+    c = rng.standard_normal((N_k, d_c))
+    r = rng.standard_normal((N_k, d_rope))
+    kpos = rng.integers(0, 6, (N_k, 3))
+    q = rng.standard_normal((N_q, n_h, d_nope + d_rope))
+    qpos = rng.integers(0, 6, (N_q, 3))
+    w_uk = rng.standard_normal((n_h, d_nope, d_c))
+    w_uv = rng.standard_normal((n_h, d_nope + d_rope, d_c))
+    w_o = rng.standard_normal((d_out, n_h * (d_nope + d_rope)))
+    kw = dict(d_nope=d_nope, rope_pairs=(1, 0, 1))
+    ref = O.output_projection(O.chunk_attention(c, r, kpos, q, qpos, w_uk, w_uv, **kw), w_o)
+    fold = O.fold_output_weights(w_o, w_uv)
+    assert fold.shape == (d_out, n_h * d_c)
+    got = O.chunk_attention_folded(c, r, kpos, q, qpos, w_uk, fold, **kw)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+    # a head block in the wrong place must not pass
+    bad = np.concatenate([fold[:, d_c:2 * d_c], fold[:, :d_c], fold[:, 2 * d_c:]], axis=1)
+    assert np.abs(O.chunk_attention_folded(c, r, kpos, q, qpos, w_uk, bad, **kw) - ref).max() > 1e-3
