@@ -48,6 +48,7 @@ class Dims:
     rope_theta: float = 10000.0
     rope_base_dims: tuple = (0, 0, 0)  # 0 = twice the pair count of the axis
     sink_frames: int = 0  # leading frames pinned in the ring (window_frames counts them)
+    d_q: int = 768  # query latent width
 
     @property
     def d_head(self) -> int:
@@ -140,6 +141,19 @@ def weights(dims: Dims, layer: int = 0, base_seed: int = 0) -> LayerWeights:
     w_o = gaussian(d, (d.d_model, d.n_heads * d.d_head), (d.n_heads * d.d_head) ** -0.5, layer, 0, 0, _T_WO,
                    base_seed)
     return LayerWeights(w_down, w_uk, w_uv, w_o)
+
+
+def query_latent_weights(dims: Dims, layer: int = 0, base_seed: int = 0):
+    """W_uq [n_heads, d_nope, d_q] and W_qr [n_heads, d_rope, d_q], N(0, 1/d_q)."""
+    d = dims
+    w_uq = gaussian(d, (d.n_heads, d.d_nope, d.d_q), d.d_q ** -0.5, layer, 0, 0, _T_WUQ, base_seed)
+    w_qr = gaussian(d, (d.n_heads, d.d_rope, d.d_q), d.d_q ** -0.5, layer, 0, 0, _T_WQR, base_seed)
+    return w_uq, w_qr
+
+
+def query_latents(dims: Dims, layer: int, chunk: int, pass_: int = 0, base_seed: int = 0) -> np.ndarray:
+    """c_Q of one chunk: [batch, chunk_frames * tokens_per_frame, d_q], N(0, 1)."""
+    return gaussian(dims, (dims.batch, dims.n_queries, dims.d_q), 1.0, layer, chunk, pass_, _T_CQ, base_seed)
 
 
 def activations(dims: Dims, layer: int, chunk: int, pass_: int = 0, n_frames: int | None = None,

@@ -304,6 +304,46 @@ def chunk_attention_folded(c, r, key_pos, q, query_pos, w_uk, w_fold, *, d_nope,
     return o_lat @ np.asarray(w_fold, dtype=np.float64).T
 
 
+def query_from_latent(c_q: np.ndarray, w_uq: np.ndarray, w_qr: np.ndarray) -> np.ndarray:
+    """Per-head queries from the query latent c_Q [N, d_q] [paperlayer §4: d_q = 768]:
+    q_h = [W_uq,h c_Q | W_qr,h c_Q] with w_uq [n_h, d_nope, d_q], w_qr [n_h, d_rope, d_q];
+    returns [N, n_h, d_nope + d_rope] (positional part not yet rotated)."""
+    c = np.asarray(c_q, dtype=np.float64)
+    return np.concatenate([np.einsum("nj,hdj->nhd", c, np.asarray(w_uq, np.float64)),
+                           np.einsum("nj,hdj->nhd", c, np.asarray(w_qr, np.float64))], axis=2)
+
+
+def fold_query_weights(w_uq: np.ndarray, w_qr: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
+    """A_h = W_uk,h^T W_uq,h stacked over W_qr,h: [n_h, d_c + d_rope, d_q] [paperlayer App. E,
+    content path absorbed into the query latent]."""
+    a = np.einsum("hnc,hnj->hcj", np.asarray(w_uk, np.float64), np.asarray(w_uq, np.float64))
+    return np.concatenate([a, np.asarray(w_qr, np.float64)], axis=1)
+
+
+def chunk_attention_query_latent(c, r, key_pos, c_q, query_pos, w_qabs, w_uv, *, d_latent, d_head, rope_pairs,
+                                 rope_theta=10000.0, rope_base_dims=None) -> np.ndarray:
+    """The absorbed form fed from the query latent: q~_h = [A_h c_Q | RoPE(W_qr,h c_Q)]
+    (w_qabs from fold_query_weights) against the shared key [c | RoPE(k_R)].  Used only to
+    check it against chunk_attention(query_from_latent(...))."""
+    freqs = rope_frequencies(rope_pairs, rope_theta, rope_base_dims)
+    key_pos = np.asarray(key_pos)
+    qpos = np.asarray(query_pos)
+    k_rope = rope_rotate(r, rope_angles(key_pos[:, 0], key_pos[:, 1], key_pos[:, 2], freqs))
+    c64 = np.asarray(c, dtype=np.float64)
+    key = np.concatenate([c64, k_rope], axis=1)
+    d_rope = key.shape[1] - d_latent
+    scale = 1.0 / math.sqrt(d_head)  # the per-head score is a (d_nope + d_rope)-dim dot product
+    n_h = w_qabs.shape[0]
+    cq = np.asarray(c_q, dtype=np.float64)
+    out = np.zeros((cq.shape[0], n_h, w_uv.shape[1]))
+    for h in range(n_h):
+        qt = cq @ np.asarray(w_qabs[h], np.float64).T
+        qt[:, d_latent:] = rope_rotate(qt[:, d_latent:], rope_angles(qpos[:, 0], qpos[:, 1], qpos[:, 2], freqs))
+        out[:, h] = softmax_attention(qt, key, c64, scale) @ np.asarray(w_uv[h], np.float64).T
+    assert d_rope == 2 * sum(rope_pairs)
+    return out
+
+
 def dense_cache_entries(c, r, key_pos, w_uk, w_uv, *, rope_pairs, rope_theta=10000.0,
                         rope_base_dims=None):
     """The per-head dense layout of the same keys and values (2 n_h d_h scalars

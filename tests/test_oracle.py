@@ -466,3 +466,32 @@ def test_folded_output_equals_projected_heads():
     # a head block in the wrong place must not pass
     bad = np.concatenate([fold[:, d_c:2 * d_c], fold[:, :d_c], fold[:, 2 * d_c:]], axis=1)
     assert np.abs(O.chunk_attention_folded(c, r, kpos, q, qpos, w_uk, bad, **kw) - ref).max() > 1e-3
+
+
+# ---------------------------------------------------------------- content path absorbed into the query latent
+def test_query_latent_absorption_equals_the_definition():
+    """q~_h = [W_uk,h^T W_uq,h c_Q | RoPE(W_qr,h c_Q)] against the shared latent key gives
+    what the per-head queries W_uq,h c_Q, W_qr,h c_Q give in the non-absorbed definition."""
+    rng = np.random.default_rng(12)
+    n_h, d_nope, d_rope, d_c, d_q, N_k, N_q = 2, 6, 4, 5, 11, 13, 6
+    c = rng.standard_normal((N_k, d_c))
+    r = rng.standard_normal((N_k, d_rope))
+    kpos = rng.integers(0, 5, (N_k, 3))
+    cq = rng.standard_normal((N_q, d_q))
+    qpos = rng.integers(0, 5, (N_q, 3))
+    w_uq = rng.standard_normal((n_h, d_nope, d_q))
+    w_qr = rng.standard_normal((n_h, d_rope, d_q))
+    w_uk = rng.standard_normal((n_h, d_nope, d_c))
+    w_uv = rng.standard_normal((n_h, d_nope + d_rope, d_c))
+    kw = dict(rope_pairs=(1, 0, 1))
+    q = O.query_from_latent(cq, w_uq, w_qr)
+    assert q.shape == (N_q, n_h, d_nope + d_rope)
+    ref = O.chunk_attention(c, r, kpos, q, qpos, w_uk, w_uv, d_nope=d_nope, **kw)
+    w_qabs = O.fold_query_weights(w_uq, w_qr, w_uk)
+    assert w_qabs.shape == (n_h, d_c + d_rope, d_q)
+    got = O.chunk_attention_query_latent(c, r, kpos, cq, qpos, w_qabs, w_uv, d_latent=d_c, d_head=d_nope + d_rope, **kw)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+    bad = w_qabs.copy()
+    bad[:, :d_c] = np.einsum("hnc,hnj->hcj", w_uk, w_uq[::-1])   # heads crossed
+    assert np.abs(O.chunk_attention_query_latent(c, r, kpos, cq, qpos, bad, w_uv, d_latent=d_c,
+                                                 d_head=d_nope + d_rope, **kw) - ref).max() > 1e-3
