@@ -400,7 +400,8 @@ def run_ours(args, rank, world, local_rank):
         line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
                         "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed),
                         "sink_window": sink_leg(dev=dev, tc=tc_burst, seed=seed),
-                        "folded_output_mixer": folded_leg(dev=dev, tc=tc_burst, seed=seed)}
+                        "folded_output_mixer": folded_leg(dev=dev, tc=tc_burst, seed=seed),
+                        "query_latent": qlatent_leg(dev=dev, seed=seed)}
     if dense:
         line["dense"] = dense
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -591,6 +592,62 @@ def folded_leg(dev, tc, seed, steps=50):
     return {"workload": "wan1.3b-layer chunk step with W_O W_uv folded (K=2304, d_out=1536)", "ms_per_step": ms,
             "attention_ms": k["attention"][0] / max(k["attention"][1], 1), "mixer_gemm_ms": gemm_ms,
             "mixer_gemm_tflops": gemm_flops / (gemm_ms * 1e-3) / 1e12}
+
+
+def qlatent_leg(dev, seed, steps=50):
+    """The content path absorbed into the query latent: the chunk step whose absorbed queries
+    come from c_Q (d_q = 768) by one K = 768 GEMM per head instead of W_uk,h^T q_nope."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    d = WORKLOAD
+    L = 4
+    m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+    pool = synth.FramePool(d, base_seed=seed)
+    bf = torch.bfloat16
+    xp = torch.from_numpy(pool.x).to(dev, bf)
+    ws = [synth.weights(d, l, seed) for l in range(L)]
+    W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv)) for w in ws]
+    qabs = []
+    for l in range(L):
+        w_uq, w_qr = synth.query_latent_weights(d, l, seed)
+        f = torch.empty(d.n_heads, d.d_latent + d.d_rope, d.d_q, dtype=bf, device=dev)
+        m.fold_query_weights(torch.from_numpy(w_uq).to(dev, bf), torch.from_numpy(w_qr).to(dev, bf), W[l][1], f)
+        qabs.append(f)
+    chunks = d.window_frames // d.chunk_frames
+    for l in range(L):
+        for c in range(chunks):
+            m.append(l, pool.activations(l, c, 0, pool=xp), W[l][0], c * d.chunk_frames, d.chunk_frames)
+    first = (chunks - 1) * d.chunk_frames
+    xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
+    cqs = [torch.from_numpy(synth.query_latents(d, l, chunks - 1, 1, seed)).to(dev, bf) for l in range(L)]
+    out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
+
+    def step(i):
+        l = i % L
+        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+        m.attention_qlatent(l, cqs[l], qabs[l], W[l][2], out, first, d.chunk_frames)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    m.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    k = {n: m.profile_read(n) for n in ("q_absorb", "attention")}
+    m.profile(False)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    q_ms = k["q_absorb"][0] / max(k["q_absorb"][1], 1)
+    q_flops = 2 * d.n_queries * d.n_heads * (d.d_latent + d.d_rope) * d.d_q
+    m.close()
+    return {"workload": "wan1.3b-layer chunk step, absorbed queries from c_Q (d_q=768)", "ms_per_step": ms,
+            "query_gemm_ms": q_ms, "query_gemm_tflops": q_flops / (q_ms * 1e-3) / 1e12,
+            "attention_ms": k["attention"][0] / max(k["attention"][1], 1)}
 
 
 def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384)):

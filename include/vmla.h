@@ -266,6 +266,22 @@ vmla_status vmla_chunk_attention_folded(vmla_handle* h, int layer, const void* q
                                         const void* w_fold, int d_out, void* out, int64_t first_frame,
                                         int n_frames, void* stream);
 
+/* The content path absorbed into the query latent [paperlayer App. E; §4: d_q = 768]:
+ * with q_h = [W_uq,h c_Q | W_qr,h c_Q] the per-head queries of the query latent c_Q,
+ *   q~_h = [A_h c_Q | RoPE(W_qr,h c_Q)],   A_h = W_uk,h^T W_uq,h  (d_latent x d_q),
+ * so the query never exists per head.  vmla_fold_query_weights writes w_qabs
+ * [n_heads][d_latent + d_rope][d_q] = [A_h ; W_qr,h] (bf16, fp32 sums; one-time weight
+ * preparation) from w_uq [n_heads][d_nope][d_q], w_qr [n_heads][d_rope][d_q] and w_uk.
+ * vmla_chunk_attention_qlatent is vmla_chunk_attention with VMLA_DESIGN_ABSORBED whose
+ * query step is one GEMM over K = d_q from c_Q [batch][n_frames*T_f][d_q] (bf16).
+ * VMLA_BF16 with d_latent 64, 128 or 192 and d_q a multiple of 64, else
+ * VMLA_ERR_UNSUPPORTED_SHAPE; frame rules and errors as vmla_chunk_attention. */
+vmla_status vmla_fold_query_weights(const vmla_config* cfg, const void* w_uq, const void* w_qr, const void* w_uk,
+                                    int d_q, void* w_qabs, void* stream);
+vmla_status vmla_chunk_attention_qlatent(vmla_handle* h, int layer, const void* c_q, const void* w_qabs, int d_q,
+                                         const void* w_uv, void* out, int64_t first_frame, int n_frames,
+                                         void* stream);
+
 /* Allocation-free chunk attention.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for example a
  * plugin inside another runtime that is handed only its input and output

@@ -72,6 +72,10 @@ _SIGS = {
     "vmla_device_status": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
     "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int]),
+    "vmla_fold_query_weights": (c_int, [ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                        c_void_p]),
+    "vmla_chunk_attention_qlatent": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
+                                             c_int64, c_int, c_void_p]),
     "vmla_fold_output_weights": (c_int, [ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
     "vmla_chunk_attention_folded": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int64,
                                             c_int, c_void_p]),
@@ -250,6 +254,17 @@ class LatentKVAttention:
         flags = c_uint32()
         st = lib().vmla_device_status(self._h, _stream(stream), ctypes.byref(flags))
         return st, flags.value
+
+    def fold_query_weights(self, w_uq, w_qr, w_uk, w_qabs, stream=None):
+        """w_qabs [n_h][d_c + d_rope][d_q] = [W_uk,h^T W_uq,h ; W_qr,h]."""
+        check(lib().vmla_fold_query_weights(ctypes.byref(self.cfg), _ptr(w_uq), _ptr(w_qr), _ptr(w_uk),
+                                            w_qabs.shape[2], _ptr(w_qabs), _stream(stream)), "vmla_fold_query_weights")
+
+    def attention_qlatent(self, layer, c_q, w_qabs, w_uv, out, first_frame, n_frames, stream=None):
+        """Absorbed chunk attention whose queries come from the query latent c_Q [B][rows][d_q]."""
+        check(lib().vmla_chunk_attention_qlatent(self._h, layer, _ptr(c_q), _ptr(w_qabs), c_q.shape[-1], _ptr(w_uv),
+                                                 _ptr(out), first_frame, n_frames, _stream(stream)),
+              "vmla_chunk_attention_qlatent")
 
     def fold_output_weights(self, w_o, w_uv, w_fold, stream=None):
         """w_fold [d_out][n_h * d_c] = W_O,h W_uv,h side by side."""

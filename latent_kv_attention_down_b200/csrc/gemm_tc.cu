@@ -771,6 +771,183 @@ __global__ void fold_weights_kernel(const __nv_bfloat16* w_o, const __nv_bfloat1
   w_fold[idx] = __float2bfloat16_rn(acc);
 }
 
+// ============================================================== query-latent absorption
+// q~_h = [A_h c_Q | RoPE(W_qr,h c_Q)] with A_h = W_uk,h^T W_uq,h [paperlayer App. E content path,
+// absorbed into the query latent c_Q; §4: d_q = 768]: per (sample, 128-query tile, head) item a
+// GEMM over K = d_q with the stacked weights [A_h ; W_qr,h] ((d_c + 32) rows), streamed in
+// 64-column blocks through a ring; the positional columns are rotated at the queries' positions
+// in the epilogue, which parks all rows unpadded and writes them with one bulk copy.
+template <int DL>
+struct QLatCfg {
+  static constexpr int N = DL + 32;
+  static constexpr int A_BLK = 128 * 128;
+  static constexpr int B_BLK = N * 128;
+  static constexpr int STAGE = A_BLK + B_BLK;
+  static constexpr int OUT_STRIDE = N * 2;
+  static constexpr int OUT_BYTES = 128 * OUT_STRIDE;
+  static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
+  static constexpr int STAGES = FIT > 6 ? 6 : FIT;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int SMEM_USED = 1024 + STAGES * STAGE + OUT_BYTES + 256;
+  static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
+  static_assert(N % 16 == 0 && N <= 256 && B_BLK % 1024 == 0 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
+};
+
+template <int DL>
+__global__ void __launch_bounds__(kThreads, 1)
+    qlat_tc_kernel(const __grid_constant__ CUtensorMap tm_cq, const __grid_constant__ CUtensorMap tm_w,
+                   const QLatTc a, int items) {
+  using C = QLatCfg<DL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sout = smem + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sout + C::OUT_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (a.n_q + 127) / 128, kblocks = a.d_q / 64;
+  const Guard g{abort_flag, a.err, a.limit_ns};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 4);
+    mbar_init(&acc_empty[1], 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_cq);
+      prefetch_tmap(&tm_w);
+      int it = 0;
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+        const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          uint8_t* st = smem + s * C::STAGE;
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          tma_load_3d(st, &tm_cq, &full[s], kb * 64, mt * 128, b);
+          tma_load_3d(st + C::A_BLK, &tm_w, &full[s], kb * 64, 0, h);
+        }
+      }
+      if (*abort_flag)
+        for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+          drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, false, false);
+      int it = 0, j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        const int acc = j & 1;
+        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          if (!(ok = wait_phase(&full[s], (it / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::STAGE);
+          const uint64_t ad = smem_desc(st, 16, 1024, LAYOUT_SW128);
+          const uint64_t bd = smem_desc(st + C::A_BLK, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (k == 0 && kb == 0)
+              mma_ss_c<false>(tbase + acc * 256, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+            else
+              mma_ss_c<true>(tbase + acc * 256, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+      }
+      mma_commit(done);
+      if (*abort_flag) drain_phase(done, 0, g);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int T = a.ring.tokens_per_frame;
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+      const int acc = j & 1;
+      const int i = mt * 128 + r;
+      const int ii = i < a.n_q ? i : 0;
+      const int tok = ii % T;
+      const int t = (int)(a.t_first + ii / T), hh = tok / a.ring.grid_w, ww = tok % a.ring.grid_w;
+      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      __syncwarp();
+      tc_fence_after();
+      const int valid_rows = ok ? min(128, a.n_q - mt * 128) : 0;
+      if (tid == 0) bulk_wait_all_read();  // the previous item's copy has read the parked rows
+      named_bar_sync(1, 128);
+      uint8_t* orow = sout + r * C::OUT_STRIDE;
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::N; c0 += 32) {
+        uint32_t raw[32];
+        tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+        float v[32];
+        raw_to_float(raw, v);
+        if (c0 >= DL) rotate16(v, a.rope, t, hh, ww);  // the 32 positional columns
+        store_bf16x32_smem(orow + c0 * 2, v);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      named_bar_sync(1, 128);
+      if (tid == 0 && valid_rows > 0) {
+        bulk_store(a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + mt * 128) * C::N, sout,
+                   (uint32_t)(valid_rows * C::OUT_STRIDE));
+        bulk_commit();
+      }
+    }
+    if (tid == 0) bulk_wait_all_read();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// [A_h ; W_qr,h] for every head (one-time weight preparation; fp32 sums, bf16 out):
+// w_qabs[h][c][j] = sum_n w_uk[h][n][c] w_uq[h][n][j] (c < d_c), w_qr[h][c - d_c][j] (c >= d_c)
+__global__ void fold_query_kernel(const __nv_bfloat16* w_uq, const __nv_bfloat16* w_qr, const __nv_bfloat16* w_uk,
+                                  __nv_bfloat16* w_qabs, int n_heads, int d_nope, int d_rope, int d_c, int d_q) {
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int rows = d_c + d_rope;
+  if (idx >= (int64_t)n_heads * rows * d_q) return;
+  const int jq = idx % d_q, c = (idx / d_q) % rows, h = idx / ((int64_t)d_q * rows);
+  float acc = 0.f;
+  if (c < d_c) {
+    for (int n = 0; n < d_nope; ++n)
+      acc = fmaf(__bfloat162float(w_uk[((int64_t)h * d_nope + n) * d_c + c]),
+                 __bfloat162float(w_uq[((int64_t)h * d_nope + n) * d_q + jq]), acc);
+  } else {
+    acc = __bfloat162float(w_qr[((int64_t)h * d_rope + (c - d_c)) * d_q + jq]);
+  }
+  w_qabs[idx] = __float2bfloat16_rn(acc);
+}
+
 template <class K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -862,6 +1039,47 @@ cudaError_t launch_fold_weights(const __nv_bfloat16* w_o, const __nv_bfloat16* w
   const int64_t total = (int64_t)d_out * n_heads * d_c;
   if (total == 0) return cudaSuccess;
   fold_weights_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(w_o, w_uv, w_fold, d_out, n_heads, d_v, d_c);
+  return cudaGetLastError();
+}
+
+template <int DL>
+cudaError_t go_qlat(const CUtensorMap& tc, const CUtensorMap& tw, const QLatTc& a, int batch, cudaStream_t s) {
+  using C = QLatCfg<DL>;
+  static const cudaError_t attr = set_smem(qlat_tc_kernel<DL>, C::SMEM);
+  if (attr != cudaSuccess) return attr;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
+  qlat_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tw, a, items);
+  return cudaGetLastError();
+}
+
+bool qlat_supported(int d_latent, int d_q) {
+  return (d_latent == 64 || d_latent == 128 || d_latent == 192) && d_q > 0 && d_q % 64 == 0;
+}
+
+cudaError_t launch_qlat_tc(const CUtensorMap& tc, const CUtensorMap& tw, const QLatTc& a, int batch, cudaStream_t s) {
+  if (a.n_q <= 0) return cudaSuccess;
+  if (!qlat_supported(a.d_latent, a.d_q)) return cudaErrorInvalidValue;
+  switch (a.d_latent) {
+    case 64: return go_qlat<64>(tc, tw, a, batch, s);
+    case 128: return go_qlat<128>(tc, tw, a, batch, s);
+    case 192: return go_qlat<192>(tc, tw, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fold_query(const __nv_bfloat16* w_uq, const __nv_bfloat16* w_qr, const __nv_bfloat16* w_uk,
+                              __nv_bfloat16* w_qabs, int n_heads, int d_nope, int d_rope, int d_c, int d_q,
+                              cudaStream_t s) {
+  const int64_t total = (int64_t)n_heads * (d_c + d_rope) * d_q;
+  if (total == 0) return cudaSuccess;
+  fold_query_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(w_uq, w_qr, w_uk, w_qabs, n_heads, d_nope, d_rope,
+                                                                   d_c, d_q);
   return cudaGetLastError();
 }
 

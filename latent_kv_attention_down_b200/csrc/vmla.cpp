@@ -582,9 +582,16 @@ struct FoldArgs {
   int d_out;
 };
 
+// The absorbed query computed from the query latent: q~ = [A_h ; W_qr,h] c_Q.
+struct QLatArgs {
+  const void* c_q;     // [B][n_q][d_q]
+  const void* w_qabs;  // [n_h][d_c + 32][d_q]
+  int d_q;
+};
+
 vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
                            int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s,
-                           const FoldArgs* fold = nullptr) {
+                           const FoldArgs* fold = nullptr, const QLatArgs* qlat = nullptr) {
   const vmla_config& c = h->cfg;
   if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   const WsLayout w = ws_layout(c);
@@ -677,7 +684,27 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
 
   __nv_bfloat16* qt = at<__nv_bfloat16>(h->ws, w.qt);
   const int dqk = c.d_latent + 32;
-  {
+  if (qlat) {
+    StageScope scope(h, 2, s);
+    CUtensorMap tcq, tw;
+    if (!map3(&tcq, qlat->c_q, qlat->d_q, nq, c.batch, (uint64_t)qlat->d_q * 2, (uint64_t)nq * qlat->d_q * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tw, qlat->w_qabs, qlat->d_q, dqk, c.n_heads, (uint64_t)qlat->d_q * 2, (uint64_t)dqk * qlat->d_q * 2, 64,
+              dqk, CU_TENSOR_MAP_SWIZZLE_128B))
+      return map_fail();
+    QLatTc a;
+    a.qt = qt;
+    a.n_q = nq;
+    a.n_heads = c.n_heads;
+    a.d_latent = c.d_latent;
+    a.d_q = qlat->d_q;
+    a.t_first = t_first;
+    a.ring = make_ring(c);
+    a.rope = make_rope(c);
+    a.err = h->err;
+    a.limit_ns = kWaitLimitNs;
+    e = launch_qlat_tc(tcq, tw, a, c.batch, s);
+  } else {
     StageScope scope(h, 2, s);
     CUtensorMap tq, tuk;
     if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 2,
@@ -814,6 +841,37 @@ vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const
     return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
   return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s);
+}
+
+vmla_status vmla_fold_query_weights(const vmla_config* cfg, const void* w_uq, const void* w_qr, const void* w_uk,
+                                    int d_q, void* w_qabs, void* stream) {
+  if (!cfg || !w_uq || !w_qr || !w_uk || !w_qabs) return VMLA_ERR_INVALID_ARG;
+  vmla_status st = vmla_config_check(cfg);
+  if (st != VMLA_OK) return st;
+  if (cfg->dtype != VMLA_BF16 || !qlat_supported(cfg->d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  return cuda_status(launch_fold_query(static_cast<const __nv_bfloat16*>(w_uq), static_cast<const __nv_bfloat16*>(w_qr),
+                                       static_cast<const __nv_bfloat16*>(w_uk), static_cast<__nv_bfloat16*>(w_qabs),
+                                       cfg->n_heads, cfg->d_nope, cfg->d_rope, cfg->d_latent, d_q,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+vmla_status vmla_chunk_attention_qlatent(vmla_handle* h, int layer, const void* c_q, const void* w_qabs, int d_q,
+                                         const void* w_uv, void* out, int64_t first, int n, void* stream) {
+  vmla_status st = check_layer(h, layer);
+  if (st != VMLA_OK) return st;
+  if (!h->ckv) return VMLA_ERR_STATE;
+  if (!c_q || !w_qabs || !w_uv || !out || !aligned16(c_q) || !aligned16(w_qabs) || !aligned16(w_uv) ||
+      !aligned16(out))
+    return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  if (c.dtype != VMLA_BF16 || !qlat_supported(c.d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  Window win;
+  if ((st = check_attention_frames(c, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
+  if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  const QLatArgs ql{c_q, w_qabs, d_q};
+  return attention_bf16(h, layer, nullptr, nullptr, w_uv, out, first, n, win, VMLA_DESIGN_ABSORBED,
+                        static_cast<cudaStream_t>(stream), nullptr, &ql);
 }
 
 vmla_status vmla_fold_output_weights(const vmla_config* cfg, const void* w_o, const void* w_uv, void* w_fold,

@@ -371,6 +371,32 @@ def test_small_bf16_folded_output_mixer():
     assert_bf16_close(out[0].cpu().numpy(), O.output_projection(heads, w.w_o), "folded output mixer")
 
 
+# ------------------------------------------------------------------ content path absorbed into the query latent
+
+@pytest.mark.parametrize("d_latent", [128, 192])
+def test_small_bf16_query_latent_absorption(d_latent):
+    """q~_h = [W_uk,h^T W_uq,h c_Q | RoPE(W_qr,h c_Q)] from the query latent (d_q = 768):
+    the library's weight fold and K = 768 query GEMM, then the absorbed attention, against the
+    oracle's per-head queries W_uq,h c_Q, W_qr,h c_Q in the non-absorbed definition."""
+    import torch
+    import oracle.vmla_oracle as O
+    d = SMALL.replace(d_latent=d_latent)
+    ro = Rollout(d)
+    _fill(ro, 7)
+    w_uq, w_qr = synth.query_latent_weights(d, 0)
+    w_qabs = torch.empty(d.n_heads, d.d_latent + d.d_rope, d.d_q, dtype=torch.bfloat16, device="cuda")
+    ro.m.fold_query_weights(to_dev(w_uq, d), to_dev(w_qr, d), ro.wd[0][1], w_qabs)
+    ref_w = O.fold_query_weights(w_uq, w_qr, ro.w[0].w_uk)
+    got_w = w_qabs.float().cpu().numpy()
+    assert np.all(np.abs(got_w - ref_w) <= 2.0 ** -8 * np.abs(ref_w) + 1e-6 * np.abs(ref_w).max())
+    c_q = synth.query_latents(d, 0, 6)
+    out = torch.full((1, d.n_queries, d.n_heads * d.d_head), float("nan"), dtype=torch.float32, device="cuda")
+    ro.m.attention_qlatent(0, to_dev(c_q, d), w_qabs, ro.wd[0][2], out, 18, 3)
+    assert ro.m.device_status()[0] == 0
+    q = O.query_from_latent(c_q[0], w_uq, w_qr)[None]
+    assert_bf16_close(out[0].cpu().numpy(), ro.oracle(0, 6, q), f"query latent, d_c={d_latent}")
+
+
 # ------------------------------------------------------------------ sink frame + local window
 
 def test_tiny_fp32_sink_window():
