@@ -650,7 +650,7 @@ def qlatent_leg(dev, seed, steps=50):
             "attention_ms": k["attention"][0] / max(k["attention"][1], 1)}
 
 
-def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384)):
+def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384, 512)):
     """Latent width sweep on the Wan layer: attention time of every built design
     and of the dense per-head cache for the same seeded x and q."""
     import torch

@@ -130,9 +130,10 @@ int vmla_abi_version(void);
 vmla_status vmla_config_init(vmla_config* cfg);
 
 /* VMLA_OK when every field is consistent and a kernel exists for it:
- * VMLA_FP32 accepts any positive sizes (d_latent, d_nope+d_rope, d_value <= 512);
+ * VMLA_FP32 accepts any positive sizes (d_latent, d_nope+d_rope, d_value <= 512; up to 64 rotary pairs);
  * VMLA_BF16 needs d_nope + d_rope = d_value = 128, d_rope = 32 and d_latent one of 64, 128,
- * 192, 256, 384 (VMLA_DESIGN_ABSORBED up to 256, VMLA_DESIGN_RECONSTRUCT up to 192).
+ * 192, 256, 384, 512 (VMLA_DESIGN_ABSORBED up to 256, VMLA_DESIGN_RECONSTRUCT up to 192;
+ * other shapes run with VMLA_FP32).
  * grid_h, grid_w, window_frames must be < 1024 (RoPE range, [paperlayer App. C.1]). */
 vmla_status vmla_config_check(const vmla_config* cfg);
 
@@ -242,7 +243,7 @@ vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* 
  * W_down x of the paperlayer paper, Sec. 3): a persistent kernel over work items
  * (sample, 128-row tile of x, column part of [c_KV | k_R]).  `n_split` column
  * parts: 0 chooses per call (two when the row tiles alone would leave SMs idle,
- * and always when d_latent > 224), 1 or 2 forces it.  `max_ctas` caps the grid
+ * and always when d_latent > 224; three when d_latent > 480), 1 or 2 forces it.  `max_ctas` caps the grid
  * (0: one CTA per SM); a small cap makes each CTA run many items.  Every split
  * gives the same bits.  n_split = 1 with d_latent > 224 makes later appends
  * return VMLA_ERR_UNSUPPORTED_SHAPE.  Host only; VMLA_ERR_INVALID_ARG for

@@ -216,8 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(raw[q]);
-            const int col = part * N_PART + c0;  // 16 columns never straddle d_latent (a multiple of 64)
-            if (a.rotate && col >= a.d_latent) {
+            // 16 columns never straddle d_latent (a multiple of 64) nor d_latent + 32
+            const int col = part * N_PART + c0;
+            if (a.rotate && col >= a.d_latent && col < a.d_latent + 32) {
               const int p0 = (col - a.d_latent) >> 1;
 #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -240,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int id = tid; id < rows_h * CH; id += 128) {
           const int row = id / CH, ch = id - row * CH;
           const int col = part * N_PART + ch * 8;
+          if (col >= a.d_latent + 32) continue;  // the last of three parts runs past [c_KV | k_R]
           const bool lat = col < a.d_latent;
           __nv_bfloat16* dst = (lat || a.contiguous ? a.ckv : a.kr) +
                                (lat ? row_lat[64 * half + row] + col : row_pos[64 * half + row] + (col - a.d_latent));
@@ -977,7 +979,10 @@ cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const Append
   if constexpr (N_OUT <= 256) {
     if (p.parts == 1) return run_append<N_OUT>(tx, tw, a, batch, 1, p.ctas, s);
   }
-  if (p.parts == 2) return run_append<N_OUT / 2>(tx, tw, a, batch, 2, p.ctas, s);
+  if constexpr (N_OUT / 2 <= 256) {
+    if (p.parts == 2) return run_append<N_OUT / 2>(tx, tw, a, batch, 2, p.ctas, s);
+  }
+  if (p.parts == 3) return run_append<append_part_cols(N_OUT, 3)>(tx, tw, a, batch, 3, p.ctas, s);
   return cudaErrorInvalidValue;
 }
 
@@ -1088,7 +1093,10 @@ AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ct
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     cudaGetLastError();
   AppendPlan p{n_split, ctas};
-  if (p.parts == 0) p.parts = (d_latent + 32 > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
+  if (d_latent + 32 > 512)
+    p.parts = 3;
+  else if (p.parts == 0)
+    p.parts = (d_latent + 32 > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
   return p;
 }
 
@@ -1102,6 +1110,7 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
     case 192: return go_append<224>(tx, tw, a, batch, s, p);
     case 256: return go_append<288>(tx, tw, a, batch, s, p);
     case 384: return go_append<416>(tx, tw, a, batch, s, p);
+    case 512: return go_append<544>(tx, tw, a, batch, s, p);
   }
   return cudaErrorInvalidValue;
 }
@@ -1127,6 +1136,7 @@ cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const
     case 192: return go_recon<192>(tc, tuk, tuv, a, batch, s);
     case 256: return go_recon<256>(tc, tuk, tuv, a, batch, s);
     case 384: return go_recon<384>(tc, tuk, tuv, a, batch, s);
+    case 512: return go_recon<512>(tc, tuk, tuv, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -7,7 +7,7 @@
 
 namespace vmla {
 
-constexpr int kMaxPairs = 32;
+constexpr int kMaxPairs = 64;  // rotary pairs (d_rope up to 128)
 
 // Bits of the library's device status word.
 enum DeviceError : unsigned {
@@ -127,7 +127,11 @@ struct AppendTc {
 // Work split of the persistent append kernel for a call: `parts` column parts
 // of [c_KV | k_R] (1 or 2) and a grid cap `ctas` (0: one CTA per SM).  n_split 0
 // chooses two parts when the 128-row tiles alone would leave SMs idle (and
-// always past 256 columns).
+// always past 256 columns); past 512 columns there are always three.
+// Columns of one part when [c_KV | k_R] (n_out columns) is split in `parts`: a multiple of 16
+// (the MMA's N); the last part may run past n_out (those rows of W_down read as zeros).
+constexpr int append_part_cols(int n_out, int parts) { return (n_out + 16 * parts - 1) / (16 * parts) * 16; }
+
 struct AppendPlan {
   int parts, ctas;
 };

@@ -76,7 +76,8 @@ Rope make_rope(const vmla_config& c) {
 
 // A forced append column split the shape can take: one MMA covers at most 256 columns.
 bool append_tiling_fits(const vmla_config& c, int n_split) {
-  return n_split != 1 || c.d_latent + 32 <= 256;
+  if (n_split == 0) return true;
+  return append_part_cols(c.d_latent + 32, n_split) <= 256;
 }
 
 Ring make_ring(const vmla_config& c) {
@@ -338,7 +339,8 @@ vmla_status vmla_config_check(const vmla_config* c) {
   if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c->dtype == VMLA_BF16) {
     if (c->d_rope != 32 || c->d_nope != 96 || c->d_value != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
-    if (!(c->d_latent == 64 || c->d_latent == 128 || c->d_latent == 192 || c->d_latent == 256 || c->d_latent == 384))
+    if (!(c->d_latent == 64 || c->d_latent == 128 || c->d_latent == 192 || c->d_latent == 256 || c->d_latent == 384 ||
+          c->d_latent == 512))
       return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (c->d_model % 64 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
   } else {
@@ -498,7 +500,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
       const int parts = plan.parts;
       if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
+          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(c.d_latent + 32, parts),
                 CU_TENSOR_MAP_SWIZZLE_128B))
         return map_fail();
       AppendTc a;
@@ -958,7 +960,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     CUtensorMap tx, tw;
     if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, (c.d_latent + 32) / parts,
+        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(c.d_latent + 32, parts),
               CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
     AppendTc a;

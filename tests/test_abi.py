@@ -88,7 +88,7 @@ def test_rope_frequencies_match_the_oracle():
 
 @pytest.mark.parametrize("field,value,status", [
     ("d_rope", 30, 1), ("rope_theta", 0.0, 1), ("batch", 0, 1), ("chunk_frames", 22, 1),
-    ("grid_w", 1024, 3), ("window_frames", 1024, 3), ("d_latent", 200, 2), ("d_latent", 512, 2),
+    ("grid_w", 1024, 3), ("window_frames", 1024, 3), ("d_latent", 200, 2), ("d_latent", 640, 2),
     ("d_nope", 64, 2), ("dtype", 7, 1), ("rope_mode", 3, 1),
 ])
 def test_config_check_rejects(field, value, status):
@@ -224,7 +224,8 @@ def test_selftest_exp2_arguments():
     assert lib.vmla_selftest_exp2(0, 0x20000, 4, None) == 1         # null
 
 
-@pytest.mark.parametrize("d_latent,status", [(64, 0), (128, 0), (192, 0), (256, 0), (384, 0), (320, 2), (448, 2), (32, 2)])
+@pytest.mark.parametrize("d_latent,status", [(64, 0), (128, 0), (192, 0), (256, 0), (384, 0), (512, 0), (320, 2), (448, 2),
+                                            (32, 2), (576, 2)])
 def test_latent_widths_with_kernels(d_latent, status):
     c = default_config()
     c.d_latent = d_latent

@@ -55,6 +55,20 @@ def test_tiny_fp32_dense():
         assert_fp32_close(out[0], ro.oracle(0, chunk, q), f"dense chunk {chunk}")
 
 
+@pytest.mark.parametrize("d_nope,d_rope,pairs", [(112, 16, (4, 2, 2)), (64, 64, (12, 10, 10)),
+                                                 (32, 96, (18, 15, 15))])
+def test_fp32_nope_rope_split_variants(d_nope, d_rope, pairs):
+    """Other splits of a 128-dim head between content and positional dims (16, 64 and 96
+    rotary dims) through the fp32 kernels, rolling past the window."""
+    d = TINY.replace(name=f"split{d_rope}", d_model=64, n_heads=2, d_nope=d_nope, d_rope=d_rope, d_latent=16,
+                     rope_pairs=pairs)
+    ro = Rollout(d)
+    for chunk in range(6):
+        ro.append_chunk(0, chunk)
+        out, q = ro.attend(0, chunk)
+        assert_fp32_close(out[0], ro.oracle(0, chunk, q), f"d_rope {d_rope} chunk {chunk}")
+
+
 def test_tiny_fp32_batch_and_layers():
     d = TINY.replace(batch=3)
     ro = Rollout(d, layers=2)
@@ -123,7 +137,7 @@ def test_small_bf16_reconstruct_once():
     assert_bf16_close(out[0], ro.oracle(0, 7, q), "reconstruct once")
 
 
-@pytest.mark.parametrize("d_latent", [64, 128, 256, 384])
+@pytest.mark.parametrize("d_latent", [64, 128, 256, 384, 512])
 def test_small_bf16_latent_width(d_latent):
     """The design AUTO picks (absorbed up to 192, reconstruct-once above) at the gate."""
     ro = Rollout(SMALL.replace(name=f"small_dc{d_latent}", d_latent=d_latent))

@@ -128,7 +128,7 @@ def test_wan_batch8_sampled_rows():
         ro.check(layer, 6, 0, samples=(0, 5) if layer == 0 else (3, 7), what="batch 8")
 
 
-@pytest.mark.parametrize("d_latent", [64, 128, 192, 256, 384])
+@pytest.mark.parametrize("d_latent", [64, 128, 192, 256, 384, 512])
 def test_wan_latent_width_sweep(d_latent):
     """The Wan-1.3B layer with latent widths 64..256 (same seeded x and q), every
     built design and the dense per-head cache, on 256 rows of every head."""
