@@ -362,9 +362,16 @@ def run_ours(args, rank, world, local_rank):
     at_ms, at_n = per_kernel["attention"]
     at_launch_ms = at_ms / max(at_n, 1)
     achieved = F["attention"] / (at_launch_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": achieved / tc_burst, "peak_source": f"{src} bf16 dense (burst, cuBLAS)",
-                "frac_of_sustained": achieved / tc_sust,
+    # the kernel runs inside a timed loop of args.steps chunk steps: past half a second of continuous
+    # load the GPU sits at its power cap, so the sustained figure is the matching denominator
+    long_run = ms_step * args.steps >= 500.0
+    peak = tc_sust if long_run else tc_burst
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": f"{src} bf16 dense, cuBLAS, " + (
+                    f"sustained (the kernel runs inside {ms_step * args.steps / 1e3:.1f} s of continuous load)"
+                    if long_run else "burst (timed region under half a second)"),
+                "frac_of_burst": achieved / tc_burst, "frac_of_sustained": achieved / tc_sust,
                 "traffic": profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"),
                 "kernel": "attn_tc_kernel<192,false>", "launch_ms": at_launch_ms,
                 "algorithmic_flops_per_launch": F["attention"]}

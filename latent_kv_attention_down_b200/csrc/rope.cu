@@ -47,17 +47,25 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * 32 + quad * 8);
   uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * 32 + quad * 8);
   const int64_t stride = ring_rows * 32 / 8;  // one sample's ring, in 16-byte units
-#pragma unroll 4
-  for (int b = 0; b < a.batch; ++b) {
-    const uint4 v = __ldg(src + b * stride);
-    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+  // up to 8 samples at a time: every load is issued before the first store
+  for (int b0 = 0; b0 < a.batch; b0 += 8) {
+    const int nb = min(8, a.batch - b0);
+    uint4 v[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float u = bf_lo(in[k]), x = bf_hi(in[k]);
-      rope_apply(u, x, cs[k]);
-      out[k] = pack2(u, x);
+    for (int k = 0; k < 8; ++k)
+      if (k < nb) v[k] = __ldg(src + (b0 + k) * stride);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= nb) break;
+      uint32_t in[4] = {v[k].x, v[k].y, v[k].z, v[k].w}, out[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        float u = bf_lo(in[p]), x = bf_hi(in[p]);
+        rope_apply(u, x, cs[p]);
+        out[p] = pack2(u, x);
+      }
+      dst[(b0 + k) * stride] = make_uint4(out[0], out[1], out[2], out[3]);
     }
-    dst[b * stride] = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
