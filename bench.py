@@ -728,7 +728,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-legs", dest="legs", action="store_false",
                     help="skip the batch-8 and latent-width legs")
-    ap.add_argument("--cpu-queries", type=int, default=2048)
+    ap.add_argument("--cpu-queries", type=int, default=4096)
     ap.add_argument("--steps-ref", type=int, default=None)
     ap.add_argument("--warmup-ref", type=int, default=None)
     args = ap.parse_args()
