@@ -53,6 +53,21 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v
   }
 }
 
+// N 16-byte chunks (8 bf16 each, from fp32 bit patterns in r) of row `row` of a column block
+// parked for a TMA tensor store with 128-byte swizzle: the block holds 64 columns, 128 bytes per
+// row, and chunk j of a row sits at position j ^ (row & 7), so the eight rows a quarter-warp
+// writes at once fall in eight different bank groups.
+template <int N>
+__device__ __forceinline__ void park_sw128(uint8_t* blk, int row, const uint32_t* r) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float* v = reinterpret_cast<const float*>(r + 8 * j);
+    *reinterpret_cast<uint4*>(blk + row * 128 + ((j ^ (row & 7)) << 4)) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                   pack_bf16x2(v[6], v[7]));
+  }
+}
+
 __device__ __forceinline__ void raw_to_float(const uint32_t (&r)[32], float (&v)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -264,10 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stage holds the head's 128-column slice of q (two [128 x 64] blocks) and W_uk,h
 // ([96 x 64] blocks, read as the MN-major B operand); a single MMA chain of 6
 // k-steps gives W_uk,h^T q_nope in TMEM (two accumulators alternate); the epilogue
-// parks the item's rows of [q~_nope (d_c) | RoPE(q_rope) (32)] unpadded (all 128 when
-// they fit, else 64 at a time) and one bulk copy writes each park out (an item's
-// output rows are consecutive in memory); the copy runs while the next item's
-// positional part is rotated and its accumulator awaited.
+// parks the item's rows of [q~_nope (d_c) | RoPE(q_rope) (32)] as 64-column blocks in
+// the 128-byte swizzled layout (all 128 rows when they fit, else 64 at a time) and TMA
+// tensor stores write each park out, clipped at the last query; the stores run while
+// the next item's positional part is rotated and its accumulator awaited.
 template <int DL>
 struct QPrepCfg {
   static constexpr int A_BYTES = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
@@ -275,9 +290,10 @@ struct QPrepCfg {
   static constexpr int B_BYTES = (DL / 64) * WB;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int ROW = DL + 32;                 // output row, elements
-  static constexpr int OUT_STRIDE = ROW * 2;          // parked rows are the output's bytes, unpadded
-  static constexpr int PARK_ROWS = 2 * STAGE + 128 * OUT_STRIDE <= 212 * 1024 ? 128 : 64;
-  static constexpr int OUT_BYTES = PARK_ROWS * OUT_STRIDE;
+  static constexpr int NCB = DL / 64 + 1;             // 64-column blocks of a row (the last one half used)
+  static constexpr int PARK_ROWS = 2 * STAGE + NCB * 128 * 128 <= 212 * 1024 ? 128 : 64;
+  static constexpr int BLK = PARK_ROWS * 128;         // one parked column block
+  static constexpr int OUT_BYTES = NCB * BLK;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 4 ? 4 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;          // two accumulators, at 0 and 256
@@ -289,7 +305,7 @@ struct QPrepCfg {
 template <int DL>
 __global__ void __launch_bounds__(kThreads, 1)
     qprep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wuk,
-                    const QPrepTc a, int items) {
+                    const __grid_constant__ CUtensorMap tm_out, const QPrepTc a, int items) {
   using C = QPrepCfg<DL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -325,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_wuk);
+      prefetch_tmap(&tm_out);
       int it = 0;
       for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x, ++it) {
         const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
@@ -388,36 +405,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       const int valid_rows = ok ? min(128, a.n_q - mt * 128) : 0;
-      __nv_bfloat16* out_tile = a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + mt * 128) * C::ROW;
 #pragma unroll 1
       for (int part = 0; part < 128 / C::PARK_ROWS; ++part) {
-        if (tid == 0) bulk_wait_all_read();  // the previous park has been read by its copy
+        if (tid == 0) bulk_wait_all_read();  // the previous park has been read by its stores
         named_bar_sync(1, 128);
         if ((r / C::PARK_ROWS) == part) {  // warps whose TMEM lanes are this park's rows
-          uint8_t* orow = sout + (r - C::PARK_ROWS * part) * C::OUT_STRIDE;
+          const int pr = r - C::PARK_ROWS * part;
 #pragma unroll 1
-          for (int c0 = 0; c0 < DL; c0 += 32) {
-            uint32_t raw[32];
-            tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-            float v[32];
-            raw_to_float(raw, v);
-            store_bf16x32_smem(orow + c0 * 2, v);
+          for (int cb = 0; cb < DL / 64; ++cb) {
+            uint32_t raw[64];
+            tmem_ld64(tmem_addr(tbase, wq * 32, acc * 256 + cb * 64), raw);
+            park_sw128<8>(sout + cb * C::BLK, pr, raw);
           }
-          store_bf16x32_smem(orow + DL * 2, qr);
-          fence_async_smem();  // the bulk copy (async proxy) reads what these threads wrote
+          park_sw128<4>(sout + (DL / 64) * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
+          fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[acc]);
         }
         named_bar_sync(1, 128);  // this park is complete
-        const int rows_p = min(C::PARK_ROWS, valid_rows - C::PARK_ROWS * part);
-        if (tid == 0 && rows_p > 0) {
-          bulk_store(out_tile + (int64_t)C::PARK_ROWS * part * C::ROW, sout, (uint32_t)(rows_p * C::OUT_STRIDE));
+        if (tid == 0) {
+          const int row0 = C::PARK_ROWS * part;
+#pragma unroll 1
+          for (int rb = 0; rb < C::PARK_ROWS; rb += 64) {
+            if (row0 + rb >= valid_rows) break;
+            for (int cb = 0; cb < C::NCB; ++cb)
+              tma_store_3d(&tm_out, sout + cb * C::BLK + rb * 128, cb * 64, mt * 128 + row0 + rb, b * a.n_heads + h);
+          }
           bulk_commit();
         }
       }
     }
-    if (tid == 0) bulk_wait_all_read();  // shared memory stays until the last copy has read it
+    if (tid == 0) bulk_wait_all();  // the last stores have read shared memory and landed
   }
   tc_fence_before();
   __syncthreads();
@@ -778,15 +797,17 @@ __global__ void fold_weights_kernel(const __nv_bfloat16* w_o, const __nv_bfloat1
 // absorbed into the query latent c_Q; §4: d_q = 768]: per (sample, 128-query tile, head) item a
 // GEMM over K = d_q with the stacked weights [A_h ; W_qr,h] ((d_c + 32) rows), streamed in
 // 64-column blocks through a ring; the positional columns are rotated at the queries' positions
-// in the epilogue, which parks all rows unpadded and writes them with one bulk copy.
+// in the epilogue, which parks the rows as 64-column blocks in the 128-byte swizzled layout and
+// writes them with TMA tensor stores, clipped at the last query.
 template <int DL>
 struct QLatCfg {
   static constexpr int N = DL + 32;
   static constexpr int A_BLK = 128 * 128;
   static constexpr int B_BLK = N * 128;
   static constexpr int STAGE = A_BLK + B_BLK;
-  static constexpr int OUT_STRIDE = N * 2;
-  static constexpr int OUT_BYTES = 128 * OUT_STRIDE;
+  static constexpr int NCB = DL / 64 + 1;  // 64-column blocks of a row (the last one half used)
+  static constexpr int BLK = 128 * 128;    // one parked column block of 128 rows
+  static constexpr int OUT_BYTES = NCB * BLK;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -798,7 +819,7 @@ struct QLatCfg {
 template <int DL>
 __global__ void __launch_bounds__(kThreads, 1)
     qlat_tc_kernel(const __grid_constant__ CUtensorMap tm_cq, const __grid_constant__ CUtensorMap tm_w,
-                   const QLatTc a, int items) {
+                   const __grid_constant__ CUtensorMap tm_out, const QLatTc a, int items) {
   using C = QLatCfg<DL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -834,6 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_cq);
       prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_out);
       int it = 0;
       for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
         const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
@@ -898,17 +920,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       const int valid_rows = ok ? min(128, a.n_q - mt * 128) : 0;
-      if (tid == 0) bulk_wait_all_read();  // the previous item's copy has read the parked rows
+      if (tid == 0) bulk_wait_all_read();  // the previous item's stores have read the parked rows
       named_bar_sync(1, 128);
-      uint8_t* orow = sout + r * C::OUT_STRIDE;
 #pragma unroll 1
-      for (int c0 = 0; c0 < C::N; c0 += 32) {
+      for (int cb = 0; cb < DL / 64; ++cb) {
+        uint32_t raw[64];
+        tmem_ld64(tmem_addr(tbase, wq * 32, acc * 256 + cb * 64), raw);
+        park_sw128<8>(sout + cb * C::BLK, r, raw);
+      }
+      {
         uint32_t raw[32];
-        tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+        tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + DL), raw);
         float v[32];
         raw_to_float(raw, v);
-        if (c0 >= DL) rotate16(v, a.rope, t, hh, ww);  // the 32 positional columns
-        store_bf16x32_smem(orow + c0 * 2, v);
+        rotate16(v, a.rope, t, hh, ww);  // the 32 positional columns
+        park_sw128<4>(sout + (DL / 64) * C::BLK, r, reinterpret_cast<const uint32_t*>(v));
       }
       fence_async_smem();
       tc_fence_before();
@@ -916,12 +942,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       named_bar_sync(1, 128);
       if (tid == 0 && valid_rows > 0) {
-        bulk_store(a.qt + (((int64_t)b * a.n_heads + h) * a.n_q + mt * 128) * C::N, sout,
-                   (uint32_t)(valid_rows * C::OUT_STRIDE));
+#pragma unroll 1
+        for (int rb = 0; rb < valid_rows; rb += 64)
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_store_3d(&tm_out, sout + cb * C::BLK + rb * 128, cb * 64, mt * 128 + rb, b * a.n_heads + h);
         bulk_commit();
       }
     }
-    if (tid == 0) bulk_wait_all_read();
+    if (tid == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -987,7 +1015,8 @@ cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const Append
 }
 
 template <int DL>
-cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc& a, int batch, cudaStream_t s) {
+cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& to, const QPrepTc& a, int batch,
+                     cudaStream_t s) {
   using C = QPrepCfg<DL>;
   static const cudaError_t attr = set_smem(qprep_tc_kernel<DL>, C::SMEM);
   if (attr != cudaSuccess) return attr;
@@ -998,7 +1027,7 @@ cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
-  qprep_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tq, tw, a, items);
+  qprep_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tq, tw, to, a, items);
   return cudaGetLastError();
 }
 
@@ -1048,7 +1077,8 @@ cudaError_t launch_fold_weights(const __nv_bfloat16* w_o, const __nv_bfloat16* w
 }
 
 template <int DL>
-cudaError_t go_qlat(const CUtensorMap& tc, const CUtensorMap& tw, const QLatTc& a, int batch, cudaStream_t s) {
+cudaError_t go_qlat(const CUtensorMap& tc, const CUtensorMap& tw, const CUtensorMap& to, const QLatTc& a, int batch,
+                    cudaStream_t s) {
   using C = QLatCfg<DL>;
   static const cudaError_t attr = set_smem(qlat_tc_kernel<DL>, C::SMEM);
   if (attr != cudaSuccess) return attr;
@@ -1059,7 +1089,7 @@ cudaError_t go_qlat(const CUtensorMap& tc, const CUtensorMap& tw, const QLatTc& 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
-  qlat_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tw, a, items);
+  qlat_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tw, to, a, items);
   return cudaGetLastError();
 }
 
@@ -1067,13 +1097,14 @@ bool qlat_supported(int d_latent, int d_q) {
   return (d_latent == 64 || d_latent == 128 || d_latent == 192) && d_q > 0 && d_q % 64 == 0;
 }
 
-cudaError_t launch_qlat_tc(const CUtensorMap& tc, const CUtensorMap& tw, const QLatTc& a, int batch, cudaStream_t s) {
+cudaError_t launch_qlat_tc(const CUtensorMap& tc, const CUtensorMap& tw, const CUtensorMap& to, const QLatTc& a,
+                           int batch, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
   if (!qlat_supported(a.d_latent, a.d_q)) return cudaErrorInvalidValue;
   switch (a.d_latent) {
-    case 64: return go_qlat<64>(tc, tw, a, batch, s);
-    case 128: return go_qlat<128>(tc, tw, a, batch, s);
-    case 192: return go_qlat<192>(tc, tw, a, batch, s);
+    case 64: return go_qlat<64>(tc, tw, to, a, batch, s);
+    case 128: return go_qlat<128>(tc, tw, to, a, batch, s);
+    case 192: return go_qlat<192>(tc, tw, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1115,14 +1146,14 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const QPrepTc& a, int batch,
-                            cudaStream_t s) {
+cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& to, const QPrepTc& a,
+                            int batch, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
   switch (a.d_latent) {
-    case 64: return go_qprep<64>(tq, tw, a, batch, s);
-    case 128: return go_qprep<128>(tq, tw, a, batch, s);
-    case 192: return go_qprep<192>(tq, tw, a, batch, s);
-    case 256: return go_qprep<256>(tq, tw, a, batch, s);
+    case 64: return go_qprep<64>(tq, tw, to, a, batch, s);
+    case 128: return go_qprep<128>(tq, tw, to, a, batch, s);
+    case 192: return go_qprep<192>(tq, tw, to, a, batch, s);
+    case 256: return go_qprep<256>(tq, tw, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -150,13 +150,15 @@ struct QPrepTc {
   unsigned* err;
   uint64_t limit_ns;
 };
-// q map: 3D (n_h*128, n_q, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64, 96, 1) SW128
-cudaError_t launch_qprep_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_wuk, const QPrepTc& a, int batch,
-                            cudaStream_t s);
+// q map: 3D (n_h*128, n_q, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64, 96, 1) SW128;
+// out map (the stores of qt): 3D (d_c + 32, n_q, B*n_h) box (64, 64, 1) SW128
+cudaError_t launch_qprep_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_wuk, const CUtensorMap& tm_out,
+                            const QPrepTc& a, int batch, cudaStream_t s);
 
 // Query-latent absorption: qt [B][n_h][n_q][d_c + 32] = [A_h ; W_qr,h] c_Q, positional part
 // rotated at the query positions.  c_Q map: 3D (d_q, n_q, B) box (64,128,1) SW128; weight map:
-// 3D (d_q, d_c + 32, n_h) box (64, d_c + 32, 1) SW128.  d_latent 64, 128 or 192; d_q % 64 == 0.
+// 3D (d_q, d_c + 32, n_h) box (64, d_c + 32, 1) SW128; out map as for launch_qprep_tc.
+// d_latent 64, 128 or 192; d_q % 64 == 0.
 struct QLatTc {
   __nv_bfloat16* qt;
   int n_q, n_heads, d_latent, d_q;
@@ -167,8 +169,8 @@ struct QLatTc {
   uint64_t limit_ns;
 };
 bool qlat_supported(int d_latent, int d_q);
-cudaError_t launch_qlat_tc(const CUtensorMap& tm_cq, const CUtensorMap& tm_w, const QLatTc& a, int batch,
-                           cudaStream_t s);
+cudaError_t launch_qlat_tc(const CUtensorMap& tm_cq, const CUtensorMap& tm_w, const CUtensorMap& tm_out,
+                           const QLatTc& a, int batch, cudaStream_t s);
 // w_qabs [n_h][d_c + d_rope][d_q] = [W_uk,h^T W_uq,h ; W_qr,h]
 cudaError_t launch_fold_query(const __nv_bfloat16* w_uq, const __nv_bfloat16* w_qr, const __nv_bfloat16* w_uk,
                               __nv_bfloat16* w_qabs, int n_heads, int d_nope, int d_rope, int d_c, int d_q,

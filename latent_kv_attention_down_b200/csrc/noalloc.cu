@@ -135,10 +135,12 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   }
   const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap tq, tuk;
+  CUtensorMap tq, tuk, tqt;
   if (!tile_map(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 256, (uint64_t)nq * c.n_heads * 256,
                 64, 128, SW128, BF) ||
       !tile_map(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+                SW128, BF) ||
+      !tile_map(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
                 SW128, BF))
     return VMLA_ERR_CUDA;
   QPrepTc qa;
@@ -152,7 +154,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   qa.rope = rope;
   qa.err = err;
   qa.limit_ns = kWaitLimitNs;
-  if (launch_qprep_tc(tq, tuk, qa, c.batch, s) != cudaSuccess) return VMLA_ERR_CUDA;
+  if (launch_qprep_tc(tq, tuk, tqt, qa, c.batch, s) != cudaSuccess) return VMLA_ERR_CUDA;
 
   const int bn = attn_absorbed_block_n(c.d_latent);
   const uint64_t bh = (uint64_t)c.batch * c.n_heads;

@@ -688,11 +688,13 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   const int dqk = c.d_latent + 32;
   if (qlat) {
     StageScope scope(h, 2, s);
-    CUtensorMap tcq, tw;
+    CUtensorMap tcq, tw, tqt;
     if (!map3(&tcq, qlat->c_q, qlat->d_q, nq, c.batch, (uint64_t)qlat->d_q * 2, (uint64_t)nq * qlat->d_q * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tw, qlat->w_qabs, qlat->d_q, dqk, c.n_heads, (uint64_t)qlat->d_q * 2, (uint64_t)dqk * qlat->d_q * 2, 64,
-              dqk, CU_TENSOR_MAP_SWIZZLE_128B))
+              dqk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
+              CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
     QLatTc a;
     a.qt = qt;
@@ -705,13 +707,15 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.rope = make_rope(c);
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    e = launch_qlat_tc(tcq, tw, a, c.batch, s);
+    e = launch_qlat_tc(tcq, tw, tqt, a, c.batch, s);
   } else {
     StageScope scope(h, 2, s);
-    CUtensorMap tq, tuk;
+    CUtensorMap tq, tuk, tqt;
     if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 2,
               (uint64_t)nq * c.n_heads * 128 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
               CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
     QPrepTc a;
@@ -725,7 +729,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.rope = make_rope(c);
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    e = launch_qprep_tc(tq, tuk, a, c.batch, s);
+    e = launch_qprep_tc(tq, tuk, tqt, a, c.batch, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   {
