@@ -388,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
         kernels[k]["algorithmic_bytes"] = b
         kernels[k]["gbs"] = b / (kernels[k]["ms_per_launch"] * 1e-3) / 1e9
         kernels[k]["frac_of_hbm"] = kernels[k]["gbs"] / hbm
+    add_copy_reference(kernels, dev)
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -405,6 +406,7 @@ def run_ours(args, rank, world, local_rank):
                        "reconstruct_in_tile": recon_in_tile}
     if args.legs:
         line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
+                        "hbm_saturation": saturation_leg(dev=dev, hbm=hbm, tc=tc_burst, seed=seed),
                         "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed),
                         "sink_window": sink_leg(dev=dev, tc=tc_burst, seed=seed),
                         "folded_output_mixer": folded_leg(dev=dev, tc=tc_burst, seed=seed),
@@ -423,12 +425,54 @@ def _pool_fill(m, d, pool, xp, W, layer, chunks):
         m.append(layer, pool.activations(layer, c, 0, pool=xp), W[0], c * d.chunk_frames, d.chunk_frames)
 
 
+def copy_gbs(nbytes, dev, reps=15):
+    """What a plain device copy achieves on the same traffic (nbytes/2 read + nbytes/2 written),
+    timed like the kernels: CUDA events around each launch, sources cycled through more than
+    the L2 so every copy reads HBM; median of `reps`."""
+    import torch
+    half = max(int(nbytes) // 2 // 16 * 16, 16)
+    nbuf = max(2, -(-512 * 2 ** 20 // half))
+    src = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
+    dst = torch.empty(half, dtype=torch.uint8, device=dev)
+    times = []
+    for i in range(reps + 3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src[i % nbuf])
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    del src, dst
+    times.sort()
+    return 2 * half / (times[len(times) // 2] * 1e-3) / 1e9
+
+
+def add_copy_reference(kernels, dev):
+    """Attach to every HBM-bound kernel entry the same-size copy rate and the kernel's fraction of it."""
+    for e in kernels.values():
+        if "algorithmic_bytes" in e:
+            c = copy_gbs(e["algorithmic_bytes"], dev)
+            e["copy_same_bytes_gbs"] = c
+            e["frac_of_same_size_copy"] = e["gbs"] / c
+
+
 def batch8_leg(m_timed, dev, hbm, tc, seed):
-    """The same layer at batch 8: 8 independent rings, 37440 queries per call;
-    two layer sets (x, q: 460 MB) alternate so inputs stay above L2."""
+    return batch_leg(8, dev, hbm, tc, seed, steps=20)
+
+
+def saturation_leg(dev, hbm, tc, seed):
+    """The HBM-bound kernels at batch 64 (one append moves 1.06 GB, one RoPE pass 268 MB, one
+    q-absorb 2.5 GB), where launch and pipeline ramp no longer hide their streaming rate."""
+    return batch_leg(64, dev, hbm, tc, seed, steps=3)
+
+
+def batch_leg(batch, dev, hbm, tc, seed, steps):
+    """The same layer at batch B: B independent rings, B*4680 queries per call; two layer sets
+    alternate so inputs stay above L2."""
     import torch
     from latent_kv_attention_down_b200 import api
-    d = WORKLOAD.replace(batch=8)
+    d = WORKLOAD.replace(batch=batch)
     L = 2
     m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
     pool = synth.FramePool(d, base_seed=seed)
@@ -451,7 +495,6 @@ def batch8_leg(m_timed, dev, hbm, tc, seed):
         m.append(l, xs[l], W[l][0], first, d.chunk_frames)
         m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, api.DESIGN_ABSORBED)
 
-    steps = 20
     for i in range(3):
         step(i)
     torch.cuda.synchronize()
@@ -474,7 +517,8 @@ def batch8_leg(m_timed, dev, hbm, tc, seed):
            "rope": B * 2 * nk * d.d_rope * 2,
            "q_absorb": B * nq * d.n_heads * d.d_head * 2 + d.n_heads * d.d_nope * d.d_latent * 2 +
            B * nq * d.n_heads * (d.d_latent + d.d_rope) * 2}
-    res = {"workload": "wan1.3b-layer chunk step at batch 8 (8 rings, N_q=37440 per call, N_k=32760 per sample)",
+    res = {"workload": f"wan1.3b-layer chunk step at batch {B} ({B} rings, N_q={B * nq} per call, "
+                       f"N_k={nk} per sample)",
            "ms_per_step": ms, "tflops": B * F["total"] / (ms * 1e-3) / 1e12,
            "query_tokens_per_s": B * nq / (ms * 1e-3), "kernels": {}}
     for n, (t, c) in k.items():
@@ -489,6 +533,7 @@ def batch8_leg(m_timed, dev, hbm, tc, seed):
             e["frac_of_bf16_peak"] = e["tflops"] / tc
         res["kernels"][n] = e
     m.close()
+    add_copy_reference(res["kernels"], dev)
     return res
 
 

@@ -30,6 +30,52 @@ __device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, int t, 
   for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], rope_cs(rp, p, t, h, w));
 }
 
+// (cos, sin) of every rotary pair at every position a chunk's queries take, one table per
+// CTA: pair p of the t axis at chunk frame f sits at p * F + f, pair p of the h axis at row
+// hh at n_t F + (p - n_t) grid_h + hh, pair p of the w axis at column ww after those.  Each
+// entry is rope_cs of the same arguments, so a lookup equals the direct evaluation.
+struct RopeTable {
+  int F, gh, gw, n;  // chunk frames, grid rows, grid columns, entries
+  __device__ __forceinline__ int index(const Rope& rp, int p, int f, int hh, int ww) const {
+    return p < rp.n_t ? p * F + f
+                      : (p < rp.n_t + rp.n_h ? rp.n_t * F + (p - rp.n_t) * gh + hh
+                                             : rp.n_t * F + rp.n_h * gh + (p - rp.n_t - rp.n_h) * gw + ww);
+  }
+};
+__device__ __forceinline__ RopeTable rope_table_shape(const Rope& rp, int n_q, const Ring& g) {
+  RopeTable t;
+  t.F = (n_q + g.tokens_per_frame - 1) / g.tokens_per_frame;
+  t.gw = g.grid_w;
+  t.gh = g.tokens_per_frame / g.grid_w;
+  t.n = rp.n_t * t.F + rp.n_h * t.gh + rp.n_w * t.gw;
+  return t;
+}
+// Fill the table (threads [tid0, tid0 + nthreads) of the caller take its entries in turn).
+__device__ __forceinline__ void rope_table_fill(float2* tab, const RopeTable& t, const Rope& rp, int64_t t_first,
+                                                int tid, int nthreads) {
+  for (int e = tid; e < t.n; e += nthreads) {
+    int p, pos;
+    if (e < rp.n_t * t.F) {
+      p = e / t.F;
+      pos = (int)(t_first + e % t.F);
+    } else if (e < rp.n_t * t.F + rp.n_h * t.gh) {
+      const int k = e - rp.n_t * t.F;
+      p = rp.n_t + k / t.gh;
+      pos = k % t.gh;
+    } else {
+      const int k = e - rp.n_t * t.F - rp.n_h * t.gh;
+      p = rp.n_t + rp.n_h + k / t.gw;
+      pos = k % t.gw;
+    }
+    tab[e] = rope_cs(rp, p, pos, pos, pos);  // the pair's own axis picks pos
+  }
+}
+__device__ __forceinline__ void rotate16_tab(float (&v)[32], const float2* tab, const RopeTable& t, const Rope& rp,
+                                             int f, int hh, int ww) {
+#pragma unroll
+  for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], tab[t.index(rp, p, f, hh, ww)]);
+}
+
 // 32 floats as bf16 into 64 bytes of shared memory (16-byte aligned)
 __device__ __forceinline__ void store_bf16x32_smem(uint8_t* dst, const float (&v)[32]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
@@ -275,58 +321,72 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================== q-absorb
-// Persistent over (sample, 128-query tile, head) items, head fastest.  Per item one
-// stage holds the head's 128-column slice of q (two [128 x 64] blocks) and W_uk,h
-// ([96 x 64] blocks, read as the MN-major B operand); a single MMA chain of 6
-// k-steps gives W_uk,h^T q_nope in TMEM (two accumulators alternate); the epilogue
-// parks the item's rows of [q~_nope (d_c) | RoPE(q_rope) (32)] as 64-column blocks in
-// the 128-byte swizzled layout (all 128 rows when they fit, else 64 at a time) and TMA
-// tensor stores write each park out, clipped at the last query; the stores run while
-// the next item's positional part is rotated and its accumulator awaited.
+// Persistent over (head, sample, 128-query tile) items: each CTA takes a contiguous
+// run of them, so it meets one or two heads and keeps W_uk,h ([96 x 64] blocks, read
+// as the MN-major B operand) resident, reloading it only when the head changes; the
+// ring stages carry only the head's 128-column slice of q (two [128 x 64] blocks),
+// which leaves room for a deeper prefetch.  Per item a single MMA chain of 6
+// k-steps gives W_uk,h^T q_nope in TMEM (two accumulators alternate); two epilogue
+// warpgroups park the item's rows of [q~_nope (d_c) | RoPE(q_rope) (32)] as 64-column
+// blocks in the 128-byte swizzled layout (all 128 rows when they fit, else 64 at a
+// time) -- the first the leading column blocks, the second the rest and the rotated
+// positional part -- and TMA tensor stores write each park out, clipped at the last
+// query; the stores run while the next item's positional part is rotated and its
+// accumulator awaited.
 template <int DL>
 struct QPrepCfg {
-  static constexpr int A_BYTES = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
-  static constexpr int WB = 96 * 128;            // one 64-col block of W_uk,h: 96 rows x 128 B
-  static constexpr int B_BYTES = (DL / 64) * WB;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGE = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
+  static constexpr int WB = 96 * 128;          // one 64-col block of W_uk,h: 96 rows x 128 B
+  static constexpr int W_BYTES = (DL / 64) * WB;
   static constexpr int ROW = DL + 32;                 // output row, elements
   static constexpr int NCB = DL / 64 + 1;             // 64-column blocks of a row (the last one half used)
-  static constexpr int PARK_ROWS = 2 * STAGE + NCB * 128 * 128 <= 212 * 1024 ? 128 : 64;
+  static constexpr int PARK_ROWS = W_BYTES + 2 * STAGE + NCB * 128 * 128 <= 212 * 1024 ? 128 : 64;
   static constexpr int BLK = PARK_ROWS * 128;         // one parked column block
   static constexpr int OUT_BYTES = NCB * BLK;
-  static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
+  static constexpr int FIT = (212 * 1024 - OUT_BYTES - W_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 4 ? 4 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;          // two accumulators, at 0 and 256
-  static constexpr int SMEM_USED = 1024 + STAGES * STAGE + OUT_BYTES + 256;
+  static constexpr int TAB_ENTRIES = 2048;            // (cos, sin) table of the chunk's positions
+  static constexpr int SMEM_USED = 1024 + STAGES * STAGE + W_BYTES + OUT_BYTES + 256 + TAB_ENTRIES * 8;
   static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;  // one CTA per SM
+  static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 two epilogue warpgroups
+  static constexpr int NB = DL / 64;   // TMEM column blocks: [0, NA) parked by warpgroup 0,
+  static constexpr int NA = (NB + 1) / 2;  // [NA, NB) and the positional block by warpgroup 1
   static_assert(DL % 64 == 0 && DL <= 256 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
 };
 
 template <int DL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
     qprep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wuk,
                     const __grid_constant__ CUtensorMap tm_out, const QPrepTc a, int items) {
   using C = QPrepCfg<DL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sout = smem + C::STAGES * C::STAGE;
+  uint8_t* sw = smem + C::STAGES * C::STAGE;  // the resident W_uk,h
+  uint8_t* sout = sw + C::W_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sout + C::OUT_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done = acc_empty + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* w_full = done + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(w_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  float2* rope_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(full) + 256);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (a.n_q + 127) / 128;
+  const int per_head = items / a.n_heads;  // (sample, query tile) items of one head
+  const int beg = (int)((int64_t)blockIdx.x * items / gridDim.x);
+  const int end = (int)((int64_t)(blockIdx.x + 1) * items / gridDim.x);
   const Guard g{abort_flag, a.err, a.limit_ns};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
+    mbar_init(w_full, 1);
     mbar_init(&acc_full[0], 1);
     mbar_init(&acc_full[1], 1);
-    mbar_init(&acc_empty[0], 4);
-    mbar_init(&acc_empty[1], 4);
+    mbar_init(&acc_empty[0], 8);  // one arrival per epilogue warp
+    mbar_init(&acc_empty[1], 8);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -342,34 +402,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_wuk);
       prefetch_tmap(&tm_out);
-      int it = 0;
-      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x, ++it) {
-        const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+      int it = 0, cur_h = -1, wloads = 0;
+      for (int item = beg; item < end && !*abort_flag; ++item, ++it) {
+        const int h = item / per_head, mt = (item % per_head) % m_tiles, b = (item % per_head) / m_tiles;
         const int s = it % C::STAGES;
+        if (h != cur_h) {
+          // the MMAs of the previous item (the last readers of the old W_uk,h) have completed:
+          // empty[] of its stage has finished the phase of that item's commit
+          if (it > 0 && !wait_phase(&empty[(it - 1) % C::STAGES], ((it - 1) / C::STAGES) & 1, g,
+                                    DEV_ERR_TIMEOUT_PRODUCER))
+            break;
+          mbar_arrive_expect_tx(w_full, C::W_BYTES);
+          for (int cb = 0; cb < DL / 64; ++cb) tma_load_3d(sw + cb * C::WB, &tm_wuk, w_full, cb * 64, 0, h);
+          cur_h = h;
+          ++wloads;
+        }
         if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
         uint8_t* st = smem + s * C::STAGE;
         mbar_arrive_expect_tx(&full[s], C::STAGE);
         tma_load_3d(st, &tm_q, &full[s], h * 128, mt * 128, b);
         tma_load_3d(st + 16384, &tm_q, &full[s], h * 128 + 64, mt * 128, b);
-        for (int cb = 0; cb < DL / 64; ++cb) tma_load_3d(st + C::A_BYTES + cb * C::WB, &tm_wuk, &full[s], cb * 64, 0, h);
       }
-      if (*abort_flag)
+      if (*abort_flag) {
         for (int i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
           drain_phase(&full[i % C::STAGES], (i / C::STAGES) & 1, g);
+        if (wloads > 0) drain_phase(w_full, (wloads - 1) & 1, g);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, DL, false, true);
-      int j = 0;
-      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      const uint64_t bd = smem_desc(smem_u32(sw), C::WB, 1024, LAYOUT_SW128);
+      int j = 0, cur_h = -1, wl = 0;
+      for (int item = beg; item < end; ++item, ++j) {
+        const int h = item / per_head;
         const int acc = j & 1, s = j % C::STAGES;
         if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        if (h != cur_h) {
+          if (!wait_phase(w_full, wl & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+          cur_h = h;
+          ++wl;
+        }
         if (!wait_phase(&full[s], (j / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::STAGE);
         const uint64_t ad = smem_desc(st, 16, 1024, LAYOUT_SW128);
-        const uint64_t bd = smem_desc(st + C::A_BYTES, C::WB, 1024, LAYOUT_SW128);
 #pragma unroll
         for (int kk = 0; kk < 6; ++kk) {  // d_nope = 96 = 6 x 16
           const uint64_t ak = desc_add(ad, (kk / 4) * 16384 + (kk % 4) * 32), bk = desc_add(bd, kk * 2048);
@@ -386,20 +464,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
+    const RopeTable tshape = rope_table_shape(a.rope, a.n_q, a.ring);
+    const bool use_tab = tshape.n <= C::TAB_ENTRIES;
+    if (use_tab) rope_table_fill(rope_tab, tshape, a.rope, a.t_first, tid, 256);
+    named_bar_sync(1, 256);  // the table is complete
+    // warpgroup 1 reads each item's positional part (64 bytes of its row) one item ahead
+    uint4 rq[4] = {};
+    auto load_rope = [&](int item) {
+      const int hh_ = item / per_head, mt_ = (item % per_head) % m_tiles, b_ = (item % per_head) / m_tiles;
+      const int i_ = mt_ * 128 + r;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.q + (((int64_t)b_ * a.n_q + (i_ < a.n_q ? i_ : 0)) * a.n_heads + hh_) * 128 + 96);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rq[k] = src[k];
+    };
+    if (wg == 1 && beg < end) load_rope(beg);
     int j = 0;
-    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
-      const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
+    for (int item = beg; item < end; ++item, ++j) {
+      const int h = item / per_head, mt = (item % per_head) % m_tiles, b = (item % per_head) / m_tiles;
       const int acc = j & 1;
       // the positional part does not wait for the tensor core
-      const int i = mt * 128 + r;
-      const int ii = i < a.n_q ? i : 0;
       float qr[32];
-      {
-        load_bf16x32(a.q + (((int64_t)b * a.n_q + ii) * a.n_heads + h) * 128 + 96, qr);
+      if (wg == 1) {
+        const int i = mt * 128 + r;
+        const int ii = i < a.n_q ? i : 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w4[4] = {rq[k].x, rq[k].y, rq[k].z, rq[k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+            qr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+          }
+        }
+        if (item + 1 < end) load_rope(item + 1);
         const int tok = ii % T;
-        rotate16(qr, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
+        if (use_tab)
+          rotate16_tab(qr, rope_tab, tshape, a.rope, ii / T, tok / a.ring.grid_w, tok % a.ring.grid_w);
+        else
+          rotate16(qr, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
       }
       const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();
@@ -408,22 +513,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int part = 0; part < 128 / C::PARK_ROWS; ++part) {
         if (tid == 0) bulk_wait_all_read();  // the previous park has been read by its stores
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 256);
         if ((r / C::PARK_ROWS) == part) {  // warps whose TMEM lanes are this park's rows
           const int pr = r - C::PARK_ROWS * part;
 #pragma unroll 1
-          for (int cb = 0; cb < DL / 64; ++cb) {
+          for (int cb = wg ? C::NA : 0; cb < (wg ? C::NB : C::NA); ++cb) {
             uint32_t raw[64];
             tmem_ld64(tmem_addr(tbase, wq * 32, acc * 256 + cb * 64), raw);
             park_sw128<8>(sout + cb * C::BLK, pr, raw);
           }
-          park_sw128<4>(sout + (DL / 64) * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
+          if (wg == 1) park_sw128<4>(sout + C::NB * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
           fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[acc]);
         }
-        named_bar_sync(1, 128);  // this park is complete
+        named_bar_sync(1, 256);  // this park is complete
         if (tid == 0) {
           const int row0 = C::PARK_ROWS * part;
 #pragma unroll 1
@@ -1027,7 +1132,7 @@ cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const CUtenso
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
-  qprep_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tq, tw, to, a, items);
+  qprep_tc_kernel<DL><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tq, tw, to, a, items);
   return cudaGetLastError();
 }
 
