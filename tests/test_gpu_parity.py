@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 from latent_kv_attention_down_b200 import api, synth
-from tests.harness import Rollout, assert_bf16_close, assert_fp32_close, to_dev
+from tests.harness import Rollout, assert_bf16_close, assert_fp32_close, sampled_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -358,6 +358,19 @@ def test_wan_layer_sampled_rows():
     rows[-1] = WAN.n_queries - 1
     ref = ro.oracle(0, 6, q, rows=rows)
     assert_bf16_close(out[0][rows], ref, "wan layer")
+
+
+def test_wide_grid_rotary_pairs_evaluated_directly():
+    """A 4 x 520 latent grid: the chunk's rotary (cos, sin) pairs no longer fit the q-absorb
+    kernel's per-CTA table (the w axis alone has 5 x 520 entries), so that kernel evaluates
+    them per row; two chunks (12480 keys, 6240 queries), 256 seeded query rows checked for
+    every head."""
+    d = SMALL.replace(name="wan_wide_grid", grid_h=4, grid_w=520)
+    ro = Rollout(d)
+    _fill(ro, 2)
+    out, q = ro.attend(0, 1)
+    rows = sampled_rows(d.n_queries)
+    assert_bf16_close(out[0][rows], ro.oracle(0, 1, q, rows=rows), "wide grid")
 
 
 # ------------------------------------------------------------------ W_uv folded into the output mixer
