@@ -557,8 +557,10 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
 // reduction over d_latent runs through a ring of [128 rows x 64] latent blocks
 // and [224 x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
 // two TMEM accumulators alternate so the epilogue of one item overlaps the
-// next; the epilogue parks 64 rows at a time as [k_h (128) | v_h (128)] bf16
-// and writes each row's two 256-byte runs out contiguously.
+// next; two epilogue warpgroups park the item's 128 rows as [k_h (128) | v_h
+// (128)] bf16 -- the first k_h (content columns from TMEM, the positional part
+// read one item ahead), the second v_h -- and all 256 threads write each row's
+// two 256-byte runs out contiguously.
 template <int DL>
 struct ReconCfg {
   static constexpr int NKB = DL / 64;
@@ -566,16 +568,17 @@ struct ReconCfg {
   static constexpr int B_BLK = 224 * 128;  // [96 rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
   static constexpr int STAGE = A_BLK + B_BLK;
   static constexpr int OUT_STRIDE = 256 * 2 + 16;  // parked row [k_h | v_h]: an odd number of 16-byte chunks
-  static constexpr int OUT_BYTES = 64 * OUT_STRIDE;
+  static constexpr int OUT_BYTES = 128 * OUT_STRIDE;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of 224 columns, at 0 and 256
   static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 128 * 8 + 256;
+  static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 two epilogue warpgroups
   static_assert(DL % 64 == 0 && STAGES >= 3 && SMEM <= 227 * 1024 && SMEM > 116 * 1024, "does not fit");
 };
 
 template <int DL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
     recon_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wuk,
                     const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a, int items) {
   using C = ReconCfg<DL>;
@@ -598,8 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
     mbar_init(&acc_full[0], 1);
     mbar_init(&acc_full[1], 1);
-    mbar_init(&acc_empty[0], 4);  // one arrival per epilogue warp
-    mbar_init(&acc_empty[1], 4);
+    mbar_init(&acc_empty[0], 8);  // one arrival per epilogue warp
+    mbar_init(&acc_empty[1], 8);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -666,61 +669,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
+    // warpgroup 0 reads each item's positional keys (64 bytes of its row) one item ahead
+    uint4 krq[4] = {};
+    auto load_kr = [&](int item) {
+      const int mt_ = (item / a.n_heads) % m_tiles, b_ = item / (a.n_heads * m_tiles);
+      const int m_ = mt_ * 128 + r;
+      if (m_ < a.rows) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.kr + ((int64_t)b_ * a.kr_rows + m_) * a.kr_stride);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) krq[k] = src[k];
+      }
+    };
+    if (wg == 0 && (int)blockIdx.x < items) load_kr(blockIdx.x);
     int j = 0;
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
       const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
       const int acc = j & 1;
+      float kr[32];
+      if (wg == 0) {
+        const int m = mt * 128 + r;
+        const int mm = m < a.rows ? m : 0;
+        const int64_t frame = a.first_frame + mm / T;
+        const int tok = mm % T;
+        const int64_t row = a.to_ring ? ring_frame_slot(a.ring, frame) * T + tok : mm;
+        row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w4[4] = {krq[k].x, krq[k].y, krq[k].z, krq[k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+            kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+          }
+        }
+        if (item + (int)gridDim.x < items) load_kr(item + gridDim.x);
+        if (a.rotate) rotate16(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
+      }
       const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();
       tc_fence_after();
-      const int m = mt * 128 + r;
-      const bool valid = ok && m < a.rows;
-      const int mm = m < a.rows ? m : 0;
-      const int64_t frame = a.first_frame + mm / T;
-      const int tok = mm % T;
-      const int64_t row = a.to_ring ? ring_frame_slot(a.ring, frame) * T + tok : mm;
-      row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
-      float kr[32];
-      if (valid) {
-        load_bf16x32(a.kr + ((int64_t)b * a.kr_rows + mm) * a.kr_stride, kr);
-        if (a.rotate) rotate16(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) kr[i] = 0.f;
-      }
-      named_bar_sync(1, 128);  // row table complete
       const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
+      uint8_t* orow = sout + r * C::OUT_STRIDE;
+      if (wg == 0) {  // TMEM columns 0..95: the content part of k_h, then its positional part
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        if ((wq >> 1) == half) {  // warps of this half hold TMEM lanes 64*half .. 64*half + 63
-          uint8_t* orow = sout + (r - 64 * half) * C::OUT_STRIDE;
+        for (int c0 = 0; c0 < 96; c0 += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+          float v[32];
+          raw_to_float(raw, v);
+          store_bf16x32_smem(orow + c0 * 2, v);
+        }
+        store_bf16x32_smem(orow + 96 * 2, kr);
+      } else {  // TMEM columns 96..223: v_h, parked from column 128
 #pragma unroll 1
-          for (int c0 = 0; c0 < 224; c0 += 32) {
-            uint32_t raw[32];
-            tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-            float v[32];
-            raw_to_float(raw, v);
-            // TMEM columns 0..95 are k_h's content part, 96..223 are v_h (parked from column 128)
-            store_bf16x32_smem(orow + (c0 < 96 ? c0 : c0 + 32) * 2, v);
-          }
-          store_bf16x32_smem(orow + 96 * 2, kr);  // positional part of k_h
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
+        for (int c0 = 96; c0 < 224; c0 += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+          float v[32];
+          raw_to_float(raw, v);
+          store_bf16x32_smem(orow + (c0 + 32) * 2, v);
         }
-        named_bar_sync(1, 128);  // this half is parked
-        const int rows_h = min(64, valid_rows - 64 * half);
-#pragma unroll 4
-        for (int id = tid; id < rows_h * 32; id += 128) {
-          const int rr = id >> 5, ch = id & 31;
-          __nv_bfloat16* dst =
-              a.dense + row_k[64 * half + rr] + (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
-          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
-        }
-        named_bar_sync(1, 128);  // the parked half is written out before it is reused
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
+      named_bar_sync(1, 256);  // the item is parked and its row table complete
+#pragma unroll 4
+      for (int id = tid; id < valid_rows * 32; id += 256) {
+        const int rr = id >> 5, ch = id & 31;
+        __nv_bfloat16* dst =
+            a.dense + row_k[rr] + (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
+      }
+      named_bar_sync(1, 256);  // the park is written out before it is reused
     }
   }
   tc_fence_before();
@@ -1149,7 +1172,7 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.rows + 127) / 128) * a.n_heads * batch;
-  recon_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tuk, tuv, a, items);
+  recon_tc_kernel<DL><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tc, tuk, tuv, a, items);
   return cudaGetLastError();
 }
 
