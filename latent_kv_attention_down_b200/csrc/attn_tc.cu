@@ -2,7 +2,7 @@
 //
 // Absorbed design [paperlayer App. E]: with W_uk folded into the query
 // (q~_h = [W_uk,h^T q_nope,h | RoPE(q_rope,h)]), every head scores the SAME
-// shared key [c_KV | RoPE(k_R)] (d_latent + 32 wide) and accumulates the SAME
+// shared key [c_KV | RoPE(k_R)] (d_latent + d_rope wide) and accumulates the SAME
 // shared values c_KV (d_latent wide): multi-query attention over the latent
 // cache.  W_uv,h is applied once per output row after the softmax-weighted
 // sum (value-path absorption), fused into the epilogue as a second tcgen05
@@ -57,17 +57,21 @@ struct Bars {
   float red[2][2][128];  // per-tile half-row maxima of the two softmax groups (tile parity, group, row)
 };
 
-template <int DL_, bool DENSE_>
+template <int DL_, bool DENSE_, int DR_ = 32>
 struct AttnCfg {
   static constexpr bool DENSE = DENSE_;
   static constexpr int DL = DL_;
-  static constexpr int DQK = DENSE ? 128 : DL + 32;  // contraction width of S = Q K^T
+  static constexpr int DR = DR_;                     // rotary dims of the shared key (absorbed)
+  static constexpr int DQK = DENSE ? 128 : DL + DR;  // contraction width of S = Q K^T
   static constexpr int DV = DENSE ? 128 : DL;
   static constexpr int BN = 128;
   static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of a query or key row
-  static constexpr int Q_BYTES = QB * 16384 + (DENSE ? 0 : 128 * 64);
+  // the rotary columns sit in one block of DR * 2 bytes per row, swizzled at that width
+  static constexpr int RB = DENSE ? 0 : DR * 2;
+  static constexpr uint32_t R_LAYOUT = RB == 128 ? LAYOUT_SW128 : (RB == 64 ? LAYOUT_SW64 : LAYOUT_SW32);
+  static constexpr int Q_BYTES = QB * 16384 + 128 * RB;
   static constexpr int KBLK = BN * 128;           // one [BN keys x 64] SW128 block
-  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * 64;
+  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * RB;
   static constexpr int SMEM_CAP = 232448;
   static constexpr int BARS = (sizeof(Bars) + 127) / 128 * 128;
   static constexpr int STAGES_FIT = (SMEM_CAP - BARS - Q_BYTES) / STAGE_BYTES;
@@ -84,6 +88,7 @@ struct AttnCfg {
   static_assert(SMEM <= SMEM_CAP, "shared memory budget");
   static_assert((DENSE || STAGE_BYTES >= DV * 256) && STAGES * STAGE_BYTES >= 65536, "epilogue staging");
   static_assert(DV % 64 == 0 && DV <= 256 && BN % 32 == 0, "tile shapes");
+  static_assert(DENSE || DR == 16 || DR == 32 || DR == 64, "rotary block of 32, 64 or 128 bytes per row");
 };
 
 // bf16 row of 32 floats into a 128B-swizzled K-major tile: row r, columns c0..c0+31
@@ -119,8 +124,9 @@ __device__ __forceinline__ void st_swizzled_row32_f32(uint8_t* tile, int r, int 
 }
 
 // S = Q K^T for one tile.  Query tile and key tile in shared memory: QB [rows x 64] SW128
-// blocks of latent (or per-head key) columns, then (absorbed) one [rows x 32] SW64 block of
-// rotated positional columns.  Descriptors are built once and advanced by compile-time offsets.
+// blocks of latent (or per-head key) columns, then (absorbed) one [rows x d_rope] block of
+// rotated positional columns, swizzled at its row width (32, 64 or 128 bytes).  Descriptors are
+// built once and advanced by compile-time offsets.
 template <class C>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t stage) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, C::BN, false, false);
@@ -137,10 +143,11 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t 
       mma_ss_c<true>(d_tmem, a, b, idesc);
   }
   if constexpr (!C::DENSE) {
-    const uint64_t krd = smem_desc(stage + C::QB * C::KBLK, 16, 512, LAYOUT_SW64);
-    const uint64_t qrd = smem_desc(sq + C::QB * 16384, 16, 512, LAYOUT_SW64);
+    const uint64_t krd = smem_desc(stage + C::QB * C::KBLK, 16, 8 * C::RB, C::R_LAYOUT);
+    const uint64_t qrd = smem_desc(sq + C::QB * 16384, 16, 8 * C::RB, C::R_LAYOUT);
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk) mma_ss_c<true>(d_tmem, desc_add(qrd, kk * 32), desc_add(krd, kk * 32), idesc);
+    for (int kk = 0; kk < C::DR / 16; ++kk)
+      mma_ss_c<true>(d_tmem, desc_add(qrd, kk * 32), desc_add(krd, kk * 32), idesc);
   }
 }
 
@@ -186,13 +193,13 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 
 // FOLD (absorbed only): the epilogue stores O_bar itself, as its bf16 pair, for an output
 // mixer that folds W_uv,h in (tm_wuv then maps O_bar's rounded part, tm_out its residual).
-template <int DL, bool DENSE, bool FOLD>
+template <int DL, bool DENSE, bool FOLD, int DR>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
                    const __grid_constant__ CUtensorMap tm_wuv, const __grid_constant__ CUtensorMap tm_out,
                    const AttnTc a) {
-  using C = AttnCfg<DL, DENSE>;
+  using C = AttnCfg<DL, DENSE, DR>;
   // The dynamic shared memory window starts 1024-byte aligned (the swizzled TMA tiles need it);
   // the whole 227 KB budget may be in use, so there is no slack to realign: check instead.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -504,16 +511,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DL, bool DENSE, bool FOLD = false>
+template <int DL, bool DENSE, bool FOLD = false, int DR = 32>
 cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk, const CUtensorMap& tkr,
                     const CUtensorMap& tuv, const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
-  using C = AttnCfg<DL, DENSE>;
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  using C = AttnCfg<DL, DENSE, DR>;
+  static const cudaError_t attr = cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE, FOLD, DR>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (attr != cudaSuccess) return attr;
   if (a.n_q <= 0 || a.n_keys <= 0) return cudaSuccess;
-  attn_tc_kernel<DL, DENSE, FOLD><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv,
-                                                                                               to, a);
+  attn_tc_kernel<DL, DENSE, FOLD, DR><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr,
+                                                                                                   tuv, to, a);
   return cudaGetLastError();
 }
 
@@ -548,14 +555,32 @@ cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, 
   return go_attn<128, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
 }
 
-cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
+bool attn_absorbed_supported(int d_latent, int d_rope) {
+  const bool dl = d_latent == 64 || d_latent == 128 || d_latent == 192 || d_latent == 256;
+  return dl && (d_rope == 16 || d_rope == 32 || (d_rope == 64 && d_latent <= 192));
+}
+
+template <int DR>
+cudaError_t go_attn_dl(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk,
+                       const CUtensorMap& tkr, const CUtensorMap& tuv, const CUtensorMap& to, const AttnTc& a,
+                       int batch, cudaStream_t s) {
+  switch (d_latent) {
+    case 64: return go_attn<64, false, false, DR>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 128: return go_attn<128, false, false, DR>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 192: return go_attn<192, false, false, DR>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 256:
+      if constexpr (DR <= 32) return go_attn<256, false, false, DR>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_absorbed_tc(int d_latent, int d_rope, const CUtensorMap& tq, const CUtensorMap& tqr,
                                     const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tuv,
                                     const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
-  switch (d_latent) {
-    case 64: return go_attn<64, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
-    case 128: return go_attn<128, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
-    case 192: return go_attn<192, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
-    case 256: return go_attn<256, false>(tq, tqr, tk, tkr, tuv, to, a, batch, s);
+  switch (d_rope) {
+    case 16: return go_attn_dl<16>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 32: return go_attn_dl<32>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 64: return go_attn_dl<64>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -24,10 +24,14 @@ namespace {
 
 constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA (+TMEM alloc), warps 4..7 epilogue; every kernel is persistent
 
-// Rotate 16 adjacent pairs held in v[0..31] at grid position (t, h, w).
-__device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, int t, int h, int w) {
+// Rotate NP adjacent pairs held in v[0..2 NP) at grid position (t, h, w).
+template <int NP>
+__device__ __forceinline__ void rotate_pairs(float (&v)[2 * NP], const Rope& rp, int t, int h, int w) {
 #pragma unroll
-  for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], rope_cs(rp, p, t, h, w));
+  for (int p = 0; p < NP; ++p) rope_apply(v[2 * p], v[2 * p + 1], rope_cs(rp, p, t, h, w));
+}
+__device__ __forceinline__ void rotate16(float (&v)[32], const Rope& rp, int t, int h, int w) {
+  rotate_pairs<16>(v, rp, t, h, w);
 }
 
 // (cos, sin) of every rotary pair at every position a chunk's queries take, one table per
@@ -70,10 +74,11 @@ __device__ __forceinline__ void rope_table_fill(float2* tab, const RopeTable& t,
     tab[e] = rope_cs(rp, p, pos, pos, pos);  // the pair's own axis picks pos
   }
 }
-__device__ __forceinline__ void rotate16_tab(float (&v)[32], const float2* tab, const RopeTable& t, const Rope& rp,
-                                             int f, int hh, int ww) {
+template <int NP>
+__device__ __forceinline__ void rotate_pairs_tab(float (&v)[2 * NP], const float2* tab, const RopeTable& t,
+                                                 const Rope& rp, int f, int hh, int ww) {
 #pragma unroll
-  for (int p = 0; p < 16; ++p) rope_apply(v[2 * p], v[2 * p + 1], tab[t.index(rp, p, f, hh, ww)]);
+  for (int p = 0; p < NP; ++p) rope_apply(v[2 * p], v[2 * p + 1], tab[t.index(rp, p, f, hh, ww)]);
 }
 
 // 32 floats as bf16 into 64 bytes of shared memory (16-byte aligned)
@@ -257,12 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t frame = a.first_frame + mm / T;
       const int tok = mm % T;
       if (a.contiguous) {
-        row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + 32);
+        row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + a.d_rope);
         row_pos[r] = row_lat[r] + a.d_latent;
       } else {
         const int64_t rr = (int64_t)b * a.ring_rows + ring_frame_slot(a.ring, frame) * T + tok;
         row_lat[r] = rr * a.d_latent;
-        row_pos[r] = rr * 32;
+        row_pos[r] = rr * a.d_rope;
       }
       named_bar_sync(1, 128);  // row table complete
       const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
@@ -277,9 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(raw[q]);
-            // 16 columns never straddle d_latent (a multiple of 64) nor d_latent + 32
+            // 16 columns never straddle d_latent (a multiple of 64) nor d_latent + d_rope
             const int col = part * N_PART + c0;
-            if (a.rotate && col >= a.d_latent && col < a.d_latent + 32) {
+            if (a.rotate && col >= a.d_latent && col < a.d_latent + a.d_rope) {
               const int p0 = (col - a.d_latent) >> 1;
 #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int id = tid; id < rows_h * CH; id += 128) {
           const int row = id / CH, ch = id - row * CH;
           const int col = part * N_PART + ch * 8;
-          if (col >= a.d_latent + 32) continue;  // the last of three parts runs past [c_KV | k_R]
+          if (col >= a.d_latent + a.d_rope) continue;  // the last part may run past [c_KV | k_R]
           const bool lat = col < a.d_latent;
           __nv_bfloat16* dst = (lat || a.contiguous ? a.ckv : a.kr) +
                                (lat ? row_lat[64 * half + row] + col : row_pos[64 * half + row] + (col - a.d_latent));
@@ -333,12 +338,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // positional part -- and TMA tensor stores write each park out, clipped at the last
 // query; the stores run while the next item's positional part is rotated and its
 // accumulator awaited.
-template <int DL>
+template <int DL, int DR>
 struct QPrepCfg {
+  static constexpr int DN = 128 - DR;          // content dims of a head (the MMA's K)
   static constexpr int STAGE = 2 * 128 * 128;  // q[:, h*128 .. h*128+128) as two 64-col blocks
-  static constexpr int WB = 96 * 128;          // one 64-col block of W_uk,h: 96 rows x 128 B
+  static constexpr int WB = DN * 128;          // one 64-col block of W_uk,h: DN rows x 128 B
   static constexpr int W_BYTES = (DL / 64) * WB;
-  static constexpr int ROW = DL + 32;                 // output row, elements
+  static constexpr int ROW = DL + DR;                 // output row, elements
   static constexpr int NCB = DL / 64 + 1;             // 64-column blocks of a row (the last one half used)
   static constexpr int PARK_ROWS = W_BYTES + 2 * STAGE + NCB * 128 * 128 <= 212 * 1024 ? 128 : 64;
   static constexpr int BLK = PARK_ROWS * 128;         // one parked column block
@@ -353,13 +359,14 @@ struct QPrepCfg {
   static constexpr int NB = DL / 64;   // TMEM column blocks: [0, NA) parked by warpgroup 0,
   static constexpr int NA = (NB + 1) / 2;  // [NA, NB) and the positional block by warpgroup 1
   static_assert(DL % 64 == 0 && DL <= 256 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
+  static_assert((DR == 16 || DR == 32 || DR == 64) && W_BYTES % 1024 == 0, "rotary dims");
 };
 
-template <int DL>
-__global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
+template <int DL, int DR>
+__global__ void __launch_bounds__(QPrepCfg<DL, DR>::THREADS, 1)
     qprep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wuk,
                     const __grid_constant__ CUtensorMap tm_out, const QPrepTc a, int items) {
-  using C = QPrepCfg<DL>;
+  using C = QPrepCfg<DL, DR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sw = smem + C::STAGES * C::STAGE;  // the resident W_uk,h
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
         const uint32_t st = smem_u32(smem + s * C::STAGE);
         const uint64_t ad = smem_desc(st, 16, 1024, LAYOUT_SW128);
 #pragma unroll
-        for (int kk = 0; kk < 6; ++kk) {  // d_nope = 96 = 6 x 16
+        for (int kk = 0; kk < C::DN / 16; ++kk) {
           const uint64_t ak = desc_add(ad, (kk / 4) * 16384 + (kk % 4) * 32), bk = desc_add(bd, kk * 2048);
           if (kk == 0)
             mma_ss_c<false>(tbase + acc * 256, ak, bk, idesc);
@@ -470,15 +477,16 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
     const bool use_tab = tshape.n <= C::TAB_ENTRIES;
     if (use_tab) rope_table_fill(rope_tab, tshape, a.rope, a.t_first, tid, 256);
     named_bar_sync(1, 256);  // the table is complete
-    // warpgroup 1 reads each item's positional part (64 bytes of its row) one item ahead
-    uint4 rq[4] = {};
+    // warpgroup 1 reads each item's positional part (DR * 2 bytes of its row) one item ahead
+    constexpr int RQ = DR / 8;  // 16-byte pieces of it
+    uint4 rq[RQ] = {};
     auto load_rope = [&](int item) {
       const int hh_ = item / per_head, mt_ = (item % per_head) % m_tiles, b_ = (item % per_head) / m_tiles;
       const int i_ = mt_ * 128 + r;
       const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + (((int64_t)b_ * a.n_q + (i_ < a.n_q ? i_ : 0)) * a.n_heads + hh_) * 128 + 96);
+          a.q + (((int64_t)b_ * a.n_q + (i_ < a.n_q ? i_ : 0)) * a.n_heads + hh_) * 128 + C::DN);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) rq[k] = src[k];
+      for (int k = 0; k < RQ; ++k) rq[k] = src[k];
     };
     if (wg == 1 && beg < end) load_rope(beg);
     int j = 0;
@@ -486,12 +494,12 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
       const int h = item / per_head, mt = (item % per_head) % m_tiles, b = (item % per_head) / m_tiles;
       const int acc = j & 1;
       // the positional part does not wait for the tensor core
-      float qr[32];
+      float qr[DR];
       if (wg == 1) {
         const int i = mt * 128 + r;
         const int ii = i < a.n_q ? i : 0;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < RQ; ++k) {
           const uint32_t w4[4] = {rq[k].x, rq[k].y, rq[k].z, rq[k].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -502,9 +510,9 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
         if (item + 1 < end) load_rope(item + 1);
         const int tok = ii % T;
         if (use_tab)
-          rotate16_tab(qr, rope_tab, tshape, a.rope, ii / T, tok / a.ring.grid_w, tok % a.ring.grid_w);
+          rotate_pairs_tab<DR / 2>(qr, rope_tab, tshape, a.rope, ii / T, tok / a.ring.grid_w, tok % a.ring.grid_w);
         else
-          rotate16(qr, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
+          rotate_pairs<DR / 2>(qr, a.rope, (int)(a.t_first + ii / T), tok / a.ring.grid_w, tok % a.ring.grid_w);
       }
       const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();
@@ -522,7 +530,7 @@ __global__ void __launch_bounds__(QPrepCfg<DL>::THREADS, 1)
             tmem_ld64(tmem_addr(tbase, wq * 32, acc * 256 + cb * 64), raw);
             park_sw128<8>(sout + cb * C::BLK, pr, raw);
           }
-          if (wg == 1) park_sw128<4>(sout + C::NB * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
+          if (wg == 1) park_sw128<DR / 8>(sout + C::NB * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
           fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
           tc_fence_before();
           __syncwarp();
@@ -1135,18 +1143,18 @@ cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const Append
   if constexpr (N_OUT <= 256) {
     if (p.parts == 1) return run_append<N_OUT>(tx, tw, a, batch, 1, p.ctas, s);
   }
-  if constexpr (N_OUT / 2 <= 256) {
-    if (p.parts == 2) return run_append<N_OUT / 2>(tx, tw, a, batch, 2, p.ctas, s);
+  if constexpr (append_part_cols(N_OUT, 2) <= 256) {
+    if (p.parts == 2) return run_append<append_part_cols(N_OUT, 2)>(tx, tw, a, batch, 2, p.ctas, s);
   }
   if (p.parts == 3) return run_append<append_part_cols(N_OUT, 3)>(tx, tw, a, batch, 3, p.ctas, s);
   return cudaErrorInvalidValue;
 }
 
-template <int DL>
+template <int DL, int DR>
 cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& to, const QPrepTc& a, int batch,
                      cudaStream_t s) {
-  using C = QPrepCfg<DL>;
-  static const cudaError_t attr = set_smem(qprep_tc_kernel<DL>, C::SMEM);
+  using C = QPrepCfg<DL, DR>;
+  static const cudaError_t attr = set_smem(qprep_tc_kernel<DL, DR>, C::SMEM);
   if (attr != cudaSuccess) return attr;
   static int sms = 0;
   if (sms == 0) {
@@ -1155,8 +1163,21 @@ cudaError_t go_qprep(const CUtensorMap& tq, const CUtensorMap& tw, const CUtenso
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
-  qprep_tc_kernel<DL><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tq, tw, to, a, items);
+  qprep_tc_kernel<DL, DR><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tq, tw, to, a, items);
   return cudaGetLastError();
+}
+
+template <int DR>
+cudaError_t go_qprep_dl(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& to, const QPrepTc& a,
+                        int batch, cudaStream_t s) {
+  switch (a.d_latent) {
+    case 64: return go_qprep<64, DR>(tq, tw, to, a, batch, s);
+    case 128: return go_qprep<128, DR>(tq, tw, to, a, batch, s);
+    case 192: return go_qprep<192, DR>(tq, tw, to, a, batch, s);
+    case 256:
+      if constexpr (DR <= 32) return go_qprep<256, DR>(tq, tw, to, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int DL>
@@ -1247,15 +1268,15 @@ cudaError_t launch_fold_query(const __nv_bfloat16* w_uq, const __nv_bfloat16* w_
   return cudaGetLastError();
 }
 
-AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ctas) {
+AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int ctas) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     cudaGetLastError();
   AppendPlan p{n_split, ctas};
-  if (d_latent + 32 > 512)
+  if (n_out > 512)
     p.parts = 3;
   else if (p.parts == 0)
-    p.parts = (d_latent + 32 > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
+    p.parts = (n_out > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
   return p;
 }
 
@@ -1263,13 +1284,20 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
                              cudaStream_t s, const AppendPlan& p) {
   if (a.rows <= 0) return cudaSuccess;
   if (a.d_model % 64 != 0) return cudaErrorInvalidValue;
-  switch (a.d_latent) {
-    case 64: return go_append<96>(tx, tw, a, batch, s, p);
-    case 128: return go_append<160>(tx, tw, a, batch, s, p);
-    case 192: return go_append<224>(tx, tw, a, batch, s, p);
-    case 256: return go_append<288>(tx, tw, a, batch, s, p);
-    case 384: return go_append<416>(tx, tw, a, batch, s, p);
-    case 512: return go_append<544>(tx, tw, a, batch, s, p);
+  switch (a.d_latent + a.d_rope) {  // n_out = [c_KV | k_R] columns
+    case 80: return go_append<80>(tx, tw, a, batch, s, p);    // d_rope 16
+    case 144: return go_append<144>(tx, tw, a, batch, s, p);
+    case 208: return go_append<208>(tx, tw, a, batch, s, p);
+    case 272: return go_append<272>(tx, tw, a, batch, s, p);
+    case 96: return go_append<96>(tx, tw, a, batch, s, p);    // d_rope 32
+    case 160: return go_append<160>(tx, tw, a, batch, s, p);
+    case 224: return go_append<224>(tx, tw, a, batch, s, p);
+    case 288: return go_append<288>(tx, tw, a, batch, s, p);
+    case 416: return go_append<416>(tx, tw, a, batch, s, p);
+    case 544: return go_append<544>(tx, tw, a, batch, s, p);
+    case 128: return go_append<128>(tx, tw, a, batch, s, p);  // d_rope 64
+    case 192: return go_append<192>(tx, tw, a, batch, s, p);
+    case 256: return go_append<256>(tx, tw, a, batch, s, p);
   }
   return cudaErrorInvalidValue;
 }
@@ -1277,11 +1305,10 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
 cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& to, const QPrepTc& a,
                             int batch, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
-  switch (a.d_latent) {
-    case 64: return go_qprep<64>(tq, tw, to, a, batch, s);
-    case 128: return go_qprep<128>(tq, tw, to, a, batch, s);
-    case 192: return go_qprep<192>(tq, tw, to, a, batch, s);
-    case 256: return go_qprep<256>(tq, tw, to, a, batch, s);
+  switch (a.d_rope) {
+    case 16: return go_qprep_dl<16>(tq, tw, to, a, batch, s);
+    case 32: return go_qprep_dl<32>(tq, tw, to, a, batch, s);
+    case 64: return go_qprep_dl<64>(tq, tw, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -115,7 +115,7 @@ cudaError_t launch_dense_reconstruct_simt(const SimtDenseReconstruct& a, cudaStr
 struct AppendTc {
   __nv_bfloat16* ckv;  // [B][ring_rows][d_c] or contiguous [B][rows][d_c + d_r] when contiguous
   __nv_bfloat16* kr;   // [B][ring_rows][d_r]
-  int rows, d_model, d_latent;  // d_rope is 32
+  int rows, d_model, d_latent, d_rope;  // d_rope 16, 32 or 64
   int64_t first_frame;
   int rotate, contiguous;
   int64_t ring_rows;
@@ -135,23 +135,24 @@ constexpr int append_part_cols(int n_out, int parts) { return (n_out + 16 * part
 struct AppendPlan {
   int parts, ctas;
 };
-AppendPlan append_tc_plan(int d_latent, int rows, int batch, int n_split, int ctas);
-// x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, d_c + 32) box (64, (d_c + 32) / parts) SW128.
+AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int ctas);
+// x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, n_out) box (64, append_part_cols(n_out, parts))
+// SW128, n_out = d_c + d_rope.
 cudaError_t launch_append_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const AppendTc& a, int batch,
                              cudaStream_t s, const AppendPlan& plan);
 
 struct QPrepTc {
-  const __nv_bfloat16* q;  // [B][n_q][n_h][128]  (rope part read directly)
-  __nv_bfloat16* qt;       // [B][n_h][n_q][d_c + 32]
-  int n_q, n_heads, d_latent;
+  const __nv_bfloat16* q;  // [B][n_q][n_h][128]: per head d_nope = 128 - d_rope content dims, then d_rope
+  __nv_bfloat16* qt;       // [B][n_h][n_q][d_c + d_rope]
+  int n_q, n_heads, d_latent, d_rope;  // d_rope 16, 32 or 64
   int64_t t_first;
   Ring ring;
   Rope rope;
   unsigned* err;
   uint64_t limit_ns;
 };
-// q map: 3D (n_h*128, n_q, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64, 96, 1) SW128;
-// out map (the stores of qt): 3D (d_c + 32, n_q, B*n_h) box (64, 64, 1) SW128
+// q map: 3D (n_h*128, n_q, B) box (64,128,1) SW128; w_uk map: 3D (d_c, d_nope, n_h) box (64, d_nope, 1)
+// SW128; out map (the stores of qt): 3D (d_c + d_rope, n_q, B*n_h) box (64, 64, 1) SW128
 cudaError_t launch_qprep_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_wuk, const CUtensorMap& tm_out,
                             const QPrepTc& a, int batch, cudaStream_t s);
 
@@ -186,7 +187,10 @@ struct AttnTc {
 // Absorbed design.  qt maps: 3D (d_c+32, n_q, B*n_h): latent box (64,128,1) SW128, rope box (32,128,1) SW64;
 // ckv map: 3D (d_c, n_keys, B) box (64,BN,1) SW128; kr map: 3D (32, n_keys, B) box (32,BN,1) SW64;
 // w_uv map: 3D (d_c, 128, n_h) box (64,128,1) SW128; out map: 3D (n_h*128, n_q, B) box (64,128,1) SW128.
-cudaError_t launch_attn_absorbed_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
+// d_rope 16, 32 or 64 (64 up to d_latent 192): tm_qr / tm_kr boxes are d_rope wide, swizzled at
+// d_rope * 2 bytes (32B, 64B or 128B)
+bool attn_absorbed_supported(int d_latent, int d_rope);
+cudaError_t launch_attn_absorbed_tc(int d_latent, int d_rope, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
                                     const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr, const CUtensorMap& tm_wuv,
                                     const CUtensorMap& tm_out, const AttnTc& a, int batch, cudaStream_t s);
 int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the key maps)

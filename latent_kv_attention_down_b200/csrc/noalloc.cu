@@ -85,6 +85,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
     return VMLA_ERR_INVALID_ARG;
   const int64_t F = frames_appended;
   if (c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;  // absorbed kernels: up to 256 latent dims
+  if (c.d_rope != 32) return VMLA_ERR_UNSUPPORTED_SHAPE;    // the 96/32 split
   if (n_frames < 1 || n_frames > c.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
   if (F < 1 || first_frame < 0 || first_frame + n_frames != F) return VMLA_ERR_STATE;
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
@@ -149,6 +150,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   qa.n_q = nq;
   qa.n_heads = c.n_heads;
   qa.d_latent = c.d_latent;
+  qa.d_rope = c.d_rope;
   qa.t_first = first_frame - (at_read ? t_origin : 0);
   qa.ring = ring;
   qa.rope = rope;
@@ -178,6 +180,6 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   a.rescale_threshold = c.softmax_rescale_log2;
   a.err = err;
   a.limit_ns = kWaitLimitNs;
-  return launch_attn_absorbed_tc(c.d_latent, mq, mqr, mk, mkr, muv, mo, a, c.batch, s) == cudaSuccess ? VMLA_OK
+  return launch_attn_absorbed_tc(c.d_latent, 32, mq, mqr, mk, mkr, muv, mo, a, c.batch, s) == cudaSuccess ? VMLA_OK
                                                                                                       : VMLA_ERR_CUDA;
 }

@@ -30,13 +30,14 @@ __device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, int t,
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// d_rope = 32: 4 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its
-// slot in every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.
+// d_rope / 8 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its slot in
+// every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.
 __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)a.n_keys * 4) return;
-  const int quad = idx & 3;
-  const int s = (int)(idx >> 2);
+  const int nq = a.d_rope >> 3;  // 16-byte pieces of a key
+  if (idx >= (int64_t)a.n_keys * nq) return;
+  const int quad = (int)(idx % nq);
+  const int s = (int)(idx / nq);
   const int64_t ring_rows = (int64_t)a.ring.window_frames * a.ring.tokens_per_frame;
   const int fslot = s / a.ring.tokens_per_frame, tok = s % a.ring.tokens_per_frame;
   const int t = ring_slot_t(a.ring, fslot, a.window_start_slot);
@@ -44,9 +45,10 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   float2 cs[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) cs[k] = rope_cs(a.rope, quad * 4 + k, t, hh, ww);
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * 32 + quad * 8);
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * 32 + quad * 8);
-  const int64_t stride = ring_rows * 32 / 8;  // one sample's ring, in 16-byte units
+  const uint4* src =
+      reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * a.d_rope + quad * 8);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * a.d_rope + quad * 8);
+  const int64_t stride = ring_rows * nq;  // one sample's ring, in 16-byte units
   // up to 8 samples at a time: every load is issued before the first store
   for (int b0 = 0; b0 < a.batch; b0 += 8) {
     const int nb = min(8, a.batch - b0);
@@ -92,8 +94,8 @@ __global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
 }  // namespace
 
 cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s) {
-  if (a.d_rope != 32) return cudaErrorInvalidValue;
-  const int64_t total = (int64_t)a.n_keys * 4;
+  if (a.d_rope % 8 != 0 || a.d_rope <= 0 || a.d_rope > 2 * kMaxPairs) return cudaErrorInvalidValue;
+  const int64_t total = (int64_t)a.n_keys * (a.d_rope / 8);
   if (total == 0 || a.batch == 0) return cudaSuccess;
   rope_window_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
   return cudaGetLastError();

@@ -77,7 +77,7 @@ Rope make_rope(const vmla_config& c) {
 // A forced append column split the shape can take: one MMA covers at most 256 columns.
 bool append_tiling_fits(const vmla_config& c, int n_split) {
   if (n_split == 0) return true;
-  return append_part_cols(c.d_latent + 32, n_split) <= 256;
+  return append_part_cols(c.d_latent + c.d_rope, n_split) <= 256;
 }
 
 Ring make_ring(const vmla_config& c) {
@@ -149,6 +149,7 @@ vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : cud
 // d_rope per key) is over twice the per-head attention's (2 d_head).
 vmla_design resolve_design(const vmla_config& c, vmla_design d) {
   if (d != VMLA_DESIGN_AUTO) return d;
+  if (c.dtype == VMLA_BF16 && c.d_rope != 32) return VMLA_DESIGN_ABSORBED;  // the only bf16 design there
   if (c.dtype == VMLA_BF16 && c.d_latent >= 256) return VMLA_DESIGN_RECON_ONCE;
   return VMLA_DESIGN_ABSORBED;
 }
@@ -338,7 +339,9 @@ vmla_status vmla_config_check(const vmla_config* c) {
   if (c->d_value != c->d_nope + c->d_rope) return VMLA_ERR_UNSUPPORTED_SHAPE;  // dense layout [2][n_h][d_head]
   if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c->dtype == VMLA_BF16) {
-    if (c->d_rope != 32 || c->d_nope != 96 || c->d_value != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    // d_head 128 split 96/32 (every design), or 112/16 and 64/64 (the absorbed design)
+    if (c->d_value != 128 || c->d_nope + c->d_rope != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_rope != 32 && !attn_absorbed_supported(c->d_latent, c->d_rope)) return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (!(c->d_latent == 64 || c->d_latent == 128 || c->d_latent == 192 || c->d_latent == 256 || c->d_latent == 384 ||
           c->d_latent == 512))
       return VMLA_ERR_UNSUPPORTED_SHAPE;
@@ -416,6 +419,7 @@ vmla_status vmla_dense_bind(vmla_handle* h, void* dense) {
   if (!h || !dense || !aligned16(dense)) return VMLA_ERR_INVALID_ARG;
   // the dense layout stores keys rotated at absolute positions: no window-relative re-indexing
   if (h->cfg.sink_frames > 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (h->cfg.dtype == VMLA_BF16 && h->cfg.d_rope != 32) return VMLA_ERR_UNSUPPORTED_SHAPE;  // 96/32 split only
   h->dense = dense;
   h->dense_frames.assign(h->cfg.layers, 0);
   return VMLA_OK;
@@ -494,13 +498,12 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
       e = launch_append_simt(a, s);
     } else {
       CUtensorMap tx, tw;
-      const int nout = c.d_latent + 32;
-      const AppendPlan plan =
-          append_tc_plan(c.d_latent, rows, c.batch, h->append_split, h->append_ctas);
+      const int nout = c.d_latent + c.d_rope;
+      const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_ctas);
       const int parts = plan.parts;
       if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(c.d_latent + 32, parts),
+          !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(nout, parts),
                 CU_TENSOR_MAP_SWIZZLE_128B))
         return map_fail();
       AppendTc a;
@@ -509,6 +512,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
       a.rows = rows;
       a.d_model = c.d_model;
       a.d_latent = c.d_latent;
+      a.d_rope = c.d_rope;
       a.first_frame = first;
       a.rotate = rotate;
       a.contiguous = 0;
@@ -596,6 +600,8 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
                            const FoldArgs* fold = nullptr, const QLatArgs* qlat = nullptr) {
   const vmla_config& c = h->cfg;
   if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  // rotary widths other than 32: the absorbed design with W_uv in its epilogue only
+  if (c.d_rope != 32 && (design != VMLA_DESIGN_ABSORBED || fold || qlat)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   const WsLayout w = ws_layout(c);
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
   const int nq = (int)(n * tokens_per_frame(c));
@@ -606,7 +612,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   cudaError_t e = cudaSuccess;
   if (at_read) {
     StageScope scope(h, 1, s);
-    RopeWindow r{kr_layer, at<__nv_bfloat16>(h->ws, w.kr_rot), c.batch, win.n_keys, 32, win.start_slot,
+    RopeWindow r{kr_layer, at<__nv_bfloat16>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
                  make_ring(c), make_rope(c)};
     e = launch_rope_window_bf16(r, s);
     kpos = at<__nv_bfloat16>(h->ws, w.kr_rot);
@@ -685,7 +691,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   }
 
   __nv_bfloat16* qt = at<__nv_bfloat16>(h->ws, w.qt);
-  const int dqk = c.d_latent + 32;
+  const int dqk = c.d_latent + c.d_rope;
   if (qlat) {
     StageScope scope(h, 2, s);
     CUtensorMap tcq, tw, tqt;
@@ -713,8 +719,8 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     CUtensorMap tq, tuk, tqt;
     if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 2,
               (uint64_t)nq * c.n_heads * 128 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
-              CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map3(&tuk, w_uk, c.d_latent, c.d_nope, c.n_heads, (uint64_t)c.d_latent * 2,
+              (uint64_t)c.d_nope * c.d_latent * 2, 64, c.d_nope, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
               CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
@@ -724,6 +730,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.n_q = nq;
     a.n_heads = c.n_heads;
     a.d_latent = c.d_latent;
+    a.d_rope = c.d_rope;
     a.t_first = t_first;
     a.ring = make_ring(c);
     a.rope = make_rope(c);
@@ -737,11 +744,15 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     const int bn = attn_absorbed_block_n(c.d_latent);
     const uint64_t bh = (uint64_t)c.batch * c.n_heads;
     CUtensorMap tq, tqr, tk, tkr, tuv, to;
+    // the rotary columns: one box c.d_rope wide, swizzled at its row width (32, 64 or 128 bytes)
+    const CUtensorMapSwizzle rsw = c.d_rope == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                  : (c.d_rope == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    const uint64_t rb = (uint64_t)c.d_rope * 2;
     if (!map3(&tq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, c.d_rope, 128, rsw) ||
         !map3(&tk, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, bn,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B))
+        !map3(&tkr, kpos, c.d_rope, win.n_keys, c.batch, rb, rr * rb, c.d_rope, bn, rsw))
       return map_fail();
     if (!fold &&
         (!map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
@@ -760,7 +771,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
     if (!fold) {
-      e = launch_attn_absorbed_tc(c.d_latent, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
+      e = launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
     } else {
       const uint64_t kf = (uint64_t)c.n_heads * c.d_latent;
       __nv_bfloat16* ob_hi = at<__nv_bfloat16>(h->ws, w.obar);
@@ -854,7 +865,8 @@ vmla_status vmla_fold_query_weights(const vmla_config* cfg, const void* w_uq, co
   if (!cfg || !w_uq || !w_qr || !w_uk || !w_qabs) return VMLA_ERR_INVALID_ARG;
   vmla_status st = vmla_config_check(cfg);
   if (st != VMLA_OK) return st;
-  if (cfg->dtype != VMLA_BF16 || !qlat_supported(cfg->d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->dtype != VMLA_BF16 || cfg->d_rope != 32 || !qlat_supported(cfg->d_latent, d_q))
+    return VMLA_ERR_UNSUPPORTED_SHAPE;
   return cuda_status(launch_fold_query(static_cast<const __nv_bfloat16*>(w_uq), static_cast<const __nv_bfloat16*>(w_qr),
                                        static_cast<const __nv_bfloat16*>(w_uk), static_cast<__nv_bfloat16*>(w_qabs),
                                        cfg->n_heads, cfg->d_nope, cfg->d_rope, cfg->d_latent, d_q,
@@ -870,7 +882,7 @@ vmla_status vmla_chunk_attention_qlatent(vmla_handle* h, int layer, const void* 
       !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
   const vmla_config& c = h->cfg;
-  if (c.dtype != VMLA_BF16 || !qlat_supported(c.d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (c.dtype != VMLA_BF16 || c.d_rope != 32 || !qlat_supported(c.d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   Window win;
   if ((st = check_attention_frames(c, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
   if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
@@ -957,14 +969,13 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     e = launch_dense_reconstruct_simt(d, s);
   } else {
     __nv_bfloat16* chunk = at<__nv_bfloat16>(h->ws, w.chunk);  // [B][rows][d_c + 32]
-    const int nout = c.d_latent + 32;
-    const AppendPlan plan =
-          append_tc_plan(c.d_latent, rows, c.batch, h->append_split, h->append_ctas);
-      const int parts = plan.parts;
+    const int nout = c.d_latent + c.d_rope;
+    const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_ctas);
+    const int parts = plan.parts;
     CUtensorMap tx, tw;
     if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(c.d_latent + 32, parts),
+        !map2(&tw, w_down, c.d_model, nout, (uint64_t)c.d_model * 2, 64, append_part_cols(nout, parts),
               CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
     AppendTc a;
@@ -973,6 +984,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     a.rows = rows;
     a.d_model = c.d_model;
     a.d_latent = c.d_latent;
+    a.d_rope = c.d_rope;
     a.first_frame = first;
     a.rotate = 0;
     a.contiguous = 1;

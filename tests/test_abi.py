@@ -97,6 +97,22 @@ def test_config_check_rejects(field, value, status):
     assert api.lib().vmla_config_check(ctypes.byref(c)) == status
 
 
+@pytest.mark.parametrize("d_nope,d_rope,pairs,d_latent,status", [
+    (112, 16, (4, 2, 2), 192, 0), (112, 16, (4, 2, 2), 256, 0), (64, 64, (12, 10, 10), 192, 0),
+    (64, 64, (12, 10, 10), 64, 0), (64, 64, (12, 10, 10), 256, 2), (112, 16, (4, 2, 2), 384, 2),
+    (32, 96, (16, 16, 16), 128, 2),
+])
+def test_bf16_rotary_splits(d_nope, d_rope, pairs, d_latent, status):
+    """d_head 128 split 112/16 and 64/64 run on the absorbed tensor-core design (64/64 up to
+    d_latent 192); 32/96 and the wider latents of those splits are refused as unsupported."""
+    c = default_config()
+    c.d_nope, c.d_rope, c.d_latent = d_nope, d_rope, d_latent
+    c.rope_pairs[:] = list(pairs)
+    assert api.lib().vmla_config_check(ctypes.byref(c)) == status
+    if status == 0:  # the automatic design is the absorbed one: no per-head K/V in the workspace
+        assert api.workspace_bytes(c, api.DESIGN_AUTO) == api.workspace_bytes(c, api.DESIGN_ABSORBED)
+
+
 def test_fp32_accepts_small_shapes():
     c = api.config_from_dims(synth.TINY)
     assert api.lib().vmla_config_check(ctypes.byref(c)) == 0

@@ -216,6 +216,36 @@ def test_small_bf16_dense_designs_short_window():
         assert_bf16_close(out[0], ro.oracle(0, 0, q), f"design {design} dense {dense}", max_abs=6e-2)
 
 
+@pytest.mark.parametrize("d_nope,d_rope,pairs,d_latent,chunks", [
+    (112, 16, (4, 2, 2), 192, 2), (112, 16, (4, 2, 2), 192, 10), (112, 16, (4, 2, 2), 64, 7),
+    (112, 16, (4, 2, 2), 256, 7), (64, 64, (12, 10, 10), 192, 2), (64, 64, (12, 10, 10), 192, 10),
+    (64, 64, (12, 10, 10), 128, 7),
+])
+def test_small_bf16_rotary_split_variants(d_nope, d_rope, pairs, d_latent, chunks):
+    """d_head 128 split 112/16 or 64/64 on the tensor-core path (absorbed design): the shared key
+    is d_latent + d_rope wide, its rotary block swizzled at d_rope * 2 bytes; short, full and
+    wrapped windows."""
+    d = SMALL.replace(name=f"wan_small_r{d_rope}_c{d_latent}", d_nope=d_nope, d_rope=d_rope, rope_pairs=pairs,
+                      d_latent=d_latent)
+    ro = Rollout(d)
+    _fill(ro, chunks)
+    out, q = ro.attend(0, chunks - 1)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"{d_nope}/{d_rope}, d_c {d_latent}, {chunks} chunks")
+
+
+def test_rotary_split_other_designs_refused():
+    """Only the absorbed design runs the 112/16 split: the per-head designs and the dense cache
+    refuse it."""
+    d = SMALL.replace(name="wan_small_r16", d_nope=112, d_rope=16, rope_pairs=(4, 2, 2))
+    ro = Rollout(d)
+    _fill(ro, 1)
+    for design in (api.DESIGN_RECON_ONCE, api.DESIGN_RECONSTRUCT):
+        with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
+            ro.attend(0, 0, design=design)
+    with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
+        Rollout(d, dense=True)
+
+
 def test_absorbed_rejects_latent_384():
     d = SMALL.replace(d_latent=384)
     ro = Rollout(d)
