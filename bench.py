@@ -410,7 +410,8 @@ def run_ours(args, rank, world, local_rank):
                         "latent_width": width_leg(m_timed=timed, dev=dev, tc=tc_burst, seed=seed),
                         "sink_window": sink_leg(dev=dev, tc=tc_burst, seed=seed),
                         "folded_output_mixer": folded_leg(dev=dev, tc=tc_burst, seed=seed),
-                        "query_latent": qlatent_leg(dev=dev, seed=seed)}
+                        "query_latent": qlatent_leg(dev=dev, seed=seed),
+                        "rotary_split": rotary_leg(dev=dev, tc=tc_burst, seed=seed)}
     if dense:
         line["dense"] = dense
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -759,6 +760,62 @@ def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384, 512)):
         res[str(dc)] = entry
         m.close()
         del xp, qp, W, qs, out, m
+        torch.cuda.empty_cache()
+    return res
+
+
+def rotary_leg(dev, tc, seed, splits=((112, 16, (4, 2, 2)), (96, 32, (6, 5, 5)), (64, 64, (12, 10, 10)))):
+    """d_head 128 split into content/rotary dims 112/16, 96/32 and 64/64 on the Wan layer (d_c 192,
+    full window): one chunk step (append + RoPE + q-absorb + absorbed attention) per split."""
+    import torch
+    from latent_kv_attention_down_b200 import api
+    res = {}
+    steps = 20
+    bf = torch.bfloat16
+    for dn, dr, pairs in splits:
+        d = WORKLOAD.replace(d_nope=dn, d_rope=dr, rope_pairs=pairs)
+        L = 2
+        m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+        pool = synth.FramePool(d, base_seed=seed)
+        xp = torch.from_numpy(pool.x).to(dev, bf)
+        qp = torch.from_numpy(pool.q).to(dev, bf)
+        W = [tuple(torch.from_numpy(a).to(dev, bf) for a in (w.w_down, w.w_uk, w.w_uv))
+             for w in (synth.weights(d, l, seed) for l in range(L))]
+        chunks = d.window_frames // d.chunk_frames
+        first = (chunks - 1) * d.chunk_frames
+        for l in range(L):
+            _pool_fill(m, d, pool, xp, W[l], l, chunks)
+        xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
+        qs = [pool.queries(l, chunks - 1, 1, pool=qp) for l in range(L)]
+        out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
+
+        def step(i):
+            l = i % L
+            m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+            m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, api.DESIGN_ABSORBED)
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        m.profile(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            step(3 + i)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        at, n = m.profile_read("attention")
+        m.profile(False)
+        st, flags = m.device_status()
+        assert st == 0, f"device status {st} flags {flags:#x}"
+        F = step_flops(d)
+        att = at / max(n, 1)
+        res[f"{dn}/{dr}"] = {"ms_per_step": ms, "attention_ms": att,
+                             "attention_tflops": F["attention"] / (att * 1e-3) / 1e12,
+                             "frac_of_bf16_peak": F["attention"] / (att * 1e-3) / 1e12 / tc,
+                             "attention_flops": F["attention"]}
+        m.close()
+        del xp, qp, W, xs, qs, out, m
         torch.cuda.empty_cache()
     return res
 
