@@ -207,8 +207,12 @@ vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q,
 
 /* One denoising pass of a chunk, end to end from HOST memory: copy x and q from
  * (preferably pinned) host buffers into the caller's device staging buffers, append,
- * attend, copy out back to the host buffer -- all enqueued on `stream`; the host
- * buffers must stay valid until the stream reaches this point.  Shapes as above. */
+ * attend, copy out back to the host buffer.  The two input copies run on a stream of the
+ * handle's own, each ordered after the previous call's last use of its staging buffer (x_dev:
+ * the append; q_dev: the attention), so consecutive calls overlap them with compute; append,
+ * attention and the output copy are enqueued on `stream`, which waits for the inputs.  The
+ * host buffers must stay valid, and out_host is complete, once `stream` reaches this point.
+ * Shapes as above. */
 vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, const void* q_host,
                                  void* out_host, const void* w_down, const void* w_uk, const void* w_uv,
                                  void* x_dev, void* q_dev, void* out_dev, int64_t first_frame, int n_frames,

@@ -174,6 +174,10 @@ struct vmla_handle {
     std::vector<cudaEvent_t> ev;  // begin/end pairs
     size_t used = 0;
   } timers[kStages];
+  // vmla_chunk_step_host: the input copies run on their own stream, each after the previous
+  // call's last reader of its staging buffer (x: the append, q: the attention)
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t x_ready = nullptr, q_ready = nullptr, x_free = nullptr, q_free = nullptr;
 };
 
 namespace {
@@ -398,6 +402,9 @@ vmla_status vmla_destroy(vmla_handle* h) {
   if (!h) return VMLA_ERR_INVALID_ARG;
   for (auto& t : h->timers)
     for (cudaEvent_t e : t.ev) cudaEventDestroy(e);
+  for (cudaEvent_t e : {h->x_ready, h->q_ready, h->x_free, h->q_free})
+    if (e) cudaEventDestroy(e);
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   delete h;
   return VMLA_OK;
 }
@@ -1083,12 +1090,28 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   const size_t ob = rows * c.n_heads * (size_t)c.d_value * sizeof(float);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if ((e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+  if (!h->copy_stream) {
+    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    for (cudaEvent_t* ev : {&h->x_ready, &h->q_ready, &h->x_free, &h->q_free})
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+  }
+  cudaStream_t cs = h->copy_stream;
+  // inputs on the copy stream: x once the previous call's append has read x_dev, q once its
+  // attention has read q_dev, so both copies overlap the previous call's attention and output
+  // copy; the compute stream waits for each copy before its consumer
+  if ((e = cudaStreamWaitEvent(cs, h->x_free, 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaEventRecord(h->x_ready, cs)) != cudaSuccess || (e = cudaStreamWaitEvent(cs, h->q_free, 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaEventRecord(h->q_ready, cs)) != cudaSuccess || (e = cudaStreamWaitEvent(s, h->x_ready, 0)) != cudaSuccess)
     return cuda_fail(e);
   if ((st = vmla_cache_append(h, layer, x_dev, w_down, first, n, stream)) != VMLA_OK) return st;
+  if ((e = cudaEventRecord(h->x_free, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s, h->q_ready, 0)) != cudaSuccess)
+    return cuda_fail(e);
   if ((st = vmla_chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream)) != VMLA_OK)
     return st;
+  if ((e = cudaEventRecord(h->q_free, s)) != cudaSuccess) return cuda_fail(e);
+  // the output copy stays on the caller's stream: the host result is there when `stream` is
   return cuda_status(cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s));
 }
 
