@@ -90,20 +90,6 @@ __device__ __forceinline__ void store_bf16x32_smem(uint8_t* dst, const float (&v
                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 u = s[q];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[8 * q + 2 * k] = __uint_as_float(w[k] << 16);
-      v[8 * q + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-    }
-  }
-}
-
 // N 16-byte chunks (8 bf16 each, from fp32 bit patterns in r) of row `row` of a column block
 // parked for a TMA tensor store with 128-byte swizzle: the block holds 64 columns, 128 bytes per
 // row, and chunk j of a row sits at position j ^ (row & 7), so the eight rows a quarter-warp
@@ -360,6 +346,7 @@ struct QPrepCfg {
   static constexpr int NA = (NB + 1) / 2;  // [NA, NB) and the positional block by warpgroup 1
   static_assert(DL % 64 == 0 && DL <= 256 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
   static_assert((DR == 16 || DR == 32 || DR == 64) && W_BYTES % 1024 == 0, "rotary dims");
+  static_assert(ROW > (NCB - 1) * 64 && ROW <= NCB * 64, "a row of q~ spans its parked column blocks");
 };
 
 template <int DL, int DR>
