@@ -65,3 +65,26 @@ def test_reference_arm_prints_on_rank0_only():
                           "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    """The roofline's `traffic` comes from a committed ncu summary only while the kernel source
+    still has the sha256 recorded beside it; an edited source (or a summary without the fields)
+    gives None rather than stale counters."""
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "latent_kv_attention_down_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    src = csrc / "k.cu"
+    src.write_text("kernel body\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles" / "k.md").write_text(f"source_sha256: {sha}\n| dram_bytes_per_launch: 42190592 | r+w |\n")
+    (tmp_path / "profiles" / "bare.md").write_text("no fields here\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k.cu", "k.md") == 42190592.0
+    assert bench.profiled_traffic("k.cu", "bare.md") is None
+    assert bench.profiled_traffic("missing.cu", "k.md") is None
+    src.write_text("kernel body, edited\n")
+    assert bench.profiled_traffic("k.cu", "k.md") is None
