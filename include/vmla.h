@@ -209,9 +209,12 @@ vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q,
  * (preferably pinned) host buffers into the caller's device staging buffers, append,
  * attend, copy out back to the host buffer.  The two input copies run on a stream of the
  * handle's own, each ordered after the previous call's last use of its staging buffer (x_dev:
- * the append; q_dev: the attention), so consecutive calls overlap them with compute; append,
- * attention and the output copy are enqueued on `stream`, which waits for the inputs.  The
- * host buffers must stay valid, and out_host is complete, once `stream` reaches this point.
+ * the append; q_dev: the attention), so consecutive calls overlap them with compute; append and
+ * attention are enqueued on `stream`, which waits for the inputs.  The absorbed attention runs
+ * as one launch per group of heads that fills the GPU once, and each group's output columns
+ * go back to out_host on a third stream while the next group computes; `stream` waits for the
+ * last of those copies (other designs copy the output back on `stream`).  The host buffers
+ * must stay valid, and out_host is complete, once `stream` reaches this point.
  * Shapes as above. */
 vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, const void* q_host,
                                  void* out_host, const void* w_down, const void* w_uk, const void* w_uv,

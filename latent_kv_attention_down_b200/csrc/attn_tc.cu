@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sKV = smem_raw + C::Q_BYTES;
   Bars* bars = reinterpret_cast<Bars*>(sKV + C::STAGES * C::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int mt = blockIdx.x, h = a.h0 + (int)blockIdx.y, b = blockIdx.z;
   const int m0 = mt * 128;
   const int n_tiles = (a.n_keys + C::BN - 1) / C::BN;
   const int epi_wuv = (n_tiles % C::STAGES) * C::STAGE_BYTES;           // W_uv,h
@@ -519,8 +519,9 @@ cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtenso
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (attr != cudaSuccess) return attr;
   if (a.n_q <= 0 || a.n_keys <= 0) return cudaSuccess;
-  attn_tc_kernel<DL, DENSE, FOLD, DR><<<dim3(a.m_tiles, a.n_heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr,
-                                                                                                   tuv, to, a);
+  const int heads = a.h_count > 0 ? a.h_count : a.n_heads;
+  attn_tc_kernel<DL, DENSE, FOLD, DR><<<dim3(a.m_tiles, heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv,
+                                                                                               to, a);
   return cudaGetLastError();
 }
 

@@ -183,6 +183,8 @@ struct AttnTc {
   float rescale_threshold;  // lazy-rescale threshold of the running max, log2 units
   unsigned* err;
   uint64_t limit_ns;
+  int h0 = 0;       // absorbed and dense attention: first head of this launch
+  int h_count = 0;  // heads of this launch (grid y); 0 = all n_heads
 };
 // Absorbed design.  qt maps: 3D (d_c+32, n_q, B*n_h): latent box (64,128,1) SW128, rope box (32,128,1) SW64;
 // ckv map: 3D (d_c, n_keys, B) box (64,BN,1) SW128; kr map: 3D (32, n_keys, B) box (32,BN,1) SW64;

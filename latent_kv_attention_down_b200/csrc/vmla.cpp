@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -178,6 +179,9 @@ struct vmla_handle {
   // call's last reader of its staging buffer (x: the append, q: the attention)
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t x_ready = nullptr, q_ready = nullptr, x_free = nullptr, q_free = nullptr;
+  // ... and the output comes back on a second one, a group of heads at a time
+  cudaStream_t out_stream = nullptr;
+  cudaEvent_t out_group = nullptr, out_done = nullptr;
 };
 
 namespace {
@@ -402,9 +406,10 @@ vmla_status vmla_destroy(vmla_handle* h) {
   if (!h) return VMLA_ERR_INVALID_ARG;
   for (auto& t : h->timers)
     for (cudaEvent_t e : t.ev) cudaEventDestroy(e);
-  for (cudaEvent_t e : {h->x_ready, h->q_ready, h->x_free, h->q_free})
+  for (cudaEvent_t e : {h->x_ready, h->q_ready, h->x_free, h->q_free, h->out_group, h->out_done})
     if (e) cudaEventDestroy(e);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  if (h->out_stream) cudaStreamDestroy(h->out_stream);
   delete h;
   return VMLA_OK;
 }
@@ -602,9 +607,19 @@ struct QLatArgs {
   int d_q;
 };
 
+// Output rows wanted in host memory (vmla_chunk_step_host): the absorbed attention then runs as
+// one launch per group of heads that fills the GPU once, and each group's columns are copied to
+// the host on `stream` while the next group computes; `copied` tells the caller it was done.
+struct HostOut {
+  void* host;
+  cudaStream_t stream;
+  cudaEvent_t group, done;
+  bool copied;
+};
+
 vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
                            int64_t first, int n, const Window& win, vmla_design design, cudaStream_t s,
-                           const FoldArgs* fold = nullptr, const QLatArgs* qlat = nullptr) {
+                           const FoldArgs* fold = nullptr, const QLatArgs* qlat = nullptr, HostOut* hout = nullptr) {
   const vmla_config& c = h->cfg;
   if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   // rotary widths other than 32: the absorbed design with W_uv in its epilogue only
@@ -777,8 +792,33 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.rescale_threshold = c.softmax_rescale_log2;
     a.err = h->err;
     a.limit_ns = kWaitLimitNs;
-    if (!fold) {
+    if (!fold && !hout) {
       e = launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
+    } else if (!fold) {
+      static int sms = 0;
+      if (sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+          sms = 148;
+      }
+      const int per_head = a.m_tiles * c.batch;  // CTAs of one head
+      const int hg = std::max(1, std::min(c.n_heads, sms / std::max(1, per_head)));
+      const size_t pitch = (size_t)c.n_heads * 128 * sizeof(float);
+      for (int g0 = 0; g0 < c.n_heads && e == cudaSuccess; g0 += hg) {
+        a.h0 = g0;
+        a.h_count = std::min(hg, c.n_heads - g0);
+        if ((e = launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, a, c.batch, s)) != cudaSuccess ||
+            (e = cudaEventRecord(hout->group, s)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(hout->stream, hout->group, 0)) != cudaSuccess)
+          break;
+        e = cudaMemcpy2DAsync(static_cast<char*>(hout->host) + (size_t)g0 * 128 * sizeof(float), pitch,
+                              static_cast<const char*>(out) + (size_t)g0 * 128 * sizeof(float), pitch,
+                              (size_t)a.h_count * 128 * sizeof(float), (size_t)c.batch * nq, cudaMemcpyDeviceToHost,
+                              hout->stream);
+      }
+      if (e == cudaSuccess && (e = cudaEventRecord(hout->done, hout->stream)) == cudaSuccess)
+        e = cudaStreamWaitEvent(s, hout->done, 0);
+      hout->copied = e == cudaSuccess;
     } else {
       const uint64_t kf = (uint64_t)c.n_heads * c.d_latent;
       __nv_bfloat16* ob_hi = at<__nv_bfloat16>(h->ws, w.obar);
@@ -846,8 +886,9 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
 
 }  // namespace
 
-vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
-                                 void* out, int64_t first, int n, vmla_design design, void* stream) {
+namespace {
+vmla_status chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
+                            int64_t first, int n, vmla_design design, void* stream, HostOut* hout) {
   vmla_status st = check_layer(h, layer);
   if (st != VMLA_OK) return st;
   if (!h->ckv) return VMLA_ERR_STATE;
@@ -864,7 +905,14 @@ vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const
   if (h->cfg.dtype == VMLA_BF16 && design == VMLA_DESIGN_ABSORBED && h->cfg.d_latent > 256)
     return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
-  return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s);
+  return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s, nullptr, nullptr,
+                        design == VMLA_DESIGN_ABSORBED ? hout : nullptr);
+}
+}  // namespace
+
+vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
+                                 void* out, int64_t first, int n, vmla_design design, void* stream) {
+  return chunk_attention(h, layer, q, w_uk, w_uv, out, first, n, design, stream, nullptr);
 }
 
 vmla_status vmla_fold_query_weights(const vmla_config* cfg, const void* w_uq, const void* w_qr, const void* w_uk,
@@ -1091,8 +1139,10 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (!h->copy_stream) {
-    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
-    for (cudaEvent_t* ev : {&h->x_ready, &h->q_ready, &h->x_free, &h->q_free})
+    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&h->out_stream, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e);
+    for (cudaEvent_t* ev : {&h->x_ready, &h->q_ready, &h->x_free, &h->q_free, &h->out_group, &h->out_done})
       if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
   }
   cudaStream_t cs = h->copy_stream;
@@ -1108,10 +1158,13 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   if ((st = vmla_cache_append(h, layer, x_dev, w_down, first, n, stream)) != VMLA_OK) return st;
   if ((e = cudaEventRecord(h->x_free, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s, h->q_ready, 0)) != cudaSuccess)
     return cuda_fail(e);
-  if ((st = vmla_chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream)) != VMLA_OK)
+  HostOut hout{out_host, h->out_stream, h->out_group, h->out_done, false};
+  if ((st = chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream, &hout)) != VMLA_OK)
     return st;
   if ((e = cudaEventRecord(h->q_free, s)) != cudaSuccess) return cuda_fail(e);
-  // the output copy stays on the caller's stream: the host result is there when `stream` is
+  // the host result is there when `stream` is: the absorbed attention copied it back a group of
+  // heads at a time (and made `stream` wait for the last copy); other paths copy it here
+  if (hout.copied) return VMLA_OK;
   return cuda_status(cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s));
 }
 

@@ -376,6 +376,37 @@ def test_step_host_matches_device_path():
     assert_bf16_close(oh.float().numpy()[0], ro.oracle(0, 7, q), "host step")
 
 
+def test_step_host_head_groups_match_device_path():
+    """Batch 4 on the small grid: the host-buffer step runs the attention as one launch per group
+    of heads that fills the GPU once (7 + 5 heads) and copies each group's output columns back
+    while the next group computes.  Two consecutive calls on the same staging buffers, issued
+    without a wait between them, must equal the device path bit for bit."""
+    import torch
+    d = SMALL.replace(batch=4)
+    dev, host = Rollout(d), Rollout(d)
+    _fill(dev, 6)
+    _fill(host, 6)
+    xd = torch.empty((d.batch, d.n_queries, d.d_model), dtype=torch.bfloat16, device="cuda")
+    qd = torch.empty((d.batch, d.n_queries, d.n_heads, d.d_head), dtype=torch.bfloat16, device="cuda")
+    od = torch.empty((d.batch, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device="cuda")
+    keep, outs = [], []
+    for chunk in (6, 7):
+        x = torch.from_numpy(synth.activations(d, 0, chunk)).to(torch.bfloat16).pin_memory()
+        q = torch.from_numpy(synth.queries(d, 0, chunk)).to(torch.bfloat16).pin_memory()
+        oh = torch.full((d.batch, d.n_queries, d.n_heads * d.d_head), float("nan")).pin_memory()
+        wd = host.wd[0]
+        host.m.step_host(0, x, q, oh, wd[0], wd[1], wd[2], xd, qd, od, chunk * d.chunk_frames, d.chunk_frames)
+        keep.append((x, q))
+        outs.append(oh)
+    torch.cuda.synchronize()
+    st, flags = host.m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    for chunk, oh in zip((6, 7), outs):
+        dev.append_chunk(0, chunk)
+        ref, _ = dev.attend(0, chunk)
+        assert np.array_equal(oh.numpy(), ref), f"chunk {chunk}: host step differs from the device path"
+
+
 # ------------------------------------------------------------------ the full Wan-1.3B layer
 
 def test_wan_layer_sampled_rows():
