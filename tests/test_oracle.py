@@ -149,6 +149,46 @@ def test_rope(check):
     check(O)
 
 
+@pytest.mark.parametrize("pairs", [(4, 2, 2), (12, 10, 10), (16, 16, 16)])
+def test_rope_other_rotary_splits(pairs):
+    """The 16, 64 and 96 rotary-dim layouts: every axis's first band turns at 1 rad per position
+    and, with the default base 2*n_a, band n_a/2 at 10000^(-1/2) = 0.01; each axis turns its own
+    2*n_a dims, in t, h, w order; scores stay invariant under a common shift on any axis and move
+    under a one-sided one."""
+    f = O.rope_frequencies(pairs)
+    assert [len(a) for a in f] == list(pairs)
+    for a, n in zip(f, pairs):
+        assert a[0] == 1.0
+        np.testing.assert_allclose(a[n // 2], 0.01, rtol=1e-14)
+        assert np.all(np.diff(a) < 0)
+    dr = 2 * sum(pairs)
+    v = _rand(3, dr)
+    zero = np.zeros(3)
+    base = O.rope_rotate(v, O.rope_angles(zero, zero, zero, f))
+    edges = np.cumsum([0] + [2 * n for n in pairs])
+    for axis in range(3):
+        pos = [zero.copy() for _ in range(3)]
+        pos[axis] = np.full(3, 5.0)
+        moved = np.any(np.abs(O.rope_rotate(v, O.rope_angles(*pos, f)) - base) > 1e-12, axis=0)
+        expect = np.zeros(dr, dtype=bool)
+        expect[edges[axis]:edges[axis + 1]] = True
+        assert np.array_equal(moved, expect), (pairs, axis)
+    a_, b_ = _rand(30, dr), _rand(30, dr)
+    p1, p2 = RNG.integers(0, 60, size=(30, 3)), RNG.integers(0, 60, size=(30, 3))
+
+    def score(pa, pb):
+        ra = O.rope_rotate(a_, O.rope_angles(pa[:, 0], pa[:, 1], pa[:, 2], f))
+        rb = O.rope_rotate(b_, O.rope_angles(pb[:, 0], pb[:, 1], pb[:, 2], f))
+        return np.sum(ra * rb, axis=1)
+
+    s0 = score(p1, p2)
+    for axis in range(3):
+        d = np.zeros(3, dtype=np.int64)
+        d[axis] = 23
+        np.testing.assert_allclose(score(p1 + d, p2 + d), s0, atol=1e-11)
+        assert np.max(np.abs(score(p1 + d, p2) - s0)) > 1e-3
+
+
 # ---------------------------------------------------------------- ring / window
 
 def check_ring_against_deque(orc, W=21, chunk=3, chunks=20):
