@@ -61,8 +61,9 @@ typedef enum vmla_dtype { VMLA_BF16 = 0, VMLA_FP32 = 1 } vmla_dtype;
 
 /* How vmla_chunk_attention evaluates the same scores and outputs. */
 typedef enum vmla_design {
-  VMLA_DESIGN_AUTO = 0,        /* ABSORBED for d_latent <= 192, RECON_ONCE from 256 on (VMLA_BF16;
-                                  VMLA_FP32 always evaluates the absorbed form) */
+  VMLA_DESIGN_AUTO = 0,        /* VMLA_BF16: ABSORBED for d_latent <= 192, RECON_ONCE from 256 on, and
+                                  ABSORBED whenever d_rope != 32; VMLA_FP32 always evaluates the
+                                  absorbed form */
   VMLA_DESIGN_ABSORBED = 1,    /* W_uk folded into the query, MQA over [c_KV | k_R], W_uv after the
                                   softmax-weighted sum [paperlayer App. E] */
   VMLA_DESIGN_RECONSTRUCT = 2, /* per KV tile, per-head K/V rebuilt from c_KV on the tensor core and kept
@@ -76,7 +77,8 @@ typedef enum vmla_design {
 /* When the positional key gets its 3D rotation. */
 typedef enum vmla_rope_mode {
   VMLA_ROPE_AT_READ = 0,  /* stored unrotated, rotated at attention time with window-relative frame
-                             indices t = frame - first frame of the window [paperlayer App. D.5, App. E] */
+                             indices: t = the frame's position in the window, oldest first (sink
+                             frames first) [paperlayer App. D.5, App. E] */
   VMLA_ROPE_AT_APPEND = 1 /* rotated at append with the absolute frame index (scores are identical
                              without a sink frame, RoPE depends on offsets only) */
 } vmla_rope_mode;
@@ -130,10 +132,14 @@ int vmla_abi_version(void);
 vmla_status vmla_config_init(vmla_config* cfg);
 
 /* VMLA_OK when every field is consistent and a kernel exists for it:
- * VMLA_FP32 accepts any positive sizes (d_latent, d_nope+d_rope, d_value <= 512; up to 64 rotary pairs);
- * VMLA_BF16 needs d_nope + d_rope = d_value = 128, d_rope = 32 and d_latent one of 64, 128,
- * 192, 256, 384, 512 (VMLA_DESIGN_ABSORBED up to 256, VMLA_DESIGN_RECONSTRUCT up to 192;
- * other shapes run with VMLA_FP32).
+ * VMLA_FP32 accepts any positive sizes (d_latent + d_rope <= 1024, d_value <= 1024, up to 64
+ * rotary pairs);
+ * VMLA_BF16 needs d_model a multiple of 64, d_nope + d_rope = d_value = 128 and d_latent one of
+ * 64, 128, 192, 256, 384, 512 (VMLA_DESIGN_ABSORBED up to 256, VMLA_DESIGN_RECONSTRUCT up to 192),
+ * with d_rope = 32 for every design, or d_rope = 16 (d_latent <= 256) or 64 (d_latent <= 192) for
+ * the absorbed design only: the other designs, the dense cache, the folded mixer, the query-latent
+ * path and the allocation-free call return VMLA_ERR_UNSUPPORTED_SHAPE for those splits.
+ * Other shapes run with VMLA_FP32.
  * grid_h, grid_w, window_frames must be < 1024 (RoPE range, [paperlayer App. C.1]). */
 vmla_status vmla_config_check(const vmla_config* cfg);
 
@@ -182,8 +188,9 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
  *   for query i of frame first_frame + i/T_f and head h,
  *     out[i, h*d_value:(h+1)*d_value] = sum_j softmax_j(s_ij) W_uv,h c_j,
  *     s_ij = ( q_nope,ih . W_uk,h c_j  +  RoPE(q_rope,ih) . RoPE(k_R,j) ) / sqrt(d_nope + d_rope)
- *   over every key j of the window frames [max(0, F-W), F) (no mask: the chunk is
- *   the newest frames and sees itself).
+ *   over every key j of the window frames [max(0, F-W), F) -- with sink frames, the first S
+ *   frames of the rollout and the newest W-S -- (no mask: the chunk is the newest frames and
+ *   sees itself).
  * q:    [batch][n_frames*T_f][n_heads][d_nope + d_rope]  (per head: content, then positional)
  * w_uk: [n_heads][d_nope][d_latent]   w_uv: [n_heads][d_value][d_latent]
  * out:  [batch][n_frames*T_f][n_heads*d_value], float32 for both dtypes (a bf16 rounding of the
