@@ -472,19 +472,29 @@ vmla_status vmla_state_set(vmla_handle* h, int layer, int64_t F) {
   return VMLA_OK;
 }
 
-vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, int64_t first,
-                              int n, void* stream) {
+namespace {
+// Every host-side check of a cache append (no CUDA call); *new_F gets the layer's frame count after it.
+vmla_status append_args(vmla_handle* h, int layer, const void* x, const void* w_down, int64_t first, int n,
+                        int64_t* new_F) {
   vmla_status st = check_layer(h, layer);
   if (st != VMLA_OK) return st;
   if (!h->ckv) return VMLA_ERR_STATE;
   if (!x || !w_down || !aligned16(x) || !aligned16(w_down)) return VMLA_ERR_INVALID_ARG;
   const vmla_config& c = h->cfg;
-  int64_t new_F;
-  if ((st = check_append_frames(c, h->frames[layer], first, n, &new_F)) != VMLA_OK) return st;
-  const bool rotate = c.rope_mode == VMLA_ROPE_AT_APPEND;
-  if (rotate && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  if ((st = check_append_frames(c, h->frames[layer], first, n, new_F)) != VMLA_OK) return st;
+  if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c.dtype == VMLA_BF16 && !append_tiling_fits(c, h->append_split)) return VMLA_ERR_UNSUPPORTED_SHAPE;
-  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  return VMLA_OK;
+}
+}  // namespace
+
+vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const void* w_down, int64_t first,
+                              int n, void* stream) {
+  int64_t new_F;
+  vmla_status st = append_args(h, layer, x, w_down, first, n, &new_F);
+  if (st != VMLA_OK || (st = ensure_err(h)) != VMLA_OK) return st;
+  const vmla_config& c = h->cfg;
+  const bool rotate = c.rope_mode == VMLA_ROPE_AT_APPEND;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = (int)(n * tokens_per_frame(c));
   cudaError_t e;
@@ -887,23 +897,40 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
 }  // namespace
 
 namespace {
-vmla_status chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
-                            int64_t first, int n, vmla_design design, void* stream, HostOut* hout) {
+// Every host-side check of a chunk attention call (no CUDA call) when the layer holds `frames`
+// frames; *design gets the design that runs and *win the window.
+vmla_status attention_args(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
+                           const void* out, int64_t first, int n, vmla_design* design, int64_t frames, Window* win) {
   vmla_status st = check_layer(h, layer);
   if (st != VMLA_OK) return st;
   if (!h->ckv) return VMLA_ERR_STATE;
   if (!q || !w_uk || !w_uv || !out || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
-  if (design < VMLA_DESIGN_AUTO || design > VMLA_DESIGN_RECON_ONCE) return VMLA_ERR_INVALID_ARG;
+  if (*design < VMLA_DESIGN_AUTO || *design > VMLA_DESIGN_RECON_ONCE) return VMLA_ERR_INVALID_ARG;
+  const vmla_config& c = h->cfg;
+  if ((st = check_attention_frames(c, frames, first, n, win)) != VMLA_OK) return st;
+  if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
+  *design = resolve_design(c, *design);
+  if (c.dtype == VMLA_BF16) {
+    // the absorbed kernels keep d_latent + d_rope query and key columns resident: up to 256 latent dims
+    if (*design == VMLA_DESIGN_ABSORBED && c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (*design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent))
+      return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c.d_rope != 32 && *design != VMLA_DESIGN_ABSORBED) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (*design == VMLA_DESIGN_RECON_ONCE) {
+      const WsLayout w = ws_layout(c);
+      if (h->ws_bytes < w.base_bytes + w.recon_bytes) return VMLA_ERR_STATE;
+    }
+  }
+  return VMLA_OK;
+}
+
+vmla_status chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
+                            int64_t first, int n, vmla_design design, void* stream, HostOut* hout) {
   Window win;
-  if ((st = check_attention_frames(h->cfg, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
-  if (h->cfg.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
-  if ((st = ensure_err(h)) != VMLA_OK) return st;
+  vmla_status st = attention_args(h, layer, q, w_uk, w_uv, out, first, n, &design, h->frames[layer], &win);
+  if (st != VMLA_OK || (st = ensure_err(h)) != VMLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  design = resolve_design(h->cfg, design);
-  // the absorbed kernels keep d_latent + 32 query and key columns resident: up to 256 latent dims
-  if (h->cfg.dtype == VMLA_BF16 && design == VMLA_DESIGN_ABSORBED && h->cfg.d_latent > 256)
-    return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
   return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s, nullptr, nullptr,
                         design == VMLA_DESIGN_ABSORBED ? hout : nullptr);
@@ -1131,6 +1158,15 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   if (st != VMLA_OK) return st;
   if (!x_host || !q_host || !out_host || !x_dev || !q_dev || !out_dev) return VMLA_ERR_INVALID_ARG;
   if (n < 1 || n > h->cfg.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
+  // everything the append and the attention would refuse is refused here, before any copy is enqueued
+  int64_t new_F;
+  if ((st = append_args(h, layer, x_dev, w_down, first, n, &new_F)) != VMLA_OK) return st;
+  {
+    vmla_design d = design;
+    Window win;
+    if ((st = attention_args(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, &d, new_F, &win)) != VMLA_OK) return st;
+  }
+  if ((st = ensure_err(h)) != VMLA_OK) return st;
   const vmla_config& c = h->cfg;
   const size_t rows = (size_t)n * tokens_per_frame(c) * c.batch;
   const size_t xb = rows * c.d_model * esize(c);

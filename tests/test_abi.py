@@ -199,6 +199,15 @@ def test_frame_rule_rejections_before_any_launch():
     # the dense calls need their own cache bound first
     assert lib.vmla_dense_cache_append(h._h, 0, x, w, w, w, 0, 3, None) == 6
     assert h.state_get(0) == 9
+    # the host-buffer step refuses what its append or its attention would refuse, before any copy
+    step = lib.vmla_chunk_step_host
+    hb = 0x50000  # host buffers: never touched when the call is refused
+    assert step(h._h, 0, hb, hb, hb, w, w, w, x, x, x, 3, 3, 0, None) == 6    # skips frames
+    assert step(h._h, 0, hb, hb, hb, w, w, w, x, x, x, 9, 3, 9, None) == 1    # bad design
+    assert step(h._h, 0, hb, hb, hb, w, w, w, 0x40008, x, x, 9, 3, 0, None) == 1  # misaligned x_dev
+    assert step(h._h, 0, hb, hb, hb, w, w, w, x, x, 0x40008, 9, 3, 0, None) == 1  # misaligned out_dev
+    assert step(h._h, 1, hb, hb, hb, w, w, w, x, x, x, 9, 3, 0, None) == 3    # layer out of range
+    assert h.state_get(0) == 9
     h.close()
 
 
