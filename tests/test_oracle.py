@@ -535,3 +535,53 @@ def test_query_latent_absorption_equals_the_definition():
     bad[:, :d_c] = np.einsum("hnc,hnj->hcj", w_uk, w_uq[::-1])   # heads crossed
     assert np.abs(O.chunk_attention_query_latent(c, r, kpos, cq, qpos, bad, w_uv, d_latent=d_c,
                                                  d_head=d_nope + d_rope, **kw) - ref).max() > 1e-3
+
+
+def test_sink_window_attention_brute_force():
+    """One sink frame and a three-frame local part (W = 4) after ten one-frame chunks, by explicit
+    loops: the context is frames 0, 7, 8, 9 at t = 0, 1, 2, 3; every key k_jh = [W_uk,h c_j |
+    R(t_j, h_j, w_j) k_R,j] and query [q_nope | R(3, h_i, w_i) q_rope] is rotated pair by pair as a
+    complex number, the softmax is taken over the 24 keys one score at a time, and v_jh = W_uv,h c_j.
+    The oracle's window, positions and attention must give the same output."""
+    rng = np.random.default_rng(21)
+    D, n_h, d_nope, d_c, gh, gw, W, S = 5, 2, 4, 3, 2, 3, 4, 1
+    pairs = (1, 0, 1)                                 # d_rope = 4: one t pair, one w pair
+    d_rope = 2 * sum(pairs)
+    T = gh * gw
+    w_down = rng.standard_normal((d_c + d_rope, D))
+    w_uk = rng.standard_normal((n_h, d_nope, d_c))
+    w_uv = rng.standard_normal((n_h, d_nope + d_rope, d_c))
+    frame_x = {f: rng.standard_normal((T, D)) for f in range(10)}
+    q = rng.standard_normal((T, n_h, d_nope + d_rope))
+    # the oracle
+    c, r, kpos, t0 = O.window_latents(frame_x, 10, W, w_down, d_c, gh, gw, sink_frames=S)
+    qpos = O.chunk_query_positions(9, 1, t0, gh, gw)
+    got = O.chunk_attention(c, r, kpos, q, qpos, w_uk, w_uv, d_nope=d_nope, rope_pairs=pairs).reshape(T, n_h, -1)
+    # brute force: base 2*n_a gives the single band of an axis a frequency of 1
+    context = [(0, 0), (7, 1), (8, 2), (9, 3)]          # (frame, window-relative t)
+
+    def rotate(v, t, hh, ww):                          # v: [t pair | w pair]
+        out = np.array(v, dtype=np.float64)
+        for k, p in ((0, t), (1, ww)):
+            z = complex(v[2 * k], v[2 * k + 1]) * np.exp(1j * p * 1.0)
+            out[2 * k], out[2 * k + 1] = z.real, z.imag
+        return out
+
+    scale = 1.0 / np.sqrt(d_nope + d_rope)
+    for i in range(T):
+        hi, wi = divmod(i, gw)
+        for h in range(n_h):
+            qv = np.concatenate([q[i, h, :d_nope], rotate(q[i, h, d_nope:], 3, hi, wi)])
+            scores, values = [], []
+            for f, t in context:
+                for j in range(T):
+                    hj, wj = divmod(j, gw)
+                    cj = w_down[:d_c] @ frame_x[f][j]
+                    kr = w_down[d_c:] @ frame_x[f][j]
+                    k = np.concatenate([w_uk[h] @ cj, rotate(kr, t, hj, wj)])
+                    scores.append(float(qv @ k) * scale)
+                    values.append(w_uv[h] @ cj)
+            m = max(scores)
+            e = [np.exp(s - m) for s in scores]
+            ref = sum(ei * v for ei, v in zip(e, values)) / sum(e)
+            np.testing.assert_allclose(got[i, h], ref, rtol=1e-11, atol=1e-12)
