@@ -394,6 +394,15 @@ def _reconstruct_no_rope(c, k_rope, w_uk, w_uv):
     return k, v
 
 
+def _sink_local_t_from_zero(frames_appended, window_frames, sink_frames=0):
+    frames = O.window_frames_list(frames_appended, window_frames, sink_frames)
+    return {f: (k if k < sink_frames else k - sink_frames) for k, f in enumerate(frames)}
+
+
+def _sink_evicted(frames_appended, window_frames, sink_frames=0):
+    return O.window_frames_list(frames_appended, window_frames, 0)
+
+
 MUTANTS = {
     "rope rotates the wrong way": dict(rope_rotate=_rope_sign_flip),
     "rope axes in the wrong order": dict(rope_angles=_rope_axis_swap),
@@ -401,6 +410,8 @@ MUTANTS = {
     "softmax scale wrong": dict(softmax_attention=_softmax_no_max),
     "window one frame short": dict(window_frame_range=_window_off_by_one),
     "positional score dropped from the per-head keys": dict(reconstruct_heads=_reconstruct_no_rope),
+    "sink window: local frames counted from t = 0": dict(window_frame_t=_sink_local_t_from_zero),
+    "sink window: the sink frame evicted like the others": dict(window_frames_list=_sink_evicted),
 }
 
 
@@ -411,6 +422,8 @@ def _all_checks(orc, golden):
         chk(orc)
     for chk in ATTN_CHECKS:
         chk(orc)
+    check_sink_slot_array(orc)
+    check_sink_attention_brute_force(orc)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -440,24 +453,28 @@ def _simulate_sink_ring(n_frames, W, S):
     return states
 
 
-@pytest.mark.parametrize("W,S", [(7, 1), (4, 1), (5, 2), (21, 0)])
-def test_sink_window_matches_an_explicit_slot_array(W, S):
+def check_sink_slot_array(orc, W=7, S=1):
     states = _simulate_sink_ring(60, W, S)
     for F in range(1, 61):
         slots = states[F - 1]
-        frames = O.window_frames_list(F, W, S)
+        frames = orc.window_frames_list(F, W, S)
         assert sorted(frames) == sorted(f for f in slots if f is not None)
         for k, f in enumerate(slots):
             if f is not None:
-                assert O.ring_slot(f, W, S) == k
+                assert orc.ring_slot(f, W, S) == k
         # sink first, locals oldest first, window-relative t = position in that order
-        t = O.window_frame_t(F, W, S)
+        t = orc.window_frame_t(F, W, S)
         sink = [f for f in frames if f < S]
         local = [f for f in frames if f >= S]
         assert frames == sink + sorted(local)
         assert [t[f] for f in frames] == list(range(len(frames)))
         if S == 0:
-            assert frames == list(range(*O.window_frame_range(F, W)))
+            assert frames == list(range(*orc.window_frame_range(F, W)))
+
+
+@pytest.mark.parametrize("W,S", [(7, 1), (4, 1), (5, 2), (21, 0)])
+def test_sink_window_matches_an_explicit_slot_array(W, S):
+    check_sink_slot_array(O, W, S)
 
 
 def test_sink_window_keeps_rope_positions_bounded():
@@ -537,7 +554,7 @@ def test_query_latent_absorption_equals_the_definition():
                                                  d_head=d_nope + d_rope, **kw) - ref).max() > 1e-3
 
 
-def test_sink_window_attention_brute_force():
+def check_sink_attention_brute_force(orc):
     """One sink frame and a three-frame local part (W = 4) after ten one-frame chunks, by explicit
     loops: the context is frames 0, 7, 8, 9 at t = 0, 1, 2, 3; every key k_jh = [W_uk,h c_j |
     R(t_j, h_j, w_j) k_R,j] and query [q_nope | R(3, h_i, w_i) q_rope] is rotated pair by pair as a
@@ -554,9 +571,9 @@ def test_sink_window_attention_brute_force():
     frame_x = {f: rng.standard_normal((T, D)) for f in range(10)}
     q = rng.standard_normal((T, n_h, d_nope + d_rope))
     # the oracle
-    c, r, kpos, t0 = O.window_latents(frame_x, 10, W, w_down, d_c, gh, gw, sink_frames=S)
-    qpos = O.chunk_query_positions(9, 1, t0, gh, gw)
-    got = O.chunk_attention(c, r, kpos, q, qpos, w_uk, w_uv, d_nope=d_nope, rope_pairs=pairs).reshape(T, n_h, -1)
+    c, r, kpos, t0 = orc.window_latents(frame_x, 10, W, w_down, d_c, gh, gw, sink_frames=S)
+    qpos = orc.chunk_query_positions(9, 1, t0, gh, gw)
+    got = orc.chunk_attention(c, r, kpos, q, qpos, w_uk, w_uv, d_nope=d_nope, rope_pairs=pairs).reshape(T, n_h, -1)
     # brute force: base 2*n_a gives the single band of an axis a frequency of 1
     context = [(0, 0), (7, 1), (8, 2), (9, 3)]          # (frame, window-relative t)
 
@@ -585,3 +602,7 @@ def test_sink_window_attention_brute_force():
             e = [np.exp(s - m) for s in scores]
             ref = sum(ei * v for ei, v in zip(e, values)) / sum(e)
             np.testing.assert_allclose(got[i, h], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_sink_window_attention_brute_force():
+    check_sink_attention_brute_force(O)
