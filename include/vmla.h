@@ -228,10 +228,12 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
                                  void* x_dev, void* q_dev, void* out_dev, int64_t first_frame, int n_frames,
                                  vmla_design design, void* stream);
 
-/* Host-side view of the window of `layer` after `frames_appended` frames: for each
- * window frame, oldest first, its absolute index, ring slot (frame mod W) and
- * window-relative index t.  `capacity` is the length of the three arrays; *n gets
- * the number of window frames. */
+/* Host-side view of the window after `frames_appended` frames (the same for every layer): for
+ * each window frame -- the sink frames, then the local frames oldest first -- its absolute index,
+ * its ring slot (frame mod W without a sink) and the window-relative index t the kernels give its
+ * keys (computed from the slot, as the window-RoPE kernel does).  `capacity` is the length of the
+ * three arrays (any may be NULL); *n gets the number of window frames; VMLA_ERR_INVALID_ARG when
+ * capacity < *n. */
 vmla_status vmla_window(const vmla_handle* h, int64_t frames_appended, int32_t* frame, int32_t* slot,
                         int32_t* t_local, int capacity, int* n);
 

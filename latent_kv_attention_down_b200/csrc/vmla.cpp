@@ -449,9 +449,11 @@ vmla_status vmla_window(const vmla_handle* h, int64_t F, int32_t* frame, int32_t
   if (count > capacity) return VMLA_ERR_INVALID_ARG;
   for (int k = 0; k < count; ++k) {  // sink frames, then local frames oldest first
     const int64_t f = k < sink ? k : w.local_start + (k - sink);
+    const int sl = (int)ring_frame_slot(g, f);
     if (frame) frame[k] = (int32_t)f;
-    if (slot) slot[k] = (int32_t)ring_frame_slot(g, f);
-    if (t_local) t_local[k] = (int32_t)(k < sink ? f : f - w.t_origin);
+    if (slot) slot[k] = (int32_t)sl;
+    // t from the slot, by the same function the window-RoPE kernel applies to every key it rotates
+    if (t_local) t_local[k] = (int32_t)ring_slot_t(g, sl, w.start_slot);
   }
   return VMLA_OK;
 }

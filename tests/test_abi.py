@@ -257,20 +257,22 @@ def test_latent_widths_with_kernels(d_latent, status):
     assert api.lib().vmla_config_check(ctypes.byref(c)) == status
 
 
-def test_sink_window_matches_the_oracle_rule():
-    """vmla_window with one sink frame and a six-frame local part (7-frame ring):
-    frames, ring slots and window-relative t as the oracle's sink rule gives them."""
+@pytest.mark.parametrize("W,S,chunk", [(7, 1, 3), (7, 1, 1), (5, 2, 3), (21, 0, 3), (4, 1, 1), (9, 3, 2)])
+def test_sink_window_matches_the_oracle_rule(W, S, chunk):
+    """vmla_window over a 200-frame rollout: frames, ring slots and window-relative t as the oracle's
+    sink rule gives them.  The t comes from the slot through the function the window-RoPE kernel
+    applies to every key, so this pins the kernels' slot -> t mapping bit for bit."""
     import oracle.vmla_oracle as O
     c = default_config()
-    c.window_frames, c.sink_frames = 7, 1
+    c.window_frames, c.sink_frames, c.chunk_frames = W, S, chunk
     assert api.lib().vmla_config_check(ctypes.byref(c)) == 0
     h = api.LatentKVAttention(c)
-    for F in range(1, 40):
+    for F in range(1, 200):
         frames, slots, ts = h.window(F)
-        want = O.window_frames_list(F, 7, 1)
-        t = O.window_frame_t(F, 7, 1)
+        want = O.window_frames_list(F, W, S)
+        t = O.window_frame_t(F, W, S)
         assert list(frames) == want
-        assert list(slots) == [O.ring_slot(f, 7, 1) for f in want]
+        assert list(slots) == [O.ring_slot(f, W, S) for f in want]
         assert list(ts) == [t[f] for f in want]
     h.close()
 
