@@ -27,6 +27,7 @@ ABI_VERSION = 2  # VMLA_ABI_VERSION of include/vmla.h that this binding's struct
 
 
 class Config(ctypes.Structure):
+    """vmla_config of include/vmla.h, field for field."""
     _fields_ = [("d_model", c_int), ("n_heads", c_int), ("d_nope", c_int), ("d_rope", c_int),
                 ("d_latent", c_int), ("d_value", c_int), ("rope_pairs", c_int * 3), ("rope_base_dims", c_int * 3),
                 ("rope_theta", c_float), ("grid_h", c_int), ("grid_w", c_int), ("window_frames", c_int),
@@ -35,6 +36,7 @@ class Config(ctypes.Structure):
 
 
 class VmlaError(RuntimeError):
+    """A vmla_status other than VMLA_OK, with its name (and the CUDA error behind VMLA_ERR_CUDA)."""
     def __init__(self, status: int, what: str):
         self.status = status
         msg = f"{what}: {lib().vmla_status_string(status).decode()}"
@@ -108,6 +110,7 @@ def lib() -> ctypes.CDLL:
 
 
 def check(status: int, what: str) -> None:
+    """Raise VmlaError unless `status` is VMLA_OK."""
     if status != 0:
         raise VmlaError(status, what)
 
@@ -131,6 +134,7 @@ def config_from_dims(dims, layers: int = 1, rope_mode: int = ROPE_AT_READ) -> Co
 
 
 def cache_bytes(cfg: Config):
+    """vmla_cache_bytes: (latent cache, positional keys, dense per-head cache) bytes of a handle."""
     a, b, d = c_size_t(), c_size_t(), c_size_t()
     check(lib().vmla_cache_bytes(ctypes.byref(cfg), ctypes.byref(a), ctypes.byref(b), ctypes.byref(d)),
           "vmla_cache_bytes")
@@ -138,12 +142,14 @@ def cache_bytes(cfg: Config):
 
 
 def workspace_bytes(cfg: Config, design: int = DESIGN_AUTO) -> int:
+    """vmla_workspace_bytes: device workspace a handle needs for `design`."""
     n = c_size_t()
     check(lib().vmla_workspace_bytes(ctypes.byref(cfg), design, ctypes.byref(n)), "vmla_workspace_bytes")
     return n.value
 
 
 def rope_frequencies(cfg: Config):
+    """vmla_rope_frequencies: angular frequency of every rotary pair, t pairs first."""
     n = cfg.d_rope // 2
     buf = (c_float * max(n, 1))()
     check(lib().vmla_rope_frequencies(ctypes.byref(cfg), buf, max(n, 1)), "vmla_rope_frequencies")
@@ -176,6 +182,7 @@ class LatentKVAttention:
         self._keep = []
 
     def close(self):
+        """vmla_destroy (idempotent)."""
         if getattr(self, "_h", None):
             lib().vmla_destroy(self._h)
             self._h = None
@@ -202,39 +209,48 @@ class LatentKVAttention:
         return self
 
     def bind(self, ckv, kr, workspace):
+        """vmla_bind: attach caller-allocated caches and workspace (uint8 device tensors)."""
         check(lib().vmla_bind(self._h, _ptr(ckv), _ptr(kr), _ptr(workspace), workspace.numel() * workspace.element_size()),
               "vmla_bind")
         self._keep = [ckv, kr, workspace]
 
     def dense_bind(self, dense_kv):
+        """vmla_dense_bind: attach the dense per-head cache."""
         check(lib().vmla_dense_bind(self._h, _ptr(dense_kv)), "vmla_dense_bind")
         self._keep.append(dense_kv)
 
     # -------------------------------------------------------------- compute
     def append(self, layer, x, w_down, first_frame, n_frames, stream=None):
+        """vmla_cache_append: x [B][n_frames*T_f][d_model], w_down [d_c + d_rope][d_model]."""
         check(lib().vmla_cache_append(self._h, layer, _ptr(x), _ptr(w_down), first_frame, n_frames, _stream(stream)),
               "vmla_cache_append")
 
     def attention(self, layer, q, w_uk, w_uv, out, first_frame, n_frames, design=DESIGN_AUTO, stream=None):
+        """vmla_chunk_attention: q [B][rows][n_h][d_head], w_uk [n_h][d_nope][d_c], w_uv [n_h][d_head][d_c], out fp32 [B][rows][n_h*d_head]."""
         check(lib().vmla_chunk_attention(self._h, layer, _ptr(q), _ptr(w_uk), _ptr(w_uv), _ptr(out), first_frame,
                                          n_frames, design, _stream(stream)), "vmla_chunk_attention")
 
     def dense_append(self, layer, x, w_down, w_uk, w_uv, first_frame, n_frames, stream=None):
+        """vmla_dense_cache_append: per-head K/V of the chunk into the dense cache."""
         check(lib().vmla_dense_cache_append(self._h, layer, _ptr(x), _ptr(w_down), _ptr(w_uk), _ptr(w_uv),
                                             first_frame, n_frames, _stream(stream)), "vmla_dense_cache_append")
 
     def dense_attention(self, layer, q, out, first_frame, n_frames, stream=None):
+        """vmla_dense_chunk_attention: d_head attention over the dense per-head cache."""
         check(lib().vmla_dense_chunk_attention(self._h, layer, _ptr(q), _ptr(out), first_frame, n_frames,
                                                _stream(stream)), "vmla_dense_chunk_attention")
 
     def step_host(self, layer, x_host, q_host, out_host, w_down, w_uk, w_uv, x_dev, q_dev, out_dev, first_frame,
                   n_frames, design=DESIGN_AUTO, stream=None):
+        """vmla_chunk_step_host: append + attention from pinned host x, q into pinned host out, through
+        the caller's device staging buffers; out_host is complete once `stream` reaches this call."""
         check(lib().vmla_chunk_step_host(self._h, layer, _ptr(x_host), _ptr(q_host), _ptr(out_host), _ptr(w_down),
                                          _ptr(w_uk), _ptr(w_uv), _ptr(x_dev), _ptr(q_dev), _ptr(out_dev),
                                          first_frame, n_frames, design, _stream(stream)), "vmla_chunk_step_host")
 
     # -------------------------------------------------------------- bookkeeping
     def window(self, frames_appended: int):
+        """vmla_window: (frames, ring slots, window-relative t) of the window, sink frames first."""
         cap = self.cfg.window_frames
         f, s, t = (ctypes.c_int32 * cap)(), (ctypes.c_int32 * cap)(), (ctypes.c_int32 * cap)()
         n = c_int()
@@ -242,11 +258,13 @@ class LatentKVAttention:
         return list(f)[:n.value], list(s)[:n.value], list(t)[:n.value]
 
     def state_get(self, layer: int) -> int:
+        """vmla_state_get: frames appended so far to `layer` (resume point)."""
         v = c_int64()
         check(lib().vmla_state_get(self._h, layer, ctypes.byref(v)), "vmla_state_get")
         return v.value
 
     def state_set(self, layer: int, frames_appended: int):
+        """vmla_state_set: resume `layer` at `frames_appended`."""
         check(lib().vmla_state_set(self._h, layer, frames_appended), "vmla_state_set")
 
     def device_status(self, stream=None):
@@ -282,9 +300,11 @@ class LatentKVAttention:
         check(lib().vmla_set_append_tiling(self._h, n_split, max_ctas), "vmla_set_append_tiling")
 
     def profile(self, enable: bool = True):
+        """vmla_profile_enable: CUDA-event timing of every stage of the following calls."""
         check(lib().vmla_profile_enable(self._h, int(enable)), "vmla_profile_enable")
 
     def profile_read(self, stage) -> tuple:
+        """vmla_profile_read: (summed milliseconds, launches) of a stage, by name or number."""
         st = STAGES[stage] if isinstance(stage, str) else stage
         ms, n = c_double(), c_int()
         check(lib().vmla_profile_read(self._h, st, ctypes.byref(ms), ctypes.byref(n)), "vmla_profile_read")
@@ -297,4 +317,5 @@ def selftest_exp2(x, y, stream=None):
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None):
+    """vmla_selftest_wait_timeout: a kernel waiting on a flag nothing sets must give up and report."""
     check(lib().vmla_selftest_wait_timeout(limit_ns, _stream(stream)), "vmla_selftest_wait_timeout")
