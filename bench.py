@@ -373,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
                     if long_run else "burst (timed region under half a second)"),
                 "frac_of_burst": achieved / tc_burst, "frac_of_sustained": achieved / tc_sust,
                 "traffic": profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"),
-                "kernel": "attn_tc_kernel<192,false>", "launch_ms": at_launch_ms,
+                "kernel": "attn_tc_kernel<192,false,false,32>", "launch_ms": at_launch_ms,
                 "algorithmic_flops_per_launch": F["attention"]}
     kernels = {}
     for k, (ms_k, n_k) in per_kernel.items():
