@@ -247,10 +247,15 @@ def run_ours(args, rank, world, local_rank):
     st, flags = m.device_status()
     assert st == 0, f"device status {st} flags {flags:#x}"
 
-    def step(i):
-        l = i % L
-        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
-        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_ABSORBED)
+    def step_with(design):
+        def step(i):
+            l = i % L
+            m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+            m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, design)
+        return step
+
+    # the headline step: the design the library's AUTO takes at this window (reconstruct-once)
+    step = step_with(api.DESIGN_AUTO)
 
     def barrier():
         if dist is not None:
@@ -276,20 +281,40 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         return s0.elapsed_time(s1)
 
+    def kernel_ms(names):
+        """Per-launch milliseconds of each profiled stage (CUDA events around each launch)."""
+        out = {}
+        for k in names:
+            tot, n = m.profile_read(k)
+            out[k] = {"ms_per_launch": tot / max(n, 1), "launches": n}
+        return out
+
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     clocks = ClockSampler(visible.split(",")[local_rank] if visible else local_rank)
     clocks.start()
     time.sleep(0.3)
-    ms = timed(step, args.steps, args.warmup, profile=True)
+    ms = timed(step, args.steps, args.warmup)  # bare: no per-stage events inside the timed loop
     clk = clocks.stop()
-    per_kernel = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "attention")}
-    m.profile(False)
     st, flags = m.device_status()
     assert st == 0, f"device status {st} flags {flags:#x}"
     ms_step = max_over_ranks(ms / args.steps)
     F = step_flops()
     value = replica_throughput(F["total"], ms_step, world) / 1e12
     tokens = replica_throughput(d.n_queries, ms_step, world)
+    # the per-kernel breakdown of the same step, from a second pass with CUDA events around each launch
+    timed(step, args.steps, 3, profile=True)
+    per_kernel = kernel_ms(("append", "rope", "q_absorb", "reconstruct_once", "dense_attention", "attention"))
+    m.profile(False)
+    auto_design = "recon_once" if per_kernel["dense_attention"]["launches"] else "absorbed"
+    per_kernel = {k: v for k, v in per_kernel.items() if v["launches"]}
+    launches_per_step = sum(v["launches"] for v in per_kernel.values()) / args.steps
+
+    # the absorbed design's step and kernel, timed the same way (bare, then profiled)
+    asteps = max(10, args.steps)
+    ms_abs = max_over_ranks(timed(step_with(api.DESIGN_ABSORBED), asteps, 3) / asteps)
+    timed(step_with(api.DESIGN_ABSORBED), asteps, 3, profile=True)
+    abs_kernels = kernel_ms(("append", "rope", "q_absorb", "attention"))
+    m.profile(False)
 
     # ------------------------------------------------ end to end from pinned host memory
     xh = [xs[l].cpu().pin_memory() for l in range(2)]
@@ -300,7 +325,7 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step(i):
         l = i % 2
         m.step_host(l, xh[l], qh[l], oh[l], W[l][0], W[l][1], W[l][2], xd, qd, od, first, d.chunk_frames,
-                    api.DESIGN_ABSORBED)
+                    api.DESIGN_AUTO)
 
     e2e_steps = max(10, args.steps // 4)
     ms_e2e = max_over_ranks(timed(e2e_step, e2e_steps, 3) / e2e_steps)
@@ -325,84 +350,85 @@ def run_ours(args, rank, world, local_rank):
                  "attention_tflops": DF["attention"] / (da_ms / max(da_n, 1) * 1e-3) / 1e12,
                  "cache_scalars_per_token": 2 * d.n_heads * d.d_head, "window_read_bytes": d.window_tokens * 2 * d.n_heads * d.d_head * 2}
 
-    # ------------------------------------------------ design (b'): per-head K/V rebuilt once per call
-    def recon_step(i):
-        l = i % L
-        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
-        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_RECON_ONCE)
-    rsteps = max(10, args.steps // 4)
-    ms_r = timed(recon_step, rsteps, 3, profile=True)
-    rk = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "reconstruct_once", "dense_attention")}
-    m.profile(False)
-    DF = dense_flops()
-    ra_ms = rk["dense_attention"][0] / max(rk["dense_attention"][1], 1)
-    recon_once = {"ms_per_step": max_over_ranks(ms_r / rsteps),
-                  "tflops_effective": world * F["total"] / (max_over_ranks(ms_r / rsteps) * 1e-3) / 1e12,
-                  "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in rk.items()},
-                  "attention_tflops_issued": DF["attention"] / (ra_ms * 1e-3) / 1e12}
-
     # ------------------------------------------------ design (b): per-head K/V rebuilt inside every key tile
-    def rt_step(i):
-        l = i % L
-        m.append(l, xs[l], W[l][0], first, d.chunk_frames)
-        m.attention(l, qs[l], W[l][1], W[l][2], outs[l], first, d.chunk_frames, api.DESIGN_RECONSTRUCT)
+    DF = dense_flops()
     tsteps = max(10, args.steps // 4)
-    ms_t = timed(rt_step, tsteps, 3, profile=True)
-    tk = {k: m.profile_read(k) for k in ("append", "rope", "q_absorb", "attention_reconstruct")}
+    ms_t = max_over_ranks(timed(step_with(api.DESIGN_RECONSTRUCT), tsteps, 3) / tsteps)
+    timed(step_with(api.DESIGN_RECONSTRUCT), tsteps, 3, profile=True)
+    tk = kernel_ms(("append", "rope", "q_absorb", "attention_reconstruct"))
     m.profile(False)
-    ms_t = max_over_ranks(ms_t / tsteps)
-    rt_attn_ms = tk["attention_reconstruct"][0] / max(tk["attention_reconstruct"][1], 1)
+    rt_attn_ms = tk["attention_reconstruct"]["ms_per_launch"]
     recon_in_tile = {"ms_per_step": ms_t, "tflops_effective": world * F["total"] / (ms_t * 1e-3) / 1e12,
-                     "kernels_ms": {k: v[0] / max(v[1], 1) for k, v in tk.items()},
+                     "kernels_ms": {k: v["ms_per_launch"] for k, v in tk.items()},
                      "attention_tflops_issued": (DF["attention"] + 2 * d.window_tokens * d.d_latent * 224 *
                                                  d.n_heads * ((d.n_queries + 127) // 128)) / (rt_attn_ms * 1e-3) / 1e12}
 
     # ------------------------------------------------ roofline of the dominant kernel (attention)
     hbm, tc_burst, tc_sust, src = load_peaks()
-    at_ms, at_n = per_kernel["attention"]
-    at_launch_ms = at_ms / max(at_n, 1)
-    achieved = F["attention"] / (at_launch_ms * 1e-3) / 1e12
     # the kernel runs inside a timed loop of args.steps chunk steps: past half a second of continuous
     # load the GPU sits at its power cap, so the sustained figure is the matching denominator
     long_run = ms_step * args.steps >= 500.0
     peak = tc_sust if long_run else tc_burst
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "peak_source": f"{src} bf16 dense, cuBLAS, " + (
-                    f"sustained (the kernel runs inside {ms_step * args.steps / 1e3:.1f} s of continuous load)"
-                    if long_run else "burst (timed region under half a second)"),
-                "frac_of_burst": achieved / tc_burst, "frac_of_sustained": achieved / tc_sust,
-                "traffic": profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"),
-                "kernel": "attn_tc_kernel<192,false,false,32>", "launch_ms": at_launch_ms,
-                "algorithmic_flops_per_launch": F["attention"]}
-    kernels = {}
-    for k, (ms_k, n_k) in per_kernel.items():
-        kernels[k] = {"ms_per_launch": ms_k / max(n_k, 1), "launches": n_k}
+    peak_source = f"{src} bf16 dense, cuBLAS, " + (
+        f"sustained (the kernel runs inside {ms_step * args.steps / 1e3:.1f} s of continuous load)"
+        if long_run else "burst (timed region under half a second)")
+
+    def tensor_roofline(kernel, launch_ms, flops, traffic):
+        achieved = flops / (launch_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": peak_source, "frac_of_burst": achieved / tc_burst,
+                "frac_of_sustained": achieved / tc_sust, "traffic": traffic, "kernel": kernel,
+                "launch_ms": launch_ms, "algorithmic_flops_per_launch": flops}
+
+    if auto_design == "recon_once":
+        # d_head = 128 attention over the window's per-head K/V: 2 * N_q * N_k * n_h * (128 + 128) FLOPs
+        roofline = tensor_roofline("attn_tc_kernel<128,true,false,32>", per_kernel["dense_attention"]["ms_per_launch"],
+                                   DF["attention"], profiled_traffic("attn_tc.cu", "attn_per_head_wan_layer.md"))
+    else:
+        roofline = tensor_roofline("attn_tc_kernel<192,false,false,32>", per_kernel["attention"]["ms_per_launch"],
+                                   F["attention"], profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"))
+    absorbed_roofline = tensor_roofline("attn_tc_kernel<192,false,false,32>", abs_kernels["attention"]["ms_per_launch"],
+                                        F["attention"], profiled_traffic("attn_tc.cu", "attn_absorbed_wan_layer.md"))
+    kernels = dict(per_kernel)
+    for k, v in abs_kernels.items():
+        kernels.setdefault(k, v)
     # HBM-bound kernels: algorithmic bytes per launch
     nq, nk = d.n_queries, d.window_tokens
     alg_bytes = {"append": nq * d.d_model * 2 + (d.d_latent + d.d_rope) * d.d_model * 2 + nq * (d.d_latent + d.d_rope) * 2,
                  "rope": 2 * nk * d.d_rope * 2,
                  "q_absorb": nq * d.n_heads * d.d_head * 2 + d.n_heads * d.d_nope * d.d_latent * 2 +
-                 nq * d.n_heads * (d.d_latent + d.d_rope) * 2}
+                 nq * d.n_heads * (d.d_latent + d.d_rope) * 2,
+                 # per-head K/V of the window: latents and rotated keys in, 2 * n_h * 128 scalars per key out
+                 "reconstruct_once": nk * (d.d_latent + d.d_rope) * 2 + nk * 2 * d.n_heads * d.d_head * 2}
     for k, b in alg_bytes.items():
+        if k not in kernels:
+            continue
         kernels[k]["algorithmic_bytes"] = b
         kernels[k]["gbs"] = b / (kernels[k]["ms_per_launch"] * 1e-3) / 1e9
         kernels[k]["frac_of_hbm"] = kernels[k]["gbs"] / hbm
     add_copy_reference(kernels, dev)
 
+    workload = ("wan1.3b-layer chunk step: append 3 frames + window rope + attention with the design AUTO takes "
+                f"({auto_design.replace('_', '-')}"
+                + (": per-head K/V of the window rebuilt once, d_head=128 attention" if auto_design == "recon_once"
+                   else ": absorbed, fused W_uv") + "); N_q=4680, N_k=32760, n_h=12, d_c=192, d_rope=32, batch 1")
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "wan1.3b-layer chunk step: append 3 frames + rope + q-absorb + absorbed attention "
-                                   "with fused W_uv; N_q=4680, N_k=32760, n_h=12, d_c=192, d_rope=32, batch 1",
+            "config": {"workload": workload, "design": auto_design,
                        "global_batch": world, "seq_len": nk, "parallelism": f"replicas x{world}",
-                       "l2": f"inputs larger than L2: {L} layer buffer sets cycled"},
+                       "l2": f"inputs larger than L2: {L} layer buffer sets cycled",
+                       "flops": "effective: 2*N_q*N_k*n_h*(2*d_c + d_rope) + append + q-absorb + W_uv per step, "
+                                "the same numerator for every design"},
             "query_tokens_per_s": tokens, "roofline": roofline, "kernels": kernels,
             "e2e": {"value": world * F["total"] / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "vmla_chunk_step_host (pinned host x, q -> device, append, attention, out -> host)"},
-            "gpu_launches": 4 * args.steps, "clocks": clk}
-    line["designs"] = {"absorbed_ms_per_step": ms_step, "recon_once": recon_once,
+                    "api": "vmla_chunk_step_host (pinned host x, q -> device, append, attention, out -> host), AUTO"},
+            "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk}
+    line["designs"] = {"auto": auto_design,
+                       "absorbed": {"ms_per_step": ms_abs, "tflops_effective": world * F["total"] / (ms_abs * 1e-3) / 1e12,
+                                    "kernels_ms": {k: v["ms_per_launch"] for k, v in abs_kernels.items()},
+                                    "roofline": absorbed_roofline},
                        "reconstruct_in_tile": recon_in_tile}
     if args.legs:
         line["legs"] = {"batch8": batch8_leg(m_timed=timed, dev=dev, hbm=hbm, tc=tc_burst, seed=seed),

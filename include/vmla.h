@@ -61,9 +61,13 @@ typedef enum vmla_dtype { VMLA_BF16 = 0, VMLA_FP32 = 1 } vmla_dtype;
 
 /* How vmla_chunk_attention evaluates the same scores and outputs. */
 typedef enum vmla_design {
-  VMLA_DESIGN_AUTO = 0,        /* VMLA_BF16: ABSORBED for d_latent <= 192, RECON_ONCE from 256 on, and
-                                  ABSORBED whenever d_rope != 32; VMLA_FP32 always evaluates the
-                                  absorbed form */
+  VMLA_DESIGN_AUTO = 0,        /* the design measured fastest that meets the accuracy gate for the call:
+                                  VMLA_BF16: RECON_ONCE past 256 latent dims, and at 192 or 256 latent
+                                  dims when the window holds at least 4096 keys; ABSORBED otherwise,
+                                  and whenever d_rope != 32.  VMLA_FP32 always evaluates the absorbed
+                                  form.  vmla_workspace_bytes(AUTO) covers the RECON_ONCE workspace
+                                  whenever the configuration's full window would take it; with a
+                                  smaller workspace bound, AUTO stays ABSORBED up to 256 latent dims */
   VMLA_DESIGN_ABSORBED = 1,    /* W_uk folded into the query, MQA over [c_KV | k_R], W_uv after the
                                   softmax-weighted sum [paperlayer App. E] */
   VMLA_DESIGN_RECONSTRUCT = 2, /* per KV tile, per-head K/V rebuilt from c_KV on the tensor core and kept
@@ -155,6 +159,19 @@ vmla_status vmla_cache_bytes(const vmla_config* cfg, size_t* ckv_bytes, size_t* 
  * (and for the dense calls, whatever design). */
 vmla_status vmla_workspace_bytes(const vmla_config* cfg, vmla_design design, size_t* bytes);
 
+/* Where the intermediates of a chunk attention call live inside the workspace, as byte offsets
+ * (for inspection and stage-by-stage checks; the workspace's contents after a call are those of
+ * the last call that wrote them):
+ *   [VMLA_WS_KR_ROT]  the window's positional keys rotated with window-relative t
+ *                     [batch][W*T_f][d_rope] (RoPE at read only; ring-slot order)
+ *   [VMLA_WS_QT]      absorbed queries [batch][n_heads][n_q][d_latent + d_rope] (ABSORBED)
+ *   [VMLA_WS_QD]      per-head queries with the positional part rotated [batch][n_heads][n_q][d_nope + d_rope]
+ *                     (RECONSTRUCT, RECON_ONCE and the dense calls)
+ *   [VMLA_WS_RECON]   the window's per-head keys and values [batch][W*T_f][2][n_heads][d_value] (RECON_ONCE)
+ * n_q = chunk_frames * T_f; dtype-sized elements.  `n` >= VMLA_WS_COUNT. */
+enum { VMLA_WS_KR_ROT = 0, VMLA_WS_QT = 1, VMLA_WS_QD = 2, VMLA_WS_RECON = 3, VMLA_WS_COUNT = 4 };
+vmla_status vmla_workspace_offsets(const vmla_config* cfg, size_t* offsets, int n);
+
 /* The angular frequency of each rotary pair, t pairs first, then h, then w
  * (w_{a,i} = theta^(-2i/B_a), i = 0..pairs_a-1 [paperlayer App. D.3]), as float. n >= pair count. */
 vmla_status vmla_rope_frequencies(const vmla_config* cfg, float* freqs, int n);
@@ -230,8 +247,10 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
 
 /* Host-side view of the window after `frames_appended` frames (the same for every layer): for
  * each window frame -- the sink frames, then the local frames oldest first -- its absolute index,
- * its ring slot (frame mod W without a sink) and the window-relative index t the kernels give its
- * keys (computed from the slot, as the window-RoPE kernel does).  `capacity` is the length of the
+ * its ring slot (frame mod W without a sink) and the frame index t its keys are rotated with:
+ * with VMLA_ROPE_AT_READ the window-relative t (computed from the slot, as the window-RoPE kernel
+ * does), with VMLA_ROPE_AT_APPEND the absolute frame index (the append rotated the keys with it).
+ * `capacity` is the length of the
  * three arrays (any may be NULL); *n gets the number of window frames; VMLA_ERR_INVALID_ARG when
  * capacity < *n. */
 vmla_status vmla_window(const vmla_handle* h, int64_t frames_appended, int32_t* frame, int32_t* slot,

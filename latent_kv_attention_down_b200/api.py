@@ -55,6 +55,7 @@ _SIGS = {
                                  ctypes.POINTER(c_size_t)]),
     "vmla_workspace_bytes": (c_int, [ctypes.POINTER(Config), c_int, ctypes.POINTER(c_size_t)]),
     "vmla_rope_frequencies": (c_int, [ctypes.POINTER(Config), ctypes.POINTER(c_float), c_int]),
+    "vmla_workspace_offsets": (c_int, [ctypes.POINTER(Config), ctypes.POINTER(c_size_t), c_int]),
     "vmla_create": (c_int, [ctypes.POINTER(Config), ctypes.POINTER(c_void_p)]),
     "vmla_destroy": (c_int, [c_void_p]),
     "vmla_bind": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_size_t]),
@@ -146,6 +147,17 @@ def workspace_bytes(cfg: Config, design: int = DESIGN_AUTO) -> int:
     n = c_size_t()
     check(lib().vmla_workspace_bytes(ctypes.byref(cfg), design, ctypes.byref(n)), "vmla_workspace_bytes")
     return n.value
+
+
+WS_KR_ROT, WS_QT, WS_QD, WS_RECON = 0, 1, 2, 3
+
+
+def workspace_offsets(cfg: Config):
+    """vmla_workspace_offsets: byte offsets of the rotated window keys, absorbed queries, per-head
+    queries and per-head K/V inside the workspace (indexed by WS_*)."""
+    buf = (c_size_t * 4)()
+    check(lib().vmla_workspace_offsets(ctypes.byref(cfg), buf, 4), "vmla_workspace_offsets")
+    return list(buf)
 
 
 def rope_frequencies(cfg: Config):

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "vmla.h"
+
 namespace vmla {
 
 constexpr int kMaxPairs = 64;  // rotary pairs (d_rope up to 128)
@@ -268,5 +270,27 @@ unsigned* device_error_word();  // address of the library's device status word (
 cudaError_t launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s);
 // y[i] = the attention kernels' polynomial 2^x[i] (exp2_poly2), n even, 8-byte aligned arrays.
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t s);
+
+// ------------------------------------------------------------------ host helpers (vmla.cpp), shared by
+// the entry points of every host file
+Rope make_rope(const vmla_config& c);  // pair frequencies theta^(-2i/B_a), t pairs first
+Ring make_ring(const vmla_config& c);
+
+// The active context after F frames [paperlayer App. D.4, D.5]: ring slots [0, n_keys / T_f);
+// a local frame f has window-relative t = f - t_origin, a sink frame t = f.
+struct Window {
+  int64_t t_origin;
+  int64_t local_start;  // oldest local frame
+  int n_keys;
+  int start_slot;       // ring slot of the oldest local frame, minus sink_frames
+};
+Window window_of(const vmla_config& c, int64_t F);
+
+// 3D TMA tensor map: dims (d0 innermost, d1, d2), byte strides s1, s2, box (b0, b1, 1); false when the
+// driver refuses it (or its encoder entry point is missing).
+bool map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+          uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+bool map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
+          CUtensorMapSwizzle sw);
 
 }  // namespace vmla

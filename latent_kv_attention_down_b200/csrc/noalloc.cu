@@ -8,6 +8,8 @@
 // not use the variable's name as a device address, so the first call on each
 // device (with that device current) looks its address up with
 // cudaGetSymbolAddress and keeps it; kernels get that pointer as an argument.
+// The library's device status word is looked up the same way, once per device
+// (device_error_word), so a later call makes no symbol lookup at all.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -44,29 +46,6 @@ vmla_status scratch_address(void** out) {
   return VMLA_OK;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool tile_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
-              uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw, CUtensorMapDataType dt) {
-  static EncodeTiledFn encode = [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeTiledFn>(nullptr);
-    return reinterpret_cast<EncodeTiledFn>(fn);
-  }();
-  if (!encode) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {s1, s2};
-  cuuint32_t box[3] = {b0, b1, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -94,11 +73,8 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   const int64_t T = (int64_t)c.grid_h * c.grid_w;
   const int64_t rr = (int64_t)c.window_frames * T;
   // active context [paperlayer App. D.4, D.5]: sink frames, then the newest W - S frames
-  const int64_t S = c.sink_frames, L = c.window_frames - c.sink_frames;
-  const bool full = F > c.window_frames;
-  const int64_t t_origin = full ? F - L - S : 0;
-  const int start_slot = full ? (int)((F - L - S) % L) : 0;
-  const int n_keys = (int)((full ? c.window_frames : F) * T);
+  const Window win = window_of(c, F);
+  const int n_keys = win.n_keys;
   const int nq = (int)(n_frames * T);
   const int dqk = c.d_latent + 32;
   const size_t kr_rot_bytes = at_read ? align256((size_t)c.batch * rr * 32 * 2) : 0;
@@ -111,16 +87,8 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   if (!err) return VMLA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  Rope rope{};
-  int p = 0;
-  for (int a = 0; a < 3; ++a) {
-    const double base = c.rope_base_dims[a] > 0 ? c.rope_base_dims[a] : 2.0 * c.rope_pairs[a];
-    for (int i = 0; i < c.rope_pairs[a]; ++i) rope.freq[p++] = (float)std::pow((double)c.rope_theta, -2.0 * i / base);
-  }
-  rope.n_t = c.rope_pairs[0];
-  rope.n_h = c.rope_pairs[1];
-  rope.n_w = c.rope_pairs[2];
-  const Ring ring{(int)T, c.grid_w, c.window_frames, c.sink_frames};
+  const Rope rope = make_rope(c);
+  const Ring ring = make_ring(c);
 
   const size_t layer_rows = (size_t)layer * c.batch * rr;
   const __nv_bfloat16* ckv_layer = static_cast<const __nv_bfloat16*>(ckv) + layer_rows * c.d_latent;
@@ -130,19 +98,18 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
 
   const __nv_bfloat16* kpos = kr_layer;
   if (at_read) {
-    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, 32, start_slot, ring, rope};
+    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, 32, win.start_slot, ring, rope};
     if (launch_rope_window_bf16(r, s) != cudaSuccess) return VMLA_ERR_CUDA;
     kpos = kr_rot;
   }
   const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
-  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tuk, tqt;
-  if (!tile_map(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 256, (uint64_t)nq * c.n_heads * 256,
-                64, 128, SW128, BF) ||
-      !tile_map(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
-                SW128, BF) ||
-      !tile_map(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
-                SW128, BF))
+  if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 256, (uint64_t)nq * c.n_heads * 256,
+                64, 128, SW128) ||
+      !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+                SW128) ||
+      !map3(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
+                SW128))
     return VMLA_ERR_CUDA;
   QPrepTc qa;
   qa.q = static_cast<const __nv_bfloat16*>(q);
@@ -151,7 +118,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   qa.n_heads = c.n_heads;
   qa.d_latent = c.d_latent;
   qa.d_rope = c.d_rope;
-  qa.t_first = first_frame - (at_read ? t_origin : 0);
+  qa.t_first = first_frame - (at_read ? win.t_origin : 0);
   qa.ring = ring;
   qa.rope = rope;
   qa.err = err;
@@ -161,14 +128,14 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   const int bn = attn_absorbed_block_n(c.d_latent);
   const uint64_t bh = (uint64_t)c.batch * c.n_heads;
   CUtensorMap mq, mqr, mk, mkr, muv, mo;
-  if (!tile_map(&mq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, SW128, BF) ||
-      !tile_map(&mqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, SW64, BF) ||
-      !tile_map(&mk, ckv_layer, c.d_latent, n_keys, c.batch, (uint64_t)c.d_latent * 2, (uint64_t)rr * c.d_latent * 2,
-                64, bn, SW128, BF) ||
-      !tile_map(&mkr, kpos, 32, n_keys, c.batch, 64, (uint64_t)rr * 64, 32, bn, SW64, BF) ||
-      !tile_map(&muv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
-                SW128, BF) ||
-      !tile_map(&mo, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 512,
+  if (!map3(&mq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, SW128) ||
+      !map3(&mqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, SW64) ||
+      !map3(&mk, ckv_layer, c.d_latent, n_keys, c.batch, (uint64_t)c.d_latent * 2, (uint64_t)rr * c.d_latent * 2,
+                64, bn, SW128) ||
+      !map3(&mkr, kpos, 32, n_keys, c.batch, 64, (uint64_t)rr * 64, 32, bn, SW64) ||
+      !map3(&muv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
+                SW128) ||
+      !map3(&mo, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 512,
                 (uint64_t)nq * c.n_heads * 512, 32, 128, SW128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
     return VMLA_ERR_CUDA;
   AttnTc a;

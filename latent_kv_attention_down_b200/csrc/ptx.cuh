@@ -379,7 +379,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // per SM, the softmax bottleneck) to the other elements.  Range reduction
 // y = n + f with n = round(y), taken from the low bits of y + 1.5*2^23, and f in
 // [-1/2, 1/2]; 2^f by the degree-3 polynomial of least maximum relative error on
-// that interval (Remez exchange, see exp2_fit.py: relative error <= 7.5e-5, far
+// that interval (Remez exchange, re-derived by tests/test_exp2_fit.py: relative error <= 7.5e-5, far
 // below the bf16 rounding of P); 2^n is added to the exponent field as an
 // integer.  y is clamped below at -125, where the result is already negligible
 // for a softmax whose largest term is 1.

@@ -1,4 +1,6 @@
 // The library's device status word and the self-test of the bounded waits.
+#include <mutex>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -6,10 +8,24 @@ namespace vmla {
 
 __device__ unsigned g_device_error;
 
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+unsigned* g_err_word[kMaxDevices] = {};
+}  // namespace
+
+// Looked up with cudaGetSymbolAddress the first time per device, with that device current, and
+// kept: later calls (a stream capture among them) make no CUDA call here but cudaGetDevice.
 unsigned* device_error_word() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-  return static_cast<unsigned*>(p);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (!g_err_word[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_word[dev] = static_cast<unsigned*>(p);
+  }
+  return g_err_word[dev];
 }
 
 namespace {

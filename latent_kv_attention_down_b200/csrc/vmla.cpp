@@ -22,6 +22,92 @@
 
 using namespace vmla;
 
+namespace vmla {
+
+// ---------------------------------------------------------------- host helpers (declared in kernels.h)
+Rope make_rope(const vmla_config& c) {
+  Rope r;
+  std::memset(&r, 0, sizeof(r));
+  int p = 0;
+  for (int a = 0; a < 3; ++a) {
+    const double base = c.rope_base_dims[a] > 0 ? c.rope_base_dims[a] : 2.0 * c.rope_pairs[a];
+    for (int i = 0; i < c.rope_pairs[a]; ++i) r.freq[p++] = (float)std::pow((double)c.rope_theta, -2.0 * i / base);
+  }
+  r.n_t = c.rope_pairs[0];
+  r.n_h = c.rope_pairs[1];
+  r.n_w = c.rope_pairs[2];
+  return r;
+}
+
+Ring make_ring(const vmla_config& c) {
+  return Ring{(int)((int64_t)c.grid_h * c.grid_w), c.grid_w, c.window_frames, c.sink_frames};
+}
+
+// The active context after F frames [paperlayer App. D.4, D.5]: ring slots [0, n_keys / T_f);
+// a local frame f has window-relative t = f - t_origin, a sink frame t = f.
+Window window_of(const vmla_config& c, int64_t F) {
+  const int64_t S = c.sink_frames, L = c.window_frames - c.sink_frames;
+  Window w;
+  if (F <= c.window_frames) {
+    w.local_start = std::min<int64_t>(S, F);
+    w.t_origin = 0;
+    w.n_keys = (int)(F * ((int64_t)c.grid_h * c.grid_w));
+    w.start_slot = 0;
+  } else {
+    w.local_start = F - L;
+    w.t_origin = w.local_start - S;
+    w.n_keys = (int)((int64_t)c.window_frames * ((int64_t)c.grid_h * c.grid_w));
+    w.start_slot = (int)((w.local_start - S) % L);
+  }
+  return w;
+}
+
+// ---------------------------------------------------------------- TMA tensor maps
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool have_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode != nullptr;
+}
+}  // namespace
+
+// 3D map: dims (d0 innermost, d1, d2), byte strides s1, s2, box (b0, b1, 1); bf16 unless told otherwise
+bool map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+          uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw, CUtensorMapDataType dt) {
+  if (!have_encode()) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
+          CUtensorMapSwizzle sw) {
+  if (!have_encode()) return false;
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {s1};
+  cuuint32_t box[2] = {b0, b1};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace vmla
+
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any healthy pipeline wait
@@ -61,71 +147,10 @@ WsLayout ws_layout(const vmla_config& c) {
   return w;
 }
 
-Rope make_rope(const vmla_config& c) {
-  Rope r;
-  std::memset(&r, 0, sizeof(r));
-  int p = 0;
-  for (int a = 0; a < 3; ++a) {
-    const double base = c.rope_base_dims[a] > 0 ? c.rope_base_dims[a] : 2.0 * c.rope_pairs[a];
-    for (int i = 0; i < c.rope_pairs[a]; ++i) r.freq[p++] = (float)std::pow((double)c.rope_theta, -2.0 * i / base);
-  }
-  r.n_t = c.rope_pairs[0];
-  r.n_h = c.rope_pairs[1];
-  r.n_w = c.rope_pairs[2];
-  return r;
-}
-
 // A forced append column split the shape can take: one MMA covers at most 256 columns.
 bool append_tiling_fits(const vmla_config& c, int n_split) {
   if (n_split == 0) return true;
   return append_part_cols(c.d_latent + c.d_rope, n_split) <= 256;
-}
-
-Ring make_ring(const vmla_config& c) {
-  return Ring{(int)tokens_per_frame(c), c.grid_w, c.window_frames, c.sink_frames};
-}
-
-// ---------------------------------------------------------------- TMA tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiledFn g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool have_encode() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-  });
-  return g_encode != nullptr;
-}
-
-// 3D map: dims (d0 innermost, d1, d2), byte strides s1, s2, box (b0, b1, 1); bf16 unless told otherwise
-bool map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
-          uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw,
-          CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
-  if (!have_encode()) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {s1, s2};
-  cuuint32_t box[3] = {b0, b1, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-bool map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
-          CUtensorMapSwizzle sw) {
-  if (!have_encode()) return false;
-  cuuint64_t dims[2] = {d0, d1};
-  cuuint64_t strides[1] = {s1};
-  cuuint32_t box[2] = {b0, b1};
-  cuuint32_t es[2] = {1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -143,16 +168,34 @@ vmla_status map_fail() {
 }
 vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : cuda_fail(e); }
 
-// AUTO: the absorbed design up to d_latent = 192; from 256 on the per-head K/V
-// are rebuilt once per call.  At 256 the rebuilt path is the more accurate one
-// (it rounds K and V per key, where the absorbed query carries one bf16
-// rounding for every key of a row) and the absorbed MMA work (2 d_latent +
-// d_rope per key) is over twice the per-head attention's (2 d_head).
-vmla_design resolve_design(const vmla_config& c, vmla_design d) {
+// AUTO keeps the design measured fastest on one B200 that also meets the accuracy gate (relative
+// L2 <= 1e-2, max |err| <= 3e-2 RMS against the fp64 definition) for the call's window:
+//  - d_latent > 256: RECON_ONCE (the absorbed tile holds at most 256 latent columns);
+//  - d_latent 192 or 256 and a window of at least kReconOnceMinKeys keys: RECON_ONCE.  Per (query,
+//    key, head) the per-head attention multiplies 2 d_head = 256 pairs where the absorbed one
+//    multiplies 2 d_latent + d_rope (416 at 192), and rebuilding the window's per-head K/V costs
+//    about 2 us per 1000 keys (Wan-1.3B layer: 0.91 ms against 1.05 ms per call).  Per-head K and V
+//    are rounded to bf16 key by key, which over a short window can put the worst output element
+//    past the max-error gate (3.4e-2 RMS at 600 keys); from a few thousand keys on it averages out.
+//  - otherwise ABSORBED: at d_latent <= 128 its extra MMA work is no larger than the
+//    reconstruction's, and it meets the gate at every window length up to 192.
+// The 112/16 and 64/64 content/rotary splits run on the absorbed design only.
+constexpr int kReconOnceMinKeys = 4096;
+
+vmla_design resolve_design(const vmla_config& c, vmla_design d, int64_t n_keys) {
   if (d != VMLA_DESIGN_AUTO) return d;
-  if (c.dtype == VMLA_BF16 && c.d_rope != 32) return VMLA_DESIGN_ABSORBED;  // the only bf16 design there
-  if (c.dtype == VMLA_BF16 && c.d_latent >= 256) return VMLA_DESIGN_RECON_ONCE;
+  if (c.dtype != VMLA_BF16) return VMLA_DESIGN_ABSORBED;
+  if (c.d_rope != 32) return VMLA_DESIGN_ABSORBED;  // the only bf16 design there
+  if (c.d_latent > 256) return VMLA_DESIGN_RECON_ONCE;
+  if (c.d_latent >= 192 && n_keys >= kReconOnceMinKeys) return VMLA_DESIGN_RECON_ONCE;
   return VMLA_DESIGN_ABSORBED;
+}
+
+// Whether some call of this configuration may run RECON_ONCE (its workspace must hold the window's
+// per-head K/V): the design AUTO takes on the largest window, or RECON_ONCE asked for.
+bool may_run_recon_once(const vmla_config& c, vmla_design d) {
+  const int64_t max_keys = (int64_t)c.window_frames * c.grid_h * c.grid_w;
+  return resolve_design(c, d, max_keys) == VMLA_DESIGN_RECON_ONCE;
 }
 
 }  // namespace
@@ -236,32 +279,6 @@ vmla_status check_append_frames(const vmla_config& c, int64_t F, int64_t first, 
   else
     return VMLA_ERR_STATE;
   return VMLA_OK;
-}
-
-// The active context after F frames [paperlayer App. D.4, D.5]: ring slots [0, n_keys / T_f);
-// a local frame f has window-relative t = f - t_origin, a sink frame t = f.
-struct Window {
-  int64_t t_origin;
-  int64_t local_start;  // oldest local frame
-  int n_keys;
-  int start_slot;       // ring slot of the oldest local frame, minus sink_frames
-};
-
-Window window_of(const vmla_config& c, int64_t F) {
-  const int64_t S = c.sink_frames, L = c.window_frames - c.sink_frames;
-  Window w;
-  if (F <= c.window_frames) {
-    w.local_start = std::min<int64_t>(S, F);
-    w.t_origin = 0;
-    w.n_keys = (int)(F * tokens_per_frame(c));
-    w.start_slot = 0;
-  } else {
-    w.local_start = F - L;
-    w.t_origin = w.local_start - S;
-    w.n_keys = (int)((int64_t)c.window_frames * tokens_per_frame(c));
-    w.start_slot = (int)((w.local_start - S) % L);
-  }
-  return w;
 }
 
 vmla_status check_attention_frames(const vmla_config& c, int64_t F, int64_t first, int n, Window* w) {
@@ -375,7 +392,19 @@ vmla_status vmla_workspace_bytes(const vmla_config* c, vmla_design d, size_t* by
   if (st != VMLA_OK) return st;
   if (!bytes || d < VMLA_DESIGN_AUTO || d > VMLA_DESIGN_RECON_ONCE) return VMLA_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(*c);
-  *bytes = w.base_bytes + (resolve_design(*c, d) == VMLA_DESIGN_RECON_ONCE ? w.recon_bytes : 0);
+  *bytes = w.base_bytes + (may_run_recon_once(*c, d) ? w.recon_bytes : 0);
+  return VMLA_OK;
+}
+
+vmla_status vmla_workspace_offsets(const vmla_config* c, size_t* offsets, int n) {
+  vmla_status st = vmla_config_check(c);
+  if (st != VMLA_OK) return st;
+  if (!offsets || n < VMLA_WS_COUNT) return VMLA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(*c);
+  offsets[VMLA_WS_KR_ROT] = w.kr_rot;
+  offsets[VMLA_WS_QT] = w.qt;
+  offsets[VMLA_WS_QD] = w.dq;
+  offsets[VMLA_WS_RECON] = w.recon;
   return VMLA_OK;
 }
 
@@ -452,8 +481,10 @@ vmla_status vmla_window(const vmla_handle* h, int64_t F, int32_t* frame, int32_t
     const int sl = (int)ring_frame_slot(g, f);
     if (frame) frame[k] = (int32_t)f;
     if (slot) slot[k] = (int32_t)sl;
-    // t from the slot, by the same function the window-RoPE kernel applies to every key it rotates
-    if (t_local) t_local[k] = (int32_t)ring_slot_t(g, sl, w.start_slot);
+    // RoPE at read: t from the slot, by the same function the window-RoPE kernel applies to every key
+    // it rotates; RoPE at append: the keys were rotated with their absolute frame index when written
+    if (t_local)
+      t_local[k] = c.rope_mode == VMLA_ROPE_AT_APPEND ? (int32_t)f : (int32_t)ring_slot_t(g, sl, w.start_slot);
   }
   return VMLA_OK;
 }
@@ -603,8 +634,52 @@ vmla_status attention_fp32(vmla_handle* h, int layer, const void* q, const void*
   return cuda_status(e);
 }
 
+// Output rows wanted in host memory (vmla_chunk_step_host): the absorbed attention then runs as
+// one launch per group of heads that fills the GPU once, and each group's columns are copied to
+// the host on `stream` while the next group computes; `copied` tells the caller it was done.
+struct HostOut {
+  void* host;
+  cudaStream_t stream;
+  cudaEvent_t group, done;
+  bool copied;
+};
+
+// Launch an attention kernel (grid y = heads) as one launch per group of heads that fills the GPU
+// once, each group's output columns copied to the host on hout->stream while the next group
+// computes; `stream` then waits for the last copy.  `launch` enqueues heads [a.h0, a.h0 + a.h_count).
+extern "C++" template <class Launch>
+cudaError_t launch_head_groups(const vmla_config& c, int nq, AttnTc a, const void* out, HostOut* hout,
+                               cudaStream_t s, Launch launch) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  const int per_head = a.m_tiles * c.batch;  // CTAs of one head
+  const int hg = std::max(1, std::min(c.n_heads, sms / std::max(1, per_head)));
+  const size_t pitch = (size_t)c.n_heads * 128 * sizeof(float);
+  cudaError_t e = cudaSuccess;
+  for (int g0 = 0; g0 < c.n_heads && e == cudaSuccess; g0 += hg) {
+    a.h0 = g0;
+    a.h_count = std::min(hg, c.n_heads - g0);
+    if ((e = launch(a)) != cudaSuccess || (e = cudaEventRecord(hout->group, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(hout->stream, hout->group, 0)) != cudaSuccess)
+      break;
+    e = cudaMemcpy2DAsync(static_cast<char*>(hout->host) + (size_t)g0 * 128 * sizeof(float), pitch,
+                          static_cast<const char*>(out) + (size_t)g0 * 128 * sizeof(float), pitch,
+                          (size_t)a.h_count * 128 * sizeof(float), (size_t)c.batch * nq, cudaMemcpyDeviceToHost,
+                          hout->stream);
+  }
+  if (e == cudaSuccess && (e = cudaEventRecord(hout->done, hout->stream)) == cudaSuccess)
+    e = cudaStreamWaitEvent(s, hout->done, 0);
+  hout->copied = e == cudaSuccess;
+  return e;
+}
+
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const void* kv_base, void* out, int nq,
-                                        int n_keys, int64_t t_first, int stage, cudaStream_t s);
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s,
+                                        HostOut* hout = nullptr);
 
 // The folded output mixer: out = O_bar W_fold^T instead of the per-head W_uv,h.
 struct FoldArgs {
@@ -617,16 +692,6 @@ struct QLatArgs {
   const void* c_q;     // [B][n_q][d_q]
   const void* w_qabs;  // [n_h][d_c + 32][d_q]
   int d_q;
-};
-
-// Output rows wanted in host memory (vmla_chunk_step_host): the absorbed attention then runs as
-// one launch per group of heads that fills the GPU once, and each group's columns are copied to
-// the host on `stream` while the next group computes; `copied` tells the caller it was done.
-struct HostOut {
-  void* host;
-  cudaStream_t stream;
-  cudaEvent_t group, done;
-  bool copied;
 };
 
 vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv, void* out,
@@ -686,7 +751,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       e = launch_recon_tc(tc, tuk, tuv, a, c.batch, s);
     }
     if (e != cudaSuccess) return cuda_fail(e);
-    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s);
+    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, hout);
   }
   if (design == VMLA_DESIGN_RECONSTRUCT) {
     __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
@@ -807,30 +872,9 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     if (!fold && !hout) {
       e = launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, a, c.batch, s);
     } else if (!fold) {
-      static int sms = 0;
-      if (sms == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-          sms = 148;
-      }
-      const int per_head = a.m_tiles * c.batch;  // CTAs of one head
-      const int hg = std::max(1, std::min(c.n_heads, sms / std::max(1, per_head)));
-      const size_t pitch = (size_t)c.n_heads * 128 * sizeof(float);
-      for (int g0 = 0; g0 < c.n_heads && e == cudaSuccess; g0 += hg) {
-        a.h0 = g0;
-        a.h_count = std::min(hg, c.n_heads - g0);
-        if ((e = launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, a, c.batch, s)) != cudaSuccess ||
-            (e = cudaEventRecord(hout->group, s)) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(hout->stream, hout->group, 0)) != cudaSuccess)
-          break;
-        e = cudaMemcpy2DAsync(static_cast<char*>(hout->host) + (size_t)g0 * 128 * sizeof(float), pitch,
-                              static_cast<const char*>(out) + (size_t)g0 * 128 * sizeof(float), pitch,
-                              (size_t)a.h_count * 128 * sizeof(float), (size_t)c.batch * nq, cudaMemcpyDeviceToHost,
-                              hout->stream);
-      }
-      if (e == cudaSuccess && (e = cudaEventRecord(hout->done, hout->stream)) == cudaSuccess)
-        e = cudaStreamWaitEvent(s, hout->done, 0);
-      hout->copied = e == cudaSuccess;
+      e = launch_head_groups(c, nq, a, out, hout, s, [&](const AttnTc& ag) {
+        return launch_attn_absorbed_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, tuv, to, ag, c.batch, s);
+      });
     } else {
       const uint64_t kf = (uint64_t)c.n_heads * c.d_latent;
       __nv_bfloat16* ob_hi = at<__nv_bfloat16>(h->ws, w.obar);
@@ -861,7 +905,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
 
 // Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128].
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const void* kv_base, void* out, int nq,
-                                        int n_keys, int64_t t_first, int stage, cudaStream_t s) {
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, HostOut* hout) {
   const vmla_config& c = h->cfg;
   const WsLayout w = ws_layout(c);
   __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
@@ -893,6 +937,10 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
   a.rescale_threshold = c.softmax_rescale_log2;
   a.err = h->err;
   a.limit_ns = kWaitLimitNs;
+  if (hout)
+    return cuda_status(launch_head_groups(c, nq, a, out, hout, s, [&](const AttnTc& ag) {
+      return launch_attn_dense_tc(tq, tkv, to, ag, c.batch, s);
+    }));
   return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s));
 }
 
@@ -912,7 +960,11 @@ vmla_status attention_args(vmla_handle* h, int layer, const void* q, const void*
   const vmla_config& c = h->cfg;
   if ((st = check_attention_frames(c, frames, first, n, win)) != VMLA_OK) return st;
   if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
-  *design = resolve_design(c, *design);
+  const bool automatic = *design == VMLA_DESIGN_AUTO;
+  *design = resolve_design(c, *design, win->n_keys);
+  if (automatic && *design == VMLA_DESIGN_RECON_ONCE && c.d_latent <= 256 &&
+      h->ws_bytes < ws_layout(c).base_bytes + ws_layout(c).recon_bytes)
+    *design = VMLA_DESIGN_ABSORBED;  // AUTO with a workspace bound without room for the per-head K/V
   if (c.dtype == VMLA_BF16) {
     // the absorbed kernels keep d_latent + d_rope query and key columns resident: up to 256 latent dims
     if (*design == VMLA_DESIGN_ABSORBED && c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;
@@ -935,7 +987,7 @@ vmla_status chunk_attention(vmla_handle* h, int layer, const void* q, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (h->cfg.dtype == VMLA_FP32) return attention_fp32(h, layer, q, w_uk, w_uv, out, first, n, win, s);
   return attention_bf16(h, layer, q, w_uk, w_uv, out, first, n, win, design, s, nullptr, nullptr,
-                        design == VMLA_DESIGN_ABSORBED ? hout : nullptr);
+                        design == VMLA_DESIGN_ABSORBED || design == VMLA_DESIGN_RECON_ONCE ? hout : nullptr);
 }
 }  // namespace
 

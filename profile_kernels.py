@@ -1,6 +1,6 @@
 """Launch one kernel of the chunk-attention path a few times, for a profiler.
 
-    python -m latent_kv_attention_down_b200.profile_kernels \
+    python profile_kernels.py \
         {absorbed,recon,reconstruct,append1,append8,step8,folded,qlatent}
 
 Fills a 21-frame window of two Wan-1.3B-shaped layers (30x52 grid, 4680 queries per chunk) from

@@ -126,6 +126,24 @@ def test_workspace_bytes_grow_with_reconstruct_once():
     assert a % 256 == 0
 
 
+def test_workspace_offsets_fit_the_workspace():
+    """The intermediates' regions are 256-byte aligned, disjoint and inside the workspace that
+    vmla_workspace_bytes asks for: rotated keys, absorbed queries and per-head queries inside the
+    base part, the per-head K/V of reconstruct-once after it."""
+    c = default_config()
+    off = api.workspace_offsets(c)
+    T, nq = c.grid_h * c.grid_w, c.chunk_frames * c.grid_h * c.grid_w
+    sizes = [c.window_frames * T * c.d_rope * 2, c.n_heads * nq * (c.d_latent + c.d_rope) * 2,
+             c.n_heads * nq * (c.d_nope + c.d_rope) * 2, c.window_frames * T * 2 * c.n_heads * c.d_value * 2]
+    base, full = api.workspace_bytes(c, api.DESIGN_ABSORBED), api.workspace_bytes(c, api.DESIGN_RECON_ONCE)
+    assert all(o % 256 == 0 for o in off)
+    spans = sorted(zip(off, sizes))
+    assert all(a + n <= b for (a, n), (b, _) in zip(spans, spans[1:]))
+    assert off[api.WS_QD] + sizes[api.WS_QD] <= base and off[api.WS_RECON] + sizes[api.WS_RECON] <= full
+    buf = (ctypes.c_size_t * 2)()
+    assert api.lib().vmla_workspace_offsets(ctypes.byref(c), buf, 2) == 1  # room for every region
+
+
 def test_window_matches_a_fifo_deque():
     """vmla_window against an independent deque model of the ring, over a
     rollout of 20 chunks of 3 frames (eviction from chunk 7)."""
@@ -143,6 +161,21 @@ def test_window_matches_a_fifo_deque():
             ring[s] = f
         assert all(ring[s] == f for f, s in zip(frames, slots))
         assert len(set(slots)) == len(slots)
+    h.close()
+
+
+def test_window_t_at_append_is_the_absolute_frame():
+    """With RoPE applied at append the keys carry their absolute frame index, so vmla_window reports
+    t = frame, also once the rollout has run past the ring (F > W) and the window-relative t would
+    differ."""
+    c = default_config()
+    c.rope_mode = api.ROPE_AT_APPEND
+    h = api.LatentKVAttention(c)
+    for F in (3, 21, 24, 60, 300):
+        frames, slots, ts = h.window(F)
+        assert frames == list(range(max(0, F - 21), F))
+        assert slots == [f % 21 for f in frames]
+        assert ts == frames
     h.close()
 
 
@@ -178,7 +211,9 @@ def test_frame_rule_rejections_before_any_launch():
     h = api.LatentKVAttention(c)
     lib = api.lib()
     ws = api.workspace_bytes(c)
-    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, ws - 256) == 1  # workspace too small
+    base = api.workspace_bytes(c, api.DESIGN_ABSORBED)  # what every design but reconstruct-once needs
+    assert base < ws
+    assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, base - 256) == 1  # workspace too small
     assert lib.vmla_bind(h._h, 0x10008, 0x20000, 0x30000, ws) == 1        # misaligned
     assert lib.vmla_bind(h._h, 0x10000, 0x20000, 0x30000, ws) == 0
     x = w = 0x40000

@@ -93,33 +93,45 @@ def test_small_bf16_absorbed(chunks):
     21-frame window, 4200 keys), 10 (evicted, wrapped ring)."""
     ro = Rollout(SMALL)
     _fill(ro, chunks)
-    out, q = ro.attend(0, chunks - 1)
+    out, q = ro.attend(0, chunks - 1, design=api.DESIGN_ABSORBED)
     assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"{chunks} chunks")
 
 
-@pytest.mark.parametrize("dense", [False, True])
-def test_small_bf16_forced_rescale(dense):
+@pytest.mark.parametrize("chunks", [7, 10])
+def test_small_bf16_auto(chunks):
+    """AUTO on the full 21-frame window (4200 keys: reconstruct-once) and on the wrapped ring."""
+    ro = Rollout(SMALL)
+    _fill(ro, chunks)
+    out, q = ro.attend(0, chunks - 1)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"AUTO, {chunks} chunks")
+
+
+@pytest.mark.parametrize("design,dense", [(api.DESIGN_ABSORBED, False), (api.DESIGN_RECON_ONCE, False),
+                                          (api.DESIGN_AUTO, True)])
+def test_small_bf16_forced_rescale(design, dense):
     """Threshold 0: the running max is raised (and O rescaled in TMEM) at every
     increase, so the correction path runs many times per row."""
-    ro = Rollout(SMALL, rescale_log2=0.0, dense=dense)
+    ro = Rollout(SMALL, rescale_log2=0.0, dense=dense, design=api.DESIGN_RECON_ONCE)
     _fill(ro, 8, dense=dense)
-    out, q = ro.attend(0, 7, dense=dense)
+    out, q = ro.attend(0, 7, design=design, dense=dense)
     assert_bf16_close(out[0], ro.oracle(0, 7, q), "forced rescale")
 
 
-def test_small_bf16_rope_at_append():
+@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE])
+def test_small_bf16_rope_at_append(design):
     ro = Rollout(SMALL, rope_mode=api.ROPE_AT_APPEND)
     _fill(ro, 9)
-    out, q = ro.attend(0, 8)
+    out, q = ro.attend(0, 8, design=design)
     assert_bf16_close(out[0], ro.oracle(0, 8, q), "rope at append")
 
 
-def test_small_bf16_denoising_passes():
+@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_AUTO])
+def test_small_bf16_denoising_passes(design):
     ro = Rollout(SMALL)
     _fill(ro, 7)
     for p in range(4):
         ro.append_chunk(0, 7, pass_=p)
-        out, q = ro.attend(0, 7, pass_=p)
+        out, q = ro.attend(0, 7, pass_=p, design=design)
         assert_bf16_close(out[0], ro.oracle(0, 7, q), f"pass {p}")
 
 
@@ -339,22 +351,23 @@ def test_small_bf16_attention_after_tiled_appends(tiling):
     assert_bf16_close(out[0], ro.oracle(0, 7, q), f"tiling {tiling}")
 
 
-def test_small_output_rows_and_guards():
+@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE, api.DESIGN_RECONSTRUCT])
+def test_small_output_rows_and_guards(design):
     """Attention writes exactly its output tensor: guard rows around it stay
     bit-identical."""
     import torch
-    ro = Rollout(SMALL)
-    _fill(ro, 3)
+    ro = Rollout(SMALL, design=api.DESIGN_RECON_ONCE)
+    _fill(ro, 8)
     d = SMALL
-    q = synth.queries(d, 0, 2)
+    q = synth.queries(d, 0, 7)
     width = d.n_heads * d.d_head
     buf = torch.full((d.n_queries + 64, width), 12345.0, dtype=torch.float32, device="cuda")
     out = buf[32:32 + d.n_queries]
-    ro.m.attention(0, to_dev(q, d), ro.wd[0][1], ro.wd[0][2], out, 6, 3)
+    ro.m.attention(0, to_dev(q, d), ro.wd[0][1], ro.wd[0][2], out, 21, 3, design)
     assert ro.m.device_status()[0] == 0
     b = buf.float().cpu().numpy()
     assert np.all(b[:32] == 12345.0) and np.all(b[32 + d.n_queries:] == 12345.0)
-    assert_bf16_close(b[32:32 + d.n_queries], ro.oracle(0, 2, q), "guarded")
+    assert_bf16_close(b[32:32 + d.n_queries], ro.oracle(0, 7, q), "guarded")
 
 
 def test_step_host_matches_device_path():
@@ -376,7 +389,8 @@ def test_step_host_matches_device_path():
     assert_bf16_close(oh.float().numpy()[0], ro.oracle(0, 7, q), "host step")
 
 
-def test_step_host_head_groups_match_device_path():
+@pytest.mark.parametrize("design", [api.DESIGN_AUTO, api.DESIGN_ABSORBED])
+def test_step_host_head_groups_match_device_path(design):
     """Batch 4 on the small grid: the host-buffer step runs the attention as one launch per group
     of heads that fills the GPU once (7 + 5 heads) and copies each group's output columns back
     while the next group computes.  Two consecutive calls on the same staging buffers, issued
@@ -395,7 +409,8 @@ def test_step_host_head_groups_match_device_path():
         q = torch.from_numpy(synth.queries(d, 0, chunk)).to(torch.bfloat16).pin_memory()
         oh = torch.full((d.batch, d.n_queries, d.n_heads * d.d_head), float("nan")).pin_memory()
         wd = host.wd[0]
-        host.m.step_host(0, x, q, oh, wd[0], wd[1], wd[2], xd, qd, od, chunk * d.chunk_frames, d.chunk_frames)
+        host.m.step_host(0, x, q, oh, wd[0], wd[1], wd[2], xd, qd, od, chunk * d.chunk_frames, d.chunk_frames,
+                         design)
         keep.append((x, q))
         outs.append(oh)
     torch.cuda.synchronize()
@@ -403,22 +418,43 @@ def test_step_host_head_groups_match_device_path():
     assert st == 0, f"device status {st} flags {flags:#x}"
     for chunk, oh in zip((6, 7), outs):
         dev.append_chunk(0, chunk)
-        ref, _ = dev.attend(0, chunk)
+        ref, _ = dev.attend(0, chunk, design=design)
         assert np.array_equal(oh.numpy(), ref), f"chunk {chunk}: host step differs from the device path"
 
 
 # ------------------------------------------------------------------ the full Wan-1.3B layer
 
-def test_wan_layer_sampled_rows():
-    """4680 queries x 12 heads over the full 32760-key window, checked on 256
-    seeded query rows (ragged last tile included) for every head."""
+def test_wan_layer_full_every_design():
+    """The Wan-1.3B layer call checked in full: all 4680 query rows x 12 heads over the 32760-key
+    window (18 past + 3 current frames, ragged last query tile) against the fp64 oracle, for the
+    design AUTO takes there (reconstruct-once), the absorbed design, reconstruct-in-tile and the
+    dense per-head cache.  One oracle evaluation serves every design."""
+    import time
+    ro = Rollout(WAN, design=api.DESIGN_RECON_ONCE, dense=True)
+    for c in range(7):
+        ro.append_chunk(0, c)
+        ro.append_chunk(0, c, dense=True)
+    got = {}
+    for name, design, dense in (("auto", api.DESIGN_AUTO, False), ("absorbed", api.DESIGN_ABSORBED, False),
+                                ("reconstruct_in_tile", api.DESIGN_RECONSTRUCT, False), ("dense", None, True)):
+        out, q = ro.attend(0, 6, design=design or api.DESIGN_AUTO, dense=dense)
+        got[name] = out[0]
+    t0 = time.perf_counter()
+    ref = ro.oracle(0, 6, q)
+    print(f"oracle, full Wan layer call: {time.perf_counter() - t0:.1f} s")
+    for name, o in got.items():
+        rel, mx = assert_bf16_close(o, ref, f"wan layer, {name}")
+        print(f"wan layer full, {name}: relative L2 {rel:.2e}, max |err| / rms {mx:.2e}")
+
+
+def test_wan_layer_first_chunk_auto():
+    """AUTO on the first chunk of a rollout (3 frames, 4680 keys: reconstruct-once from 4096 keys
+    on), 256 seeded query rows of every head."""
     ro = Rollout(WAN)
-    _fill(ro, 7)
-    out, q = ro.attend(0, 6)
-    rows = np.sort(np.random.default_rng(0).choice(WAN.n_queries, 256, replace=False))
-    rows[-1] = WAN.n_queries - 1
-    ref = ro.oracle(0, 6, q, rows=rows)
-    assert_bf16_close(out[0][rows], ref, "wan layer")
+    _fill(ro, 1)
+    out, q = ro.attend(0, 0)
+    rows = sampled_rows(WAN.n_queries, 256, seed=3)
+    assert_bf16_close(out[0][rows], ro.oracle(0, 0, q, rows=rows), "wan layer, first chunk")
 
 
 def test_wide_grid_rotary_pairs_evaluated_directly():

@@ -85,10 +85,13 @@ class PoolRollout:
             assert_bf16_close(out[b][rows], ref, f"{what} layer {layer} chunk {chunk} pass {pass_} sample {b}")
 
 
-def test_wan_rollout_30_layers_20_chunks_4_passes():
+@pytest.mark.parametrize("design", [api.DESIGN_AUTO, api.DESIGN_ABSORBED])
+def test_wan_rollout_30_layers_20_chunks_4_passes(design):
+    """AUTO runs reconstruct-once on every window of this rollout (4680 keys and more); the
+    absorbed design is rolled out the same way."""
     import torch
     layers, chunks, passes = 30, 20, 4
-    ro = PoolRollout(WAN, layers)
+    ro = PoolRollout(WAN, layers, design=design)
     checks = {(0, 0, 0), (17, 5, 2), (29, 6, 3), (3, 7, 0), (11, 13, 1), (29, 19, 3)}
     resume_at, resume_layers = 10, (0, 21)  # snapshot before chunk 10, replay it on a second handle
     kept = {}

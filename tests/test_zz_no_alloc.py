@@ -8,11 +8,10 @@ that a run stopping at its first failure has already run every other test.
 """
 import ctypes
 
-import numpy as np
 import pytest
 
 from latent_kv_attention_down_b200 import api, synth
-from tests.harness import Rollout, assert_bf16_close, to_dev
+from tests.harness import Rollout, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -32,9 +31,13 @@ def _noalloc(ro, q, out, first, n, frames):
         w[2].data_ptr(), out.data_ptr(), first, n, torch.cuda.current_stream().cuda_stream)
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
+@pytest.mark.parametrize("dims", [synth.WAN_SMALL, synth.WAN], ids=lambda d: d.name)
+def test_noalloc_matches_workspace_entry_point_twice(dims):
+    """Both entry points launch the same kernels with the same arguments, so the outputs must be
+    equal bit for bit, on two calls in a row (the second one reuses the array as the first left
+    it), on the small grid and on the full Wan-1.3B layer (27.3 MB of scratch)."""
     import torch
-    d = synth.WAN_SMALL
+    d = dims
     ro = Rollout(d)
     for c in range(8):  # 24 frames through the 21-frame ring
         ro.append_chunk(0, c)
@@ -43,12 +46,12 @@ def test_noalloc_matches_workspace_entry_point_twice():
     ref = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
     ro.m.attention(0, q, ro.wd[0][1], ro.wd[0][2], ref, 21, 3, api.DESIGN_ABSORBED)
     assert ro.m.device_status()[0] == 0
-    ref = ref.cpu().numpy()[0]
+    assert torch.isfinite(ref).all()
     for call in range(2):
         out = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(ro, q, out, 21, 3, 24) == 0
         assert ro.m.device_status()[0] == 0
-        assert_bf16_close(out.cpu().numpy()[0], ref, f"no-alloc call {call}")
+        assert torch.equal(out, ref), f"no-alloc call {call} differs from the workspace entry point"
 
 
 def test_noalloc_rejects_calls_beyond_its_array():
