@@ -790,9 +790,11 @@ def width_leg(m_timed, dev, tc, seed, widths=(64, 128, 192, 256, 384, 512)):
     return res
 
 
-def rotary_leg(dev, tc, seed, splits=((112, 16, (4, 2, 2)), (96, 32, (6, 5, 5)), (64, 64, (12, 10, 10)))):
-    """d_head 128 split into content/rotary dims 112/16, 96/32 and 64/64 on the Wan layer (d_c 192,
-    full window): one chunk step (append + RoPE + q-absorb + absorbed attention) per split."""
+def rotary_leg(dev, tc, seed, splits=((112, 16, (4, 2, 2)), (96, 32, (6, 5, 5)), (64, 64, (12, 10, 10)),
+                                      (32, 96, (16, 16, 16)))):
+    """d_head 128 split into content/rotary dims 112/16, 96/32, 64/64 and 32/96 on the Wan layer (d_c
+    192, full window): one chunk step per split and design -- the absorbed design, reconstruct-once
+    (AUTO's choice) and the dense per-head cache -- with the attention kernel's time and rate."""
     import torch
     from latent_kv_attention_down_b200 import api
     res = {}
@@ -801,7 +803,8 @@ def rotary_leg(dev, tc, seed, splits=((112, 16, (4, 2, 2)), (96, 32, (6, 5, 5)),
     for dn, dr, pairs in splits:
         d = WORKLOAD.replace(d_nope=dn, d_rope=dr, rope_pairs=pairs)
         L = 2
-        m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev)
+        m = api.LatentKVAttention(api.config_from_dims(d, layers=L)).allocate(device=dev, design=api.DESIGN_RECON_ONCE,
+                                                                             dense=True)
         pool = synth.FramePool(d, base_seed=seed)
         xp = torch.from_numpy(pool.x).to(dev, bf)
         qp = torch.from_numpy(pool.q).to(dev, bf)
@@ -811,35 +814,48 @@ def rotary_leg(dev, tc, seed, splits=((112, 16, (4, 2, 2)), (96, 32, (6, 5, 5)),
         first = (chunks - 1) * d.chunk_frames
         for l in range(L):
             _pool_fill(m, d, pool, xp, W[l], l, chunks)
+            for c in range(chunks):
+                m.dense_append(l, pool.activations(l, c, 0, pool=xp), W[l][0], W[l][1], W[l][2], c * d.chunk_frames,
+                               d.chunk_frames)
         xs = [pool.activations(l, chunks - 1, 1, pool=xp) for l in range(L)]
         qs = [pool.queries(l, chunks - 1, 1, pool=qp) for l in range(L)]
         out = torch.empty((1, d.n_queries, d.n_heads * d.d_head), dtype=torch.float32, device=dev)
-
-        def step(i):
-            l = i % L
-            m.append(l, xs[l], W[l][0], first, d.chunk_frames)
-            m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, api.DESIGN_ABSORBED)
-        for i in range(3):
-            step(i)
-        torch.cuda.synchronize()
-        m.profile(True)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(steps):
-            step(3 + i)
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / steps
-        at, n = m.profile_read("attention")
-        m.profile(False)
-        st, flags = m.device_status()
-        assert st == 0, f"device status {st} flags {flags:#x}"
-        F = step_flops(d)
-        att = at / max(n, 1)
-        res[f"{dn}/{dr}"] = {"ms_per_step": ms, "attention_ms": att,
-                             "attention_tflops": F["attention"] / (att * 1e-3) / 1e12,
-                             "frac_of_bf16_peak": F["attention"] / (att * 1e-3) / 1e12 / tc,
-                             "attention_flops": F["attention"]}
+        F, DF = step_flops(d), dense_flops(d)
+        per = {}
+        for name, design, stage, flops in (("absorbed", api.DESIGN_ABSORBED, "attention", F["attention"]),
+                                           ("recon_once", api.DESIGN_RECON_ONCE, "dense_attention", DF["attention"]),
+                                           ("dense", None, "dense_attention", DF["attention"])):
+            def step(i):
+                l = i % L
+                if design is None:
+                    m.dense_append(l, xs[l], W[l][0], W[l][1], W[l][2], first, d.chunk_frames)
+                    m.dense_attention(l, qs[l], out, first, d.chunk_frames)
+                else:
+                    m.append(l, xs[l], W[l][0], first, d.chunk_frames)
+                    m.attention(l, qs[l], W[l][1], W[l][2], out, first, d.chunk_frames, design)
+            for i in range(3):
+                step(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(steps):
+                step(3 + i)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            m.profile(True)
+            for i in range(steps):
+                step(3 + steps + i)
+            at, n = m.profile_read(stage)
+            m.profile(False)
+            st, flags = m.device_status()
+            assert st == 0, f"device status {st} flags {flags:#x}"
+            att = at / max(n, 1)
+            per[name] = {"ms_per_step": ms, "attention_ms": att,
+                         "tflops_effective": F["total"] / (ms * 1e-3) / 1e12,
+                         "attention_tflops_issued": flops / (att * 1e-3) / 1e12,
+                         "frac_of_bf16_peak": flops / (att * 1e-3) / 1e12 / tc}
+        res[f"{dn}/{dr}"] = per
         m.close()
         del xp, qp, W, xs, qs, out, m
         torch.cuda.empty_cache()

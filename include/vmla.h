@@ -54,19 +54,21 @@ typedef enum vmla_status {
   VMLA_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
   VMLA_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up on a pipeline wait (device status word) */
   VMLA_ERR_STATE = 6,             /* frame sequence not allowed (skips or rewinds), buffers not bound */
-  VMLA_ERR_DEVICE_BOUNDS = 7      /* a kernel found an index outside its buffer (device status word) */
+  VMLA_ERR_DEVICE_BOUNDS = 7,     /* a kernel found an index outside its buffer (device status word) */
+  VMLA_ERR_DEVICE_RANGE = 8       /* a kernel produced a value past the range of its storage type: a per-head
+                                     query, key or value above 65504 in the fp16 reconstruct-once
+                                     workspace (device status word) */
 } vmla_status;
 
 typedef enum vmla_dtype { VMLA_BF16 = 0, VMLA_FP32 = 1 } vmla_dtype;
 
 /* How vmla_chunk_attention evaluates the same scores and outputs. */
 typedef enum vmla_design {
-  VMLA_DESIGN_AUTO = 0,        /* the design measured fastest that meets the accuracy gate for the call:
-                                  VMLA_BF16: RECON_ONCE past 256 latent dims, and at 192 or 256 latent
-                                  dims when the window holds at least 4096 keys; ABSORBED otherwise,
-                                  and whenever d_rope != 32.  VMLA_FP32 always evaluates the absorbed
-                                  form.  vmla_workspace_bytes(AUTO) covers the RECON_ONCE workspace
-                                  whenever the configuration's full window would take it; with a
+  VMLA_DESIGN_AUTO = 0,        /* the design measured fastest that meets the accuracy gate:
+                                  VMLA_BF16: RECON_ONCE from 192 latent dims on (and for the splits the
+                                  absorbed kernel does not take), ABSORBED at 64 and 128.  VMLA_FP32
+                                  always evaluates the absorbed form.  vmla_workspace_bytes(AUTO)
+                                  covers the RECON_ONCE workspace whenever AUTO takes it; with a
                                   smaller workspace bound, AUTO stays ABSORBED up to 256 latent dims */
   VMLA_DESIGN_ABSORBED = 1,    /* W_uk folded into the query, MQA over [c_KV | k_R], W_uv after the
                                   softmax-weighted sum [paperlayer App. E] */
@@ -75,7 +77,9 @@ typedef enum vmla_design {
                                   On-demand reconstruction]; VMLA_BF16 with d_latent 64, 128 or 192
                                   (VMLA_ERR_UNSUPPORTED_SHAPE otherwise), no extra workspace */
   VMLA_DESIGN_RECON_ONCE = 3   /* per-head K/V of the whole window rebuilt once into the workspace, then
-                                  d_head attention */
+                                  d_head attention; the rebuilt K/V, the per-head queries and the
+                                  probabilities are fp16 (rounding 2^-11 against bf16's 2^-8), and a
+                                  value past fp16's range is reported (VMLA_ERR_DEVICE_RANGE) */
 } vmla_design;
 
 /* When the positional key gets its 3D rotation. */
@@ -233,9 +237,11 @@ vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q,
  * (preferably pinned) host buffers into the caller's device staging buffers, append,
  * attend, copy out back to the host buffer.  The two input copies run on a stream of the
  * handle's own, each ordered after the previous call's last use of its staging buffer (x_dev:
- * the append; q_dev: the attention), so consecutive calls overlap them with compute; append and
- * attention are enqueued on `stream`, which waits for the inputs.  The absorbed attention runs
- * as one launch per group of heads that fills the GPU once, and each group's output columns
+ * the append; q_dev: the kernel that prepares the queries, the first kernel of the attention), so
+ * consecutive calls overlap them with compute; append and
+ * attention are enqueued on `stream`, which waits for the inputs.  The absorbed and the
+ * reconstruct-once attention run as one launch per group of heads that fills the GPU once, and each
+ * group's output columns
  * go back to out_host on a third stream while the next group computes; `stream` waits for the
  * last of those copies (other designs copy the output back on `stream`).  The host buffers
  * must stay valid, and out_host is complete, once `stream` reaches this point.
@@ -261,8 +267,8 @@ vmla_status vmla_state_get(const vmla_handle* h, int layer, int64_t* frames_appe
 vmla_status vmla_state_set(vmla_handle* h, int layer, int64_t frames_appended);
 
 /* Synchronise `stream`, read and clear the library's device status word:
- * VMLA_OK, VMLA_ERR_DEVICE_TIMEOUT or VMLA_ERR_DEVICE_BOUNDS; *flags (may be NULL)
- * gets the raw bits. */
+ * VMLA_OK, VMLA_ERR_DEVICE_TIMEOUT, VMLA_ERR_DEVICE_BOUNDS or VMLA_ERR_DEVICE_RANGE; *flags (may
+ * be NULL) gets the raw bits. */
 vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
 
 /* Per-stage CUDA-event timing of the kernels each call launches, recorded on the
@@ -327,11 +333,12 @@ vmla_status vmla_chunk_attention_qlatent(vmla_handle* h, int layer, const void* 
  *
  * It computes exactly what vmla_chunk_attention computes with
  * VMLA_DESIGN_ABSORBED (same kernels, same arguments and layouts; VMLA_BF16
- * only), for the window of a layer that has `frames_appended` frames in it.
+ * only, the shapes that design takes), for the window of a layer that has
+ * `frames_appended` frames in it.
  * `ckv` and `kr` are the caches of all layers as laid out by vmla_cache_bytes.
  * Its scratch (the window's rotated positional keys and the absorbed queries:
- * batch*W*T_f*32*2 bytes, rounded up to 256, plus batch*n_heads*n_frames*T_f*
- * (d_latent + 32)*2 bytes) lives in a fixed 32 MiB array inside the library
+ * batch*W*T_f*d_rope*2 bytes, rounded up to 256, plus batch*n_heads*n_frames*T_f*
+ * (d_latent + d_rope)*2 bytes) lives in a fixed 32 MiB array inside the library
  * that every GPU which loads the library holds until the process exits;
  * larger calls return VMLA_ERR_OUT_OF_RANGE and enqueue nothing.  The call
  * makes no cudaMalloc or cudaFree and calls no allocating routine.

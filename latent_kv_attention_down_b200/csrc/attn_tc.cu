@@ -44,9 +44,9 @@ struct Bars {
   uint64_t q_full;
   uint64_t kv_full[kMaxStages];
   uint64_t kv_empty[kMaxStages];
-  uint64_t s_full[2];  // S_j computed (MMA commit)
-  uint64_t p_full[2];  // P_j stored over S_j by every softmax warp
-  uint64_t p_done[2];  // P V_j has completed (MMA commit), by tile parity
+  uint64_t s_full[3];  // S_j computed (MMA commit), by S buffer j % NSB
+  uint64_t p_full[3];  // P_j stored over S_j by every softmax warp
+  uint64_t p_done[3];  // P V_j has completed (MMA commit)
   uint64_t o_final;
   uint64_t wuv_full;
   uint64_t ob_full;
@@ -57,27 +57,37 @@ struct Bars {
   float red[2][2][128];  // per-tile half-row maxima of the two softmax groups (tile parity, group, row)
 };
 
-template <int DL_, bool DENSE_, int DR_ = 32>
+template <int DL_, bool DENSE_, int DR_ = 32, bool F16_ = false>
 struct AttnCfg {
   static constexpr bool DENSE = DENSE_;
+  // per-head operands (Q, K, V and P) in fp16 instead of bf16: the reconstruct-once workspace
+  static constexpr bool F16 = F16_;
+  static_assert(!F16 || DENSE, "fp16 operands: per-head tiles only");
   static constexpr int DL = DL_;
   static constexpr int DR = DR_;                     // rotary dims of the shared key (absorbed)
   static constexpr int DQK = DENSE ? 128 : DL + DR;  // contraction width of S = Q K^T
   static constexpr int DV = DENSE ? 128 : DL;
   static constexpr int BN = 128;
   static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of a query or key row
-  // the rotary columns sit in one block of DR * 2 bytes per row, swizzled at that width
-  static constexpr int RB = DENSE ? 0 : DR * 2;
+  // the rotary columns sit in NRB blocks of RB bytes per row, each swizzled at its width: one block
+  // of DR * 2 bytes for 16, 32 or 64 rotary dims, three 64-byte blocks for 96
+  static constexpr int NRB = DENSE ? 0 : (DR == 96 ? 3 : 1);
+  static constexpr int RB = DENSE ? 0 : (DR == 96 ? 64 : DR * 2);
   static constexpr uint32_t R_LAYOUT = RB == 128 ? LAYOUT_SW128 : (RB == 64 ? LAYOUT_SW64 : LAYOUT_SW32);
-  static constexpr int Q_BYTES = QB * 16384 + 128 * RB;
+  static constexpr int Q_BYTES = QB * 16384 + NRB * 128 * RB;
   static constexpr int KBLK = BN * 128;           // one [BN keys x 64] SW128 block
-  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + BN * RB;
+  static constexpr int STAGE_BYTES = DENSE ? 4 * KBLK : QB * KBLK + NRB * BN * RB;
   static constexpr int SMEM_CAP = 232448;
   static constexpr int BARS = (sizeof(Bars) + 127) / 128 * 128;
   static constexpr int STAGES_FIT = (SMEM_CAP - BARS - Q_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
-  static constexpr int S_COL = 0;  // S buffer b (and P_j over it) at S_COL + b*BN
-  static constexpr int O_COL = 2 * BN;
+  // S buffers: S_j (and P_j over it) in buffer j % NSB at S_COL + (j % NSB) * BN.  Two: Q K^T
+  // runs one tile ahead of the softmax.  (Per-head tiles would leave TMEM for a third; with Q K^T
+  // two tiles ahead the MMA thread then waits for the K/V stage of tile j+2 -- free only once
+  // P V_{j-1} is done -- before it can issue P V_j, which measured 1.6x slower.)
+  static constexpr int NSB = 2;
+  static constexpr int S_COL = 0;
+  static constexpr int O_COL = NSB * BN;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int SMEM = Q_BYTES + STAGES * STAGE_BYTES + BARS;
   // epilogue images: O_bar rounded over the query tile; W_uv,h in the ring stage that tile n_tiles
@@ -88,7 +98,7 @@ struct AttnCfg {
   static_assert(SMEM <= SMEM_CAP, "shared memory budget");
   static_assert((DENSE || STAGE_BYTES >= DV * 256) && STAGES * STAGE_BYTES >= 65536, "epilogue staging");
   static_assert(DV % 64 == 0 && DV <= 256 && BN % 32 == 0, "tile shapes");
-  static_assert(DENSE || DR == 16 || DR == 32 || DR == 64, "rotary block of 32, 64 or 128 bytes per row");
+  static_assert(DENSE || DR == 16 || DR == 32 || DR == 64 || DR == 96, "rotary blocks of 32, 64 or 128 bytes per row");
 };
 
 // bf16 row of 32 floats into a 128B-swizzled K-major tile: row r, columns c0..c0+31
@@ -124,12 +134,12 @@ __device__ __forceinline__ void st_swizzled_row32_f32(uint8_t* tile, int r, int 
 }
 
 // S = Q K^T for one tile.  Query tile and key tile in shared memory: QB [rows x 64] SW128
-// blocks of latent (or per-head key) columns, then (absorbed) one [rows x d_rope] block of
-// rotated positional columns, swizzled at its row width (32, 64 or 128 bytes).  Descriptors are
-// built once and advanced by compile-time offsets.
+// blocks of latent (or per-head key) columns, then (absorbed) the rotated positional columns: one
+// [rows x d_rope] block swizzled at its row width (32, 64 or 128 bytes), or three [rows x 32] SW64
+// blocks for 96 rotary dims.  Descriptors are built once and advanced by compile-time offsets.
 template <class C>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t stage) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, C::BN, false, false);
+  constexpr uint32_t idesc = C::F16 ? idesc_f16_f32(128, C::BN, false, false) : idesc_bf16_f32(128, C::BN, false, false);
   constexpr int KL = C::QB * 4;  // k-steps over the SW128 blocks
   const uint64_t kd = smem_desc(stage, 16, 1024, LAYOUT_SW128);
   const uint64_t qd = smem_desc(sq, 16, 1024, LAYOUT_SW128);
@@ -143,17 +153,20 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sq, uint32_t 
       mma_ss_c<true>(d_tmem, a, b, idesc);
   }
   if constexpr (!C::DENSE) {
-    const uint64_t krd = smem_desc(stage + C::QB * C::KBLK, 16, 8 * C::RB, C::R_LAYOUT);
-    const uint64_t qrd = smem_desc(sq + C::QB * 16384, 16, 8 * C::RB, C::R_LAYOUT);
 #pragma unroll
-    for (int kk = 0; kk < C::DR / 16; ++kk)
-      mma_ss_c<true>(d_tmem, desc_add(qrd, kk * 32), desc_add(krd, kk * 32), idesc);
+    for (int rb = 0; rb < C::NRB; ++rb) {
+      const uint64_t krd = smem_desc(stage + C::QB * C::KBLK + rb * C::BN * C::RB, 16, 8 * C::RB, C::R_LAYOUT);
+      const uint64_t qrd = smem_desc(sq + C::QB * 16384 + rb * 128 * C::RB, 16, 8 * C::RB, C::R_LAYOUT);
+#pragma unroll
+      for (int kk = 0; kk < C::RB / 32; ++kk)
+        mma_ss_c<true>(d_tmem, desc_add(qrd, kk * 32), desc_add(krd, kk * 32), idesc);
+    }
   }
 }
 
 template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t stage, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, C::DV, false, true);
+  constexpr uint32_t idesc = C::F16 ? idesc_f16_f32(128, C::DV, false, true) : idesc_bf16_f32(128, C::DV, false, true);
   const uint64_t vd = smem_desc(C::DENSE ? stage + 2 * C::KBLK : stage, C::KBLK, 1024, LAYOUT_SW128);
   if (accumulate)
     mma_ts_c<true>(o_tmem, p_tmem, vd, idesc);
@@ -193,13 +206,13 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 
 // FOLD (absorbed only): the epilogue stores O_bar itself, as its bf16 pair, for an output
 // mixer that folds W_uv,h in (tm_wuv then maps O_bar's rounded part, tm_out its residual).
-template <int DL, bool DENSE, bool FOLD, int DR>
+template <int DL, bool DENSE, bool FOLD, int DR, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
                    const __grid_constant__ CUtensorMap tm_wuv, const __grid_constant__ CUtensorMap tm_out,
                    const AttnTc a) {
-  using C = AttnCfg<DL, DENSE, DR>;
+  using C = AttnCfg<DL, DENSE, DR, F16>;
   // The dynamic shared memory window starts 1024-byte aligned (the swizzled TMA tiles need it);
   // the whole 227 KB budget may be in use, so there is no slack to realign: check instead.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < C::NSB; ++k) {
       mbar_init(&bars->s_full[k], 1);
       mbar_init(&bars->p_full[k], kSoftmaxWarps);
       mbar_init(&bars->p_done[k], 1);
@@ -251,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qrow = b * a.n_heads + h;
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int qb = 0; qb < C::QB; ++qb) tma_load_3d(sQ + qb * 16384, &tm_q, &bars->q_full, qb * 64, m0, qrow);
-      if constexpr (!C::DENSE) tma_load_3d(sQ + C::QB * 16384, &tm_qr, &bars->q_full, DL, m0, qrow);
+      if constexpr (!C::DENSE)
+        for (int rb = 0; rb < C::NRB; ++rb)
+          tma_load_3d(sQ + C::QB * 16384 + rb * 128 * C::RB, &tm_qr, &bars->q_full, DL + rb * (C::RB / 2), m0, qrow);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % C::STAGES;
@@ -267,7 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           for (int kb = 0; kb < C::QB; ++kb)
             tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], kb * 64, j * C::BN, b);
-          tma_load_3d(st + C::QB * C::KBLK, &tm_kr, &bars->kv_full[s], 0, j * C::BN, b);
+          for (int rb = 0; rb < C::NRB; ++rb)
+            tma_load_3d(st + C::QB * C::KBLK + rb * C::BN * C::RB, &tm_kr, &bars->kv_full[s], rb * (C::RB / 2),
+                        j * C::BN, b);
         }
         ++issued;
       }
@@ -292,26 +309,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // order: QK_0, then per tile j: QK_{j+1}, P V_j
+    // order: QK_0 .. QK_{NSB-2}, then per tile j: QK_{j+NSB-1}, P V_j.  QK_{j+NSB-1} goes into the
+    // buffer that held P_{j-1}; P V_{j-1} was issued before it, and the tensor pipe runs in order.
     if (lane == 0) {
       const uint32_t sq = smem_u32(sQ), skv = smem_u32(sKV);
-      bool ok = wait_phase(&bars->q_full, 0, g, DEV_ERR_TIMEOUT_MMA) &&
-                wait_phase(&bars->kv_full[0], 0, g, DEV_ERR_TIMEOUT_MMA);
-      if (ok) {
+      bool ok = wait_phase(&bars->q_full, 0, g, DEV_ERR_TIMEOUT_MMA);
+      for (int j0 = 0; ok && j0 < C::NSB - 1 && j0 < n_tiles; ++j0) {
+        const int s0 = j0 % C::STAGES;
+        if (!(ok = wait_phase(&bars->kv_full[s0], (j0 / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
         tc_fence_after();
-        issue_qk<C>(tbase + C::S_COL, sq, skv);
-        mma_commit(&bars->s_full[0]);
+        issue_qk<C>(tbase + C::S_COL + j0 * C::BN, sq, skv + s0 * C::STAGE_BYTES);
+        mma_commit(&bars->s_full[j0]);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int buf = j & 1;
-        if (j + 1 < n_tiles) {
-          const int s1 = (j + 1) % C::STAGES;
-          if (!(ok = wait_phase(&bars->kv_full[s1], ((j + 1) / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+        const int buf = j % C::NSB;
+        const int jn = j + C::NSB - 1;
+        if (jn < n_tiles) {
+          const int s1 = jn % C::STAGES;
+          if (!(ok = wait_phase(&bars->kv_full[s1], (jn / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
           tc_fence_after();
-          issue_qk<C>(tbase + C::S_COL + (buf ^ 1) * C::BN, sq, skv + s1 * C::STAGE_BYTES);
-          mma_commit(&bars->s_full[buf ^ 1]);
+          issue_qk<C>(tbase + C::S_COL + (jn % C::NSB) * C::BN, sq, skv + s1 * C::STAGE_BYTES);
+          mma_commit(&bars->s_full[jn % C::NSB]);
         }
-        if (!(ok = wait_phase(&bars->p_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+        if (!(ok = wait_phase(&bars->p_full[buf], (j / C::NSB) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
         tc_fence_after();
         const int s = j % C::STAGES;
         issue_pv<C>(tbase + C::O_COL, tbase + C::S_COL + buf * C::BN, skv + s * C::STAGE_BYTES, j > 0);
@@ -350,9 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Two warpgroups share the 128 rows: group wg takes score columns [wg*BN/2, (wg+1)*BN/2)
     // of every tile and O columns [wg*DV/2, (wg+1)*DV/2); warp w of either group reads TMEM
     // lanes 32*(w%4).. (the same rows).  The row max of a tile is the larger of the two
-    // halves' maxima, swapped through shared memory once per tile.  Every thread of both
-    // groups passes the same named barriers in the same order, whatever happens: a thread
-    // that gave up skips the work, never the barrier.
+    // halves' maxima, swapped through shared memory once per tile by the two warps of a lane
+    // quarter alone (named barrier 2 + quarter, 64 threads).  Every thread of both groups
+    // passes the same named barriers in the same order, whatever happens: a thread that gave
+    // up skips the work, never the barrier.
     const int wg = (warp - 4) >> 2;
     const int wq = (warp - 4) & 3;
     const int r = wq * 32 + lane;  // query row inside the tile == TMEM lane
@@ -364,8 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int buf = j & 1;
-      ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->s_full[buf], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+      const int buf = j % C::NSB;  // S buffer of tile j
+      const int xp = j & 1;        // exchange slot of tile j
+      ok = ok && __all_sync(0xffffffffu, wait_phase(&bars->s_full[buf], (j / C::NSB) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
       uint32_t sraw[HS];
       float mx = -INFINITY;
       if (ok) {
@@ -391,9 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 1; k < HS / 16; ++k) mx = fmaxf(mx, mxc[k]);
       }
-      bars->red[buf][wg][r] = mx;
-      named_bar_sync(2, 256);
-      const float m_tile = fmaxf(mx, bars->red[buf][wg ^ 1][r]) * a.scale_log2;
+      bars->red[xp][wg][r] = mx;
+      named_bar_sync(2 + wq, 64);  // the two warps of this lane quarter (one per group) exchange
+      const float m_tile = fmaxf(mx, bars->red[xp][wg ^ 1][r]) * a.scale_log2;
       if (ok) {
         if (j == 0) {
           m_run = m_tile;
@@ -402,8 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // once the previous P V is done (both groups take the same decision for a row)
           const float m_new = fmaxf(m_run, m_tile);
           const float alpha = ex2_approx(m_run - m_new);
-          ok = __all_sync(0xffffffffu,
-                          wait_phase(&bars->p_done[(j - 1) & 1], ((j - 1) >> 1) & 1, g, DEV_ERR_TIMEOUT_SOFTMAX));
+          ok = __all_sync(0xffffffffu, wait_phase(&bars->p_done[(j - 1) % C::NSB], ((j - 1) / C::NSB) & 1, g,
+                                                  DEV_ERR_TIMEOUT_SOFTMAX));
           if (ok) {
             tc_fence_after();
 #pragma unroll 1
@@ -431,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 y = __ffma2_rn(x, sc2, nm2);
           const float2 pr = exp2_mixed(y, k);
           acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
-          packed[k] = pack_bf16x2(pr.x, pr.y);
+          packed[k] = C::F16 ? pack_f16x2(pr.x, pr.y) : pack_bf16x2(pr.x, pr.y);
         }
         st_packed<HS / 2>(lane_base + C::S_COL + buf * C::BN + wg * (HS / 2), packed);
         const float2 acc4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
@@ -444,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) tc_fence_after();
     // row sum = both halves' partial sums (the other parity's exchange slot is free by now)
     bars->red[n_tiles & 1][wg][r] = l_run;
-    named_bar_sync(2, 256);
+    named_bar_sync(2 + wq, 64);
     const float inv_l = 1.f / (l_run + bars->red[n_tiles & 1][wg ^ 1][r]);
     if constexpr (!C::DENSE) {
       // O_bar = O / l as a bf16 pair (A operands of the two W_uv GEMMs): rounded part over the
@@ -511,17 +533,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DL, bool DENSE, bool FOLD = false, int DR = 32>
+template <int DL, bool DENSE, bool FOLD = false, int DR = 32, bool F16 = false>
 cudaError_t go_attn(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk, const CUtensorMap& tkr,
                     const CUtensorMap& tuv, const CUtensorMap& to, const AttnTc& a, int batch, cudaStream_t s) {
-  using C = AttnCfg<DL, DENSE, DR>;
-  static const cudaError_t attr = cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE, FOLD, DR>,
+  using C = AttnCfg<DL, DENSE, DR, F16>;
+  static const cudaError_t attr = cudaFuncSetAttribute(attn_tc_kernel<DL, DENSE, FOLD, DR, F16>,
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (attr != cudaSuccess) return attr;
   if (a.n_q <= 0 || a.n_keys <= 0) return cudaSuccess;
   const int heads = a.h_count > 0 ? a.h_count : a.n_heads;
-  attn_tc_kernel<DL, DENSE, FOLD, DR><<<dim3(a.m_tiles, heads, batch), kThreads, C::SMEM, s>>>(tq, tqr, tk, tkr, tuv,
-                                                                                               to, a);
+  attn_tc_kernel<DL, DENSE, FOLD, DR, F16><<<dim3(a.m_tiles, heads, batch), kThreads, C::SMEM, s>>>(
+      tq, tqr, tk, tkr, tuv, to, a);
   return cudaGetLastError();
 }
 
@@ -539,26 +561,41 @@ int attn_absorbed_block_n(int d_latent) {
 
 int attn_dense_block_n() { return AttnCfg<128, true>::BN; }
 
-cudaError_t launch_attn_absorbed_obar_tc(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr,
+template <int DR>
+cudaError_t go_attn_obar_dl(int d_latent, const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tk,
+                            const CUtensorMap& tkr, const CUtensorMap& tob_hi, const CUtensorMap& tob_lo,
+                            const AttnTc& a, int batch, cudaStream_t s) {
+  switch (d_latent) {
+    case 64: return go_attn<64, false, true, DR>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 128: return go_attn<128, false, true, DR>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 192: return go_attn<192, false, true, DR>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 256:
+      if constexpr (DR <= 32) return go_attn<256, false, true, DR>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_absorbed_obar_tc(int d_latent, int d_rope, const CUtensorMap& tq, const CUtensorMap& tqr,
                                          const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tob_hi,
                                          const CUtensorMap& tob_lo, const AttnTc& a, int batch, cudaStream_t s) {
-  switch (d_latent) {
-    case 64: return go_attn<64, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
-    case 128: return go_attn<128, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
-    case 192: return go_attn<192, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
-    case 256: return go_attn<256, false, true>(tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+  switch (d_rope) {
+    case 16: return go_attn_obar_dl<16>(d_latent, tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 32: return go_attn_obar_dl<32>(d_latent, tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 64: return go_attn_obar_dl<64>(d_latent, tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
+    case 96: return go_attn_obar_dl<96>(d_latent, tq, tqr, tk, tkr, tob_hi, tob_lo, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& to,
-                                 const AttnTc& a, int batch, cudaStream_t s) {
+                                 const AttnTc& a, int batch, cudaStream_t s, bool f16) {
+  if (f16) return go_attn<128, true, false, 32, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
   return go_attn<128, true>(tq, tq, tkv, tkv, tq, to, a, batch, s);
 }
 
 bool attn_absorbed_supported(int d_latent, int d_rope) {
   const bool dl = d_latent == 64 || d_latent == 128 || d_latent == 192 || d_latent == 256;
-  return dl && (d_rope == 16 || d_rope == 32 || (d_rope == 64 && d_latent <= 192));
+  return dl && (d_rope == 16 || d_rope == 32 || ((d_rope == 64 || d_rope == 96) && d_latent <= 192));
 }
 
 template <int DR>
@@ -582,6 +619,7 @@ cudaError_t launch_attn_absorbed_tc(int d_latent, int d_rope, const CUtensorMap&
     case 16: return go_attn_dl<16>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
     case 32: return go_attn_dl<32>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
     case 64: return go_attn_dl<64>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
+    case 96: return go_attn_dl<96>(d_latent, tq, tqr, tk, tkr, tuv, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -15,6 +15,8 @@
 //    next to its rotated positional part.
 //  * recon_tc   [gist.it pt. 2; paperlayer §3 On-demand reconstruction]: the
 //    per-head dense entries k_h = [W_uk,h c | RoPE(k_R)], v_h = W_uv,h c.
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -94,14 +96,15 @@ __device__ __forceinline__ void store_bf16x32_smem(uint8_t* dst, const float (&v
 // parked for a TMA tensor store with 128-byte swizzle: the block holds 64 columns, 128 bytes per
 // row, and chunk j of a row sits at position j ^ (row & 7), so the eight rows a quarter-warp
 // writes at once fall in eight different bank groups.
-template <int N>
+// F16: the chunks are written as fp16 instead of bf16.
+template <int N, bool F16 = false>
 __device__ __forceinline__ void park_sw128(uint8_t* blk, int row, const uint32_t* r) {
+  auto pk = [](float lo, float hi) { return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi); };
 #pragma unroll
   for (int j = 0; j < N; ++j) {
     const float* v = reinterpret_cast<const float*>(r + 8 * j);
     *reinterpret_cast<uint4*>(blk + row * 128 + ((j ^ (row & 7)) << 4)) =
-        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                   pack_bf16x2(v[6], v[7]));
+        make_uint4(pk(v[0], v[1]), pk(v[2], v[3]), pk(v[4], v[5]), pk(v[6], v[7]));
   }
 }
 
@@ -331,7 +334,7 @@ struct QPrepCfg {
   static constexpr int WB = DN * 128;          // one 64-col block of W_uk,h: DN rows x 128 B
   static constexpr int W_BYTES = (DL / 64) * WB;
   static constexpr int ROW = DL + DR;                 // output row, elements
-  static constexpr int NCB = DL / 64 + 1;             // 64-column blocks of a row (the last one half used)
+  static constexpr int NCB = (ROW + 63) / 64;        // 64-column blocks of a row (the last one partly used)
   static constexpr int PARK_ROWS = W_BYTES + 2 * STAGE + NCB * 128 * 128 <= 212 * 1024 ? 128 : 64;
   static constexpr int BLK = PARK_ROWS * 128;         // one parked column block
   static constexpr int OUT_BYTES = NCB * BLK;
@@ -345,7 +348,7 @@ struct QPrepCfg {
   static constexpr int NB = DL / 64;   // TMEM column blocks: [0, NA) parked by warpgroup 0,
   static constexpr int NA = (NB + 1) / 2;  // [NA, NB) and the positional block by warpgroup 1
   static_assert(DL % 64 == 0 && DL <= 256 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
-  static_assert((DR == 16 || DR == 32 || DR == 64) && W_BYTES % 1024 == 0, "rotary dims");
+  static_assert((DR == 16 || DR == 32 || DR == 64 || DR == 96) && W_BYTES % 1024 == 0, "rotary dims");
   static_assert(ROW > (NCB - 1) * 64 && ROW <= NCB * 64, "a row of q~ spans its parked column blocks");
 };
 
@@ -517,7 +520,12 @@ __global__ void __launch_bounds__(QPrepCfg<DL, DR>::THREADS, 1)
             tmem_ld64(tmem_addr(tbase, wq * 32, acc * 256 + cb * 64), raw);
             park_sw128<8>(sout + cb * C::BLK, pr, raw);
           }
-          if (wg == 1) park_sw128<DR / 8>(sout + C::NB * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
+          if (wg == 1) {  // the positional part: DR / 8 chunks from column block NB on, 8 per block
+            constexpr int RC = DR / 8;
+            park_sw128<(RC < 8 ? RC : 8)>(sout + C::NB * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr));
+            if constexpr (RC > 8)
+              park_sw128<RC - 8>(sout + (C::NB + 1) * C::BLK, pr, reinterpret_cast<const uint32_t*>(qr) + 64);
+          }
           fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
           tc_fence_before();
           __syncwarp();
@@ -550,33 +558,54 @@ __global__ void __launch_bounds__(QPrepCfg<DL, DR>::THREADS, 1)
 // Persistent over (sample, 128-row tile, head) items, head fastest so that the
 // CTAs working at one time share the latent tile in L2.  Per item the
 // reduction over d_latent runs through a ring of [128 rows x 64] latent blocks
-// and [224 x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
+// and [(d_nope + 128) x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
 // two TMEM accumulators alternate so the epilogue of one item overlaps the
 // next; two epilogue warpgroups park the item's 128 rows as [k_h (128) | v_h
-// (128)] bf16 -- the first k_h (content columns from TMEM, the positional part
-// read one item ahead), the second v_h -- and all 256 threads write each row's
-// two 256-byte runs out contiguously.
-template <int DL>
+// (128)] bf16 -- the first k_h (d_nope content columns from TMEM, the d_rope
+// positional columns read one item ahead), the second v_h -- and all 256 threads
+// write each row's two 256-byte runs out contiguously.
+__device__ __forceinline__ bool m_valid(int mt, int r, int rows) { return mt * 128 + r < rows; }
+
+template <int DL, int DR>
 struct ReconCfg {
+  static constexpr int DN = 128 - DR;        // content dims of a head's key
+  static constexpr int N = DN + 128;         // MMA N: [W_uk,h ; W_uv,h] rows
   static constexpr int NKB = DL / 64;
   static constexpr int A_BLK = 128 * 128;  // 128 latent rows x 64 cols
-  static constexpr int B_BLK = 224 * 128;  // [96 rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
+  static constexpr int B_BLK = N * 128;    // [d_nope rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
   static constexpr int STAGE = A_BLK + B_BLK;
   static constexpr int OUT_STRIDE = 256 * 2 + 16;  // parked row [k_h | v_h]: an odd number of 16-byte chunks
   static constexpr int OUT_BYTES = 128 * OUT_STRIDE;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
-  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of 224 columns, at 0 and 256
+  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of N columns, at 0 and 256
   static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 128 * 8 + 256;
   static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 two epilogue warpgroups
+  static_assert(DR == 16 || DR == 32 || DR == 64 || DR == 96, "rotary dims");
+  static_assert(N % 16 == 0 && N <= 256 && (DN * 128) % 1024 == 0, "MMA shape / swizzle atoms");
   static_assert(DL % 64 == 0 && STAGES >= 3 && SMEM <= 227 * 1024 && SMEM > 116 * 1024, "does not fit");
 };
 
-template <int DL>
-__global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
+// 16 floats as bf16 (or fp16) into 32 bytes of shared memory (16-byte aligned); amax tracks the
+// largest magnitude stored
+template <bool F16>
+__device__ __forceinline__ void store_x16_smem(uint8_t* dst, const float* v, float& amax) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  auto pk = [](float lo, float hi) { return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi); };
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[8 * q + k]));
+    d[q] = make_uint4(pk(v[8 * q + 0], v[8 * q + 1]), pk(v[8 * q + 2], v[8 * q + 3]), pk(v[8 * q + 4], v[8 * q + 5]),
+                      pk(v[8 * q + 6], v[8 * q + 7]));
+  }
+}
+
+template <int DL, int DR, bool F16>
+__global__ void __launch_bounds__(ReconCfg<DL, DR>::THREADS, 1)
     recon_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wuk,
                     const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a, int items) {
-  using C = ReconCfg<DL>;
+  using C = ReconCfg<DL, DR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sout = smem + C::STAGES * C::STAGE;
@@ -623,7 +652,7 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
           mbar_arrive_expect_tx(&full[s], C::STAGE);
           tma_load_3d(st, &tm_c, &full[s], kb * 64, mt * 128, b);
           tma_load_3d(st + C::A_BLK, &tm_wuk, &full[s], kb * 64, 0, h);
-          tma_load_3d(st + C::A_BLK + 96 * 128, &tm_wuv, &full[s], kb * 64, 0, h);
+          tma_load_3d(st + C::A_BLK + C::DN * 128, &tm_wuv, &full[s], kb * 64, 0, h);
         }
       }
       if (*abort_flag)
@@ -633,7 +662,7 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 224, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, false, false);
       int it = 0, j = 0;
       for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
         const int acc = j & 1;
@@ -666,15 +695,17 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
-    // warpgroup 0 reads each item's positional keys (64 bytes of its row) one item ahead
-    uint4 krq[4] = {};
+    // warpgroup 0 reads each item's positional keys (DR * 2 bytes of its row) one item ahead
+    constexpr int RQ = DR / 8;  // 16-byte pieces of a positional key
+    uint4 krq[RQ] = {};
     auto load_kr = [&](int item) {
       const int mt_ = (item / a.n_heads) % m_tiles, b_ = item / (a.n_heads * m_tiles);
       const int m_ = mt_ * 128 + r;
       if (m_ < a.rows) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.kr + ((int64_t)b_ * a.kr_rows + m_) * a.kr_stride);
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kr) +
+                                                          ((int64_t)b_ * a.kr_rows + m_) * a.kr_stride);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) krq[k] = src[k];
+        for (int k = 0; k < RQ; ++k) krq[k] = src[k];
       }
     };
     if (wg == 0 && (int)blockIdx.x < items) load_kr(blockIdx.x);
@@ -682,7 +713,7 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
       const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
       const int acc = j & 1;
-      float kr[32];
+      float kr[DR];
       if (wg == 0) {
         const int m = mt * 128 + r;
         const int mm = m < a.rows ? m : 0;
@@ -691,42 +722,48 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
         const int64_t row = a.to_ring ? ring_frame_slot(a.ring, frame) * T + tok : mm;
         row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < RQ; ++k) {
           const uint32_t w4[4] = {krq[k].x, krq[k].y, krq[k].z, krq[k].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
-            kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+            if constexpr (F16) {  // fp16 pairs (the workspace's window keys)
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
+              kr[8 * k + 2 * e] = f.x;
+              kr[8 * k + 2 * e + 1] = f.y;
+            } else {
+              kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+              kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+            }
           }
         }
         if (item + (int)gridDim.x < items) load_kr(item + gridDim.x);
-        if (a.rotate) rotate16(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
+        if (a.rotate) rotate_pairs<DR / 2>(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
       }
       const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();
       tc_fence_after();
       const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
       uint8_t* orow = sout + r * C::OUT_STRIDE;
-      if (wg == 0) {  // TMEM columns 0..95: the content part of k_h, then its positional part
+      float amax = 0.f;
+      if (wg == 0) {  // TMEM columns 0..DN-1: the content part of k_h, then its positional part
 #pragma unroll 1
-        for (int c0 = 0; c0 < 96; c0 += 32) {
-          uint32_t raw[32];
-          tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-          float v[32];
-          raw_to_float(raw, v);
-          store_bf16x32_smem(orow + c0 * 2, v);
+        for (int c0 = 0; c0 < C::DN; c0 += 16) {
+          uint32_t raw[16];
+          tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+          store_x16_smem<F16>(orow + c0 * 2, reinterpret_cast<const float*>(raw), amax);
         }
-        store_bf16x32_smem(orow + 96 * 2, kr);
-      } else {  // TMEM columns 96..223: v_h, parked from column 128
+#pragma unroll
+        for (int c0 = 0; c0 < DR; c0 += 16) store_x16_smem<F16>(orow + (C::DN + c0) * 2, kr + c0, amax);
+      } else {  // TMEM columns DN..DN+127: v_h, parked from column 128 (16-column loads: DN is a multiple of 16)
 #pragma unroll 1
-        for (int c0 = 96; c0 < 224; c0 += 32) {
-          uint32_t raw[32];
-          tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-          float v[32];
-          raw_to_float(raw, v);
-          store_bf16x32_smem(orow + (c0 + 32) * 2, v);
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+          uint32_t raw[16];
+          tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
+          store_x16_smem<F16>(orow + (128 + c0) * 2, reinterpret_cast<const float*>(raw), amax);
         }
       }
+      // fp16 holds magnitudes up to 65504: a row past it is reported, not stored as inf silently
+      if (F16 && m_valid(mt, r, a.rows) && !(amax <= 65504.f)) atomicOr(a.err, DEV_ERR_RANGE);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
@@ -734,8 +771,8 @@ __global__ void __launch_bounds__(ReconCfg<DL>::THREADS, 1)
 #pragma unroll 4
       for (int id = tid; id < valid_rows * 32; id += 256) {
         const int rr = id >> 5, ch = id & 31;
-        __nv_bfloat16* dst =
-            a.dense + row_k[rr] + (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
+        uint16_t* dst = static_cast<uint16_t*>(a.dense) + row_k[rr] +
+                        (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
       }
       named_bar_sync(1, 256);  // the park is written out before it is reused
@@ -922,28 +959,29 @@ __global__ void fold_weights_kernel(const __nv_bfloat16* w_o, const __nv_bfloat1
 // 64-column blocks through a ring; the positional columns are rotated at the queries' positions
 // in the epilogue, which parks the rows as 64-column blocks in the 128-byte swizzled layout and
 // writes them with TMA tensor stores, clipped at the last query.
-template <int DL>
+template <int DL, int DR>
 struct QLatCfg {
-  static constexpr int N = DL + 32;
+  static constexpr int N = DL + DR;        // [A_h ; W_qr,h] rows: the MMA's N
   static constexpr int A_BLK = 128 * 128;
   static constexpr int B_BLK = N * 128;
   static constexpr int STAGE = A_BLK + B_BLK;
-  static constexpr int NCB = DL / 64 + 1;  // 64-column blocks of a row (the last one half used)
-  static constexpr int BLK = 128 * 128;    // one parked column block of 128 rows
+  static constexpr int NCB = (N + 63) / 64;  // 64-column blocks of a row (the last one partly used)
+  static constexpr int BLK = 128 * 128;      // one parked column block of 128 rows
   static constexpr int OUT_BYTES = NCB * BLK;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int SMEM_USED = 1024 + STAGES * STAGE + OUT_BYTES + 256;
   static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
+  static_assert(DR % 16 == 0 && DR <= 96 && DL % 64 == 0, "rotary dims");
   static_assert(N % 16 == 0 && N <= 256 && B_BLK % 1024 == 0 && STAGES >= 2 && SMEM <= 227 * 1024, "bad d_latent");
 };
 
-template <int DL>
+template <int DL, int DR>
 __global__ void __launch_bounds__(kThreads, 1)
     qlat_tc_kernel(const __grid_constant__ CUtensorMap tm_cq, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_out, const QLatTc a, int items) {
-  using C = QLatCfg<DL>;
+  using C = QLatCfg<DL, DR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sout = smem + C::STAGES * C::STAGE;
@@ -1052,12 +1090,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         park_sw128<8>(sout + cb * C::BLK, r, raw);
       }
       {
-        uint32_t raw[32];
-        tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + DL), raw);
-        float v[32];
-        raw_to_float(raw, v);
-        rotate16(v, a.rope, t, hh, ww);  // the 32 positional columns
-        park_sw128<4>(sout + (DL / 64) * C::BLK, r, reinterpret_cast<const uint32_t*>(v));
+        float v[DR];  // the DR positional columns, rotated; parked 8 chunks of 8 per column block
+#pragma unroll
+        for (int c0 = 0; c0 < DR; c0 += 16) tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + DL + c0),
+                                                       *reinterpret_cast<uint32_t(*)[16]>(v + c0));
+        rotate_pairs<DR / 2>(v, a.rope, t, hh, ww);
+        constexpr int RC = DR / 8;
+        park_sw128<(RC < 8 ? RC : 8)>(sout + (DL / 64) * C::BLK, r, reinterpret_cast<const uint32_t*>(v));
+        if constexpr (RC > 8)
+          park_sw128<RC - 8>(sout + (DL / 64 + 1) * C::BLK, r, reinterpret_cast<const uint32_t*>(v) + 64);
       }
       fence_async_smem();
       tc_fence_before();
@@ -1167,11 +1208,11 @@ cudaError_t go_qprep_dl(const CUtensorMap& tq, const CUtensorMap& tw, const CUte
   return cudaErrorInvalidValue;
 }
 
-template <int DL>
+template <int DL, int DR, bool F16>
 cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
                      int batch, cudaStream_t s) {
-  using C = ReconCfg<DL>;
-  static const cudaError_t attr = set_smem(recon_tc_kernel<DL>, C::SMEM);
+  using C = ReconCfg<DL, DR>;
+  static const cudaError_t attr = set_smem(recon_tc_kernel<DL, DR, F16>, C::SMEM);
   if (attr != cudaSuccess) return attr;
   static int sms = 0;
   if (sms == 0) {
@@ -1180,8 +1221,32 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.rows + 127) / 128) * a.n_heads * batch;
-  recon_tc_kernel<DL><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tc, tuk, tuv, a, items);
+  recon_tc_kernel<DL, DR, F16><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tc, tuk, tuv, a, items);
   return cudaGetLastError();
+}
+
+template <int DR, bool F16>
+cudaError_t go_recon_dl(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
+                        int batch, cudaStream_t s) {
+  switch (a.d_latent) {
+    case 64: return go_recon<64, DR, F16>(tc, tuk, tuv, a, batch, s);
+    case 128: return go_recon<128, DR, F16>(tc, tuk, tuv, a, batch, s);
+    case 192: return go_recon<192, DR, F16>(tc, tuk, tuv, a, batch, s);
+    case 256: return go_recon<256, DR, F16>(tc, tuk, tuv, a, batch, s);
+    case 384:
+      if constexpr (DR == 32) return go_recon<384, DR, F16>(tc, tuk, tuv, a, batch, s);
+      break;
+    case 512:
+      if constexpr (DR == 32) return go_recon<512, DR, F16>(tc, tuk, tuv, a, batch, s);
+      break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int DR>
+cudaError_t go_recon_t(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
+                       int batch, cudaStream_t s) {
+  return a.f16 ? go_recon_dl<DR, true>(tc, tuk, tuv, a, batch, s) : go_recon_dl<DR, false>(tc, tuk, tuv, a, batch, s);
 }
 
 }  // namespace
@@ -1212,35 +1277,53 @@ cudaError_t launch_fold_weights(const __nv_bfloat16* w_o, const __nv_bfloat16* w
   return cudaGetLastError();
 }
 
-template <int DL>
+template <int DL, int DR>
 cudaError_t go_qlat(const CUtensorMap& tc, const CUtensorMap& tw, const CUtensorMap& to, const QLatTc& a, int batch,
                     cudaStream_t s) {
-  using C = QLatCfg<DL>;
-  static const cudaError_t attr = set_smem(qlat_tc_kernel<DL>, C::SMEM);
-  if (attr != cudaSuccess) return attr;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if constexpr (DL + DR > 256) {
+    return cudaErrorInvalidValue;
+  } else {
+    using C = QLatCfg<DL, DR>;
+    static const cudaError_t attr = set_smem(qlat_tc_kernel<DL, DR>, C::SMEM);
+    if (attr != cudaSuccess) return attr;
+    static int sms = 0;
+    if (sms == 0) {
+      int dev = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
+    qlat_tc_kernel<DL, DR><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tw, to, a, items);
+    return cudaGetLastError();
   }
-  const int items = ((a.n_q + 127) / 128) * a.n_heads * batch;
-  qlat_tc_kernel<DL><<<std::min(items, sms), kThreads, C::SMEM, s>>>(tc, tw, to, a, items);
-  return cudaGetLastError();
 }
 
-bool qlat_supported(int d_latent, int d_q) {
-  return (d_latent == 64 || d_latent == 128 || d_latent == 192) && d_q > 0 && d_q % 64 == 0;
+template <int DR>
+cudaError_t go_qlat_dl(const CUtensorMap& tc, const CUtensorMap& tw, const CUtensorMap& to, const QLatTc& a,
+                       int batch, cudaStream_t s) {
+  switch (a.d_latent) {
+    case 64: return go_qlat<64, DR>(tc, tw, to, a, batch, s);
+    case 128: return go_qlat<128, DR>(tc, tw, to, a, batch, s);
+    case 192: return go_qlat<192, DR>(tc, tw, to, a, batch, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+bool qlat_supported(int d_latent, int d_rope, int d_q) {
+  return (d_latent == 64 || d_latent == 128 || d_latent == 192) &&
+         (d_rope == 16 || d_rope == 32 || d_rope == 64 || d_rope == 96) && d_latent + d_rope <= 256 && d_q > 0 &&
+         d_q % 64 == 0;
 }
 
 cudaError_t launch_qlat_tc(const CUtensorMap& tc, const CUtensorMap& tw, const CUtensorMap& to, const QLatTc& a,
                            int batch, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
-  if (!qlat_supported(a.d_latent, a.d_q)) return cudaErrorInvalidValue;
-  switch (a.d_latent) {
-    case 64: return go_qlat<64>(tc, tw, to, a, batch, s);
-    case 128: return go_qlat<128>(tc, tw, to, a, batch, s);
-    case 192: return go_qlat<192>(tc, tw, to, a, batch, s);
+  if (!qlat_supported(a.d_latent, a.d_rope, a.d_q)) return cudaErrorInvalidValue;
+  switch (a.d_rope) {
+    case 16: return go_qlat_dl<16>(tc, tw, to, a, batch, s);
+    case 32: return go_qlat_dl<32>(tc, tw, to, a, batch, s);
+    case 64: return go_qlat_dl<64>(tc, tw, to, a, batch, s);
+    case 96: return go_qlat_dl<96>(tc, tw, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1285,6 +1368,8 @@ cudaError_t launch_append_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
     case 128: return go_append<128>(tx, tw, a, batch, s, p);  // d_rope 64
     case 192: return go_append<192>(tx, tw, a, batch, s, p);
     case 256: return go_append<256>(tx, tw, a, batch, s, p);
+    case 320: return go_append<320>(tx, tw, a, batch, s, p);
+    case 352: return go_append<352>(tx, tw, a, batch, s, p);  // d_rope 96 (160, 224, 288 above)
   }
   return cudaErrorInvalidValue;
 }
@@ -1296,6 +1381,7 @@ cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const 
     case 16: return go_qprep_dl<16>(tq, tw, to, a, batch, s);
     case 32: return go_qprep_dl<32>(tq, tw, to, a, batch, s);
     case 64: return go_qprep_dl<64>(tq, tw, to, a, batch, s);
+    case 96: return go_qprep_dl<96>(tq, tw, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1303,13 +1389,11 @@ cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const 
 cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
                             int batch, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
-  switch (a.d_latent) {
-    case 64: return go_recon<64>(tc, tuk, tuv, a, batch, s);
-    case 128: return go_recon<128>(tc, tuk, tuv, a, batch, s);
-    case 192: return go_recon<192>(tc, tuk, tuv, a, batch, s);
-    case 256: return go_recon<256>(tc, tuk, tuv, a, batch, s);
-    case 384: return go_recon<384>(tc, tuk, tuv, a, batch, s);
-    case 512: return go_recon<512>(tc, tuk, tuv, a, batch, s);
+  switch (a.d_rope) {
+    case 16: return go_recon_t<16>(tc, tuk, tuv, a, batch, s);
+    case 32: return go_recon_t<32>(tc, tuk, tuv, a, batch, s);
+    case 64: return go_recon_t<64>(tc, tuk, tuv, a, batch, s);
+    case 96: return go_recon_t<96>(tc, tuk, tuv, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

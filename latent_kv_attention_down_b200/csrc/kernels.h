@@ -19,6 +19,7 @@ enum DeviceError : unsigned {
   DEV_ERR_TIMEOUT_EPILOGUE = 1u << 3,
   DEV_ERR_TIMEOUT_SELFTEST = 1u << 4,
   DEV_ERR_BOUNDS = 1u << 5,
+  DEV_ERR_RANGE = 1u << 6,  // a value past the range of its storage type (fp16 per-head operands)
 };
 constexpr unsigned DEV_ERR_BOUNDS_MASK = DEV_ERR_BOUNDS;
 
@@ -67,12 +68,14 @@ struct SimtAppend {
 cudaError_t launch_append_simt(const SimtAppend& a, cudaStream_t s);
 
 struct RopeWindow {  // rotate the window's positional keys with window-relative t
-  const void* kr;    // [B][W*T_f][d_r]
-  void* kr_rot;      // [B][W*T_f][d_r]
+  const void* kr;    // [B][W*T_f][d_r]  (bf16 path: bf16)
+  void* kr_rot;      // [B][W*T_f][d_r]  (bf16 path: bf16, or fp16 with out_f16)
   int batch, n_keys, d_rope;
   int window_start_slot;  // (ring slot of the oldest local frame) - sink_frames
   Ring ring;
   Rope rope;
+  int rotate = 1;    // bf16 path: 0 only converts (keys rotated at append)
+  int out_f16 = 0;   // bf16 path: write fp16 (the per-head keys of reconstruct-once)
 };
 cudaError_t launch_rope_window_f32(const RopeWindow& a, cudaStream_t s);
 cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s);
@@ -158,20 +161,20 @@ struct QPrepTc {
 cudaError_t launch_qprep_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_wuk, const CUtensorMap& tm_out,
                             const QPrepTc& a, int batch, cudaStream_t s);
 
-// Query-latent absorption: qt [B][n_h][n_q][d_c + 32] = [A_h ; W_qr,h] c_Q, positional part
+// Query-latent absorption: qt [B][n_h][n_q][d_c + d_rope] = [A_h ; W_qr,h] c_Q, positional part
 // rotated at the query positions.  c_Q map: 3D (d_q, n_q, B) box (64,128,1) SW128; weight map:
-// 3D (d_q, d_c + 32, n_h) box (64, d_c + 32, 1) SW128; out map as for launch_qprep_tc.
-// d_latent 64, 128 or 192; d_q % 64 == 0.
+// 3D (d_q, d_c + d_rope, n_h) box (64, d_c + d_rope, 1) SW128; out map as for launch_qprep_tc.
+// d_latent 64, 128 or 192, d_rope 16, 32, 64 or 96 with d_latent + d_rope <= 256; d_q % 64 == 0.
 struct QLatTc {
   __nv_bfloat16* qt;
-  int n_q, n_heads, d_latent, d_q;
+  int n_q, n_heads, d_latent, d_rope, d_q;
   int64_t t_first;
   Ring ring;
   Rope rope;
   unsigned* err;
   uint64_t limit_ns;
 };
-bool qlat_supported(int d_latent, int d_q);
+bool qlat_supported(int d_latent, int d_rope, int d_q);
 cudaError_t launch_qlat_tc(const CUtensorMap& tm_cq, const CUtensorMap& tm_w, const CUtensorMap& tm_out,
                            const QLatTc& a, int batch, cudaStream_t s);
 // w_qabs [n_h][d_c + d_rope][d_q] = [W_uk,h^T W_uq,h ; W_qr,h]
@@ -191,8 +194,8 @@ struct AttnTc {
 // Absorbed design.  qt maps: 3D (d_c+32, n_q, B*n_h): latent box (64,128,1) SW128, rope box (32,128,1) SW64;
 // ckv map: 3D (d_c, n_keys, B) box (64,BN,1) SW128; kr map: 3D (32, n_keys, B) box (32,BN,1) SW64;
 // w_uv map: 3D (d_c, 128, n_h) box (64,128,1) SW128; out map: 3D (n_h*128, n_q, B) box (64,128,1) SW128.
-// d_rope 16, 32 or 64 (64 up to d_latent 192): tm_qr / tm_kr boxes are d_rope wide, swizzled at
-// d_rope * 2 bytes (32B, 64B or 128B)
+// d_rope 16, 32, 64 or 96 (64 and 96 up to d_latent 192): tm_qr / tm_kr boxes are d_rope wide, swizzled
+// at d_rope * 2 bytes (32B, 64B or 128B), except for 96: boxes 32 wide, SW64 (three loads per tile)
 bool attn_absorbed_supported(int d_latent, int d_rope);
 cudaError_t launch_attn_absorbed_tc(int d_latent, int d_rope, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
                                     const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr, const CUtensorMap& tm_wuv,
@@ -202,7 +205,7 @@ int attn_absorbed_block_n(int d_latent);  // keys per tile (TMA box rows of the 
 // Absorbed attention that stores O_bar = softmax-weighted latents / l (per head, d_c wide) as a
 // bf16 pair instead of applying W_uv,h: maps 3D (n_h*d_c, n_q, B) bf16 box (64,128,1) SW128 for
 // the rounded part (tob_hi) and the residual (tob_lo).
-cudaError_t launch_attn_absorbed_obar_tc(int d_latent, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
+cudaError_t launch_attn_absorbed_obar_tc(int d_latent, int d_rope, const CUtensorMap& tm_q, const CUtensorMap& tm_qr,
                                          const CUtensorMap& tm_ckv, const CUtensorMap& tm_kr,
                                          const CUtensorMap& tob_hi, const CUtensorMap& tob_lo, const AttnTc& a,
                                          int batch, cudaStream_t s);
@@ -232,23 +235,28 @@ int attn_dense_block_n();
 
 // Dense per-head attention, d_head = 128.  q map: 3D (128, n_q, B*n_h) box (64,128,1);
 // kv map: 3D (2*n_h*128, n_keys, B) box (64,128,1); out: 3D fp32 (n_h*128, n_q, B) box (32,128,1) SW128.
+// f16: q and kv hold fp16 (the reconstruct-once workspace) instead of bf16 (the dense cache).
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_out,
-                                 const AttnTc& a, int batch, cudaStream_t s);
+                                 const AttnTc& a, int batch, cudaStream_t s, bool f16);
 
 struct DenseQTc {  // q' = [q_nope | RoPE(q_rope)] -> [B][n_h][n_q][128]
   const __nv_bfloat16* q;
-  __nv_bfloat16* qd;
-  int batch, n_q, n_heads;
+  void* qd;                         // bf16, or fp16 when f16
+  int batch, n_q, n_heads, d_rope;  // d_rope a multiple of 8: the last d_rope of a head's 128 dims
   int64_t t_first;
   Ring ring;
   Rope rope;
+  int f16 = 0;            // write fp16 (DEV_ERR_RANGE in *err for a value past 65504)
+  unsigned* err = nullptr;
 };
 cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s);
 
 struct ReconTc {  // per-head dense entries from latents (tcgen05)
-  const __nv_bfloat16* kr;  // positional keys [B][rows_per_sample][32] (rotated iff !rotate)
-  __nv_bfloat16* dense;     // [B][ring_rows][2][n_h][128]
-  int rows, n_heads, d_latent;
+  const void* kr;           // positional keys [B][rows_per_sample][d_rope] (rotated iff !rotate): bf16, or
+                            // (f16) the fp16 window keys of the workspace
+  void* dense;              // [B][ring_rows][2][n_h][128], bf16 or (f16) fp16
+  int f16;                  // fp16 entries (DEV_ERR_RANGE for a value past 65504)
+  int rows, n_heads, d_latent, d_rope;  // d_rope 16, 32, 64 or 96 (d_nope = 128 - d_rope)
   int64_t first_frame;      // frame of row 0 (ring placement and absolute t)
   int rotate;               // rotate kr with the absolute frame index
   int to_ring;              // 1: row m -> ring slot of its frame; 0: row m -> row m
@@ -260,7 +268,7 @@ struct ReconTc {  // per-head dense entries from latents (tcgen05)
   unsigned* err;
   uint64_t limit_ns;
 };
-// c map: 3D (d_c, rows, B) box (64,128,1) SW128; w_uk map: 3D (d_c, 96, n_h) box (64,96,1);
+// c map: 3D (d_c, rows, B) box (64,128,1) SW128; w_uk map: 3D (d_c, d_nope, n_h) box (64,d_nope,1);
 // w_uv map: 3D (d_c, 128, n_h) box (64,128,1)
 cudaError_t launch_recon_tc(const CUtensorMap& tm_c, const CUtensorMap& tm_wuk, const CUtensorMap& tm_wuv,
                             const ReconTc& a, int batch, cudaStream_t s);

@@ -63,8 +63,8 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   if (!aligned16(ckv) || !aligned16(kr) || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
   const int64_t F = frames_appended;
-  if (c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;  // absorbed kernels: up to 256 latent dims
-  if (c.d_rope != 32) return VMLA_ERR_UNSUPPORTED_SHAPE;    // the 96/32 split
+  // the absorbed kernels: up to 256 latent dims, up to 192 with 64 or 96 rotary dims
+  if (!attn_absorbed_supported(c.d_latent, c.d_rope)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   if (n_frames < 1 || n_frames > c.chunk_frames) return VMLA_ERR_OUT_OF_RANGE;
   if (F < 1 || first_frame < 0 || first_frame + n_frames != F) return VMLA_ERR_STATE;
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
@@ -76,8 +76,8 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   const Window win = window_of(c, F);
   const int n_keys = win.n_keys;
   const int nq = (int)(n_frames * T);
-  const int dqk = c.d_latent + 32;
-  const size_t kr_rot_bytes = at_read ? align256((size_t)c.batch * rr * 32 * 2) : 0;
+  const int dqk = c.d_latent + c.d_rope;
+  const size_t kr_rot_bytes = at_read ? align256((size_t)c.batch * rr * c.d_rope * 2) : 0;
   const size_t qt_bytes = (size_t)c.batch * c.n_heads * nq * dqk * 2;
   if (kr_rot_bytes + qt_bytes > kNoallocScratchBytes) return VMLA_ERR_OUT_OF_RANGE;
 
@@ -92,22 +92,22 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
 
   const size_t layer_rows = (size_t)layer * c.batch * rr;
   const __nv_bfloat16* ckv_layer = static_cast<const __nv_bfloat16*>(ckv) + layer_rows * c.d_latent;
-  const __nv_bfloat16* kr_layer = static_cast<const __nv_bfloat16*>(kr) + layer_rows * 32;
-  __nv_bfloat16* kr_rot = static_cast<__nv_bfloat16*>(scratch);
+  const __nv_bfloat16* kr_layer = static_cast<const __nv_bfloat16*>(kr) + layer_rows * c.d_rope;
+  void* kr_rot = scratch;  // the window's positional keys rotated for this call (bf16)
   __nv_bfloat16* qt = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(scratch) + kr_rot_bytes);
 
-  const __nv_bfloat16* kpos = kr_layer;
+  const void* kpos = kr_layer;
   if (at_read) {
-    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, 32, win.start_slot, ring, rope};
+    RopeWindow r{kr_layer, kr_rot, c.batch, n_keys, c.d_rope, win.start_slot, ring, rope};
     if (launch_rope_window_bf16(r, s) != cudaSuccess) return VMLA_ERR_CUDA;
     kpos = kr_rot;
   }
-  const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B, SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
   CUtensorMap tq, tuk, tqt;
   if (!map3(&tq, q, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 256, (uint64_t)nq * c.n_heads * 256,
                 64, 128, SW128) ||
-      !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
-                SW128) ||
+      !map3(&tuk, w_uk, c.d_latent, c.d_nope, c.n_heads, (uint64_t)c.d_latent * 2,
+            (uint64_t)c.d_nope * c.d_latent * 2, 64, c.d_nope, SW128) ||
       !map3(&tqt, qt, dqk, nq, (uint64_t)c.batch * c.n_heads, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 64,
                 SW128))
     return VMLA_ERR_CUDA;
@@ -126,13 +126,18 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   if (launch_qprep_tc(tq, tuk, tqt, qa, c.batch, s) != cudaSuccess) return VMLA_ERR_CUDA;
 
   const int bn = attn_absorbed_block_n(c.d_latent);
+  // the rotary columns: one box d_rope wide swizzled at its row width, or three boxes of 32 for 96
+  const int rbox = c.d_rope == 96 ? 32 : c.d_rope;
+  const CUtensorMapSwizzle rsw = rbox == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                            : (rbox == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
   const uint64_t bh = (uint64_t)c.batch * c.n_heads;
   CUtensorMap mq, mqr, mk, mkr, muv, mo;
   if (!map3(&mq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, SW128) ||
-      !map3(&mqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 32, 128, SW64) ||
+      !map3(&mqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, rbox, 128, rsw) ||
       !map3(&mk, ckv_layer, c.d_latent, n_keys, c.batch, (uint64_t)c.d_latent * 2, (uint64_t)rr * c.d_latent * 2,
                 64, bn, SW128) ||
-      !map3(&mkr, kpos, 32, n_keys, c.batch, 64, (uint64_t)rr * 64, 32, bn, SW64) ||
+      !map3(&mkr, kpos, c.d_rope, n_keys, c.batch, (uint64_t)c.d_rope * 2, (uint64_t)rr * c.d_rope * 2, rbox, bn,
+            rsw) ||
       !map3(&muv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
                 SW128) ||
       !map3(&mo, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 512,
@@ -147,6 +152,7 @@ extern "C" vmla_status vmla_chunk_attention_noalloc(const vmla_config* cfg, int 
   a.rescale_threshold = c.softmax_rescale_log2;
   a.err = err;
   a.limit_ns = kWaitLimitNs;
-  return launch_attn_absorbed_tc(c.d_latent, 32, mq, mqr, mk, mkr, muv, mo, a, c.batch, s) == cudaSuccess ? VMLA_OK
-                                                                                                      : VMLA_ERR_CUDA;
+  return launch_attn_absorbed_tc(c.d_latent, c.d_rope, mq, mqr, mk, mkr, muv, mo, a, c.batch, s) == cudaSuccess
+             ? VMLA_OK
+             : VMLA_ERR_CUDA;
 }

@@ -1,9 +1,13 @@
 // 3D-RoPE kernels of the bf16 path [paperlayer App. C.1, App. D.3, App. D.5]:
 //  * rope_window_bf16: rotate every positional key of the window with its
-//    window-relative (t, h, w) into the workspace.  HBM-bound: each thread
-//    moves one 16-byte vector (4 rotary pairs) in and out, fully coalesced.
+//    window-relative (t, h, w) into the workspace (bf16, or fp16 for the per-head
+//    keys of reconstruct-once).  HBM-bound: each thread moves one 16-byte vector
+//    (4 rotary pairs) in and out, fully coalesced.
 //  * dense_q_bf16: the dense path's query [q_nope | RoPE(q_rope)], re-laid out
-//    head-major for the attention kernel's TMA tiles.
+//    head-major for the attention kernel's TMA tiles, in bf16 (the dense cache) or fp16 (the
+//    reconstruct-once workspace).
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "rope.cuh"
 
@@ -30,8 +34,17 @@ __device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, int t,
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 // d_rope / 8 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its slot in
-// every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.
+// every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.  The stored
+// bf16 keys are rotated (or, when they were rotated at append, only converted) and written as bf16,
+// or as fp16 for the per-head keys of reconstruct-once: one rounding of 2^-11 relative there, where
+// a second bf16 rounding would add 2^-8.
 __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int nq = a.d_rope >> 3;  // 16-byte pieces of a key
@@ -44,7 +57,7 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   const int hh = tok / a.ring.grid_w, ww = tok % a.ring.grid_w;
   float2 cs[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) cs[k] = rope_cs(a.rope, quad * 4 + k, t, hh, ww);
+  for (int k = 0; k < 4; ++k) cs[k] = a.rotate ? rope_cs(a.rope, quad * 4 + k, t, hh, ww) : make_float2(1.f, 0.f);
   const uint4* src =
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * a.d_rope + quad * 8);
   uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * a.d_rope + quad * 8);
@@ -64,14 +77,15 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
       for (int p = 0; p < 4; ++p) {
         float u = bf_lo(in[p]), x = bf_hi(in[p]);
         rope_apply(u, x, cs[p]);
-        out[p] = pack2(u, x);
+        out[p] = a.out_f16 ? pack_h2(u, x) : pack2(u, x);
       }
       dst[(b0 + k) * stride] = make_uint4(out[0], out[1], out[2], out[3]);
     }
   }
 }
 
-// 16 threads per (sample, query, head): 12 copy the content dims, 4 rotate the positional ones
+// 16 threads per (sample, query, head), 8 dims each: those of the content dims copy them, those
+// of the positional dims (the last d_rope of the 128) rotate them
 __global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
@@ -81,14 +95,33 @@ __global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
   const int i = ((idx >> 4) / a.n_heads) % a.n_q;
   const int b = (idx >> 4) / ((int64_t)a.n_heads * a.n_q);
   const __nv_bfloat16* src = a.q + (((int64_t)b * a.n_q + i) * a.n_heads + h) * 128 + chunk * 8;
-  __nv_bfloat16* dst = a.qd + (((int64_t)b * a.n_heads + h) * a.n_q + i) * 128 + chunk * 8;
+  const int64_t dst = (((int64_t)b * a.n_heads + h) * a.n_q + i) * 128 + chunk * 8;  // element offset
   uint4 v = *reinterpret_cast<const uint4*>(src);
-  if (chunk >= 12) {
-    const int tok = i % a.ring.tokens_per_frame;
-    const int t = (int)(a.t_first + i / a.ring.tokens_per_frame);
-    v = rotate4(v, a.rope, (chunk - 12) * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
+  const int first_rope_chunk = (128 - a.d_rope) >> 3;
+  const bool rope = chunk >= first_rope_chunk;
+  const int tok = i % a.ring.tokens_per_frame;
+  const int t = (int)(a.t_first + i / a.ring.tokens_per_frame);
+  if (!a.f16) {
+    if (rope) v = rotate4(v, a.rope, (chunk - first_rope_chunk) * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.qd) + dst) = v;
+    return;
   }
-  *reinterpret_cast<uint4*>(dst) = v;
+  // fp16 out: the content dims converted (exact for bf16 values in fp16's range), the positional
+  // ones rotated in fp32 and rounded once
+  uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float u = bf_lo(in[k]), x = bf_hi(in[k]);
+    if (rope) rope_apply(u, x, rope_cs(a.rope, (chunk - first_rope_chunk) * 4 + k, t, tok / a.ring.grid_w,
+                                       tok % a.ring.grid_w));
+    amax = fmaxf(amax, fmaxf(fabsf(u), fabsf(x)));
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x), "f"(u));
+    out[k] = d;
+  }
+  if (!(amax <= 65504.f)) atomicOr(a.err, DEV_ERR_RANGE);
+  *reinterpret_cast<uint4*>(static_cast<__half*>(a.qd) + dst) = make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 }  // namespace
@@ -102,6 +135,7 @@ cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s) {
+  if (a.d_rope <= 0 || a.d_rope > 128 || a.d_rope % 8 != 0 || (a.f16 && !a.err)) return cudaErrorInvalidValue;
   const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
   if (total == 0) return cudaSuccess;
   dense_q_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);

@@ -169,25 +169,20 @@ vmla_status map_fail() {
 vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : cuda_fail(e); }
 
 // AUTO keeps the design measured fastest on one B200 that also meets the accuracy gate (relative
-// L2 <= 1e-2, max |err| <= 3e-2 RMS against the fp64 definition) for the call's window:
-//  - d_latent > 256: RECON_ONCE (the absorbed tile holds at most 256 latent columns);
-//  - d_latent 192 or 256 and a window of at least kReconOnceMinKeys keys: RECON_ONCE.  Per (query,
-//    key, head) the per-head attention multiplies 2 d_head = 256 pairs where the absorbed one
-//    multiplies 2 d_latent + d_rope (416 at 192), and rebuilding the window's per-head K/V costs
-//    about 2 us per 1000 keys (Wan-1.3B layer: 0.91 ms against 1.05 ms per call).  Per-head K and V
-//    are rounded to bf16 key by key, which over a short window can put the worst output element
-//    past the max-error gate (3.4e-2 RMS at 600 keys); from a few thousand keys on it averages out.
-//  - otherwise ABSORBED: at d_latent <= 128 its extra MMA work is no larger than the
-//    reconstruction's, and it meets the gate at every window length up to 192.
-// The 112/16 and 64/64 content/rotary splits run on the absorbed design only.
-constexpr int kReconOnceMinKeys = 4096;
-
+// L2 <= 1e-2, max |err| <= 3e-2 RMS against the fp64 definition):
+//  - d_latent >= 192, or a split the absorbed kernel does not hold (past 256 latent dims; 64 or 96
+//    rotary dims past 192): RECON_ONCE.  Per (query, key, head) the per-head attention multiplies
+//    2 d_head = 256 pairs where the absorbed one multiplies 2 d_latent + d_rope (416 at 192), and
+//    rebuilding the window's per-head K/V costs about 2 us per 1000 keys (Wan-1.3B layer: 0.91 ms
+//    against 1.05 ms per call).  Its per-head K, V, queries and probabilities are fp16, which keeps
+//    it inside the gate on every window, the shortest (600 keys) included;
+//  - d_latent 64 or 128: ABSORBED, whose extra MMA work is then no larger than the reconstruction's
+//    (0.83 / 0.87 ms against 0.92 ms per call at the Wan layer).
 vmla_design resolve_design(const vmla_config& c, vmla_design d, int64_t n_keys) {
+  (void)n_keys;
   if (d != VMLA_DESIGN_AUTO) return d;
   if (c.dtype != VMLA_BF16) return VMLA_DESIGN_ABSORBED;
-  if (c.d_rope != 32) return VMLA_DESIGN_ABSORBED;  // the only bf16 design there
-  if (c.d_latent > 256) return VMLA_DESIGN_RECON_ONCE;
-  if (c.d_latent >= 192 && n_keys >= kReconOnceMinKeys) return VMLA_DESIGN_RECON_ONCE;
+  if (!attn_absorbed_supported(c.d_latent, c.d_rope) || c.d_latent >= 192) return VMLA_DESIGN_RECON_ONCE;
   return VMLA_DESIGN_ABSORBED;
 }
 
@@ -311,6 +306,7 @@ const char* vmla_status_string(vmla_status s) {
     case VMLA_ERR_DEVICE_TIMEOUT: return "VMLA_ERR_DEVICE_TIMEOUT";
     case VMLA_ERR_STATE: return "VMLA_ERR_STATE";
     case VMLA_ERR_DEVICE_BOUNDS: return "VMLA_ERR_DEVICE_BOUNDS";
+    case VMLA_ERR_DEVICE_RANGE: return "VMLA_ERR_DEVICE_RANGE";
   }
   return "VMLA_ERR_UNKNOWN";
 }
@@ -364,11 +360,12 @@ vmla_status vmla_config_check(const vmla_config* c) {
   if (c->d_value != c->d_nope + c->d_rope) return VMLA_ERR_UNSUPPORTED_SHAPE;  // dense layout [2][n_h][d_head]
   if (c->grid_h >= kMaxPos || c->grid_w >= kMaxPos || c->window_frames >= kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
   if (c->dtype == VMLA_BF16) {
-    // d_head 128 split 96/32 (every design), or 112/16 and 64/64 (the absorbed design)
+    // d_head 128 split 96/32 with d_latent 64..512, or 112/16, 64/64, 32/96 with d_latent 64..256
     if (c->d_value != 128 || c->d_nope + c->d_rope != 128) return VMLA_ERR_UNSUPPORTED_SHAPE;
-    if (c->d_rope != 32 && !attn_absorbed_supported(c->d_latent, c->d_rope)) return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (!(c->d_latent == 64 || c->d_latent == 128 || c->d_latent == 192 || c->d_latent == 256 || c->d_latent == 384 ||
           c->d_latent == 512))
+      return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_rope != 32 && !((c->d_rope == 16 || c->d_rope == 64 || c->d_rope == 96) && c->d_latent <= 256))
       return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (c->d_model % 64 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
   } else {
@@ -460,7 +457,6 @@ vmla_status vmla_dense_bind(vmla_handle* h, void* dense) {
   if (!h || !dense || !aligned16(dense)) return VMLA_ERR_INVALID_ARG;
   // the dense layout stores keys rotated at absolute positions: no window-relative re-indexing
   if (h->cfg.sink_frames > 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
-  if (h->cfg.dtype == VMLA_BF16 && h->cfg.d_rope != 32) return VMLA_ERR_UNSUPPORTED_SHAPE;  // 96/32 split only
   h->dense = dense;
   h->dense_frames.assign(h->cfg.layers, 0);
   return VMLA_OK;
@@ -642,7 +638,17 @@ struct HostOut {
   cudaStream_t stream;
   cudaEvent_t group, done;
   bool copied;
+  cudaEvent_t q_read = nullptr;  // recorded once the query-prep kernel has read q (its last reader)
+  bool q_recorded = false;
 };
+
+// Record hout->q_read right after the kernel that last reads q.
+cudaError_t note_q_read(HostOut* hout, cudaStream_t s) {
+  if (!hout || !hout->q_read) return cudaSuccess;
+  cudaError_t e = cudaEventRecord(hout->q_read, s);
+  hout->q_recorded = e == cudaSuccess;
+  return e;
+}
 
 // Launch an attention kernel (grid y = heads) as one launch per group of heads that fills the GPU
 // once, each group's output columns copied to the host on hout->stream while the next group
@@ -678,7 +684,7 @@ cudaError_t launch_head_groups(const vmla_config& c, int nq, AttnTc a, const voi
 }
 
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const void* kv_base, void* out, int nq,
-                                        int n_keys, int64_t t_first, int stage, cudaStream_t s,
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, bool f16,
                                         HostOut* hout = nullptr);
 
 // The folded output mixer: out = O_bar W_fold^T instead of the per-head W_uv,h.
@@ -699,22 +705,29 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
                            const FoldArgs* fold = nullptr, const QLatArgs* qlat = nullptr, HostOut* hout = nullptr) {
   const vmla_config& c = h->cfg;
   if (design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent)) return VMLA_ERR_UNSUPPORTED_SHAPE;
-  // rotary widths other than 32: the absorbed design with W_uv in its epilogue only
-  if (c.d_rope != 32 && (design != VMLA_DESIGN_ABSORBED || fold || qlat)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  // rotary widths other than 32: every design but reconstruct-in-tile
+  if (c.d_rope != 32 && design == VMLA_DESIGN_RECONSTRUCT) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (design == VMLA_DESIGN_ABSORBED && !attn_absorbed_supported(c.d_latent, c.d_rope)) return VMLA_ERR_UNSUPPORTED_SHAPE;
   const WsLayout w = ws_layout(c);
   const bool at_read = c.rope_mode == VMLA_ROPE_AT_READ;
   const int nq = (int)(n * tokens_per_frame(c));
   const int64_t t_first = first - (at_read ? win.t_origin : 0);
   __nv_bfloat16* ckv_layer = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
   __nv_bfloat16* kr_layer = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
-  const __nv_bfloat16* kpos = kr_layer;
+  // the window's positional keys, rotated with window-relative t into the workspace; reconstruct-once
+  // takes them in fp16 (converted there too when they were rotated at append: its per-head keys are
+  // fp16), the other designs in bf16 (the cache's own values when rotated at append)
+  const bool kr_f16 = design == VMLA_DESIGN_RECON_ONCE;
+  const void* kpos = kr_layer;
   cudaError_t e = cudaSuccess;
-  if (at_read) {
+  if (at_read || kr_f16) {
     StageScope scope(h, 1, s);
-    RopeWindow r{kr_layer, at<__nv_bfloat16>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
+    RopeWindow r{kr_layer, at<char>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
                  make_ring(c), make_rope(c)};
+    r.rotate = at_read;
+    r.out_f16 = kr_f16;
     e = launch_rope_window_bf16(r, s);
-    kpos = at<__nv_bfloat16>(h->ws, w.kr_rot);
+    kpos = at<char>(h->ws, w.kr_rot);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   const uint64_t rr = ring_rows(c);
@@ -727,7 +740,8 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       CUtensorMap tc, tuk, tuv;
       if (!map3(&tc, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64,
                 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+          !map3(&tuk, w_uk, c.d_latent, c.d_nope, c.n_heads, (uint64_t)c.d_latent * 2,
+                (uint64_t)c.d_nope * c.d_latent * 2, 64, c.d_nope,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B))
@@ -735,14 +749,16 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       ReconTc a;
       a.kr = kpos;
       a.dense = recon;
+      a.f16 = 1;  // the window's per-head K/V in fp16: 2^-11 rounding per entry, past bf16's 2^-8
       a.rows = win.n_keys;
       a.n_heads = c.n_heads;
       a.d_latent = c.d_latent;
+      a.d_rope = c.d_rope;
       a.first_frame = 0;
       a.rotate = 0;  // positional keys are already rotated (at read into the workspace, or at append)
       a.to_ring = 0;
       a.kr_rows = rr;
-      a.kr_stride = 32;
+      a.kr_stride = c.d_rope;
       a.ring_rows = rr;
       a.ring = make_ring(c);
       a.rope = make_rope(c);
@@ -751,13 +767,13 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       e = launch_recon_tc(tc, tuk, tuv, a, c.batch, s);
     }
     if (e != cudaSuccess) return cuda_fail(e);
-    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, hout);
+    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, true, hout);
   }
   if (design == VMLA_DESIGN_RECONSTRUCT) {
     __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
     {
       StageScope scope(h, 2, s);
-      DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, t_first, make_ring(c),
+      DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, c.d_rope, t_first, make_ring(c),
                  make_rope(c)};
       e = launch_dense_q_bf16(a, s);
     }
@@ -769,7 +785,8 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
         !map3(&tc, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tkr, kpos, 32, win.n_keys, c.batch, 64, rr * 64, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+        !map3(&tuk, w_uk, c.d_latent, c.d_nope, c.n_heads, (uint64_t)c.d_latent * 2,
+              (uint64_t)c.d_nope * c.d_latent * 2, 64, c.d_nope,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -806,6 +823,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.n_q = nq;
     a.n_heads = c.n_heads;
     a.d_latent = c.d_latent;
+    a.d_rope = c.d_rope;
     a.d_q = qlat->d_q;
     a.t_first = t_first;
     a.ring = make_ring(c);
@@ -837,6 +855,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     a.limit_ns = kWaitLimitNs;
     e = launch_qprep_tc(tq, tuk, tqt, a, c.batch, s);
   }
+  if (e == cudaSuccess) e = note_q_read(hout, s);
   if (e != cudaSuccess) return cuda_fail(e);
   {
     StageScope scope(h, 3, s);
@@ -844,14 +863,16 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     const uint64_t bh = (uint64_t)c.batch * c.n_heads;
     CUtensorMap tq, tqr, tk, tkr, tuv, to;
     // the rotary columns: one box c.d_rope wide, swizzled at its row width (32, 64 or 128 bytes)
-    const CUtensorMapSwizzle rsw = c.d_rope == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                                  : (c.d_rope == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    // (96 rotary dims: three boxes of 32, 64-byte swizzle)
+    const int rbox = c.d_rope == 96 ? 32 : c.d_rope;
+    const CUtensorMapSwizzle rsw = rbox == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                              : (rbox == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     const uint64_t rb = (uint64_t)c.d_rope * 2;
     if (!map3(&tq, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, c.d_rope, 128, rsw) ||
+        !map3(&tqr, qt, dqk, nq, bh, (uint64_t)dqk * 2, (uint64_t)nq * dqk * 2, rbox, 128, rsw) ||
         !map3(&tk, ckv_layer, c.d_latent, win.n_keys, c.batch, (uint64_t)c.d_latent * 2, rr * c.d_latent * 2, 64, bn,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tkr, kpos, c.d_rope, win.n_keys, c.batch, rb, rr * rb, c.d_rope, bn, rsw))
+        !map3(&tkr, kpos, c.d_rope, win.n_keys, c.batch, rb, rr * rb, rbox, bn, rsw))
       return map_fail();
     if (!fold &&
         (!map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
@@ -883,7 +904,7 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       if (!map3(&thi, ob_hi, kf, nq, c.batch, kf * 2, (uint64_t)nq * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3(&tlo, ob_lo, kf, nq, c.batch, kf * 2, (uint64_t)nq * kf * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return map_fail();
-      e = launch_attn_absorbed_obar_tc(c.d_latent, tq, tqr, tk, tkr, thi, tlo, a, c.batch, s);
+      e = launch_attn_absorbed_obar_tc(c.d_latent, c.d_rope, tq, tqr, tk, tkr, thi, tlo, a, c.batch, s);
     }
   }
   if (e != cudaSuccess || !fold) return cuda_status(e);
@@ -903,28 +924,34 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   return cuda_status(launch_fold_gemm_tc(thi, tlo, tw, to, fa, s));
 }
 
-// Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128].
+// Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128]: bf16 (the
+// dense cache) or, with f16, fp16 (the reconstruct-once workspace; the queries then go fp16 too).
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const void* kv_base, void* out, int nq,
-                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, HostOut* hout) {
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, bool f16,
+                                        HostOut* hout) {
   const vmla_config& c = h->cfg;
   const WsLayout w = ws_layout(c);
-  __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
+  void* qd = at<char>(h->ws, w.dq);
   cudaError_t e;
   {
     StageScope scope(h, 2, s);
-    DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, t_first, make_ring(c),
+    DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, c.d_rope, t_first, make_ring(c),
                make_rope(c)};
+    a.f16 = f16;
+    a.err = h->err;
     e = launch_dense_q_bf16(a, s);
   }
+  if (e == cudaSuccess) e = note_q_read(hout, s);
   if (e != cudaSuccess) return cuda_fail(e);
   StageScope scope(h, stage, s);
   const uint64_t rr = ring_rows(c);
   const uint64_t row_bytes = 2ull * c.n_heads * 128 * 2;
   CUtensorMap tq, tkv, to;
+  const CUtensorMapDataType et = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!map3(&tq, qd, 128, nq, (uint64_t)c.batch * c.n_heads, 256, (uint64_t)nq * 256, 64, 128,
-            CU_TENSOR_MAP_SWIZZLE_128B) ||
+            CU_TENSOR_MAP_SWIZZLE_128B, et) ||
       !map3(&tkv, kv_base, 2ull * c.n_heads * 128, n_keys, c.batch, row_bytes, rr * row_bytes, 64,
-            attn_dense_block_n(), CU_TENSOR_MAP_SWIZZLE_128B) ||
+            attn_dense_block_n(), CU_TENSOR_MAP_SWIZZLE_128B, et) ||
       !map3(&to, out, (uint64_t)c.n_heads * 128, nq, c.batch, (uint64_t)c.n_heads * 128 * 4,
             (uint64_t)nq * c.n_heads * 128 * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
     return map_fail();
@@ -939,9 +966,9 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
   a.limit_ns = kWaitLimitNs;
   if (hout)
     return cuda_status(launch_head_groups(c, nq, a, out, hout, s, [&](const AttnTc& ag) {
-      return launch_attn_dense_tc(tq, tkv, to, ag, c.batch, s);
+      return launch_attn_dense_tc(tq, tkv, to, ag, c.batch, s, f16);
     }));
-  return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s));
+  return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s, f16));
 }
 
 }  // namespace
@@ -970,7 +997,9 @@ vmla_status attention_args(vmla_handle* h, int layer, const void* q, const void*
     if (*design == VMLA_DESIGN_ABSORBED && c.d_latent > 256) return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (*design == VMLA_DESIGN_RECONSTRUCT && !attn_reconstruct_supported(c.d_latent))
       return VMLA_ERR_UNSUPPORTED_SHAPE;
-    if (c.d_rope != 32 && *design != VMLA_DESIGN_ABSORBED) return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (*design == VMLA_DESIGN_ABSORBED && !attn_absorbed_supported(c.d_latent, c.d_rope))
+      return VMLA_ERR_UNSUPPORTED_SHAPE;
+    if (c.d_rope != 32 && *design == VMLA_DESIGN_RECONSTRUCT) return VMLA_ERR_UNSUPPORTED_SHAPE;
     if (*design == VMLA_DESIGN_RECON_ONCE) {
       const WsLayout w = ws_layout(c);
       if (h->ws_bytes < w.base_bytes + w.recon_bytes) return VMLA_ERR_STATE;
@@ -1001,7 +1030,7 @@ vmla_status vmla_fold_query_weights(const vmla_config* cfg, const void* w_uq, co
   if (!cfg || !w_uq || !w_qr || !w_uk || !w_qabs) return VMLA_ERR_INVALID_ARG;
   vmla_status st = vmla_config_check(cfg);
   if (st != VMLA_OK) return st;
-  if (cfg->dtype != VMLA_BF16 || cfg->d_rope != 32 || !qlat_supported(cfg->d_latent, d_q))
+  if (cfg->dtype != VMLA_BF16 || !qlat_supported(cfg->d_latent, cfg->d_rope, d_q))
     return VMLA_ERR_UNSUPPORTED_SHAPE;
   return cuda_status(launch_fold_query(static_cast<const __nv_bfloat16*>(w_uq), static_cast<const __nv_bfloat16*>(w_qr),
                                        static_cast<const __nv_bfloat16*>(w_uk), static_cast<__nv_bfloat16*>(w_qabs),
@@ -1018,7 +1047,8 @@ vmla_status vmla_chunk_attention_qlatent(vmla_handle* h, int layer, const void* 
       !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
   const vmla_config& c = h->cfg;
-  if (c.dtype != VMLA_BF16 || c.d_rope != 32 || !qlat_supported(c.d_latent, d_q)) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (c.dtype != VMLA_BF16 || !qlat_supported(c.d_latent, c.d_rope, d_q) || !attn_absorbed_supported(c.d_latent, c.d_rope))
+    return VMLA_ERR_UNSUPPORTED_SHAPE;
   Window win;
   if ((st = check_attention_frames(c, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
   if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
@@ -1050,7 +1080,8 @@ vmla_status vmla_chunk_attention_folded(vmla_handle* h, int layer, const void* q
   if (!q || !w_uk || !w_fold || !out || !aligned16(q) || !aligned16(w_uk) || !aligned16(w_fold) || !aligned16(out))
     return VMLA_ERR_INVALID_ARG;
   const vmla_config& c = h->cfg;
-  if (c.dtype != VMLA_BF16 || c.d_latent > 256 || d_out < 128 || d_out % 128 != 0) return VMLA_ERR_UNSUPPORTED_SHAPE;
+  if (c.dtype != VMLA_BF16 || !attn_absorbed_supported(c.d_latent, c.d_rope) || d_out < 128 || d_out % 128 != 0)
+    return VMLA_ERR_UNSUPPORTED_SHAPE;
   Window win;
   if ((st = check_attention_frames(c, h->frames[layer], first, n, &win)) != VMLA_OK) return st;
   if (c.rope_mode == VMLA_ROPE_AT_APPEND && first + n > kMaxPos) return VMLA_ERR_OUT_OF_RANGE;
@@ -1133,17 +1164,20 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     CUtensorMap tc, tuk, tuv;
     if (!map3(&tc, chunk, c.d_latent, rows, c.batch, (uint64_t)nout * 2, (uint64_t)rows * nout * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map3(&tuk, w_uk, c.d_latent, 96, c.n_heads, (uint64_t)c.d_latent * 2, 96ull * c.d_latent * 2, 64, 96,
+        !map3(&tuk, w_uk, c.d_latent, c.d_nope, c.n_heads, (uint64_t)c.d_latent * 2,
+              (uint64_t)c.d_nope * c.d_latent * 2, 64, c.d_nope,
               CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map3(&tuv, w_uv, c.d_latent, 128, c.n_heads, (uint64_t)c.d_latent * 2, 128ull * c.d_latent * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B))
       return map_fail();
     ReconTc r;
+    r.f16 = 0;  // the dense comparison caches bf16 entries
     r.kr = chunk + c.d_latent;  // positional key columns of the chunk rows (row stride d_c + 32)
     r.dense = at<__nv_bfloat16>(h->dense, dense_off);
     r.rows = rows;
     r.n_heads = c.n_heads;
     r.d_latent = c.d_latent;
+    r.d_rope = c.d_rope;
     r.first_frame = first;
     r.rotate = 1;
     r.to_ring = 1;
@@ -1177,7 +1211,7 @@ vmla_status vmla_dense_chunk_attention(vmla_handle* h, int layer, const void* q,
   const int nq = (int)(n * tokens_per_frame(c));
   const size_t dense_off = (size_t)layer * c.batch * ring_rows(c) * 2 * c.n_heads * c.d_value * esize(c);
   if (c.dtype == VMLA_BF16)
-    return dense_attention_bf16_launch(h, q, at<char>(h->dense, dense_off), out, nq, win.n_keys, first, 6, s);
+    return dense_attention_bf16_launch(h, q, at<char>(h->dense, dense_off), out, nq, win.n_keys, first, 6, s, false);
   cudaError_t e;
   {
     StageScope scope(h, 2, s);
@@ -1248,10 +1282,12 @@ vmla_status vmla_chunk_step_host(vmla_handle* h, int layer, const void* x_host, 
   if ((st = vmla_cache_append(h, layer, x_dev, w_down, first, n, stream)) != VMLA_OK) return st;
   if ((e = cudaEventRecord(h->x_free, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s, h->q_ready, 0)) != cudaSuccess)
     return cuda_fail(e);
-  HostOut hout{out_host, h->out_stream, h->out_group, h->out_done, false};
+  // q_free is recorded as soon as the query-prep kernel has read q_dev, so the next call's q copy
+  // overlaps this call's attention kernel
+  HostOut hout{out_host, h->out_stream, h->out_group, h->out_done, false, h->q_free, false};
   if ((st = chunk_attention(h, layer, q_dev, w_uk, w_uv, out_dev, first, n, design, stream, &hout)) != VMLA_OK)
     return st;
-  if ((e = cudaEventRecord(h->q_free, s)) != cudaSuccess) return cuda_fail(e);
+  if (!hout.q_recorded && (e = cudaEventRecord(h->q_free, s)) != cudaSuccess) return cuda_fail(e);
   // the host result is there when `stream` is: the absorbed attention copied it back a group of
   // heads at a time (and made `stream` wait for the last copy); other paths copy it here
   if (hout.copied) return VMLA_OK;
@@ -1270,6 +1306,7 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
   if (v && (e = cudaMemset(err, 0, sizeof(v))) != cudaSuccess) return cuda_fail(e);
   if (flags) *flags = v;
   if (v & DEV_ERR_BOUNDS_MASK) return VMLA_ERR_DEVICE_BOUNDS;
+  if (v & DEV_ERR_RANGE) return VMLA_ERR_DEVICE_RANGE;
   if (v) return VMLA_ERR_DEVICE_TIMEOUT;
   return VMLA_OK;
 }

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     lib = api.lib()
     assert lib.vmla_abi_version() == api.ABI_VERSION == 2
-    for code in range(8):
+    for code in range(9):
         assert lib.vmla_status_string(code).decode().startswith("VMLA_")
     assert lib.vmla_status_string(99).decode() == "VMLA_ERR_UNKNOWN"
 
@@ -99,18 +99,25 @@ def test_config_check_rejects(field, value, status):
 
 @pytest.mark.parametrize("d_nope,d_rope,pairs,d_latent,status", [
     (112, 16, (4, 2, 2), 192, 0), (112, 16, (4, 2, 2), 256, 0), (64, 64, (12, 10, 10), 192, 0),
-    (64, 64, (12, 10, 10), 64, 0), (64, 64, (12, 10, 10), 256, 2), (112, 16, (4, 2, 2), 384, 2),
-    (32, 96, (16, 16, 16), 128, 2),
+    (64, 64, (12, 10, 10), 64, 0), (64, 64, (12, 10, 10), 256, 0), (32, 96, (16, 16, 16), 128, 0),
+    (32, 96, (16, 16, 16), 256, 0), (112, 16, (4, 2, 2), 384, 2), (32, 96, (16, 16, 16), 512, 2),
+    (80, 48, (8, 8, 8), 192, 2),
 ])
 def test_bf16_rotary_splits(d_nope, d_rope, pairs, d_latent, status):
-    """d_head 128 split 112/16 and 64/64 run on the absorbed tensor-core design (64/64 up to
-    d_latent 192); 32/96 and the wider latents of those splits are refused as unsupported."""
+    """d_head 128 split 112/16, 64/64 and 32/96 on the tensor-core path with d_latent up to 256 (the
+    absorbed kernel up to 192 for 64 and 96 rotary dims); wider latents of those splits and other
+    splits are refused as unsupported.  AUTO's workspace holds reconstruct-once's per-head K/V
+    exactly when the full window would take it: from 192 latent dims on, or where the absorbed
+    kernel does not take the split."""
     c = default_config()
     c.d_nope, c.d_rope, c.d_latent = d_nope, d_rope, d_latent
     c.rope_pairs[:] = list(pairs)
     assert api.lib().vmla_config_check(ctypes.byref(c)) == status
-    if status == 0:  # the automatic design is the absorbed one: no per-head K/V in the workspace
-        assert api.workspace_bytes(c, api.DESIGN_AUTO) == api.workspace_bytes(c, api.DESIGN_ABSORBED)
+    if status == 0:
+        recon = d_latent >= 192
+        auto, absorbed = api.workspace_bytes(c, api.DESIGN_AUTO), api.workspace_bytes(c, api.DESIGN_ABSORBED)
+        assert (auto > absorbed) == recon
+        assert auto == api.workspace_bytes(c, api.DESIGN_RECON_ONCE if recon else api.DESIGN_ABSORBED)
 
 
 def test_fp32_accepts_small_shapes():

@@ -158,21 +158,16 @@ def test_small_bf16_latent_width(d_latent):
     assert_bf16_close(out[0], ro.oracle(0, 7, q), f"d_latent {d_latent}")
 
 
-def test_small_bf16_absorbed_at_latent_256():
-    """The absorbed design is still exact up to rounding at d_latent = 256, but
-    its bf16 query (W_uk^T q_nope, rounded once per row and reused against
-    every key) adds a coherent score error on top of the bf16 cache: an fp64
-    emulation of this rounding chain on these inputs gives max |err| = 3.4e-2
-    RMS (cache rounding alone: 1.8e-2).  Held to relative L2 <= 1e-2 and
-    max |err| <= 5e-2 RMS; AUTO uses reconstruct-once at this width."""
-    import numpy as np
-    from tests.harness import rel_l2
+@pytest.mark.parametrize("chunks", [1, 3, pytest.param(8, marks=pytest.mark.xfail(
+    strict=True, reason="fails the max-error gate (3.4e-2 RMS): the absorbed query's bf16 rounding at 256 "
+                        "latent dims; AUTO takes reconstruct-once there"))])
+def test_small_bf16_absorbed_at_latent_256(chunks):
+    """The absorbed design at d_latent = 256 (its bf16 query, one rounding per row reused against
+    every key, adds a coherent score error to the cache's) on short, mid and full windows."""
     ro = Rollout(SMALL.replace(name="small_dc256", d_latent=256), design=api.DESIGN_ABSORBED)
-    _fill(ro, 8)
-    out, q = ro.attend(0, 7, design=api.DESIGN_ABSORBED)
-    ref = ro.oracle(0, 7, q)
-    assert rel_l2(out[0], ref) <= 1e-2
-    assert np.max(np.abs(out[0] - ref)) <= 5e-2 * np.sqrt(np.mean(ref ** 2))
+    _fill(ro, chunks)
+    out, q = ro.attend(0, chunks - 1, design=api.DESIGN_ABSORBED)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"absorbed d_c 256, {chunks} chunks")
 
 
 def test_small_bf16_batch_and_layers():
@@ -187,18 +182,23 @@ def test_small_bf16_batch_and_layers():
             assert_bf16_close(out[b], ro.oracle(layer, 7, q, b), f"layer {layer} sample {b}")
 
 
-@pytest.mark.parametrize("chunks", [1, 7, 10])
+# Per-head designs that round each key's K_h and V_h to bf16 (reconstruct-in-tile and the dense
+# comparison, whose cache is bf16 by definition) fail the max-error gate on the shortest window:
+# over 600 keys the per-key roundings do not average out (measured 4.55e-2 RMS on these inputs;
+# relative L2 2.8e-3 passes).  These cases are kept as strict expected failures at the gate, next
+# to the stage-wise checks that hold the same kernels to their own rounding bounds.
+SHORT_WINDOW_FAILS = pytest.mark.xfail(strict=True, reason="fails the max-error gate on a 600-key window: "
+                                                          "bf16 rounding of every key's per-head K and V")
+
+
+@pytest.mark.parametrize("chunks", [pytest.param(1, marks=SHORT_WINDOW_FAILS), 2, 7, 10])
 def test_small_bf16_reconstruct_in_tile(chunks):
     """Design (b): per-head K/V rebuilt from the latent tile on the tensor core
     inside the attention kernel; partial window, full window, wrapped ring."""
     ro = Rollout(SMALL)
     _fill(ro, chunks)
     out, q = ro.attend(0, chunks - 1, design=api.DESIGN_RECONSTRUCT)
-    # per-head K and V are rounded to bf16 key by key (as in the dense layout): over a
-    # 600-key window that rounding alone puts the worst element at ~3.4e-2 RMS (fp64
-    # emulation of the roundings on the same inputs); the relative L2 gate is unchanged
-    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"reconstruct, {chunks} chunks",
-                      max_abs=6e-2 if chunks == 1 else 3e-2)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"reconstruct, {chunks} chunks")
 
 
 @pytest.mark.parametrize("d_latent", [64, 128])
@@ -217,45 +217,123 @@ def test_small_bf16_reconstruct_in_tile_rope_at_append_and_rescale():
     assert_bf16_close(out[0], ro.oracle(0, 7, q), "reconstruct, rope at append, rescale every tile")
 
 
-def test_small_bf16_dense_designs_short_window():
-    """The per-head designs on a 600-key window next to design (b): the same
-    rounding of per-head K and V, the same widened max-abs term."""
-    ro = Rollout(SMALL, design=api.DESIGN_RECON_ONCE, dense=True)
-    ro.append_chunk(0, 0)
-    ro.append_chunk(0, 0, dense=True)
-    for design, dense in ((api.DESIGN_RECON_ONCE, False), (api.DESIGN_RECONSTRUCT, False), (None, True)):
-        out, q = ro.attend(0, 0, design=design or api.DESIGN_AUTO, dense=dense)
-        assert_bf16_close(out[0], ro.oracle(0, 0, q), f"design {design} dense {dense}", max_abs=6e-2)
+@pytest.mark.parametrize("design,dense", [(api.DESIGN_RECON_ONCE, False),
+                                          pytest.param(api.DESIGN_RECONSTRUCT, False, marks=SHORT_WINDOW_FAILS),
+                                          pytest.param(api.DESIGN_AUTO, True, marks=SHORT_WINDOW_FAILS)])
+def test_small_bf16_per_head_designs_short_window(design, dense):
+    """The per-head designs on a 600-key window (the first chunk): reconstruct-once, whose per-head
+    K, V, queries and probabilities are fp16, meets the gate; the bf16 per-head tiles of
+    reconstruct-in-tile and of the dense cache do not."""
+    ro = Rollout(SMALL, design=api.DESIGN_RECON_ONCE, dense=dense)
+    ro.append_chunk(0, 0, dense=dense)
+    out, q = ro.attend(0, 0, design=design, dense=dense)
+    assert_bf16_close(out[0], ro.oracle(0, 0, q), f"design {design} dense {dense}")
 
 
-@pytest.mark.parametrize("d_nope,d_rope,pairs,d_latent,chunks", [
-    (112, 16, (4, 2, 2), 192, 2), (112, 16, (4, 2, 2), 192, 10), (112, 16, (4, 2, 2), 64, 7),
-    (112, 16, (4, 2, 2), 256, 7), (64, 64, (12, 10, 10), 192, 2), (64, 64, (12, 10, 10), 192, 10),
-    (64, 64, (12, 10, 10), 128, 7),
-])
-def test_small_bf16_rotary_split_variants(d_nope, d_rope, pairs, d_latent, chunks):
-    """d_head 128 split 112/16 or 64/64 on the tensor-core path (absorbed design): the shared key
-    is d_latent + d_rope wide, its rotary block swizzled at d_rope * 2 bytes; short, full and
-    wrapped windows."""
-    d = SMALL.replace(name=f"wan_small_r{d_rope}_c{d_latent}", d_nope=d_nope, d_rope=d_rope, rope_pairs=pairs,
-                      d_latent=d_latent)
-    ro = Rollout(d)
-    _fill(ro, chunks)
-    out, q = ro.attend(0, chunks - 1)
-    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"{d_nope}/{d_rope}, d_c {d_latent}, {chunks} chunks")
+# content/rotary splits of a 128-dim head [paperlayer App. F]: 112/16, 96/32, 64/64, 32/96, with the
+# rotary pairs split over (t, h, w) as (4,2,2), (6,5,5), (12,10,10), (16,16,16)
+SPLITS = {16: (112, (4, 2, 2)), 64: (64, (12, 10, 10)), 96: (32, (16, 16, 16))}
 
 
-def test_rotary_split_other_designs_refused():
-    """Only the absorbed design runs the 112/16 split: the per-head designs and the dense cache
-    refuse it."""
-    d = SMALL.replace(name="wan_small_r16", d_nope=112, d_rope=16, rope_pairs=(4, 2, 2))
+def split_dims(base, d_rope, d_latent=192):
+    d_nope, pairs = SPLITS[d_rope]
+    return base.replace(name=f"{base.name}_r{d_rope}_c{d_latent}", d_nope=d_nope, d_rope=d_rope, rope_pairs=pairs,
+                        d_latent=d_latent)
+
+
+SPLIT_WINDOWS = [(192, 2), (192, 7), (192, 10), (64, 7), (128, 7), (256, 7)]
+
+
+def _split_rollout(d_rope, d_latent, chunks, dense):
+    d = split_dims(SMALL, d_rope, d_latent)
+    ro = Rollout(d, design=api.DESIGN_RECON_ONCE, dense=dense)
+    for c in range(chunks):
+        ro.append_chunk(0, c, dense=dense)
+    return d, ro
+
+
+@pytest.mark.parametrize("d_rope", [16, 64, 96])
+@pytest.mark.parametrize("d_latent,chunks", SPLIT_WINDOWS)
+def test_small_bf16_rotary_split_reconstruct_once_and_auto(d_rope, d_latent, chunks):
+    """Every content/rotary split through reconstruct-once (fp16 per-head operands) and through
+    the design AUTO takes: partial, full and wrapped windows, in full, at the gate."""
+    d, ro = _split_rollout(d_rope, d_latent, chunks, dense=False)
+    ref = None
+    for name, design in (("recon_once", api.DESIGN_RECON_ONCE), ("auto", api.DESIGN_AUTO)):
+        out, q = ro.attend(0, chunks - 1, design=design)
+        if ref is None:
+            ref = ro.oracle(0, chunks - 1, q)
+        assert_bf16_close(out[0], ref, f"{d.d_nope}/{d_rope}, d_c {d_latent}, {chunks} chunks, {name}")
+
+
+# Where the max-error gate fails for the designs that round per row or per key to bf16 (the absorbed
+# query q~; every key's per-head K and V in the dense cache), measured on these seeded inputs; the
+# stage-wise tests hold the same kernels to their own rounding bounds.
+def _gate_fails(reason):
+    return pytest.mark.xfail(strict=True, reason="fails the max-error gate: " + reason)
+
+
+DENSE_FAILS = {(64, 192, 2), (96, 192, 10)}
+
+
+@pytest.mark.parametrize("d_rope,d_latent,chunks", [
+    pytest.param(r, dl, ch, marks=_gate_fails("bf16 per-head cache entries") if (r, dl, ch) in DENSE_FAILS else ())
+    for r in (16, 64, 96) for dl, ch in SPLIT_WINDOWS])
+def test_small_bf16_rotary_split_dense_cache(d_rope, d_latent, chunks):
+    """The dense per-head cache (bf16 K/V per head and key) with every content/rotary split."""
+    d, ro = _split_rollout(d_rope, d_latent, chunks, dense=True)
+    out, q = ro.attend(0, chunks - 1, dense=True)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"{d.d_nope}/{d_rope}, d_c {d_latent}, {chunks}, dense")
+
+
+ABSORBED_FAILS = {(96, 192, 2), (96, 192, 10)}  # 3.2e-2 and 4.0e-2 RMS: 96 rotary dims leave 32 content dims
+
+
+@pytest.mark.parametrize("d_rope,d_latent,chunks", [
+    pytest.param(r, dl, ch, marks=_gate_fails("the absorbed query's bf16 rounding") if (r, dl, ch) in ABSORBED_FAILS
+                 else ())
+    for r in (16, 64, 96) for dl, ch in SPLIT_WINDOWS if r == 16 or dl <= 192])
+def test_small_bf16_rotary_split_absorbed(d_rope, d_latent, chunks):
+    """The absorbed kernel with every content/rotary split it takes (rotary blocks swizzled at their
+    width; 96 dims as three 32-column blocks; 64 and 96 up to d_latent 192)."""
+    d, ro = _split_rollout(d_rope, d_latent, chunks, dense=False)
+    out, q = ro.attend(0, chunks - 1, design=api.DESIGN_ABSORBED)
+    assert_bf16_close(out[0], ro.oracle(0, chunks - 1, q), f"{d.d_nope}/{d_rope}, d_c {d_latent}, {chunks}, absorbed")
+
+
+@pytest.mark.parametrize("d_rope", [16, 64, 96])
+def test_rotary_split_reconstruct_in_tile_refused(d_rope):
+    """Reconstruct-in-tile keeps the 96/32 split; the others return VMLA_ERR_UNSUPPORTED_SHAPE, and
+    the absorbed design refuses 64 and 96 rotary dims past d_latent 192."""
+    d = split_dims(SMALL, d_rope)
     ro = Rollout(d)
     _fill(ro, 1)
-    for design in (api.DESIGN_RECON_ONCE, api.DESIGN_RECONSTRUCT):
-        with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
-            ro.attend(0, 0, design=design)
     with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
-        Rollout(d, dense=True)
+        ro.attend(0, 0, design=api.DESIGN_RECONSTRUCT)
+    if d_rope != 16:
+        ro = Rollout(split_dims(SMALL, d_rope, 256))
+        _fill(ro, 1)
+        with pytest.raises(api.VmlaError, match="UNSUPPORTED"):
+            ro.attend(0, 0, design=api.DESIGN_ABSORBED)
+
+
+@pytest.mark.parametrize("d_rope", [16, 64, 96])
+def test_wan_layer_rotary_split_every_design(d_rope):
+    """The Wan-1.3B layer with each split (4680 queries over 32760 keys), 256 seeded rows of every
+    head, for the absorbed design, reconstruct-once (what AUTO takes) and the dense cache."""
+    d = split_dims(WAN, d_rope)
+    ro = Rollout(d, design=api.DESIGN_RECON_ONCE, dense=True)
+    for c in range(7):
+        ro.append_chunk(0, c)
+        ro.append_chunk(0, c, dense=True)
+    rows = sampled_rows(d.n_queries, 256, seed=d_rope)
+    ref = None
+    for name, design, dense in (("absorbed", api.DESIGN_ABSORBED, False), ("auto", api.DESIGN_AUTO, False),
+                                ("dense", api.DESIGN_AUTO, True)):
+        out, q = ro.attend(0, 6, design=design, dense=dense)
+        if ref is None:
+            ref = ro.oracle(0, 6, q, rows=rows)
+        assert_bf16_close(out[0][rows], ref, f"Wan layer {d.d_nope}/{d_rope}, {name}")
 
 
 def test_absorbed_rejects_latent_384():
@@ -472,13 +550,14 @@ def test_wide_grid_rotary_pairs_evaluated_directly():
 
 # ------------------------------------------------------------------ W_uv folded into the output mixer
 
-def test_small_bf16_folded_output_mixer():
+@pytest.mark.parametrize("d_rope", [32, 16, 64, 96])
+def test_small_bf16_folded_output_mixer(d_rope):
     """out = sum_h (W_O,h W_uv,h) o~_h through the library (weight fold, absorbed
     attention handing o~ over as a bf16 pair, one K = 12 x 192 GEMM) against W_O
-    applied to the oracle's per-head outputs."""
+    applied to the oracle's per-head outputs; every content/rotary split."""
     import torch
     import oracle.vmla_oracle as O
-    d = SMALL
+    d = SMALL if d_rope == 32 else split_dims(SMALL, d_rope)
     ro = Rollout(d)
     _fill(ro, 7)
     w = ro.w[0]
@@ -497,14 +576,15 @@ def test_small_bf16_folded_output_mixer():
 
 # ------------------------------------------------------------------ content path absorbed into the query latent
 
-@pytest.mark.parametrize("d_latent", [128, 192])
-def test_small_bf16_query_latent_absorption(d_latent):
+@pytest.mark.parametrize("d_latent,d_rope", [(128, 32), (192, 32), (192, 16), (192, 64), (128, 96)])
+def test_small_bf16_query_latent_absorption(d_latent, d_rope):
     """q~_h = [W_uk,h^T W_uq,h c_Q | RoPE(W_qr,h c_Q)] from the query latent (d_q = 768):
     the library's weight fold and K = 768 query GEMM, then the absorbed attention, against the
-    oracle's per-head queries W_uq,h c_Q, W_qr,h c_Q in the non-absorbed definition."""
+    oracle's per-head queries W_uq,h c_Q, W_qr,h c_Q in the non-absorbed definition; the splits
+    whose d_latent + d_rope fits one MMA (<= 256)."""
     import torch
     import oracle.vmla_oracle as O
-    d = SMALL.replace(d_latent=d_latent)
+    d = SMALL.replace(d_latent=d_latent) if d_rope == 32 else split_dims(SMALL, d_rope, d_latent)
     ro = Rollout(d)
     _fill(ro, 7)
     w_uq, w_qr = synth.query_latent_weights(d, 0)
@@ -534,29 +614,41 @@ def test_tiny_fp32_sink_window():
         assert_fp32_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk}")
 
 
-@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE, api.DESIGN_RECONSTRUCT])
-def test_small_bf16_sink_window_rolling(design):
+@pytest.mark.parametrize("design,first", [(api.DESIGN_ABSORBED, 0), (api.DESIGN_RECON_ONCE, 0),
+                                          (api.DESIGN_RECONSTRUCT, 1)])
+def test_small_bf16_sink_window_rolling(design, first):
     """The long-horizon context of the pages (one sink frame + six recent frames,
     window-relative RoPE) over 9 chunks of 3 frames: the sink stays, the local
-    frames rotate, positions stay within 0..6; every chunk checked in full."""
+    frames rotate, positions stay within 0..6; every chunk checked in full (from the second
+    for reconstruct-in-tile, whose first 600-key window is the strict expected failure below)."""
     d = synth.WAN_SMALL_SINK
     ro = Rollout(d, design=api.DESIGN_RECON_ONCE)
     for chunk in range(9):
         ro.append_chunk(0, chunk)
         out, q = ro.attend(0, chunk, design=design)
-        # per-head bf16 K/V on the 600-key first window: see test_small_bf16_dense_designs_short_window
-        loose = design != api.DESIGN_ABSORBED and chunk == 0
-        assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk}", max_abs=6e-2 if loose else 3e-2)
+        if chunk >= first:
+            assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk}")
+
+
+@SHORT_WINDOW_FAILS
+def test_small_bf16_sink_window_first_chunk_reconstruct_in_tile():
+    d = synth.WAN_SMALL_SINK
+    ro = Rollout(d)
+    ro.append_chunk(0, 0)
+    out, q = ro.attend(0, 0, design=api.DESIGN_RECONSTRUCT)
+    assert_bf16_close(out[0], ro.oracle(0, 0, q), "sink chunk 0, reconstruct-in-tile")
 
 
 def test_small_bf16_sink_window_passes_and_noalloc():
+    """Two denoising passes per chunk on the sink window (absorbed design), then the allocation-free
+    entry point on the same window: equal bit for bit."""
     import torch
     d = synth.WAN_SMALL_SINK
     ro = Rollout(d)
     for chunk in range(5):
         for p in range(2):
             ro.append_chunk(0, chunk, pass_=p)
-            out, q = ro.attend(0, chunk, pass_=p)
+            out, q = ro.attend(0, chunk, pass_=p, design=api.DESIGN_ABSORBED)
             assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk} pass {p}")
     qd = to_dev(q, d)
     out2 = torch.empty_like(torch.from_numpy(out)).cuda()
@@ -566,6 +658,21 @@ def test_small_bf16_sink_window_passes_and_noalloc():
               "noalloc")
     assert ro.m.device_status()[0] == 0
     assert torch.equal(out2.cpu(), torch.from_numpy(out)), "allocation-free path differs on the sink window"
+
+
+@pytest.mark.parametrize("chunk,pass_", [(0, 0), pytest.param(0, 1, marks=pytest.mark.xfail(
+    strict=True, reason="fails the max-error gate at the bf16 cache's own floor: on this 600-key window the "
+                        "cache rounding alone gives 2.8e-2 RMS (fp64 emulation), reconstruct-once 3.08e-2")),
+    (1, 1), (4, 1)])
+def test_small_bf16_sink_window_passes_reconstruct_once(chunk, pass_):
+    """Reconstruct-once (AUTO at d_latent 192) on the sink window's denoising passes."""
+    d = synth.WAN_SMALL_SINK
+    ro = Rollout(d)
+    for c in range(chunk + 1):
+        for p in range(2 if c < chunk else pass_ + 1):
+            ro.append_chunk(0, c, pass_=p)
+    out, q = ro.attend(0, chunk, pass_=pass_, design=api.DESIGN_RECON_ONCE)
+    assert_bf16_close(out[0], ro.oracle(0, chunk, q), f"sink chunk {chunk} pass {pass_}, reconstruct-once")
 
 
 # ------------------------------------------------------------------ numerics of the kernels' helpers

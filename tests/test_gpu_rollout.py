@@ -155,14 +155,7 @@ def test_wan_latent_width_sweep(d_latent):
     got["dense"] = out[0][rows]
     ref = ro.oracle(0, 6, q, rows=rows)
     for name, o in got.items():
-        if name == "absorbed" and d_latent >= 256:
-            # one bf16 rounding of the absorbed query is shared by every key of a
-            # row; at 256 latent dims that alone reaches ~3.4e-2 of RMS
-            rel = np.linalg.norm(o - ref) / np.linalg.norm(ref)
-            mx = np.max(np.abs(o - ref)) / np.sqrt(np.mean(ref ** 2))
-            assert rel <= 1e-2 and mx <= 5e-2, f"absorbed d_c={d_latent}: rel {rel:.3e} max {mx:.3e}"
-        else:
-            assert_bf16_close(o, ref, f"{name} d_c={d_latent}")
+        assert_bf16_close(o, ref, f"{name} d_c={d_latent}")
 
 
 def test_wan_sink_window_sampled_rows():

@@ -31,7 +31,11 @@ def _noalloc(ro, q, out, first, n, frames):
         w[2].data_ptr(), out.data_ptr(), first, n, torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("dims", [synth.WAN_SMALL, synth.WAN], ids=lambda d: d.name)
+SPLIT_64 = synth.WAN_SMALL.replace(name="wan_small_r64", d_nope=64, d_rope=64, rope_pairs=(12, 10, 10))
+SPLIT_96 = synth.WAN_SMALL.replace(name="wan_small_r96", d_nope=32, d_rope=96, rope_pairs=(16, 16, 16))
+
+
+@pytest.mark.parametrize("dims", [synth.WAN_SMALL, synth.WAN, SPLIT_64, SPLIT_96], ids=lambda d: d.name)
 def test_noalloc_matches_workspace_entry_point_twice(dims):
     """Both entry points launch the same kernels with the same arguments, so the outputs must be
     equal bit for bit, on two calls in a row (the second one reuses the array as the first left
