@@ -14,24 +14,14 @@
 namespace vmla {
 namespace {
 
+constexpr int kMaxHeads16 = 1024;  // threads of a per-head query block: 16 per head, up to 64 heads
+
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
-}
-
-// rotate the 4 pairs held in one 16-byte vector; first pair index p0
-__device__ __forceinline__ uint4 rotate4(uint4 v, const Rope& rp, int p0, int t, int h, int w) {
-  uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float u = bf_lo(in[k]), x = bf_hi(in[k]);
-    rope_apply(u, x, rope_cs(rp, p0 + k, t, h, w));
-    out[k] = pack2(u, x);
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -84,44 +74,44 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   }
 }
 
-// 16 threads per (sample, query, head), 8 dims each: those of the content dims copy them, those
-// of the positional dims (the last d_rope of the 128) rotate them
-__global__ void __launch_bounds__(256) dense_q_bf16_kernel(const DenseQTc a) {
-  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
-  if (idx >= total) return;
-  const int chunk = idx & 15;
-  const int h = (idx >> 4) % a.n_heads;
-  const int i = ((idx >> 4) / a.n_heads) % a.n_q;
-  const int b = (idx >> 4) / ((int64_t)a.n_heads * a.n_q);
-  const __nv_bfloat16* src = a.q + (((int64_t)b * a.n_q + i) * a.n_heads + h) * 128 + chunk * 8;
-  const int64_t dst = (((int64_t)b * a.n_heads + h) * a.n_q + i) * 128 + chunk * 8;  // element offset
-  uint4 v = *reinterpret_cast<const uint4*>(src);
-  const int first_rope_chunk = (128 - a.d_rope) >> 3;
-  const bool rope = chunk >= first_rope_chunk;
+// One block per (sample, query row): 16 threads per head, 8 dims each (n_heads * 16 threads).
+// Those of the content dims copy them, those of the positional dims (the last d_rope of the 128)
+// rotate them; the (cos, sin) of the row's rotary pairs are computed once for all heads.
+__global__ void __launch_bounds__(kMaxHeads16) dense_q_bf16_kernel(const DenseQTc a) {
+  __shared__ float2 cs[kMaxPairs];
+  const int row = blockIdx.x;  // b * n_q + i
+  const int i = row % a.n_q;
   const int tok = i % a.ring.tokens_per_frame;
   const int t = (int)(a.t_first + i / a.ring.tokens_per_frame);
-  if (!a.f16) {
-    if (rope) v = rotate4(v, a.rope, (chunk - first_rope_chunk) * 4, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.qd) + dst) = v;
-    return;
-  }
-  // fp16 out: the content dims converted (exact for bf16 values in fp16's range), the positional
-  // ones rotated in fp32 and rounded once
+  const int n_pairs = a.d_rope >> 1;
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x)
+    cs[p] = rope_cs(a.rope, p, t, tok / a.ring.grid_w, tok % a.ring.grid_w);
+  __syncthreads();
+  const int chunk = threadIdx.x & 15;
+  const int h = threadIdx.x >> 4;
+  if (h >= a.n_heads) return;
+  const int b = row / a.n_q;
+  const __nv_bfloat16* src = a.q + ((int64_t)row * a.n_heads + h) * 128 + chunk * 8;
+  const int64_t dst = (((int64_t)b * a.n_heads + h) * a.n_q + i) * 128 + chunk * 8;  // element offset
+  const uint4 v = *reinterpret_cast<const uint4*>(src);
+  const int first_rope_chunk = (128 - a.d_rope) >> 3;
+  const bool rope = chunk >= first_rope_chunk;
+  const int p0 = (chunk - first_rope_chunk) * 4;
   uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
   float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     float u = bf_lo(in[k]), x = bf_hi(in[k]);
-    if (rope) rope_apply(u, x, rope_cs(a.rope, (chunk - first_rope_chunk) * 4 + k, t, tok / a.ring.grid_w,
-                                       tok % a.ring.grid_w));
+    if (rope) rope_apply(u, x, cs[p0 + k]);
     amax = fmaxf(amax, fmaxf(fabsf(u), fabsf(x)));
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x), "f"(u));
-    out[k] = d;
+    out[k] = a.f16 ? pack_h2(u, x) : pack2(u, x);
   }
-  if (!(amax <= 65504.f)) atomicOr(a.err, DEV_ERR_RANGE);
-  *reinterpret_cast<uint4*>(static_cast<__half*>(a.qd) + dst) = make_uint4(out[0], out[1], out[2], out[3]);
+  // fp16 out (the reconstruct-once workspace): the content dims convert exactly for bf16 values in
+  // fp16's range; a value past it is reported
+  if (a.f16 && !(amax <= 65504.f)) atomicOr(a.err, DEV_ERR_RANGE);
+  uint4* d = a.f16 ? reinterpret_cast<uint4*>(static_cast<__half*>(a.qd) + dst)
+                   : reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.qd) + dst);
+  *d = make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 }  // namespace
@@ -136,9 +126,10 @@ cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s) {
 
 cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s) {
   if (a.d_rope <= 0 || a.d_rope > 128 || a.d_rope % 8 != 0 || (a.f16 && !a.err)) return cudaErrorInvalidValue;
-  const int64_t total = (int64_t)a.batch * a.n_q * a.n_heads * 16;
-  if (total == 0) return cudaSuccess;
-  dense_q_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
+  if (a.n_heads * 16 > kMaxHeads16) return cudaErrorInvalidValue;
+  const int64_t rows = (int64_t)a.batch * a.n_q;
+  if (rows == 0) return cudaSuccess;
+  dense_q_bf16_kernel<<<(unsigned)rows, a.n_heads * 16, 0, s>>>(a);
   return cudaGetLastError();
 }
 
