@@ -282,14 +282,18 @@ vmla_status vmla_profile_read(vmla_handle* h, int stage, double* total_ms, int* 
 
 /* Work split of the bf16 append kernel (the down-projection GEMM [c_KV | k_R] =
  * W_down x of the paperlayer paper, Sec. 3): a persistent kernel over work items
- * (sample, 128-row tile of x, column part of [c_KV | k_R]).  `n_split` column
+ * (column part of [c_KV | k_R], one or two 128-row tiles of x).  `n_split` column
  * parts: 0 chooses per call (two when the row tiles alone would leave SMs idle,
- * and always when d_latent > 224; three when d_latent > 480), 1 or 2 forces it.  `max_ctas` caps the grid
- * (0: one CTA per SM); a small cap makes each CTA run many items.  Every split
- * gives the same bits.  n_split = 1 with d_latent > 224 makes later appends
- * return VMLA_ERR_UNSUPPORTED_SHAPE.  Host only; VMLA_ERR_INVALID_ARG for
- * n_split outside 0..2 or a negative cap. */
-vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas);
+ * and always when d_latent > 224; three when d_latent > 480), 1 or 2 forces it.
+ * `row_tiles` 128-row tiles per item: 0 or 1 takes one, 2 shares every W_down
+ * stage between two MMA chains (fewer L2 reads of W_down per row, but the item's
+ * epilogue no longer overlaps the next item's MMAs: slower on the Wan-1.3B layer
+ * at batch 1 to 64); two apply only where the call runs one column part.  `max_ctas`
+ * caps the grid (0: one CTA per SM); a small cap makes each CTA run many items.
+ * Every split gives the same bits.  n_split = 1 with d_latent > 224 makes later
+ * appends return VMLA_ERR_UNSUPPORTED_SHAPE.  Host only; VMLA_ERR_INVALID_ARG for
+ * n_split or row_tiles outside 0..2, both 2, or a negative cap. */
+vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int row_tiles, int max_ctas);
 
 /* The value path absorbed all the way into the layer's output mixer [paperlayer App. E]:
  * with B_h = W_O,h W_uv,h (W_O,h the d_value columns of W_O that read head h),

@@ -74,7 +74,7 @@ _SIGS = {
     "vmla_state_set": (c_int, [c_void_p, c_int, c_int64]),
     "vmla_device_status": (c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "vmla_profile_enable": (c_int, [c_void_p, c_int]),
-    "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int]),
+    "vmla_set_append_tiling": (c_int, [c_void_p, c_int, c_int, c_int]),
     "vmla_fold_query_weights": (c_int, [ctypes.POINTER(Config), c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                         c_void_p]),
     "vmla_chunk_attention_qlatent": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
@@ -307,9 +307,10 @@ class LatentKVAttention:
                                                 _ptr(out), first_frame, n_frames, _stream(stream)),
               "vmla_chunk_attention_folded")
 
-    def set_append_tiling(self, n_split: int = 0, max_ctas: int = 0):
-        """Column parts (0: chosen per call) and grid cap (0: one CTA per SM) of the append kernel."""
-        check(lib().vmla_set_append_tiling(self._h, n_split, max_ctas), "vmla_set_append_tiling")
+    def set_append_tiling(self, n_split: int = 0, row_tiles: int = 0, max_ctas: int = 0):
+        """Column parts, 128-row tiles per work item (0: chosen per call) and grid cap (0: one CTA
+        per SM) of the append kernel."""
+        check(lib().vmla_set_append_tiling(self._h, n_split, row_tiles, max_ctas), "vmla_set_append_tiling")
 
     def profile(self, enable: bool = True):
         """vmla_profile_enable: CUDA-event timing of every stage of the following calls."""

@@ -114,37 +114,42 @@ __device__ __forceinline__ void raw_to_float(const uint32_t (&r)[32], float (&v)
 }
 
 // ============================================================== append
-// Persistent: each CTA takes work items (sample, 128-row tile, column part) in
-// a grid-stride loop.  The column parts split [c_KV | k_R] into NP pieces of
-// N_PART columns (NP = 2 gives small calls -- one chunk of one sample, 37 row
-// tiles -- work for twice as many SMs, at the price of reading x twice from
-// L2).  Two TMEM accumulators alternate, so the epilogue of one item overlaps
-// the loads and MMAs of the next; the epilogue parks the bf16 tile in shared
-// memory and writes it out row-contiguous (ring rows of one frame are
-// consecutive).
-template <int N_PART>
+// Persistent: each CTA takes work items in a grid-stride loop.  An item is a
+// column part of [c_KV | k_R] (NP pieces of N_PART columns) over MT consecutive
+// 128-row tiles of the flattened (sample, row tile) sequence.  NP = 2 gives small
+// calls -- one chunk of one sample, 37 row tiles -- work for twice as many SMs, at
+// the price of reading x twice from L2.  MT = 2 reuses every W_down stage for two
+// row tiles (two MMA chains, one accumulator each), which cuts the L2 -> SM bytes
+// per row by a third when the row tiles outnumber the SMs.  With MT = 1 two TMEM
+// accumulators alternate, so the epilogue of one item overlaps the loads and MMAs
+// of the next; with MT = 2 the item's two accumulators fill TMEM and only the loads
+// run ahead.  The epilogue parks the bf16 tile in shared memory, PARK rows at a
+// time, and writes it out row-contiguous (ring rows of one frame are consecutive).
+template <int N_PART, int MT = 1>
 struct AppendCfg {
   static constexpr int A_BYTES = 128 * 128;  // 128 rows x 64 bf16
   static constexpr int B_BYTES = N_PART * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGE_BYTES = MT * A_BYTES + B_BYTES;
   static constexpr int OUT_STRIDE = N_PART * 2 + 16;  // bytes per parked row: an odd number of 16-byte chunks
-  static constexpr int OUT_BYTES = 64 * OUT_STRIDE;   // half a tile is parked at a time
+  static constexpr int PARK = (212 * 1024 - 64 * OUT_STRIDE) / STAGE_BYTES >= 3 ? 64 : 32;  // rows parked at a time
+  static constexpr int OUT_BYTES = PARK * OUT_STRIDE;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = FIT > 8 ? 8 : FIT;
-  static constexpr uint32_t TMEM_COLS = 512;  // two accumulators, at columns 0 and 256
+  static constexpr int NACC = 2 / MT;         // accumulator slots (items in flight between MMA and epilogue)
+  static constexpr uint32_t TMEM_COLS = 512;  // 128-lane accumulators at columns 0 and 256
   static constexpr int SMEM_USED = 1024 + STAGES * STAGE_BYTES + OUT_BYTES + 2 * 128 * 8 + 256;
   // more than half of an SM's shared memory: one CTA per SM, so the 512 TMEM columns are always free
   static constexpr int SMEM = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
-  static_assert(N_PART % 16 == 0 && N_PART <= 256, "bad N");
+  static_assert(N_PART % 16 == 0 && N_PART <= 256 && (MT == 1 || MT == 2), "bad N or MT");
   static_assert(B_BYTES % 1024 == 0 && OUT_BYTES % 16 == 0, "alignment");
   static_assert(STAGES >= 3 && SMEM <= 227 * 1024, "does not fit");
 };
 
-template <int N_PART>
+template <int N_PART, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     append_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const AppendTc a, int n_parts, int items) {
-  using C = AppendCfg<N_PART>;
+                     const AppendTc a, int n_parts, int tiles, int items) {
+  using C = AppendCfg<N_PART, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sout = smem + C::STAGES * C::STAGE_BYTES;
@@ -184,14 +189,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_w);
       int it = 0;  // global stage counter
       for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
-        const int part = item % n_parts, mt = (item / n_parts) % m_tiles, b = item / (n_parts * m_tiles);
+        const int part = item % n_parts, t0 = (item / n_parts) * MT, nt = min(MT, tiles - t0);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           if (!wait_phase(&empty[s], ((it / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
           uint8_t* sa = smem + s * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_3d(sa, &tm_x, &full[s], kb * 64, mt * 128, b);
-          tma_load_2d(sa + C::A_BYTES, &tm_w, &full[s], kb * 64, part * N_PART);
+          mbar_arrive_expect_tx(&full[s], nt * C::A_BYTES + C::B_BYTES);
+          for (int u = 0; u < nt; ++u)
+            tma_load_3d(sa + u * C::A_BYTES, &tm_x, &full[s], kb * 64, ((t0 + u) % m_tiles) * 128, (t0 + u) / m_tiles);
+          tma_load_2d(sa + MT * C::A_BYTES, &tm_w, &full[s], kb * 64, part * N_PART);
         }
       }
       if (*abort_flag)  // let the copies in flight land before the CTA goes away
@@ -204,10 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(128, N_PART, false, false);
       int it = 0, j = 0;
       for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
-        const int acc = j & 1;
-        if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
+        const int acc = j % C::NACC, use = j / C::NACC;
+        const int nt = min(MT, tiles - (item / n_parts) * MT);
+        if (!wait_phase(&acc_empty[acc], (use & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t d = tbase + acc * 256;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % C::STAGES;
@@ -217,14 +223,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-          const uint64_t ad = smem_desc(sa, 16, 1024, LAYOUT_SW128);
-          const uint64_t bd = smem_desc(sa + C::A_BYTES, 16, 1024, LAYOUT_SW128);
+          const uint64_t bd = smem_desc(sa + MT * C::A_BYTES, 16, 1024, LAYOUT_SW128);
+          for (int u = 0; u < nt; ++u) {  // one MMA chain per row tile, all on this W_down stage
+            const uint32_t d = tbase + (acc * MT + u) * 256;
+            const uint64_t ad = smem_desc(sa + u * C::A_BYTES, 16, 1024, LAYOUT_SW128);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if (k == 0 && kb == 0)
-              mma_ss_c<false>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
-            else
-              mma_ss_c<true>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+            for (int k = 0; k < 4; ++k) {
+              if (k == 0 && kb == 0)
+                mma_ss_c<false>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+              else
+                mma_ss_c<true>(d, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc);
+            }
           }
           mma_commit(&empty[s]);
         }
@@ -238,71 +247,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     const int wq = warp - 4, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
-    constexpr int CH = N_PART / 8;  // 16-byte chunks per row
+    constexpr int CH = N_PART / 8;          // 16-byte chunks per row
+    constexpr int WPP = C::PARK / 32;       // epilogue warps whose TMEM lanes fill one park
     int j = 0;
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
-      const int part = item % n_parts, mt = (item / n_parts) % m_tiles, b = item / (n_parts * m_tiles);
-      const int acc = j & 1;
-      const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
+      const int part = item % n_parts, t0 = (item / n_parts) * MT, nt = min(MT, tiles - t0);
+      const int acc = j % C::NACC, use = j / C::NACC;
+      const bool ok = wait_phase(&acc_full[acc], use & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();
       tc_fence_after();
-      const int m = mt * 128 + r;
-      const int mm = m < a.rows ? m : 0;
-      const int64_t frame = a.first_frame + mm / T;
-      const int tok = mm % T;
-      if (a.contiguous) {
-        row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + a.d_rope);
-        row_pos[r] = row_lat[r] + a.d_latent;
-      } else {
-        const int64_t rr = (int64_t)b * a.ring_rows + ring_frame_slot(a.ring, frame) * T + tok;
-        row_lat[r] = rr * a.d_latent;
-        row_pos[r] = rr * a.d_rope;
-      }
-      named_bar_sync(1, 128);  // row table complete
-      const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        if ((wq >> 1) == half) {  // warps of this half hold TMEM lanes 64*half .. 64*half + 63
-          uint8_t* orow = sout + (r - 64 * half) * C::OUT_STRIDE;
+      for (int u = 0; u < nt; ++u) {
+        const int mt = (t0 + u) % m_tiles, b = (t0 + u) / m_tiles;
+        const int m = mt * 128 + r;
+        const int mm = m < a.rows ? m : 0;
+        const int64_t frame = a.first_frame + mm / T;
+        const int tok = mm % T;
+        if (a.contiguous) {
+          row_lat[r] = ((int64_t)b * a.rows + mm) * (a.d_latent + a.d_rope);
+          row_pos[r] = row_lat[r] + a.d_latent;
+        } else {
+          const int64_t rr = (int64_t)b * a.ring_rows + ring_frame_slot(a.ring, frame) * T + tok;
+          row_lat[r] = rr * a.d_latent;
+          row_pos[r] = rr * a.d_rope;
+        }
+        named_bar_sync(1, 128);  // row table complete
+        const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
+        const uint32_t col_base = (acc * MT + u) * 256;
 #pragma unroll 1
-          for (int c0 = 0; c0 < N_PART; c0 += 16) {
-            uint32_t raw[16];
-            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-            float v[16];
+        for (int pk = 0; pk < 128 / C::PARK; ++pk) {
+          if (wq / WPP == pk) {  // warps of this park hold TMEM lanes PARK*pk .. PARK*pk + PARK - 1
+            uint8_t* orow = sout + (r - C::PARK * pk) * C::OUT_STRIDE;
+#pragma unroll 1
+            for (int c0 = 0; c0 < N_PART; c0 += 16) {
+              uint32_t raw[16];
+              tmem_ld16(tmem_addr(tbase, wq * 32, col_base + c0), raw);
+              float v[16];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(raw[q]);
-            // 16 columns never straddle d_latent (a multiple of 64) nor d_latent + d_rope
-            const int col = part * N_PART + c0;
-            if (a.rotate && col >= a.d_latent && col < a.d_latent + a.d_rope) {
-              const int p0 = (col - a.d_latent) >> 1;
+              for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(raw[q]);
+              // 16 columns never straddle d_latent (a multiple of 64) nor d_latent + d_rope
+              const int col = part * N_PART + c0;
+              if (a.rotate && col >= a.d_latent && col < a.d_latent + a.d_rope) {
+                const int p0 = (col - a.d_latent) >> 1;
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                rope_apply(v[2 * q], v[2 * q + 1],
-                           rope_cs(a.rope, p0 + q, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w));
+                for (int q = 0; q < 8; ++q)
+                  rope_apply(v[2 * q], v[2 * q + 1],
+                             rope_cs(a.rope, p0 + q, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w));
+              }
+              uint4* o = reinterpret_cast<uint4*>(orow + c0 * 2);
+              o[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                pack_bf16x2(v[6], v[7]));
+              o[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                pack_bf16x2(v[14], v[15]));
             }
-            uint4* o = reinterpret_cast<uint4*>(orow + c0 * 2);
-            o[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                              pack_bf16x2(v[6], v[7]));
-            o[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                              pack_bf16x2(v[14], v[15]));
+            tc_fence_before();
+            __syncwarp();
+            // after its last tile, each warp's lanes are read; all four free the slot for item j + NACC
+            if (u == nt - 1 && lane == 0) mbar_arrive(&acc_empty[acc]);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read; all four free it for item j + 2
-        }
-        named_bar_sync(1, 128);  // this half is parked
-        const int rows_h = min(64, valid_rows - 64 * half);
+          named_bar_sync(1, 128);  // this park is complete
+          const int rows_p = min(C::PARK, valid_rows - C::PARK * pk);
 #pragma unroll 4
-        for (int id = tid; id < rows_h * CH; id += 128) {
-          const int row = id / CH, ch = id - row * CH;
-          const int col = part * N_PART + ch * 8;
-          if (col >= a.d_latent + a.d_rope) continue;  // the last part may run past [c_KV | k_R]
-          const bool lat = col < a.d_latent;
-          __nv_bfloat16* dst = (lat || a.contiguous ? a.ckv : a.kr) +
-                               (lat ? row_lat[64 * half + row] + col : row_pos[64 * half + row] + (col - a.d_latent));
-          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + row * C::OUT_STRIDE + ch * 16);
+          for (int id = tid; id < rows_p * CH; id += 128) {
+            const int row = id / CH, ch = id - row * CH;
+            const int col = part * N_PART + ch * 8;
+            if (col >= a.d_latent + a.d_rope) continue;  // the last part may run past [c_KV | k_R]
+            const bool lat = col < a.d_latent;
+            const int rt = C::PARK * pk + row;
+            __nv_bfloat16* dst =
+                (lat || a.contiguous ? a.ckv : a.kr) + (lat ? row_lat[rt] + col : row_pos[rt] + (col - a.d_latent));
+            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + row * C::OUT_STRIDE + ch * 16);
+          }
+          named_bar_sync(1, 128);  // the park is written out before it is reused
         }
-        named_bar_sync(1, 128);  // the parked half is written out before it is reused
       }
     }
   }
@@ -561,12 +578,16 @@ __global__ void __launch_bounds__(QPrepCfg<DL, DR>::THREADS, 1)
 // and [(d_nope + 128) x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
 // two TMEM accumulators alternate so the epilogue of one item overlaps the
 // next; two epilogue warpgroups park the item's 128 rows as [k_h (128) | v_h
-// (128)] bf16 -- the first k_h (d_nope content columns from TMEM, the d_rope
-// positional columns read one item ahead), the second v_h -- and all 256 threads
-// write each row's two 256-byte runs out contiguously.
+// (128)] -- the first k_h (d_nope content columns from TMEM, the d_rope
+// positional columns read one item ahead), the second v_h.  With TMA_OUT (rows
+// written to consecutive rows: the window of reconstruct-once) the park is four
+// 128-byte-swizzled [128 x 64] blocks that four TMA tensor stores write out,
+// clipped at the last key, while the threads go on to the next item; otherwise
+// (rows to the ring slots of their frames: the dense cache) all 256 threads write
+// each row's two 256-byte runs out contiguously.
 __device__ __forceinline__ bool m_valid(int mt, int r, int rows) { return mt * 128 + r < rows; }
 
-template <int DL, int DR>
+template <int DL, int DR, bool TMA_OUT = false>
 struct ReconCfg {
   static constexpr int DN = 128 - DR;        // content dims of a head's key
   static constexpr int N = DN + 128;         // MMA N: [W_uk,h ; W_uv,h] rows
@@ -575,7 +596,7 @@ struct ReconCfg {
   static constexpr int B_BLK = N * 128;    // [d_nope rows of W_uk,h ; 128 rows of W_uv,h] x 64 cols
   static constexpr int STAGE = A_BLK + B_BLK;
   static constexpr int OUT_STRIDE = 256 * 2 + 16;  // parked row [k_h | v_h]: an odd number of 16-byte chunks
-  static constexpr int OUT_BYTES = 128 * OUT_STRIDE;
+  static constexpr int OUT_BYTES = TMA_OUT ? 4 * 16384 : 128 * OUT_STRIDE;
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of N columns, at 0 and 256
@@ -601,11 +622,30 @@ __device__ __forceinline__ void store_x16_smem(uint8_t* dst, const float* v, flo
   }
 }
 
-template <int DL, int DR, bool F16>
-__global__ void __launch_bounds__(ReconCfg<DL, DR>::THREADS, 1)
+// 16 floats as bf16 (or fp16) into columns c0 .. c0 + 15 (c0 a multiple of 16) of row r of a parked
+// tile made of 128-byte-swizzled [128 x 64] blocks of 16 KB: 16-byte chunk j of a row's block at
+// position j ^ (r & 7)
+template <bool F16>
+__device__ __forceinline__ void store_sw16_smem(uint8_t* tile, int r, int c0, const float* v, float& amax) {
+  auto pk = [](float lo, float hi) { return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi); };
+  uint8_t* row = tile + (c0 >> 6) * 16384 + r * 128;
+  const int j = (c0 & 63) >> 3;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[8 * q + k]));
+    *reinterpret_cast<uint4*>(row + (((j + q) ^ (r & 7)) << 4)) =
+        make_uint4(pk(v[8 * q + 0], v[8 * q + 1]), pk(v[8 * q + 2], v[8 * q + 3]), pk(v[8 * q + 4], v[8 * q + 5]),
+                   pk(v[8 * q + 6], v[8 * q + 7]));
+  }
+}
+
+template <int DL, int DR, bool F16, bool TMA_OUT>
+__global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
     recon_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wuk,
-                    const __grid_constant__ CUtensorMap tm_wuv, const ReconTc a, int items) {
-  using C = ReconCfg<DL, DR>;
+                    const __grid_constant__ CUtensorMap tm_wuv, const __grid_constant__ CUtensorMap tm_out,
+                    const ReconTc a, int items) {
+  using C = ReconCfg<DL, DR, TMA_OUT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sout = smem + C::STAGES * C::STAGE;
@@ -743,23 +783,46 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR>::THREADS, 1)
       __syncwarp();
       tc_fence_after();
       const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
-      uint8_t* orow = sout + r * C::OUT_STRIDE;
       float amax = 0.f;
-      if (wg == 0) {  // TMEM columns 0..DN-1: the content part of k_h, then its positional part
+      if constexpr (TMA_OUT) {
+        if (tid == 0) bulk_wait_all_read();  // the previous item's stores have read the park
+        named_bar_sync(1, 256);
+        if (wg == 0) {  // k_h: TMEM columns 0..DN-1, then the positional part, into blocks 0 and 1
 #pragma unroll 1
-        for (int c0 = 0; c0 < C::DN; c0 += 16) {
-          uint32_t raw[16];
-          tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-          store_x16_smem<F16>(orow + c0 * 2, reinterpret_cast<const float*>(raw), amax);
-        }
+          for (int c0 = 0; c0 < C::DN; c0 += 16) {
+            uint32_t raw[16];
+            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            store_sw16_smem<F16>(sout, r, c0, reinterpret_cast<const float*>(raw), amax);
+          }
 #pragma unroll
-        for (int c0 = 0; c0 < DR; c0 += 16) store_x16_smem<F16>(orow + (C::DN + c0) * 2, kr + c0, amax);
-      } else {  // TMEM columns DN..DN+127: v_h, parked from column 128 (16-column loads: DN is a multiple of 16)
+          for (int c0 = 0; c0 < DR; c0 += 16) store_sw16_smem<F16>(sout, r, C::DN + c0, kr + c0, amax);
+        } else {  // v_h: TMEM columns DN..DN+127 into blocks 2 and 3
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          uint32_t raw[16];
-          tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
-          store_x16_smem<F16>(orow + (128 + c0) * 2, reinterpret_cast<const float*>(raw), amax);
+          for (int c0 = 0; c0 < 128; c0 += 16) {
+            uint32_t raw[16];
+            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
+            store_sw16_smem<F16>(sout + 2 * 16384, r, c0, reinterpret_cast<const float*>(raw), amax);
+          }
+        }
+        fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
+      } else {
+        uint8_t* orow = sout + r * C::OUT_STRIDE;
+        if (wg == 0) {  // TMEM columns 0..DN-1: the content part of k_h, then its positional part
+#pragma unroll 1
+          for (int c0 = 0; c0 < C::DN; c0 += 16) {
+            uint32_t raw[16];
+            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            store_x16_smem<F16>(orow + c0 * 2, reinterpret_cast<const float*>(raw), amax);
+          }
+#pragma unroll
+          for (int c0 = 0; c0 < DR; c0 += 16) store_x16_smem<F16>(orow + (C::DN + c0) * 2, kr + c0, amax);
+        } else {  // TMEM columns DN..DN+127: v_h, parked from column 128 (16-column loads: DN is a multiple of 16)
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 16) {
+            uint32_t raw[16];
+            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
+            store_x16_smem<F16>(orow + (128 + c0) * 2, reinterpret_cast<const float*>(raw), amax);
+          }
         }
       }
       // fp16 holds magnitudes up to 65504: a row past it is reported, not stored as inf silently
@@ -768,14 +831,26 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
       named_bar_sync(1, 256);  // the item is parked and its row table complete
+      if constexpr (TMA_OUT) {
+        if (tid == 0 && valid_rows > 0) {  // rows past the window are clipped by the tensor map
+          for (int blk = 0; blk < 4; ++blk)
+            tma_store_3d(&tm_out, sout + blk * 16384, ((blk >> 1) * a.n_heads + h) * 128 + (blk & 1) * 64, mt * 128,
+                         b);
+          bulk_commit();
+        }
+      } else {
 #pragma unroll 4
-      for (int id = tid; id < valid_rows * 32; id += 256) {
-        const int rr = id >> 5, ch = id & 31;
-        uint16_t* dst = static_cast<uint16_t*>(a.dense) + row_k[rr] +
-                        (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
+        for (int id = tid; id < valid_rows * 32; id += 256) {
+          const int rr = id >> 5, ch = id & 31;
+          uint16_t* dst = static_cast<uint16_t*>(a.dense) + row_k[rr] +
+                          (ch < 16 ? ch * 8 : (int64_t)a.n_heads * 128 + (ch - 16) * 8);
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sout + rr * C::OUT_STRIDE + ch * 16);
+        }
+        named_bar_sync(1, 256);  // the park is written out before it is reused
       }
-      named_bar_sync(1, 256);  // the park is written out before it is reused
+    }
+    if constexpr (TMA_OUT) {
+      if (tid == 0) bulk_wait_all();  // the last stores have read shared memory and landed
     }
   }
   tc_fence_before();
@@ -1147,11 +1222,11 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int N_PART>
+template <int N_PART, int MT>
 cudaError_t run_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, int n_parts,
                        int ctas, cudaStream_t s) {
-  using C = AppendCfg<N_PART>;
-  static const cudaError_t attr = set_smem(append_tc_kernel<N_PART>, C::SMEM);
+  using C = AppendCfg<N_PART, MT>;
+  static const cudaError_t attr = set_smem(append_tc_kernel<N_PART, MT>, C::SMEM);
   if (attr != cudaSuccess) return attr;
   static int sms = 0;
   if (sms == 0) {
@@ -1159,9 +1234,10 @@ cudaError_t run_append(const CUtensorMap& tx, const CUtensorMap& tw, const Appen
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  const int items = ((a.rows + 127) / 128) * n_parts * batch;
+  const int tiles = ((a.rows + 127) / 128) * batch;
+  const int items = (tiles + MT - 1) / MT * n_parts;
   const int grid = std::min(items, ctas > 0 ? ctas : sms);
-  append_tc_kernel<N_PART><<<grid, kThreads, C::SMEM, s>>>(tx, tw, a, n_parts, items);
+  append_tc_kernel<N_PART, MT><<<grid, kThreads, C::SMEM, s>>>(tx, tw, a, n_parts, tiles, items);
   return cudaGetLastError();
 }
 
@@ -1169,12 +1245,14 @@ template <int N_OUT>
 cudaError_t go_append(const CUtensorMap& tx, const CUtensorMap& tw, const AppendTc& a, int batch, cudaStream_t s,
                       const AppendPlan& p) {
   if constexpr (N_OUT <= 256) {
-    if (p.parts == 1) return run_append<N_OUT>(tx, tw, a, batch, 1, p.ctas, s);
+    if (p.parts == 1)
+      return p.row_tiles == 2 ? run_append<N_OUT, 2>(tx, tw, a, batch, 1, p.ctas, s)
+                              : run_append<N_OUT, 1>(tx, tw, a, batch, 1, p.ctas, s);
   }
   if constexpr (append_part_cols(N_OUT, 2) <= 256) {
-    if (p.parts == 2) return run_append<append_part_cols(N_OUT, 2)>(tx, tw, a, batch, 2, p.ctas, s);
+    if (p.parts == 2) return run_append<append_part_cols(N_OUT, 2), 1>(tx, tw, a, batch, 2, p.ctas, s);
   }
-  if (p.parts == 3) return run_append<append_part_cols(N_OUT, 3)>(tx, tw, a, batch, 3, p.ctas, s);
+  if (p.parts == 3) return run_append<append_part_cols(N_OUT, 3), 1>(tx, tw, a, batch, 3, p.ctas, s);
   return cudaErrorInvalidValue;
 }
 
@@ -1208,11 +1286,13 @@ cudaError_t go_qprep_dl(const CUtensorMap& tq, const CUtensorMap& tw, const CUte
   return cudaErrorInvalidValue;
 }
 
+// F16 runs are the reconstruct-once window (fp16 entries, consecutive rows: TMA tensor stores of the
+// park through tm_out); the others the dense cache (bf16 entries placed in ring slots by the threads)
 template <int DL, int DR, bool F16>
-cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
-                     int batch, cudaStream_t s) {
-  using C = ReconCfg<DL, DR>;
-  static const cudaError_t attr = set_smem(recon_tc_kernel<DL, DR, F16>, C::SMEM);
+cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const CUtensorMap& to,
+                     const ReconTc& a, int batch, cudaStream_t s) {
+  using C = ReconCfg<DL, DR, F16>;
+  static const cudaError_t attr = set_smem(recon_tc_kernel<DL, DR, F16, F16>, C::SMEM);
   if (attr != cudaSuccess) return attr;
   static int sms = 0;
   if (sms == 0) {
@@ -1221,32 +1301,36 @@ cudaError_t go_recon(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtens
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int items = ((a.rows + 127) / 128) * a.n_heads * batch;
-  recon_tc_kernel<DL, DR, F16><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tc, tuk, tuv, a, items);
+  recon_tc_kernel<DL, DR, F16, F16><<<std::min(items, sms), C::THREADS, C::SMEM, s>>>(tc, tuk, tuv, to, a, items);
   return cudaGetLastError();
 }
 
 template <int DR, bool F16>
-cudaError_t go_recon_dl(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
-                        int batch, cudaStream_t s) {
+cudaError_t go_recon_dl(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const CUtensorMap& to,
+                        const ReconTc& a, int batch, cudaStream_t s) {
   switch (a.d_latent) {
-    case 64: return go_recon<64, DR, F16>(tc, tuk, tuv, a, batch, s);
-    case 128: return go_recon<128, DR, F16>(tc, tuk, tuv, a, batch, s);
-    case 192: return go_recon<192, DR, F16>(tc, tuk, tuv, a, batch, s);
-    case 256: return go_recon<256, DR, F16>(tc, tuk, tuv, a, batch, s);
+    case 64: return go_recon<64, DR, F16>(tc, tuk, tuv, to, a, batch, s);
+    case 128: return go_recon<128, DR, F16>(tc, tuk, tuv, to, a, batch, s);
+    case 192: return go_recon<192, DR, F16>(tc, tuk, tuv, to, a, batch, s);
+    case 256: return go_recon<256, DR, F16>(tc, tuk, tuv, to, a, batch, s);
     case 384:
-      if constexpr (DR == 32) return go_recon<384, DR, F16>(tc, tuk, tuv, a, batch, s);
+      if constexpr (DR == 32) return go_recon<384, DR, F16>(tc, tuk, tuv, to, a, batch, s);
       break;
     case 512:
-      if constexpr (DR == 32) return go_recon<512, DR, F16>(tc, tuk, tuv, a, batch, s);
+      if constexpr (DR == 32) return go_recon<512, DR, F16>(tc, tuk, tuv, to, a, batch, s);
       break;
   }
   return cudaErrorInvalidValue;
 }
 
 template <int DR>
-cudaError_t go_recon_t(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
-                       int batch, cudaStream_t s) {
-  return a.f16 ? go_recon_dl<DR, true>(tc, tuk, tuv, a, batch, s) : go_recon_dl<DR, false>(tc, tuk, tuv, a, batch, s);
+cudaError_t go_recon_t(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const CUtensorMap* to,
+                       const ReconTc& a, int batch, cudaStream_t s) {
+  if (a.f16) {
+    if (!to || a.to_ring) return cudaErrorInvalidValue;
+    return go_recon_dl<DR, true>(tc, tuk, tuv, *to, a, batch, s);
+  }
+  return go_recon_dl<DR, false>(tc, tuk, tuv, tc, a, batch, s);
 }
 
 }  // namespace
@@ -1338,15 +1422,19 @@ cudaError_t launch_fold_query(const __nv_bfloat16* w_uq, const __nv_bfloat16* w_
   return cudaGetLastError();
 }
 
-AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int ctas) {
+AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int row_tiles, int ctas) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     cudaGetLastError();
-  AppendPlan p{n_split, ctas};
+  const int64_t tiles = (int64_t)((rows + 127) / 128) * batch;
+  AppendPlan p{n_split, ctas, row_tiles};
   if (n_out > 512)
     p.parts = 3;
   else if (p.parts == 0)
-    p.parts = (n_out > 256 || (int64_t)((rows + 127) / 128) * batch < sms) ? 2 : 1;
+    p.parts = (n_out > 256 || tiles < sms) ? 2 : 1;
+  // two row tiles per item measured slower at every batch (Wan layer, batch 1 to 64: the item's two
+  // accumulators fill TMEM, so its epilogue no longer overlaps the next item's MMAs)
+  if (p.parts != 1 || p.row_tiles == 0) p.row_tiles = 1;
   return p;
 }
 
@@ -1386,14 +1474,14 @@ cudaError_t launch_qprep_tc(const CUtensorMap& tq, const CUtensorMap& tw, const 
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv, const ReconTc& a,
-                            int batch, cudaStream_t s) {
+cudaError_t launch_recon_tc(const CUtensorMap& tc, const CUtensorMap& tuk, const CUtensorMap& tuv,
+                            const CUtensorMap* to, const ReconTc& a, int batch, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
   switch (a.d_rope) {
-    case 16: return go_recon_t<16>(tc, tuk, tuv, a, batch, s);
-    case 32: return go_recon_t<32>(tc, tuk, tuv, a, batch, s);
-    case 64: return go_recon_t<64>(tc, tuk, tuv, a, batch, s);
-    case 96: return go_recon_t<96>(tc, tuk, tuv, a, batch, s);
+    case 16: return go_recon_t<16>(tc, tuk, tuv, to, a, batch, s);
+    case 32: return go_recon_t<32>(tc, tuk, tuv, to, a, batch, s);
+    case 64: return go_recon_t<64>(tc, tuk, tuv, to, a, batch, s);
+    case 96: return go_recon_t<96>(tc, tuk, tuv, to, a, batch, s);
   }
   return cudaErrorInvalidValue;
 }

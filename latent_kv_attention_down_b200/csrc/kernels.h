@@ -130,17 +130,19 @@ struct AppendTc {
   uint64_t limit_ns;
 };
 // Work split of the persistent append kernel for a call: `parts` column parts
-// of [c_KV | k_R] (1 or 2) and a grid cap `ctas` (0: one CTA per SM).  n_split 0
+// of [c_KV | k_R] (1, 2 or 3), `row_tiles` 128-row tiles per work item (1 or 2;
+// 2 only with one part) and a grid cap `ctas` (0: one CTA per SM).  n_split 0
 // chooses two parts when the 128-row tiles alone would leave SMs idle (and
-// always past 256 columns); past 512 columns there are always three.
+// always past 256 columns); past 512 columns there are always three.  row_tiles
+// 0 takes one row tile (two measured slower).
 // Columns of one part when [c_KV | k_R] (n_out columns) is split in `parts`: a multiple of 16
 // (the MMA's N); the last part may run past n_out (those rows of W_down read as zeros).
 constexpr int append_part_cols(int n_out, int parts) { return (n_out + 16 * parts - 1) / (16 * parts) * 16; }
 
 struct AppendPlan {
-  int parts, ctas;
+  int parts, ctas, row_tiles;
 };
-AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int ctas);
+AppendPlan append_tc_plan(int n_out, int rows, int batch, int n_split, int row_tiles, int ctas);
 // x map: 3D (D, rows, B) box (64,128,1) SW128; w map: 2D (D, n_out) box (64, append_part_cols(n_out, parts))
 // SW128, n_out = d_c + d_rope.
 cudaError_t launch_append_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const AppendTc& a, int batch,
@@ -239,6 +241,31 @@ int attn_dense_block_n();
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_out,
                                  const AttnTc& a, int batch, cudaStream_t s, bool f16);
 
+// Per-head attention, d_head = 128, two query tiles per CTA and a stream-K split of the
+// (tile pair, key tile) iterations over `ctas` CTAs (attn_pp.cu).  Maps as launch_attn_dense_tc;
+// the output rows go straight from registers to `out` ([B][n_q][n_h*128] fp32).  Pairs whose keys
+// are split leave partials in `part` / `part_ml` (attn_pp_partial_bytes), combined by a second
+// kernel in the same launch call.
+constexpr int kAttnPPMaxCtas = 160;
+struct AttnPP {
+  int n_q, n_keys, n_heads, m_tiles;
+  float scale_log2;
+  float rescale_threshold;
+  unsigned* err;
+  uint64_t limit_ns;
+  int h0 = 0, h_count = 0;  // heads of this launch
+  // filled by attn_pp_plan
+  int pairs_per_bh = 0, n_kt = 0, ctas = 0;
+  int64_t iters = 0;
+  float* out = nullptr;      // [B][n_q][n_h*128]
+  float* part = nullptr;     // [2*kAttnPPMaxCtas][2][128][128]
+  float* part_ml = nullptr;  // [2*kAttnPPMaxCtas][2][128][2]
+};
+constexpr size_t attn_pp_partial_bytes() { return (size_t)2 * kAttnPPMaxCtas * 2 * 128 * (128 + 2) * 4; }
+AttnPP attn_pp_plan(AttnPP a, int batch, int sms);
+cudaError_t launch_attn_pp(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const AttnPP& a, cudaStream_t s,
+                           bool f16);
+
 struct DenseQTc {  // q' = [q_nope | RoPE(q_rope)] -> [B][n_h][n_q][128]
   const __nv_bfloat16* q;
   void* qd;                         // bf16, or fp16 when f16
@@ -269,9 +296,11 @@ struct ReconTc {  // per-head dense entries from latents (tcgen05)
   uint64_t limit_ns;
 };
 // c map: 3D (d_c, rows, B) box (64,128,1) SW128; w_uk map: 3D (d_c, d_nope, n_h) box (64,d_nope,1);
-// w_uv map: 3D (d_c, 128, n_h) box (64,128,1)
+// w_uv map: 3D (d_c, 128, n_h) box (64,128,1).  f16 (the reconstruct-once window, to_ring 0) also
+// needs tm_out: 3D fp16 (2*n_h*128, rows, B) over `dense`, box (64,128,1) SW128 (its row extent
+// clips the last tile); the bf16 dense cache passes NULL.
 cudaError_t launch_recon_tc(const CUtensorMap& tm_c, const CUtensorMap& tm_wuk, const CUtensorMap& tm_wuv,
-                            const ReconTc& a, int batch, cudaStream_t s);
+                            const CUtensorMap* tm_out, const ReconTc& a, int batch, cudaStream_t s);
 
 // ------------------------------------------------------------------ device status
 unsigned* device_error_word();  // address of the library's device status word (current device)

@@ -120,7 +120,7 @@ int64_t ring_rows(const vmla_config& c) { return (int64_t)c.window_frames * toke
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, obar = 0, recon = 0;  // offsets
+  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, obar = 0, part = 0, recon = 0;  // offsets
   size_t base_bytes = 0;   // every design but RECON_ONCE
   size_t recon_bytes = 0;  // extra for RECON_ONCE
 };
@@ -141,6 +141,8 @@ WsLayout ws_layout(const vmla_config& c) {
   off = align256(off + B * (size_t)c.window_frames * tokens_per_frame(c) * (size_t)(c.d_latent + 2 * c.d_rope) * e);
   w.obar = off;  // the folded output mixer's input: O_bar as a bf16 pair [2][B][rows][n_h * d_c]
   off = align256(off + (c.dtype == VMLA_BF16 ? 2 * B * nq * c.n_heads * (size_t)c.d_latent * 2 : 0));
+  w.part = off;  // partial rows of the per-head attention's split pairs (fp32)
+  off = align256(off + (c.dtype == VMLA_BF16 ? attn_pp_partial_bytes() : 0));
   w.recon = off;
   w.base_bytes = off;
   w.recon_bytes = B * ring_rows(c) * 2 * (size_t)c.n_heads * c.d_value * e;
@@ -207,6 +209,7 @@ struct vmla_handle {
   std::vector<int64_t> dense_frames;  // dense cache, per layer
   unsigned* err = nullptr;            // device status word (resolved at bind)
   int append_split = 0;               // append work split (0: chosen per call), see vmla_set_append_tiling
+  int append_rows = 0;                // 128-row tiles per append work item (0: chosen per call)
   int append_ctas = 0;
   bool profiling = false;
   struct Timer {
@@ -550,7 +553,7 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
     } else {
       CUtensorMap tx, tw;
       const int nout = c.d_latent + c.d_rope;
-      const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_ctas);
+      const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_rows, h->append_ctas);
       const int parts = plan.parts;
       if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -764,7 +767,12 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       a.rope = make_rope(c);
       a.err = h->err;
       a.limit_ns = kWaitLimitNs;
-      e = launch_recon_tc(tc, tuk, tuv, a, c.batch, s);
+      CUtensorMap to;
+      const uint64_t row_bytes = 2ull * c.n_heads * 128 * 2;
+      if (!map3(&to, recon, 2ull * c.n_heads * 128, win.n_keys, c.batch, row_bytes, rr * row_bytes, 64, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return map_fail();
+      e = launch_recon_tc(tc, tuk, tuv, &to, a, c.batch, s);
     }
     if (e != cudaSuccess) return cuda_fail(e);
     return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, true, hout);
@@ -964,11 +972,41 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
   a.rescale_threshold = c.softmax_rescale_log2;
   a.err = h->err;
   a.limit_ns = kWaitLimitNs;
+#ifndef VMLA_PER_HEAD_PAIRS
+  // one query tile per CTA (the absorbed kernel's pipeline with per-head tiles)
   if (hout)
     return cuda_status(launch_head_groups(c, nq, a, out, hout, s, [&](const AttnTc& ag) {
       return launch_attn_dense_tc(tq, tkv, to, ag, c.batch, s, f16);
     }));
   return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s, f16));
+#else
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  float* part = at<float>(h->ws, w.part);
+  auto pp = [&](const AttnTc& ag) {
+    AttnPP p;
+    p.n_q = ag.n_q;
+    p.n_keys = ag.n_keys;
+    p.n_heads = ag.n_heads;
+    p.m_tiles = ag.m_tiles;
+    p.scale_log2 = ag.scale_log2;
+    p.rescale_threshold = ag.rescale_threshold;
+    p.err = ag.err;
+    p.limit_ns = ag.limit_ns;
+    p.h0 = ag.h0;
+    p.h_count = ag.h_count;
+    p.out = static_cast<float*>(out);
+    p.part = part;
+    p.part_ml = part + (size_t)2 * kAttnPPMaxCtas * 2 * 128 * 128;
+    return launch_attn_pp(tq, tkv, attn_pp_plan(p, c.batch, sms), s, f16);
+  };
+  if (hout) return cuda_status(launch_head_groups(c, nq, a, out, hout, s, pp));
+  return cuda_status(pp(a));
+#endif
 }
 
 }  // namespace
@@ -1137,7 +1175,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
   } else {
     __nv_bfloat16* chunk = at<__nv_bfloat16>(h->ws, w.chunk);  // [B][rows][d_c + 32]
     const int nout = c.d_latent + c.d_rope;
-    const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_ctas);
+    const AppendPlan plan = append_tc_plan(nout, rows, c.batch, h->append_split, h->append_rows, h->append_ctas);
     const int parts = plan.parts;
     CUtensorMap tx, tw;
     if (!map3(&tx, x, c.d_model, rows, c.batch, (uint64_t)c.d_model * 2, (uint64_t)rows * c.d_model * 2, 64, 128,
@@ -1188,7 +1226,7 @@ vmla_status vmla_dense_cache_append(vmla_handle* h, int layer, const void* x, co
     r.rope = make_rope(c);
     r.err = h->err;
     r.limit_ns = kWaitLimitNs;
-    e = launch_recon_tc(tc, tuk, tuv, r, c.batch, s);
+    e = launch_recon_tc(tc, tuk, tuv, nullptr, r, c.batch, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   h->dense_frames[layer] = new_F;
@@ -1311,9 +1349,11 @@ vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags) {
   return VMLA_OK;
 }
 
-vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int max_ctas) {
-  if (!h || n_split < 0 || n_split > 2 || max_ctas < 0) return VMLA_ERR_INVALID_ARG;
+vmla_status vmla_set_append_tiling(vmla_handle* h, int n_split, int row_tiles, int max_ctas) {
+  if (!h || n_split < 0 || n_split > 2 || row_tiles < 0 || row_tiles > 2 || max_ctas < 0) return VMLA_ERR_INVALID_ARG;
+  if (row_tiles == 2 && n_split == 2) return VMLA_ERR_INVALID_ARG;
   h->append_split = n_split;
+  h->append_rows = row_tiles;
   h->append_ctas = max_ctas;
   return VMLA_OK;
 }

@@ -269,16 +269,17 @@ def test_append_tiling_arguments():
     c = default_config()
     h = api.LatentKVAttention(c)
     lib = api.lib()
-    for t in ((3, 0), (-1, 0), (1, -1)):
+    # (column parts, row tiles per item, grid cap); two row tiles exist only with one column part
+    for t in ((3, 0, 0), (-1, 0, 0), (1, 0, -1), (0, 3, 0), (0, -1, 0), (2, 2, 0)):
         assert lib.vmla_set_append_tiling(h._h, *t) == 1, t
-    for t in ((0, 0), (1, 0), (2, 0), (1, 3), (2, 148), (0, 7)):
+    for t in ((0, 0, 0), (1, 0, 0), (2, 0, 0), (1, 0, 3), (2, 0, 148), (0, 0, 7), (1, 2, 0), (0, 2, 5), (2, 1, 0)):
         assert lib.vmla_set_append_tiling(h._h, *t) == 0, t
     # one MMA covers at most 256 columns: d_latent 256 (+32) needs two column parts
     c256 = default_config()
     c256.d_latent = 256
     h2 = api.LatentKVAttention(c256)
     assert lib.vmla_bind(h2._h, 0x10000, 0x20000, 0x30000, api.workspace_bytes(c256)) == 0
-    assert lib.vmla_set_append_tiling(h2._h, 1, 0) == 0
+    assert lib.vmla_set_append_tiling(h2._h, 1, 0, 0) == 0
     assert lib.vmla_cache_append(h2._h, 0, 0x40000, 0x40000, 0, 3, None) == 2
     for x in (h, h2):
         x.close()

@@ -377,20 +377,23 @@ def test_small_append_writes_only_its_slots():
     assert np.all(raw_ckv == 0x7F) and np.all(raw_kr == 0x7F)
 
 
-TILINGS = [(0, 0), (1, 0), (2, 0), (1, 1), (2, 3)]
+# (column parts, 128-row tiles per item, grid cap)
+TILINGS = [(0, 0, 0), (1, 1, 0), (2, 0, 0), (1, 1, 1), (2, 0, 3), (1, 2, 0), (1, 2, 3), (1, 2, 1)]
 
 
-@pytest.mark.parametrize("tiling", TILINGS, ids=lambda t: "np%d_ctas%d" % t)
+@pytest.mark.parametrize("tiling", TILINGS, ids=lambda t: "np%d_mt%d_ctas%d" % t)
 @pytest.mark.parametrize("rope_mode", [api.ROPE_AT_READ, api.ROPE_AT_APPEND])
 def test_append_tilings(tiling, rope_mode):
     """Every work split of the persistent append kernel (one or two column
-    parts; a grid of one CTA per SM, or capped so each CTA runs many items
-    through both TMEM accumulators) writes bf16(W_down x) -- k_R rotated with the absolute frame
-    when RoPE is applied at append -- into exactly its ring rows, for two
-    samples and a ragged last tile (600 rows per sample)."""
+    parts; one or two row tiles per item, a pair crossing from one sample's
+    ragged last tile into the next sample and the last item holding a single
+    tile; a grid of one CTA per SM, or capped so each CTA runs many items
+    through its TMEM accumulators) writes bf16(W_down x) -- k_R rotated with the
+    absolute frame when RoPE is applied at append -- into exactly its ring rows,
+    for three samples and a ragged last tile (600 rows per sample: 5 tiles)."""
     import torch
     import oracle.vmla_oracle as O
-    d = SMALL.replace(name="small_b2", batch=2)
+    d = SMALL.replace(name="small_b3", batch=3)
     ro = Rollout(d, rope_mode=rope_mode)
     ro.m.set_append_tiling(*tiling)
     ro.m.ckv.fill_(0x7F)
@@ -419,7 +422,79 @@ def test_append_tilings(tiling, rope_mode):
     assert np.all(raw_ckv == 0x7F) and np.all(raw_kr == 0x7F)
 
 
-@pytest.mark.parametrize("tiling", [(1, 0), (2, 0), (2, 1)], ids=lambda t: "np%d_ctas%d" % t)
+# The tiny layer (d_model 32, 2 heads of 10 + 6, d_c 8, rotary pairs (1, 1, 1), a 4x6
+# grid, a 4-frame window of 1-frame chunks: 96 keys, 24 queries) zero-padded into the
+# widths the tensor-core kernels take: d_model 64, d_c 64, heads of 96 + 32 with the
+# rotary pairs (14, 1, 1).  The first pair of every axis turns at theta^0 = 1 whatever
+# the band size, so the tiny layer's three pairs become pairs 0, 14 and 15 of the
+# padded head and every other pair carries zeros.  Every tile is mostly padding: the
+# TMA zero fill past the last key and query and the ragged-tile masks decide the result.
+TINY_BF16 = TINY.replace(dtype="bf16")
+TINY_PADDED = TINY.replace(name="tiny_padded", d_model=64, d_nope=96, d_rope=32, d_latent=64,
+                           rope_pairs=(14, 1, 1), dtype="bf16")
+_PAD_PAIR = (0, 14, 15)  # padded pair of each of the tiny layer's (t, h, w) pairs
+
+
+def _pad_rotary(dst, src):
+    """Tiny rotary pairs [..., 6] into the padded [..., 32] layout."""
+    for k, p in enumerate(_PAD_PAIR):
+        dst[..., 2 * p:2 * p + 2] = src[..., 2 * k:2 * k + 2]
+
+
+@pytest.mark.parametrize("design", [api.DESIGN_AUTO, api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE,
+                                    api.DESIGN_RECONSTRUCT])
+def test_tiny_layer_zero_padded_through_tensor_cores(design):
+    """The tiny layer, zero-padded, through the bf16 tensor-core kernels over a
+    rollout that wraps the ring (chunk 6 of 1-frame chunks, 4-frame window),
+    against the fp64 definition of the unpadded layer; the padded value columns
+    come out exactly zero.  The softmax scale of the padded head is
+    1/sqrt(128) against the tiny head's 1/sqrt(16): the padded queries carry
+    the factor sqrt(8), and the oracle takes them divided back."""
+    import torch
+    from tests.harness import oracle_chunk
+    t, d = TINY_BF16, TINY_PADDED
+    w = synth.weights(t, 0)
+    wd = np.zeros((d.d_latent + d.d_rope, d.d_model), np.float32)
+    wd[:t.d_latent, :t.d_model] = w.w_down[:t.d_latent]
+    _pad_rotary(wd[d.d_latent:, :t.d_model].T, w.w_down[t.d_latent:].T)
+    wuk = np.zeros((d.n_heads, d.d_nope, d.d_latent), np.float32)
+    wuk[:, :t.d_nope, :t.d_latent] = w.w_uk
+    wuv = np.zeros((d.n_heads, d.d_head, d.d_latent), np.float32)
+    wuv[:, :t.d_head, :t.d_latent] = w.w_uv
+    cfg = api.config_from_dims(d)
+    m = api.LatentKVAttention(cfg).allocate(design=design)
+    W = [to_dev(a, d) for a in (wd, wuk, wuv)]
+    frame_x = {}
+    chunk = 6
+    for c in range(chunk + 1):
+        x = synth.activations(t, 0, c)
+        xp = np.zeros((1, x.shape[1], d.d_model), np.float32)
+        xp[..., :t.d_model] = x
+        m.append(0, to_dev(xp, d), W[0], c, 1)
+        frame_x[c] = x[0]
+    s8 = np.float32(np.sqrt(8.0))
+    q = synth.queries(t, 0, chunk)
+    qp = np.zeros((1, q.shape[1], d.n_heads, d.d_head), np.float32)
+    qp[..., :t.d_nope] = q[..., :t.d_nope] * s8
+    _pad_rotary(qp[..., d.d_nope:], q[..., t.d_nope:] * s8)
+    qp_dev = to_dev(qp, d)
+    out = torch.full((1, d.n_queries, d.n_heads * d.d_head), float("nan"), dtype=torch.float32, device="cuda")
+    m.attention(0, qp_dev, W[1], W[2], out, chunk, 1, design)
+    st, flags = m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    got = out.cpu().numpy().reshape(d.n_queries, d.n_heads, d.d_head)
+    m.close()
+    qb = qp_dev.float().cpu().numpy().astype(np.float64) / np.sqrt(8.0)  # the padded queries as stored, rescaled
+    q_oracle = np.concatenate([qb[0, :, :, :t.d_nope],
+                               np.stack([qb[0, :, :, d.d_nope + 2 * p + e] for p in _PAD_PAIR for e in (0, 1)],
+                                        axis=-1)], axis=-1)
+    ref = oracle_chunk(t, w, frame_x, chunk, q_oracle).reshape(t.n_queries, t.n_heads, t.d_head)
+    assert np.all(got[:, :, t.d_head:] == 0), "padded value columns"
+    assert_bf16_close(got[:, :, :t.d_head].reshape(t.n_queries, -1), ref.reshape(t.n_queries, -1),
+                      f"tiny layer zero-padded, design {design}")
+
+
+@pytest.mark.parametrize("tiling", [(1, 1, 0), (2, 0, 0), (2, 0, 1), (1, 2, 1)], ids=lambda t: "np%d_mt%d_ctas%d" % t)
 def test_small_bf16_attention_after_tiled_appends(tiling):
     """The full path with a forced append tiling, against the oracle."""
     ro = Rollout(SMALL)
