@@ -241,31 +241,6 @@ int attn_dense_block_n();
 cudaError_t launch_attn_dense_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_out,
                                  const AttnTc& a, int batch, cudaStream_t s, bool f16);
 
-// Per-head attention, d_head = 128, two query tiles per CTA and a stream-K split of the
-// (tile pair, key tile) iterations over `ctas` CTAs (attn_pp.cu).  Maps as launch_attn_dense_tc;
-// the output rows go straight from registers to `out` ([B][n_q][n_h*128] fp32).  Pairs whose keys
-// are split leave partials in `part` / `part_ml` (attn_pp_partial_bytes), combined by a second
-// kernel in the same launch call.
-constexpr int kAttnPPMaxCtas = 160;
-struct AttnPP {
-  int n_q, n_keys, n_heads, m_tiles;
-  float scale_log2;
-  float rescale_threshold;
-  unsigned* err;
-  uint64_t limit_ns;
-  int h0 = 0, h_count = 0;  // heads of this launch
-  // filled by attn_pp_plan
-  int pairs_per_bh = 0, n_kt = 0, ctas = 0;
-  int64_t iters = 0;
-  float* out = nullptr;      // [B][n_q][n_h*128]
-  float* part = nullptr;     // [2*kAttnPPMaxCtas][2][128][128]
-  float* part_ml = nullptr;  // [2*kAttnPPMaxCtas][2][128][2]
-};
-constexpr size_t attn_pp_partial_bytes() { return (size_t)2 * kAttnPPMaxCtas * 2 * 128 * (128 + 2) * 4; }
-AttnPP attn_pp_plan(AttnPP a, int batch, int sms);
-cudaError_t launch_attn_pp(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const AttnPP& a, cudaStream_t s,
-                           bool f16);
-
 struct DenseQTc {  // q' = [q_nope | RoPE(q_rope)] -> [B][n_h][n_q][128]
   const __nv_bfloat16* q;
   void* qd;                         // bf16, or fp16 when f16

@@ -313,28 +313,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       : "memory");
 }
 
-// Load 128 consecutive columns (four x32 loads) with a single wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
-      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : VMLA_R8(0), VMLA_R8(8), VMLA_R8(16), VMLA_R8(24), VMLA_R8(32), VMLA_R8(40), VMLA_R8(48), VMLA_R8(56),
-        VMLA_R8(64), VMLA_R8(72), VMLA_R8(80), VMLA_R8(88), VMLA_R8(96), VMLA_R8(104), VMLA_R8(112), VMLA_R8(120)
-      : "r"(taddr), "r"(taddr + 32u), "r"(taddr + 64u), "r"(taddr + 96u)
-      : "memory");
-}
-
 // Load 48 consecutive columns (x32 at taddr, x16 at taddr + 32) with a single wait.
 __device__ __forceinline__ void tmem_ld48(uint32_t taddr, uint32_t (&r)[48]) {
   asm volatile(

@@ -120,7 +120,7 @@ int64_t ring_rows(const vmla_config& c) { return (int64_t)c.window_frames * toke
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, obar = 0, part = 0, recon = 0;  // offsets
+  size_t kr_rot = 0, qt = 0, dq = 0, chunk = 0, obar = 0, recon = 0;  // offsets
   size_t base_bytes = 0;   // every design but RECON_ONCE
   size_t recon_bytes = 0;  // extra for RECON_ONCE
 };
@@ -141,8 +141,6 @@ WsLayout ws_layout(const vmla_config& c) {
   off = align256(off + B * (size_t)c.window_frames * tokens_per_frame(c) * (size_t)(c.d_latent + 2 * c.d_rope) * e);
   w.obar = off;  // the folded output mixer's input: O_bar as a bf16 pair [2][B][rows][n_h * d_c]
   off = align256(off + (c.dtype == VMLA_BF16 ? 2 * B * nq * c.n_heads * (size_t)c.d_latent * 2 : 0));
-  w.part = off;  // partial rows of the per-head attention's split pairs (fp32)
-  off = align256(off + (c.dtype == VMLA_BF16 ? attn_pp_partial_bytes() : 0));
   w.recon = off;
   w.base_bytes = off;
   w.recon_bytes = B * ring_rows(c) * 2 * (size_t)c.n_heads * c.d_value * e;
@@ -209,7 +207,7 @@ struct vmla_handle {
   std::vector<int64_t> dense_frames;  // dense cache, per layer
   unsigned* err = nullptr;            // device status word (resolved at bind)
   int append_split = 0;               // append work split (0: chosen per call), see vmla_set_append_tiling
-  int append_rows = 0;                // 128-row tiles per append work item (0: chosen per call)
+  int append_rows = 0;                // 128-row tiles per append work item (0 or 1: one; 2: two)
   int append_ctas = 0;
   bool profiling = false;
   struct Timer {
@@ -972,41 +970,11 @@ vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const voi
   a.rescale_threshold = c.softmax_rescale_log2;
   a.err = h->err;
   a.limit_ns = kWaitLimitNs;
-#ifndef VMLA_PER_HEAD_PAIRS
-  // one query tile per CTA (the absorbed kernel's pipeline with per-head tiles)
   if (hout)
     return cuda_status(launch_head_groups(c, nq, a, out, hout, s, [&](const AttnTc& ag) {
       return launch_attn_dense_tc(tq, tkv, to, ag, c.batch, s, f16);
     }));
   return cuda_status(launch_attn_dense_tc(tq, tkv, to, a, c.batch, s, f16));
-#else
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
-  }
-  float* part = at<float>(h->ws, w.part);
-  auto pp = [&](const AttnTc& ag) {
-    AttnPP p;
-    p.n_q = ag.n_q;
-    p.n_keys = ag.n_keys;
-    p.n_heads = ag.n_heads;
-    p.m_tiles = ag.m_tiles;
-    p.scale_log2 = ag.scale_log2;
-    p.rescale_threshold = ag.rescale_threshold;
-    p.err = ag.err;
-    p.limit_ns = ag.limit_ns;
-    p.h0 = ag.h0;
-    p.h_count = ag.h_count;
-    p.out = static_cast<float*>(out);
-    p.part = part;
-    p.part_ml = part + (size_t)2 * kAttnPPMaxCtas * 2 * 128 * 128;
-    return launch_attn_pp(tq, tkv, attn_pp_plan(p, c.batch, sms), s, f16);
-  };
-  if (hout) return cuda_status(launch_head_groups(c, nq, a, out, hout, s, pp));
-  return cuda_status(pp(a));
-#endif
 }
 
 }  // namespace
