@@ -167,7 +167,8 @@ vmla_status vmla_workspace_bytes(const vmla_config* cfg, vmla_design design, siz
  * (for inspection and stage-by-stage checks; the workspace's contents after a call are those of
  * the last call that wrote them):
  *   [VMLA_WS_KR_ROT]  the window's positional keys rotated with window-relative t
- *                     [batch][W*T_f][d_rope] (RoPE at read only; ring-slot order)
+ *                     [batch][W*T_f][d_rope] (RoPE at read only; ring-slot order; ABSORBED and
+ *                     RECONSTRUCT: RECON_ONCE rotates them inside the reconstruction)
  *   [VMLA_WS_QT]      absorbed queries [batch][n_heads][n_q][d_latent + d_rope] (ABSORBED)
  *   [VMLA_WS_QD]      per-head queries with the positional part rotated [batch][n_heads][n_q][d_nope + d_rope]
  *                     (RECONSTRUCT, RECON_ONCE and the dense calls)

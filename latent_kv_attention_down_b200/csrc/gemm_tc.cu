@@ -572,14 +572,17 @@ __global__ void __launch_bounds__(QPrepCfg<DL, DR>::THREADS, 1)
 }
 
 // ============================================================== per-head reconstruction
-// Persistent over (sample, 128-row tile, head) items, head fastest so that the
-// CTAs working at one time share the latent tile in L2.  Per item the
+// Persistent over (sample, 128-row tile, head) items, head fastest, each CTA taking a
+// contiguous run of them: the heads of a key tile follow each other in one CTA, which
+// reads the tile's latents from L2 once per head and its positional keys once (one
+// tile ahead), rotating them with the window-relative t when asked (reconstruct-once
+// at read time) or the absolute frame (the dense cache).  Per item the
 // reduction over d_latent runs through a ring of [128 rows x 64] latent blocks
 // and [(d_nope + 128) x 64] blocks of [W_uk,h ; W_uv,h] (any d_latent a multiple of 64);
 // two TMEM accumulators alternate so the epilogue of one item overlaps the
 // next; two epilogue warpgroups park the item's 128 rows as [k_h (128) | v_h
-// (128)] -- the first k_h (d_nope content columns from TMEM, the d_rope
-// positional columns read one item ahead), the second v_h.  With TMA_OUT (rows
+// (128)] -- the first k_h (d_nope content columns from TMEM, then the d_rope
+// positional columns), the second v_h.  With TMA_OUT (rows
 // written to consecutive rows: the window of reconstruct-once) the park is four
 // 128-byte-swizzled [128 x 64] blocks that four TMA tensor stores write out,
 // clipped at the last key, while the threads go on to the next item; otherwise
@@ -600,7 +603,8 @@ struct ReconCfg {
   static constexpr int FIT = (212 * 1024 - OUT_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 6 ? 6 : FIT;
   static constexpr uint32_t TMEM_COLS = 512;  // two accumulators of N columns, at 0 and 256
-  static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 128 * 8 + 256;
+  static constexpr int TAB = 1024;  // (cos, sin) entries of the window's rotary positions (window_t)
+  static constexpr int SMEM = 1024 + STAGES * STAGE + OUT_BYTES + 128 * 8 + 256 + TAB * 8;
   static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 two epilogue warpgroups
   static_assert(DR == 16 || DR == 32 || DR == 64 || DR == 96, "rotary dims");
   static_assert(N % 16 == 0 && N <= 256 && (DN * 128) % 1024 == 0, "MMA shape / swizzle atoms");
@@ -657,9 +661,19 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
   uint64_t* done = acc_empty + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  float2* rtab = reinterpret_cast<float2*>(sout + C::OUT_BYTES + 128 * 8 + 256);  // C::TAB entries
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (a.rows + 127) / 128;
   const Guard g{abort_flag, a.err, a.limit_ns};
+  // window-relative rotation: (cos, sin) of every pair at every t of the window (0..W-1) and every
+  // grid row and column, looked up per key (equal to the direct evaluation); wider windows or grids
+  // than the table holds evaluate directly
+  const RopeTable rt = rope_table_shape(a.rope, a.ring.window_frames * a.ring.tokens_per_frame, a.ring);
+  const bool use_tab = a.window_t && !a.rotate && rt.n <= C::TAB;
+  // a contiguous run of items per CTA (head fastest): the heads of a key tile follow each other,
+  // so its positional keys are read and rotated once for all of them
+  const int it_begin = (int)((int64_t)items * blockIdx.x / gridDim.x);
+  const int it_end = (int)((int64_t)items * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * C::STAGES; ++i) mbar_init(&full[i], 1);  // full[], empty[]
@@ -683,7 +697,7 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
       prefetch_tmap(&tm_wuk);
       prefetch_tmap(&tm_wuv);
       int it = 0;
-      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+      for (int item = it_begin; item < it_end && !*abort_flag; ++item) {
         const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
         for (int kb = 0; kb < C::NKB; ++kb, ++it) {
           const int s = it % C::STAGES;
@@ -704,7 +718,7 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, false, false);
       int it = 0, j = 0;
-      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      for (int item = it_begin; item < it_end; ++item, ++j) {
         const int acc = j & 1;
         if (!wait_phase(&acc_empty[acc], ((j >> 1) & 1) ^ 1, g, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
@@ -735,7 +749,7 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128;
     const int T = a.ring.tokens_per_frame;
-    // warpgroup 0 reads each item's positional keys (DR * 2 bytes of its row) one item ahead
+    // warpgroup 0 reads each key tile's positional keys (DR * 2 bytes of its row) one tile ahead
     constexpr int RQ = DR / 8;  // 16-byte pieces of a positional key
     uint4 krq[RQ] = {};
     auto load_kr = [&](int item) {
@@ -748,12 +762,15 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
         for (int k = 0; k < RQ; ++k) krq[k] = src[k];
       }
     };
-    if (wg == 0 && (int)blockIdx.x < items) load_kr(blockIdx.x);
+    if (wg == 0 && it_begin < it_end) load_kr(it_begin);
+    if (use_tab) rope_table_fill(rtab, rt, a.rope, 0, tid, 256);
+    named_bar_sync(1, 256);  // the table is complete
     int j = 0;
-    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+    float kr[DR];      // warpgroup 0: this row's positional key, decoded and rotated, of key tile kr_tile
+    int kr_tile = -1;
+    for (int item = it_begin; item < it_end; ++item, ++j) {
       const int h = item % a.n_heads, mt = (item / a.n_heads) % m_tiles, b = item / (a.n_heads * m_tiles);
       const int acc = j & 1;
-      float kr[DR];
       if (wg == 0) {
         const int m = mt * 128 + r;
         const int mm = m < a.rows ? m : 0;
@@ -761,23 +778,33 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
         const int tok = mm % T;
         const int64_t row = a.to_ring ? ring_frame_slot(a.ring, frame) * T + tok : mm;
         row_k[r] = (((int64_t)b * a.ring_rows + row) * 2 * a.n_heads + h) * 128;
+        if (item / a.n_heads != kr_tile) {  // a new key tile: decode, prefetch the next, rotate
+          kr_tile = item / a.n_heads;
 #pragma unroll
-        for (int k = 0; k < RQ; ++k) {
-          const uint32_t w4[4] = {krq[k].x, krq[k].y, krq[k].z, krq[k].w};
+          for (int k = 0; k < RQ; ++k) {
+            const uint32_t w4[4] = {krq[k].x, krq[k].y, krq[k].z, krq[k].w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if constexpr (F16) {  // fp16 pairs (the workspace's window keys)
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
-              kr[8 * k + 2 * e] = f.x;
-              kr[8 * k + 2 * e + 1] = f.y;
-            } else {
-              kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
-              kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+            for (int e = 0; e < 4; ++e) {
+              if (a.kr_f16) {  // fp16 pairs
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
+                kr[8 * k + 2 * e] = f.x;
+                kr[8 * k + 2 * e + 1] = f.y;
+              } else {
+                kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+                kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+              }
             }
           }
+          if ((kr_tile + 1) * a.n_heads < it_end) load_kr((kr_tile + 1) * a.n_heads);
+          if (a.rotate || a.window_t) {
+            // absolute frame, or the window-relative t of ring frame slot mm / T (to_ring 0)
+            const int tt = a.rotate ? (int)frame : ring_slot_t(a.ring, mm / T, a.window_start_slot);
+            if (use_tab)
+              rotate_pairs_tab<DR / 2>(kr, rtab, rt, a.rope, tt, tok / a.ring.grid_w, tok % a.ring.grid_w);
+            else
+              rotate_pairs<DR / 2>(kr, a.rope, tt, tok / a.ring.grid_w, tok % a.ring.grid_w);
+          }
         }
-        if (item + (int)gridDim.x < items) load_kr(item + gridDim.x);
-        if (a.rotate) rotate_pairs<DR / 2>(kr, a.rope, (int)frame, tok / a.ring.grid_w, tok % a.ring.grid_w);
       }
       const bool ok = wait_phase(&acc_full[acc], (j >> 1) & 1, g, DEV_ERR_TIMEOUT_EPILOGUE);
       __syncwarp();

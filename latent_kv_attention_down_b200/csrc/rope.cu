@@ -32,9 +32,7 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 
 // d_rope / 8 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its slot in
 // every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.  The stored
-// bf16 keys are rotated (or, when they were rotated at append, only converted) and written as bf16,
-// or as fp16 for the per-head keys of reconstruct-once: one rounding of 2^-11 relative there, where
-// a second bf16 rounding would add 2^-8.
+// bf16 keys are rotated (or, when they were rotated at append, only copied) and written as bf16.
 __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int nq = a.d_rope >> 3;  // 16-byte pieces of a key
@@ -67,7 +65,7 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
       for (int p = 0; p < 4; ++p) {
         float u = bf_lo(in[p]), x = bf_hi(in[p]);
         rope_apply(u, x, cs[p]);
-        out[p] = a.out_f16 ? pack_h2(u, x) : pack2(u, x);
+        out[p] = pack2(u, x);
       }
       dst[(b0 + k) * stride] = make_uint4(out[0], out[1], out[2], out[3]);
     }

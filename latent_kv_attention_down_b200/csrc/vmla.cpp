@@ -715,18 +715,17 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   const int64_t t_first = first - (at_read ? win.t_origin : 0);
   __nv_bfloat16* ckv_layer = at<__nv_bfloat16>(h->ckv, layer_cache_offset(c, layer, c.d_latent));
   __nv_bfloat16* kr_layer = at<__nv_bfloat16>(h->kr, layer_cache_offset(c, layer, c.d_rope));
-  // the window's positional keys, rotated with window-relative t into the workspace; reconstruct-once
-  // takes them in fp16 (converted there too when they were rotated at append: its per-head keys are
-  // fp16), the other designs in bf16 (the cache's own values when rotated at append)
-  const bool kr_f16 = design == VMLA_DESIGN_RECON_ONCE;
+  // the window's positional keys, rotated with window-relative t into the workspace (bf16; the
+  // cache's own values when rotated at append).  Reconstruct-once rotates them itself while it
+  // rebuilds the per-head keys, so it takes the cache's keys as they are.
+  const bool recon_once = design == VMLA_DESIGN_RECON_ONCE;
   const void* kpos = kr_layer;
   cudaError_t e = cudaSuccess;
-  if (at_read || kr_f16) {
+  if (at_read && !recon_once) {
     StageScope scope(h, 1, s);
     RopeWindow r{kr_layer, at<char>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
                  make_ring(c), make_rope(c)};
-    r.rotate = at_read;
-    r.out_f16 = kr_f16;
+    r.rotate = 1;
     e = launch_rope_window_bf16(r, s);
     kpos = at<char>(h->ws, w.kr_rot);
   }
@@ -756,7 +755,9 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
       a.d_latent = c.d_latent;
       a.d_rope = c.d_rope;
       a.first_frame = 0;
-      a.rotate = 0;  // positional keys are already rotated (at read into the workspace, or at append)
+      a.rotate = 0;
+      a.window_t = at_read;  // rotated here with window-relative t (or already at append)
+      a.window_start_slot = win.start_slot;
       a.to_ring = 0;
       a.kr_rows = rr;
       a.kr_stride = c.d_rope;

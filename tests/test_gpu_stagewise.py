@@ -231,8 +231,10 @@ def test_stages_of_the_reconstruct_once_design(dims, chunks):
     pos, frames, ts = slot_positions(ro, F)
     n_keys = len(frames) * d.tokens_per_frame
     fr = freqs_of(d)
-    # the window's positional keys, rotated for this call and kept in fp16 for the per-head keys
-    kr_rot = workspace(ro, api.WS_KR_ROT, (d.batch, d.window_tokens, d.d_rope), fp16=True)[0, :n_keys]
+    # the window's positional keys, rotated for this call by the reconstruction and kept in fp16 in
+    # every head's key (head 0's copy here; the others must equal it)
+    recon = workspace(ro, api.WS_RECON, (d.batch, d.window_tokens, 2, d.n_heads, d.d_head), fp16=True)[0, :n_keys]
+    kr_rot = recon[:, 0, 0, d.d_nope:]
     ang = O.rope_angles(pos[:n_keys, 0], pos[:n_keys, 1], pos[:n_keys, 2], fr)
     pair = np.repeat(np.sqrt(kr[0, :n_keys, 0::2] ** 2 + kr[0, :n_keys, 1::2] ** 2), 2, axis=1)
     assert_rounded_once(kr_rot, O.rope_rotate(kr[0, :n_keys], ang), 16 * pair, "window RoPE (fp16)", u=U_F16,
@@ -254,7 +256,6 @@ def test_stages_of_the_reconstruct_once_design(dims, chunks):
                             f"q rope, head {h}", u=U_F16, floor=F16_TINY)
 
     # reconstruction in fp16: K_h = [W_uk,h c | k_R rotated], V_h = W_uv,h c from the stored cache
-    recon = workspace(ro, api.WS_RECON, (d.batch, d.window_tokens, 2, d.n_heads, d.d_head), fp16=True)[0, :n_keys]
     c = ckv[0, :n_keys]
     keys = np.arange(n_keys) if n_keys <= 8192 else np.sort(np.random.default_rng(1).choice(n_keys, 8192, False))
     for h in range(d.n_heads):
