@@ -221,6 +221,10 @@ struct vmla_handle {
   // ... and the output comes back on a second one, a group of heads at a time
   cudaStream_t out_stream = nullptr;
   cudaEvent_t out_group = nullptr, out_done = nullptr;
+  // reconstruct-once: the per-head queries are prepared on a stream of the handle's own while the
+  // reconstruction runs on the caller's
+  cudaStream_t side_stream = nullptr;
+  cudaEvent_t side_fork = nullptr, side_join = nullptr;
 };
 
 namespace {
@@ -433,10 +437,12 @@ vmla_status vmla_destroy(vmla_handle* h) {
   if (!h) return VMLA_ERR_INVALID_ARG;
   for (auto& t : h->timers)
     for (cudaEvent_t e : t.ev) cudaEventDestroy(e);
-  for (cudaEvent_t e : {h->x_ready, h->q_ready, h->x_free, h->q_free, h->out_group, h->out_done})
+  for (cudaEvent_t e : {h->x_ready, h->q_ready, h->x_free, h->q_free, h->out_group, h->out_done, h->side_fork,
+                        h->side_join})
     if (e) cudaEventDestroy(e);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   if (h->out_stream) cudaStreamDestroy(h->out_stream);
+  if (h->side_stream) cudaStreamDestroy(h->side_stream);
   delete h;
   return VMLA_OK;
 }
@@ -684,9 +690,11 @@ cudaError_t launch_head_groups(const vmla_config& c, int nq, AttnTc a, const voi
   return e;
 }
 
+vmla_status dense_q_launch(vmla_handle* h, const void* q, int nq, int64_t t_first, cudaStream_t s, bool f16,
+                           HostOut* hout);
 vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q_dev, const void* kv_base, void* out, int nq,
                                         int n_keys, int64_t t_first, int stage, cudaStream_t s, bool f16,
-                                        HostOut* hout = nullptr);
+                                        HostOut* hout = nullptr, bool q_done = false);
 
 // The folded output mixer: out = O_bar W_fold^T instead of the per-head W_uv,h.
 struct FoldArgs {
@@ -735,6 +743,19 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
   if (design == VMLA_DESIGN_RECON_ONCE) {
     if (h->ws_bytes < w.base_bytes + w.recon_bytes) return VMLA_ERR_STATE;
     __nv_bfloat16* recon = at<__nv_bfloat16>(h->ws, w.recon);
+    // the per-head queries (independent of the reconstruction) on the handle's side stream, forked
+    // from and joined back into `s`
+    if (!h->side_stream) {
+      if ((e = cudaStreamCreateWithFlags(&h->side_stream, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+      for (cudaEvent_t* ev : {&h->side_fork, &h->side_join})
+        if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+    }
+    if ((e = cudaEventRecord(h->side_fork, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(h->side_stream, h->side_fork, 0)) != cudaSuccess)
+      return cuda_fail(e);
+    vmla_status qs = dense_q_launch(h, q, nq, t_first, h->side_stream, true, hout);
+    if (qs != VMLA_OK) return qs;
+    if ((e = cudaEventRecord(h->side_join, h->side_stream)) != cudaSuccess) return cuda_fail(e);
     {
       StageScope scope(h, 7, s);
       CUtensorMap tc, tuk, tuv;
@@ -773,8 +794,8 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
         return map_fail();
       e = launch_recon_tc(tc, tuk, tuv, &to, a, c.batch, s);
     }
-    if (e != cudaSuccess) return cuda_fail(e);
-    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, true, hout);
+    if (e != cudaSuccess || (e = cudaStreamWaitEvent(s, h->side_join, 0)) != cudaSuccess) return cuda_fail(e);
+    return dense_attention_bf16_launch(h, q, recon, out, nq, win.n_keys, t_first, 6, s, true, hout, true);
   }
   if (design == VMLA_DESIGN_RECONSTRUCT) {
     __nv_bfloat16* qd = at<__nv_bfloat16>(h->ws, w.dq);
@@ -933,23 +954,32 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
 
 // Dense d_head = 128 attention on a per-head K/V buffer [B][ring_rows][2][n_h][128]: bf16 (the
 // dense cache) or, with f16, fp16 (the reconstruct-once workspace; the queries then go fp16 too).
-vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const void* kv_base, void* out, int nq,
-                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, bool f16,
-                                        HostOut* hout) {
+// The per-head queries [B][n_h][n_q][128] in the workspace: q_nope copied, q_rope rotated.
+vmla_status dense_q_launch(vmla_handle* h, const void* q, int nq, int64_t t_first, cudaStream_t s, bool f16,
+                           HostOut* hout) {
   const vmla_config& c = h->cfg;
   const WsLayout w = ws_layout(c);
-  void* qd = at<char>(h->ws, w.dq);
   cudaError_t e;
   {
     StageScope scope(h, 2, s);
-    DenseQTc a{static_cast<const __nv_bfloat16*>(q), qd, c.batch, nq, c.n_heads, c.d_rope, t_first, make_ring(c),
-               make_rope(c)};
+    DenseQTc a{static_cast<const __nv_bfloat16*>(q), at<char>(h->ws, w.dq), c.batch, nq, c.n_heads, c.d_rope,
+               t_first, make_ring(c), make_rope(c)};
     a.f16 = f16;
     a.err = h->err;
     e = launch_dense_q_bf16(a, s);
   }
   if (e == cudaSuccess) e = note_q_read(hout, s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  return e == cudaSuccess ? VMLA_OK : cuda_fail(e);
+}
+
+vmla_status dense_attention_bf16_launch(vmla_handle* h, const void* q, const void* kv_base, void* out, int nq,
+                                        int n_keys, int64_t t_first, int stage, cudaStream_t s, bool f16,
+                                        HostOut* hout, bool q_done) {
+  const vmla_config& c = h->cfg;
+  const WsLayout w = ws_layout(c);
+  void* qd = at<char>(h->ws, w.dq);
+  vmla_status st;
+  if (!q_done && (st = dense_q_launch(h, q, nq, t_first, s, f16, hout)) != VMLA_OK) return st;
   StageScope scope(h, stage, s);
   const uint64_t rr = ring_rows(c);
   const uint64_t row_bytes = 2ull * c.n_heads * 128 * 2;
