@@ -784,15 +784,9 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
           for (int k = 0; k < RQ; ++k) {
             const uint32_t w4[4] = {krq[k].x, krq[k].y, krq[k].z, krq[k].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (a.kr_f16) {  // fp16 pairs
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
-                kr[8 * k + 2 * e] = f.x;
-                kr[8 * k + 2 * e + 1] = f.y;
-              } else {
-                kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
-                kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
-              }
+            for (int e = 0; e < 4; ++e) {  // bf16 pairs
+              kr[8 * k + 2 * e] = __uint_as_float(w4[e] << 16);
+              kr[8 * k + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
             }
           }
           if ((kr_tile + 1) * a.n_heads < it_end) load_kr((kr_tile + 1) * a.n_heads);

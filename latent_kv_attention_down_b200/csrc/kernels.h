@@ -74,7 +74,6 @@ struct RopeWindow {  // rotate the window's positional keys with window-relative
   int window_start_slot;  // (ring slot of the oldest local frame) - sink_frames
   Ring ring;
   Rope rope;
-  int rotate = 1;    // bf16 path: 0 only converts (keys rotated at append)
 };
 cudaError_t launch_rope_window_f32(const RopeWindow& a, cudaStream_t s);
 cudaError_t launch_rope_window_bf16(const RopeWindow& a, cudaStream_t s);
@@ -253,15 +252,14 @@ struct DenseQTc {  // q' = [q_nope | RoPE(q_rope)] -> [B][n_h][n_q][128]
 cudaError_t launch_dense_q_bf16(const DenseQTc& a, cudaStream_t s);
 
 struct ReconTc {  // per-head dense entries from latents (tcgen05)
-  const void* kr;           // positional keys [B][kr_rows][d_rope], bf16 or (kr_f16) fp16; unrotated
-                            // when rotate or window_t is set
+  const void* kr;           // positional keys [B][kr_rows][d_rope], bf16; unrotated when rotate or
+                            // window_t is set
   void* dense;              // [B][ring_rows][2][n_h][128], bf16 or (f16) fp16
   int f16;                  // fp16 entries (DEV_ERR_RANGE for a value past 65504)
   int rows, n_heads, d_latent, d_rope;  // d_rope 16, 32, 64 or 96 (d_nope = 128 - d_rope)
   int64_t first_frame;      // frame of row 0 (ring placement and absolute t)
   int rotate;               // rotate kr with the absolute frame index
   int to_ring;              // 1: row m -> ring slot of its frame; 0: row m -> row m
-  int kr_f16 = 0;           // kr holds fp16 (else bf16)
   int window_t = 0;         // rotate kr with the window-relative t of row m's ring slot (to_ring 0)
   int window_start_slot = 0;  // (ring slot of the oldest local frame) - sink_frames, for window_t
   int64_t kr_rows;          // rows per sample of kr

@@ -32,7 +32,7 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 
 // d_rope / 8 threads per key slot, 16 bytes (4 rotary pairs) each; a thread takes its slot in
 // every sample, so the (cos, sin) of its 4 pairs are computed once for the batch.  The stored
-// bf16 keys are rotated (or, when they were rotated at append, only copied) and written as bf16.
+// bf16 keys are rotated and written as bf16.
 __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow a) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int nq = a.d_rope >> 3;  // 16-byte pieces of a key
@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256) rope_window_bf16_kernel(const RopeWindow 
   const int hh = tok / a.ring.grid_w, ww = tok % a.ring.grid_w;
   float2 cs[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) cs[k] = a.rotate ? rope_cs(a.rope, quad * 4 + k, t, hh, ww) : make_float2(1.f, 0.f);
+  for (int k = 0; k < 4; ++k) cs[k] = rope_cs(a.rope, quad * 4 + k, t, hh, ww);
   const uint4* src =
       reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.kr) + (int64_t)s * a.d_rope + quad * 8);
   uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.kr_rot) + (int64_t)s * a.d_rope + quad * 8);

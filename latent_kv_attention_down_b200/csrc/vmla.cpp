@@ -733,7 +733,6 @@ vmla_status attention_bf16(vmla_handle* h, int layer, const void* q, const void*
     StageScope scope(h, 1, s);
     RopeWindow r{kr_layer, at<char>(h->ws, w.kr_rot), c.batch, win.n_keys, c.d_rope, win.start_slot,
                  make_ring(c), make_rope(c)};
-    r.rotate = 1;
     e = launch_rope_window_bf16(r, s);
     kpos = at<char>(h->ws, w.kr_rot);
   }
