@@ -415,6 +415,10 @@ def run_ours(args, rank, world, local_rank):
     kernels = {("per_head_queries" if auto_design == "recon_once" and k == "q_absorb" else k): dict(v)
                for k, v in per_kernel.items()}
     kernels = with_bytes(kernels, recon_bytes if auto_design == "recon_once" else absorbed_bytes)
+    if "per_head_queries" in kernels:
+        # launched on the handle's side stream beside the reconstruction: its event time spans the
+        # overlap, not the kernel alone
+        kernels["per_head_queries"]["overlapped_with"] = "reconstruct_once"
     abs_kernels = with_bytes({k: dict(v) for k, v in abs_kernels.items()}, absorbed_bytes)
 
     workload = ("wan1.3b-layer chunk step: append 3 frames + attention with the design AUTO takes "
