@@ -610,17 +610,18 @@ def test_wan_layer_first_chunk_auto():
     assert_bf16_close(out[0][rows], ro.oracle(0, 0, q, rows=rows), "wan layer, first chunk")
 
 
-def test_wide_grid_rotary_pairs_evaluated_directly():
-    """A 4 x 520 latent grid: the chunk's rotary (cos, sin) pairs no longer fit the q-absorb
-    kernel's per-CTA table (the w axis alone has 5 x 520 entries), so that kernel evaluates
-    them per row; two chunks (12480 keys, 6240 queries), 256 seeded query rows checked for
-    every head."""
+@pytest.mark.parametrize("design", [api.DESIGN_ABSORBED, api.DESIGN_RECON_ONCE])
+def test_wide_grid_rotary_pairs_evaluated_directly(design):
+    """A 4 x 520 latent grid: the rotary (cos, sin) pairs no longer fit the per-CTA tables (the w
+    axis alone has 5 x 520 entries), so the q-absorb kernel (absorbed design) evaluates them per
+    query row and the reconstruction (reconstruct-once) per key; two chunks (12480 keys, 6240
+    queries), 256 seeded query rows checked for every head."""
     d = SMALL.replace(name="wan_wide_grid", grid_h=4, grid_w=520)
-    ro = Rollout(d)
+    ro = Rollout(d, design=design)
     _fill(ro, 2)
-    out, q = ro.attend(0, 1)
+    out, q = ro.attend(0, 1, design=design)
     rows = sampled_rows(d.n_queries)
-    assert_bf16_close(out[0][rows], ro.oracle(0, 1, q, rows=rows), "wide grid")
+    assert_bf16_close(out[0][rows], ro.oracle(0, 1, q, rows=rows), f"wide grid, design {design}")
 
 
 # ------------------------------------------------------------------ W_uv folded into the output mixer
