@@ -218,7 +218,11 @@ vmla_status vmla_cache_append(vmla_handle* h, int layer, const void* x, const vo
  * out:  [batch][n_frames*T_f][n_heads*d_value], float32 for both dtypes (a bf16 rounding of the
  *       output alone would take two thirds of a 3e-2*RMS max-error budget: max |out| is about 5 RMS)
  * The chunk must be the newest appended frames: first_frame + n_frames == F,
- * 1 <= n_frames <= chunk_frames; otherwise VMLA_ERR_STATE. */
+ * 1 <= n_frames <= chunk_frames; otherwise VMLA_ERR_STATE.
+ * Everything is enqueued on `stream`; VMLA_DESIGN_RECON_ONCE prepares the per-head queries on a
+ * stream of the handle's own (created at its first such call), forked from `stream` by an event
+ * and joined back into it before the attention kernel, so the call stays ordered on `stream`
+ * (and can be captured in a CUDA graph from it). */
 vmla_status vmla_chunk_attention(vmla_handle* h, int layer, const void* q, const void* w_uk, const void* w_uv,
                                  void* out, int64_t first_frame, int n_frames, vmla_design design, void* stream);
 
@@ -273,9 +277,11 @@ vmla_status vmla_state_set(vmla_handle* h, int layer, int64_t frames_appended);
 vmla_status vmla_device_status(vmla_handle* h, void* stream, uint32_t* flags);
 
 /* Per-stage CUDA-event timing of the kernels each call launches, recorded on the
- * call's stream.  Stages: 0 append, 1 rope, 2 q-absorb, 3 attention (absorbed),
- * 4 attention (reconstruct), 5 dense append, 6 dense attention, 7 reconstruct-once,
- * 8 folded output mixer.
+ * stream each launches on.  Stages: 0 append, 1 rope, 2 query preparation (q-absorb; the
+ * per-head queries, which reconstruct-once runs on the handle's side stream beside the
+ * reconstruction, so their time there spans the overlap), 3 attention (absorbed), 4 attention
+ * (reconstruct), 5 dense append, 6 dense attention (also the reconstruct-once attention),
+ * 7 reconstruct-once (the reconstruction), 8 folded output mixer.
  * vmla_profile_read synchronises, then returns the summed milliseconds and the
  * launch count of one stage since profiling was enabled. */
 vmla_status vmla_profile_enable(vmla_handle* h, int enable);
