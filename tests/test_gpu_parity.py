@@ -575,6 +575,45 @@ def test_step_host_head_groups_match_device_path(design):
         assert np.array_equal(oh.numpy(), ref), f"chunk {chunk}: host step differs from the device path"
 
 
+@pytest.mark.parametrize("design", [api.DESIGN_AUTO, api.DESIGN_ABSORBED])
+def test_chunk_step_replayed_from_a_cuda_graph(design):
+    """One denoising pass of a chunk (append + attention) captured into a CUDA graph from the
+    caller's stream and replayed gives the bits of the same calls made eagerly: every launch is
+    enqueued on that stream, and reconstruct-once's side stream (the per-head queries) joins the
+    capture through its fork and join events.  The eager call comes first, so the handle's stream
+    and events exist before the capture."""
+    import torch
+    d = SMALL
+    ro = Rollout(d, design=design)
+    _fill(ro, 7)
+    chunk = 6
+    first = chunk * d.chunk_frames
+    x = to_dev(synth.activations(d, 0, chunk, 1), d)
+    q = to_dev(synth.queries(d, 0, chunk, 1), d)
+    wd = ro.wd[0]
+    out_e = torch.full((d.batch, d.n_queries, d.n_heads * d.d_head), float("nan"), dtype=torch.float32,
+                       device="cuda")
+    out_g = torch.full_like(out_e, float("nan"))
+    ro.m.append(0, x, wd[0], first, d.chunk_frames)
+    ro.m.attention(0, q, wd[1], wd[2], out_e, first, d.chunk_frames, design)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            ro.m.append(0, x, wd[0], first, d.chunk_frames)
+            ro.m.attention(0, q, wd[1], wd[2], out_g, first, d.chunk_frames, design)
+    torch.cuda.synchronize()
+    assert torch.isnan(out_g).all(), "capture must not run the kernels"
+    g.replay()
+    torch.cuda.synchronize()
+    st, flags = ro.m.device_status()
+    assert st == 0, f"device status {st} flags {flags:#x}"
+    assert torch.equal(out_g, out_e), "graph replay differs from the eager calls"
+    del g
+
+
 # ------------------------------------------------------------------ the full Wan-1.3B layer
 
 def test_wan_layer_full_every_design():
