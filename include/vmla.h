@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define VMLA_ABI_VERSION 2
+#define VMLA_ABI_VERSION 3
 
 typedef enum vmla_status {
   VMLA_OK = 0,

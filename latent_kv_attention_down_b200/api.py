@@ -23,7 +23,7 @@ STAGES = {"append": 0, "rope": 1, "q_absorb": 2, "attention": 3, "attention_reco
           "dense_append": 5, "dense_attention": 6, "reconstruct_once": 7, "folded_mixer": 8}
 
 
-ABI_VERSION = 2  # VMLA_ABI_VERSION of include/vmla.h that this binding's structures follow
+ABI_VERSION = 3  # VMLA_ABI_VERSION of include/vmla.h that this binding's structures follow
 
 
 class Config(ctypes.Structure):

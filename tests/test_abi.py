@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = api.lib()
-    assert lib.vmla_abi_version() == api.ABI_VERSION == 2
+    assert lib.vmla_abi_version() == api.ABI_VERSION == 3
     for code in range(9):
         assert lib.vmla_status_string(code).decode().startswith("VMLA_")
     assert lib.vmla_status_string(99).decode() == "VMLA_ERR_UNKNOWN"
