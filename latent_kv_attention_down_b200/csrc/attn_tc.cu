@@ -14,7 +14,8 @@
 // One CTA owns 128 query rows of one head of one sample and streams the whole
 // window in tiles of BN keys:
 //   warp 0      TMA producer: the query tile once, then K/V tiles into a ring
-//   warp 1      tcgen05.mma issuer (one thread) + TMEM owner
+//   warp 1      TMEM owner; tcgen05.mma issuer (one thread) of the absorbed design
+//   warps 2, 3  per-head tiles: the Q K^T and the P V issuers (one thread each)
 //   warps 4-11  two softmax warpgroups; thread r of either group owns query
 //               row r = TMEM lane r, each group half of every tile's keys
 // TMEM (512 columns): S0 [0,BN), S1 [BN,2BN), O [2BN, 2BN+DV).
@@ -26,6 +27,8 @@
 //   reuses S[j&1] once P V_j has read P_j (in-order tensor pipe).  Letting QK
 //   run further ahead would need a third resident K/V tile, and the 227 KB of
 //   shared memory then leave no room to prefetch the next one.
+// Per-head tiles (d_head 128) take 192 keys per tile (S0, S1 of 192 columns,
+//   O at 384) and release the K and V halves of a stage separately.
 // The running max is only raised when it grows by more than 2^threshold (lazy
 // rescale, 2^8 by default); O is then rescaled in TMEM after the previous P V
 // has finished.  Every mbarrier wait is bounded; a CTA that gives up records
@@ -42,8 +45,10 @@ constexpr int kSoftmaxWarps = 8;
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[kMaxStages];
-  uint64_t kv_empty[kMaxStages];
+  uint64_t kv_full[kMaxStages];   // the stage's tile landed (per-head tiles: its K half)
+  uint64_t kv_empty[kMaxStages];  // the stage may be reloaded (per-head tiles: its K half)
+  uint64_t v_full[kMaxStages];    // per-head tiles: the stage's V half landed
+  uint64_t v_empty[kMaxStages];   // per-head tiles: the stage's V half may be reloaded
   uint64_t s_full[3];  // S_j computed (MMA commit), by S buffer j % NSB
   uint64_t p_full[3];  // P_j stored over S_j by every softmax warp
   uint64_t p_done[3];  // P V_j has completed (MMA commit)
@@ -52,6 +57,7 @@ struct Bars {
   uint64_t ob_full;
   uint64_t epi_done;
   uint64_t drain;
+  uint64_t drain_pv;  // per-head tiles: the P V issuer's own drain
   uint32_t tslot;
   int abort_flag;
   float red[2][2][128];  // per-tile half-row maxima of the two softmax groups (tile parity, group, row)
@@ -67,7 +73,10 @@ struct AttnCfg {
   static constexpr int DR = DR_;                     // rotary dims of the shared key (absorbed)
   static constexpr int DQK = DENSE ? 128 : DL + DR;  // contraction width of S = Q K^T
   static constexpr int DV = DENSE ? 128 : DL;
-  static constexpr int BN = 128;
+  // keys per tile: 192 for per-head tiles (the softmax's fixed cost per tile -- loading S, the
+  // row max and its exchange, handing P over -- is spread over 1.5x the keys; TMEM holds two
+  // 192-column S buffers and O), 128 for the absorbed design's wider O
+  static constexpr int BN = DENSE ? 192 : 128;
   static constexpr int QB = DENSE ? 2 : DL / 64;  // 64-wide SW128 blocks of a query or key row
   // the rotary columns sit in NRB blocks of RB bytes per row, each swizzled at its width: one block
   // of DR * 2 bytes for 16, 32 or 64 rotary dims, three 64-byte blocks for 96
@@ -81,10 +90,10 @@ struct AttnCfg {
   static constexpr int BARS = (sizeof(Bars) + 127) / 128 * 128;
   static constexpr int STAGES_FIT = (SMEM_CAP - BARS - Q_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
-  // S buffers: S_j (and P_j over it) in buffer j % NSB at S_COL + (j % NSB) * BN.  Two: Q K^T
-  // runs one tile ahead of the softmax.  (Per-head tiles would leave TMEM for a third; with Q K^T
-  // two tiles ahead the MMA thread then waits for the K/V stage of tile j+2 -- free only once
-  // P V_{j-1} is done -- before it can issue P V_j, which measured 1.6x slower.)
+  // S buffers: S_j (and P_j over it) in buffer j % NSB at S_COL + (j % NSB) * BN: two, Q K^T one
+  // tile ahead of the softmax.  Per-head tiles have their K and V halves on barriers of their own
+  // (K_j is free once Q K_j^T is done, V_j once P V_j is), so a K tile is never held back by the
+  // P V of an older one.
   static constexpr int NSB = 2;
   static constexpr int S_COL = 0;
   static constexpr int O_COL = NSB * BN;
@@ -178,7 +187,10 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 
 template <int HS>
 __device__ __forceinline__ void ld_half_tile(uint32_t taddr, uint32_t (&r)[HS]) {
-  if constexpr (HS == 64) {
+  if constexpr (HS == 96) {
+    tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(&r[0]));
+    tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+  } else if constexpr (HS == 64) {
     tmem_ld64(taddr, r);
   } else if constexpr (HS == 48) {
     tmem_ld48(taddr, r);
@@ -236,6 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int k = 0; k < C::NSB; ++k) {
       mbar_init(&bars->s_full[k], 1);
@@ -247,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->ob_full, kSoftmaxWarps);
     mbar_init(&bars->epi_done, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain_pv, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -267,26 +282,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (!C::DENSE)
         for (int rb = 0; rb < C::NRB; ++rb)
           tma_load_3d(sQ + C::QB * 16384 + rb * 128 * C::RB, &tm_qr, &bars->q_full, DL + rb * (C::RB / 2), m0, qrow);
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % C::STAGES;
-        if (!wait_phase(&bars->kv_empty[s], ((j / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
-        uint8_t* st = sKV + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_BYTES);
-        if constexpr (C::DENSE) {
-          for (int kb = 0; kb < 2; ++kb) {
-            tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], h * 128 + kb * 64, j * C::BN, b);
-            tma_load_3d(st + (2 + kb) * C::KBLK, &tm_k, &bars->kv_full[s], (a.n_heads + h) * 128 + kb * 64,
-                        j * C::BN, b);
+      int issued = 0, issued_v = 0;  // tiles (per-head: K halves) and per-head V halves in flight
+      if constexpr (C::DENSE) {
+        // K_t, then V_{t-1}: a K half waits behind a V half whose stage frees one tile earlier
+        for (int t = 0; t <= n_tiles; ++t) {
+          if (t < n_tiles) {
+            const int s = t % C::STAGES;
+            if (!wait_phase(&bars->kv_empty[s], ((t / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+            uint8_t* st = sKV + s * C::STAGE_BYTES;
+            mbar_arrive_expect_tx(&bars->kv_full[s], 2 * C::KBLK);
+            for (int kb = 0; kb < 2; ++kb)
+              tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], h * 128 + kb * 64, t * C::BN, b);
+            ++issued;
           }
-        } else {
+          if (t > 0) {
+            const int v = t - 1, s = v % C::STAGES;
+            if (!wait_phase(&bars->v_empty[s], ((v / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+            uint8_t* st = sKV + s * C::STAGE_BYTES;
+            mbar_arrive_expect_tx(&bars->v_full[s], 2 * C::KBLK);
+            for (int kb = 0; kb < 2; ++kb)
+              tma_load_3d(st + (2 + kb) * C::KBLK, &tm_k, &bars->v_full[s], (a.n_heads + h) * 128 + kb * 64,
+                          v * C::BN, b);
+            ++issued_v;
+          }
+        }
+      } else {
+        for (int j = 0; j < n_tiles; ++j) {
+          const int s = j % C::STAGES;
+          if (!wait_phase(&bars->kv_empty[s], ((j / C::STAGES) & 1) ^ 1, g, DEV_ERR_TIMEOUT_PRODUCER)) break;
+          uint8_t* st = sKV + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&bars->kv_full[s], C::STAGE_BYTES);
           for (int kb = 0; kb < C::QB; ++kb)
             tma_load_3d(st + kb * C::KBLK, &tm_k, &bars->kv_full[s], kb * 64, j * C::BN, b);
           for (int rb = 0; rb < C::NRB; ++rb)
             tma_load_3d(st + C::QB * C::KBLK + rb * C::BN * C::RB, &tm_kr, &bars->kv_full[s], rb * (C::RB / 2),
                         j * C::BN, b);
+          ++issued;
         }
-        ++issued;
       }
       bool wuv_issued = false;
       if constexpr (!C::DENSE && !FOLD) {
@@ -304,11 +336,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_phase(&bars->q_full, 0, g);
         for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
           drain_phase(&bars->kv_full[j % C::STAGES], (j / C::STAGES) & 1, g);
+        for (int j = issued_v > C::STAGES ? issued_v - C::STAGES : 0; j < issued_v; ++j)
+          drain_phase(&bars->v_full[j % C::STAGES], (j / C::STAGES) & 1, g);
         if (wuv_issued) drain_phase(&bars->wuv_full, 0, g);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 && !C::DENSE) {
+    // ------------------------------------------------------------ MMA issuer (absorbed)
     // order: QK_0 .. QK_{NSB-2}, then per tile j: QK_{j+NSB-1}, P V_j.  QK_{j+NSB-1} goes into the
     // buffer that held P_{j-1}; P V_{j-1} was issued before it, and the tensor pipe runs in order.
     if (lane == 0) {
@@ -363,6 +397,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bars->abort_flag) {
         mma_commit(&bars->drain);
         drain_phase(&bars->drain, 0, g);
+      }
+    }
+  } else if (C::DENSE && (warp == 2 || warp == 3)) {
+    // ------------------------------------------------------------ per-head MMA issuers
+    // Q K^T from warp 2 and P V from warp 3 (one thread each, on SM sub-partitions of their own), so
+    // neither stream of MMAs waits behind the other's issue.  Ordering between them is by barriers:
+    // Q K_t^T overwrites the S buffer of P_{t-NSB} only once P V_{t-NSB} has completed.
+    if (lane == 0) {
+      const uint32_t sq = smem_u32(sQ), skv = smem_u32(sKV);
+      bool ok = true;
+      if (warp == 2) {
+        ok = wait_phase(&bars->q_full, 0, g, DEV_ERR_TIMEOUT_MMA);
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const int sb = t % C::NSB, s = t % C::STAGES;
+          if (t >= C::NSB &&
+              !(ok = wait_phase(&bars->p_done[sb], ((t - C::NSB) / C::NSB) & 1, g, DEV_ERR_TIMEOUT_MMA)))
+            break;
+          if (!(ok = wait_phase(&bars->kv_full[s], (t / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          issue_qk<C>(tbase + C::S_COL + sb * C::BN, sq, skv + s * C::STAGE_BYTES);
+          mma_commit(&bars->kv_empty[s]);
+          mma_commit(&bars->s_full[sb]);
+        }
+        if (bars->abort_flag) {
+          mma_commit(&bars->drain);
+          drain_phase(&bars->drain, 0, g);
+        }
+      } else {
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int sb = j % C::NSB, s = j % C::STAGES;
+          if (!(ok = wait_phase(&bars->p_full[sb], (j / C::NSB) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          if (!(ok = wait_phase(&bars->v_full[s], (j / C::STAGES) & 1, g, DEV_ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          issue_pv<C>(tbase + C::O_COL, tbase + C::S_COL + sb * C::BN, skv + s * C::STAGE_BYTES, j > 0);
+          mma_commit(&bars->v_empty[s]);
+          mma_commit(&bars->p_done[sb]);
+        }
+        if (ok) mma_commit(&bars->o_final);
+        if (bars->abort_flag) {
+          mma_commit(&bars->drain_pv);
+          drain_phase(&bars->drain_pv, 0, g);
+        }
       }
     }
   } else if (warp >= 4) {
@@ -446,16 +522,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         // row sum in four independent packed accumulators, bf16 pairs back into TMEM over S
         const float2 nm2 = make_float2(-m_run, -m_run);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        uint32_t packed[HS / 2];
+        if constexpr (HS % 32 == 0 && HS > 64) {
+          // wide tiles: P leaves in 16-column pieces as it is made, so the pieces' registers recycle
 #pragma unroll
-        for (int k = 0; k < HS / 2; ++k) {
-          const float2 x = make_float2(__uint_as_float(sraw[2 * k]), __uint_as_float(sraw[2 * k + 1]));
-          const float2 y = __ffma2_rn(x, sc2, nm2);
-          const float2 pr = exp2_mixed(y, k);
-          acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
-          packed[k] = C::F16 ? pack_f16x2(pr.x, pr.y) : pack_bf16x2(pr.x, pr.y);
+          for (int c = 0; c < HS / 32; ++c) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+              const int k = 16 * c + kk;
+              const float2 x = make_float2(__uint_as_float(sraw[2 * k]), __uint_as_float(sraw[2 * k + 1]));
+              const float2 y = __ffma2_rn(x, sc2, nm2);
+              const float2 pr = exp2_mixed(y, k);
+              acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
+              packed[kk] = C::F16 ? pack_f16x2(pr.x, pr.y) : pack_bf16x2(pr.x, pr.y);
+            }
+            tmem_st16_async(lane_base + C::S_COL + buf * C::BN + wg * (HS / 2) + 16 * c, packed);
+          }
+          tmem_wait_st();
+        } else {
+          uint32_t packed[HS / 2];
+#pragma unroll
+          for (int k = 0; k < HS / 2; ++k) {
+            const float2 x = make_float2(__uint_as_float(sraw[2 * k]), __uint_as_float(sraw[2 * k + 1]));
+            const float2 y = __ffma2_rn(x, sc2, nm2);
+            const float2 pr = exp2_mixed(y, k);
+            acc[k & 3] = __fadd2_rn(acc[k & 3], pr);
+            packed[k] = C::F16 ? pack_f16x2(pr.x, pr.y) : pack_bf16x2(pr.x, pr.y);
+          }
+          st_packed<HS / 2>(lane_base + C::S_COL + buf * C::BN + wg * (HS / 2), packed);
         }
-        st_packed<HS / 2>(lane_base + C::S_COL + buf * C::BN + wg * (HS / 2), packed);
         const float2 acc4 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         l_run += acc4.x + acc4.y;
         tc_fence_before();

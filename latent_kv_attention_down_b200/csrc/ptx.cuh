@@ -337,6 +337,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// Store 16 consecutive columns without waiting (tmem_wait_st before the data is relied on).
+__device__ __forceinline__ void tmem_st16_async(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      VMLA_W8(0), VMLA_W8(8)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Store 24 consecutive columns (x16 at taddr, x8 at taddr + 16), then wait.
 __device__ __forceinline__ void tmem_st24(uint32_t taddr, const uint32_t (&r)[24]) {
   asm volatile(

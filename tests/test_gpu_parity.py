@@ -273,7 +273,7 @@ def _gate_fails(reason):
     return pytest.mark.xfail(strict=True, reason="fails the max-error gate: " + reason)
 
 
-DENSE_FAILS = {(64, 192, 2), (96, 192, 10)}
+DENSE_FAILS = {(96, 192, 10)}
 
 
 @pytest.mark.parametrize("d_rope,d_latent,chunks", [
