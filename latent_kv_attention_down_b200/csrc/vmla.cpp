@@ -173,11 +173,12 @@ vmla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VMLA_OK : cud
 //  - d_latent >= 192, or a split the absorbed kernel does not hold (past 256 latent dims; 64 or 96
 //    rotary dims past 192): RECON_ONCE.  Per (query, key, head) the per-head attention multiplies
 //    2 d_head = 256 pairs where the absorbed one multiplies 2 d_latent + d_rope (416 at 192), and
-//    rebuilding the window's per-head K/V costs about 2 us per 1000 keys (Wan-1.3B layer: 0.91 ms
+//    rebuilding the window's per-head K/V costs about 2 us per 1000 keys (Wan-1.3B layer: 0.87 ms
 //    against 1.05 ms per call).  Its per-head K, V, queries and probabilities are fp16, which keeps
 //    it inside the gate on every window, the shortest (600 keys) included;
 //  - d_latent 64 or 128: ABSORBED, whose extra MMA work is then no larger than the reconstruction's
-//    (0.83 / 0.87 ms against 0.92 ms per call at the Wan layer).
+//    (0.84 against 0.86 ms per call at d_latent 64, 0.87 against 0.87 at 128, Wan layer), and which
+//    needs no per-head workspace.
 vmla_design resolve_design(const vmla_config& c, vmla_design d, int64_t n_keys) {
   (void)n_keys;
   if (d != VMLA_DESIGN_AUTO) return d;
