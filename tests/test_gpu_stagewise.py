@@ -170,6 +170,17 @@ CASES = [(synth.WAN_SMALL, 1), (synth.WAN_SMALL, 7), (synth.WAN_SMALL, 10), (syn
          (_split(16), 7), (_split(64), 7), (_split(96), 7)]
 
 
+def _grid(h, w):
+    return synth.WAN_SMALL.replace(name=f"wan_grid{h}x{w}", grid_h=h, grid_w=w)
+
+
+# Windows whose last 192-key tile of the per-head kernel ends at each softmax group's edge (each
+# group takes 96 of a tile's keys): 96 keys (the second group's half empty), 192 (one full tile),
+# 195 (3 keys past it), 291 (the second group's half holding 3 keys), 672 (three tiles and an
+# empty half); 96, 195 and 291 queries make one to three ragged query tiles.
+TILE_EDGE_CASES = [(_grid(4, 8), 1), (_grid(4, 8), 2), (_grid(4, 8), 7), (_grid(5, 13), 1), (_grid(1, 97), 1)]
+
+
 @pytest.mark.parametrize("dims,chunks", CASES, ids=lambda v: getattr(v, "name", v))
 def test_stages_of_the_absorbed_design(dims, chunks):
     """Window RoPE, q-absorb and the absorbed attention core (with the fused W_uv) each against the
@@ -218,7 +229,7 @@ def test_stages_of_the_absorbed_design(dims, chunks):
           f"max err/rms {max(x[1] for x in worst):.2e}")
 
 
-@pytest.mark.parametrize("dims,chunks", CASES, ids=lambda v: getattr(v, "name", v))
+@pytest.mark.parametrize("dims,chunks", CASES + TILE_EDGE_CASES, ids=lambda v: getattr(v, "name", v))
 def test_stages_of_the_reconstruct_once_design(dims, chunks):
     """Per-head queries, the reconstruction of the window's per-head K/V and the d_head = 128
     attention core, each against the fp64 definition fed the GPU's inputs of that stage."""
@@ -278,11 +289,12 @@ def test_stages_of_the_reconstruct_once_design(dims, chunks):
           f"max err/rms {max(x[1] for x in worst):.2e}")
 
 
-@pytest.mark.parametrize("chunks", [1, 7])
-def test_stages_of_the_dense_comparison(chunks):
+@pytest.mark.parametrize("dims,chunks", [(synth.WAN_SMALL, 1), (synth.WAN_SMALL, 7)] + TILE_EDGE_CASES[1:4:2],
+                         ids=lambda v: getattr(v, "name", v))
+def test_stages_of_the_dense_comparison(dims, chunks):
     """The dense per-head cache (3072 scalars per token): its stored keys and values against the
     fp64 reconstruction from x's bf16 latents, and the attention core over the stored entries."""
-    d = synth.WAN_SMALL
+    d = dims
     ro = Rollout(d, dense=True)
     for c in range(chunks):
         ro.append_chunk(0, c, dense=True)
@@ -323,4 +335,4 @@ def test_stages_of_the_dense_comparison(chunks):
     for h in range(d.n_heads):
         got = out[0][:, h * d.d_head:(h + 1) * d.d_head]
         worst.append(attention_core_check(qd[h], dense[:, 0, h], dense[:, 1, h], got, f"dense core, head {h}"))
-    print(f"dense core {chunks} chunks: max err/sigma {max(x[0] for x in worst):.2f}")
+    print(f"dense core {d.name} {chunks} chunks: max err/sigma {max(x[0] for x in worst):.2f}")
