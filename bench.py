@@ -382,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
 
     if auto_design == "recon_once":
         # d_head = 128 attention over the window's per-head K/V: 2 * N_q * N_k * n_h * (128 + 128) FLOPs
-        roofline = tensor_roofline("attn_tc_kernel<128,true,false,32>", per_kernel["dense_attention"]["ms_per_launch"],
+        roofline = tensor_roofline("attn_tc_kernel<128,true,false,32,true>", per_kernel["dense_attention"]["ms_per_launch"],
                                    DF["attention"], profiled_traffic("attn_tc.cu", "attn_per_head_wan_layer.md"))
     else:
         roofline = tensor_roofline("attn_tc_kernel<192,false,false,32>", per_kernel["attention"]["ms_per_launch"],
