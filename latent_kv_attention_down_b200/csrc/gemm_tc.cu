@@ -747,7 +747,7 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128;
+    const int wg = (warp - 4) >> 2, wq = warp & 3, r = wq * 32 + lane, tid = threadIdx.x - 128, wt = tid & 127;
     const int T = a.ring.tokens_per_frame;
     // warpgroup 0 reads each key tile's positional keys (DR * 2 bytes of its row) one tile ahead
     constexpr int RQ = DR / 8;  // 16-byte pieces of a positional key
@@ -805,45 +805,45 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
       tc_fence_after();
       const int valid_rows = ok ? min(128, a.rows - mt * 128) : 0;
       float amax = 0.f;
-      if constexpr (TMA_OUT) {
-        if (tid == 0) bulk_wait_all_read();  // the previous item's stores have read the park
-        named_bar_sync(1, 256);
-        if (wg == 0) {  // k_h: TMEM columns 0..DN-1, then the positional part, into blocks 0 and 1
+      // TMEM columns [c_begin, c_end) of this row (a multiple of 16 wide) through `put`, 32 per wait
+      auto drain_cols = [&](int c_begin, int c_end, auto put) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < C::DN; c0 += 16) {
+        for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+          if (c0 + 32 <= c_end) {
+            uint32_t raw[32];
+            tmem_ld32(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
+            put(c0 - c_begin, reinterpret_cast<const float*>(raw));
+            put(c0 - c_begin + 16, reinterpret_cast<const float*>(raw) + 16);
+          } else {
             uint32_t raw[16];
             tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-            store_sw16_smem<F16>(sout, r, c0, reinterpret_cast<const float*>(raw), amax);
+            put(c0 - c_begin, reinterpret_cast<const float*>(raw));
           }
+        }
+      };
+      if constexpr (TMA_OUT) {
+        // each warpgroup parks and stores its own half of the item (k_h: blocks 0 and 1, v_h: blocks
+        // 2 and 3), waiting only for its own earlier stores and its own 128 threads
+        uint8_t* park = sout + wg * 2 * 16384;
+        if (wt == 0) bulk_wait_all_read();  // this warpgroup's previous stores have read its park
+        named_bar_sync(2 + wg, 128);
+        if (wg == 0) {  // k_h: TMEM columns 0..DN-1, then the positional part
+          drain_cols(0, C::DN, [&](int c, const float* v) { store_sw16_smem<F16>(park, r, c, v, amax); });
 #pragma unroll
-          for (int c0 = 0; c0 < DR; c0 += 16) store_sw16_smem<F16>(sout, r, C::DN + c0, kr + c0, amax);
-        } else {  // v_h: TMEM columns DN..DN+127 into blocks 2 and 3
-#pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 16) {
-            uint32_t raw[16];
-            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
-            store_sw16_smem<F16>(sout + 2 * 16384, r, c0, reinterpret_cast<const float*>(raw), amax);
-          }
+          for (int c0 = 0; c0 < DR; c0 += 16) store_sw16_smem<F16>(park, r, C::DN + c0, kr + c0, amax);
+        } else {  // v_h: TMEM columns DN..DN+127
+          drain_cols(C::DN, C::DN + 128, [&](int c, const float* v) { store_sw16_smem<F16>(park, r, c, v, amax); });
         }
         fence_async_smem();  // the tensor stores (async proxy) read what these threads wrote
       } else {
         uint8_t* orow = sout + r * C::OUT_STRIDE;
         if (wg == 0) {  // TMEM columns 0..DN-1: the content part of k_h, then its positional part
-#pragma unroll 1
-          for (int c0 = 0; c0 < C::DN; c0 += 16) {
-            uint32_t raw[16];
-            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + c0), raw);
-            store_x16_smem<F16>(orow + c0 * 2, reinterpret_cast<const float*>(raw), amax);
-          }
+          drain_cols(0, C::DN, [&](int c, const float* v) { store_x16_smem<F16>(orow + c * 2, v, amax); });
 #pragma unroll
           for (int c0 = 0; c0 < DR; c0 += 16) store_x16_smem<F16>(orow + (C::DN + c0) * 2, kr + c0, amax);
-        } else {  // TMEM columns DN..DN+127: v_h, parked from column 128 (16-column loads: DN is a multiple of 16)
-#pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 16) {
-            uint32_t raw[16];
-            tmem_ld16(tmem_addr(tbase, wq * 32, acc * 256 + C::DN + c0), raw);
-            store_x16_smem<F16>(orow + (128 + c0) * 2, reinterpret_cast<const float*>(raw), amax);
-          }
+        } else {  // TMEM columns DN..DN+127: v_h, parked from column 128
+          drain_cols(C::DN, C::DN + 128,
+                     [&](int c, const float* v) { store_x16_smem<F16>(orow + (128 + c) * 2, v, amax); });
         }
       }
       // fp16 holds magnitudes up to 65504: a row past it is reported, not stored as inf silently
@@ -851,15 +851,16 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);  // this warp's lanes are read
-      named_bar_sync(1, 256);  // the item is parked and its row table complete
       if constexpr (TMA_OUT) {
-        if (tid == 0 && valid_rows > 0) {  // rows past the window are clipped by the tensor map
-          for (int blk = 0; blk < 4; ++blk)
+        named_bar_sync(2 + wg, 128);  // this warpgroup's half of the item is parked
+        if (wt == 0 && valid_rows > 0) {  // rows past the window are clipped by the tensor map
+          for (int blk = 2 * wg; blk < 2 * wg + 2; ++blk)
             tma_store_3d(&tm_out, sout + blk * 16384, ((blk >> 1) * a.n_heads + h) * 128 + (blk & 1) * 64, mt * 128,
                          b);
           bulk_commit();
         }
       } else {
+        named_bar_sync(1, 256);  // the item is parked and its row table complete
 #pragma unroll 4
         for (int id = tid; id < valid_rows * 32; id += 256) {
           const int rr = id >> 5, ch = id & 31;
@@ -871,7 +872,7 @@ __global__ void __launch_bounds__(ReconCfg<DL, DR, TMA_OUT>::THREADS, 1)
       }
     }
     if constexpr (TMA_OUT) {
-      if (tid == 0) bulk_wait_all();  // the last stores have read shared memory and landed
+      if (wt == 0) bulk_wait_all();  // this warpgroup's last stores have read shared memory and landed
     }
   }
   tc_fence_before();
